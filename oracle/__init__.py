@@ -1,0 +1,147 @@
+"""fp64 CPU oracle for LoZA streaming sparse attention (SSA).
+
+TEST INFRASTRUCTURE. This package is the plain, slow reference that the CUDA
+library is checked against. Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline / reference legs of ``bench.py`` may import it. It shares no
+code with the CUDA library, and the library never imports it.
+
+The arithmetic lives in ``ssa_ref.c`` (plain C, double precision, OpenMP over
+rows); this module only compiles it with gcc and marshals numpy arrays. What it
+computes is stated in the header of ``ssa_ref.c`` with the passages it follows
+(Efficient Context Scaling with LongCat ZigZag Attention: page 1 section 01,
+page 2 section 2.2, page 5).
+
+Every array argument holding model values is a numpy ``uint16`` array of bf16
+bit patterns; the C side widens each exactly to double.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssa_ref.c")
+_LIB_PATH = os.path.join(_HERE, "libssa_oracle.so")
+_lib = None
+
+_u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+
+
+def build(force: bool = False) -> str:
+    """Compile ssa_ref.c into libssa_oracle.so next to it (gcc -O2 -fopenmp)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
+                    "-o", tmp, _SRC, "-lm"], check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.ssa_oracle_forward_rows.restype = ctypes.c_int
+        lib.ssa_oracle_forward_rows.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            _i64p, ctypes.c_int64, _f64p, _f64p]
+        lib.ssa_oracle_decode.restype = ctypes.c_int
+        lib.ssa_oracle_decode.argtypes = [
+            _u16p, _u16p, _u16p, ctypes.c_int64, _i32p, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            _f64p, _f64p]
+        lib.ssa_oracle_backward_rows.restype = ctypes.c_int
+        lib.ssa_oracle_backward_rows.argtypes = [
+            _u16p, _u16p, _u16p, _u16p, _i32p, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            _i64p, ctypes.c_int64, _i64p, ctypes.c_int64,
+            _f64p, _f64p, _f64p]
+        lib.ssa_oracle_visible_count.restype = ctypes.c_int64
+        lib.ssa_oracle_visible_count.argtypes = [
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (numpy uint16)")
+    return a
+
+
+def forward(q, k, v, cu_seqlens, n_heads, n_kv_heads, block_size=128, n_sink=1,
+            n_local=7, scale=1.0, rows=None):
+    """O [R,H,d_v] and LSE [R,H] (float64) for the query rows ``rows`` (all rows
+    when None). q [T,H,d_qk], k [T,Hkv,d_qk], v [T,Hkv,d_v] uint16 bf16 bits;
+    cu_seqlens int32 [B+1]. ``n_local=-1`` means an unbounded local window."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    T = int(cu[-1])
+    d_qk, d_v = q.shape[-1], v.shape[-1]
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    o = np.zeros((len(rows), n_heads, d_v), np.float64)
+    lse = np.zeros((len(rows), n_heads), np.float64)
+    rc = _load().ssa_oracle_forward_rows(q, k, v, cu, len(cu) - 1, n_heads, n_kv_heads,
+                                         d_qk, d_v, block_size, n_sink, n_local,
+                                         float(scale), rows, len(rows), o, lse)
+    if rc != 0:
+        raise ValueError("oracle forward rejected its arguments")
+    return o, lse
+
+
+def decode(q, k_cache, v_cache, seqlens, n_heads, n_kv_heads, block_size=128,
+           n_sink=1, n_local=7, scale=1.0):
+    """O [B,H,d_v], LSE [B,H] for one query per sequence (position L_n - 1).
+    q [B,H,d_qk]; k_cache [B,Lcap,Hkv,d_qk]; v_cache [B,Lcap,Hkv,d_v]."""
+    q, kc, vc = _u16(q), _u16(k_cache), _u16(v_cache)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    B = q.shape[0]
+    d_qk, d_v = q.shape[-1], vc.shape[-1]
+    o = np.zeros((B, n_heads, d_v), np.float64)
+    lse = np.zeros((B, n_heads), np.float64)
+    rc = _load().ssa_oracle_decode(q, kc, vc, kc.shape[1], sl, B, n_heads, n_kv_heads,
+                                   d_qk, d_v, block_size, n_sink, n_local, float(scale),
+                                   o, lse)
+    if rc != 0:
+        raise ValueError("oracle decode rejected its arguments")
+    return o, lse
+
+
+def backward(q, k, v, dout, cu_seqlens, n_heads, n_kv_heads, block_size=128,
+             n_sink=1, n_local=7, scale=1.0, q_rows=None, k_rows=None):
+    """dQ [Rq,H,d_qk] for ``q_rows`` and dK [Rk,Hkv,d_qk], dV [Rk,Hkv,d_v] for
+    ``k_rows`` (float64); None selects every row."""
+    q, k, v, dout = _u16(q), _u16(k), _u16(v), _u16(dout)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    T = int(cu[-1])
+    d_qk, d_v = q.shape[-1], v.shape[-1]
+    q_rows = np.arange(T, dtype=np.int64) if q_rows is None else np.ascontiguousarray(q_rows, dtype=np.int64)
+    k_rows = np.arange(T, dtype=np.int64) if k_rows is None else np.ascontiguousarray(k_rows, dtype=np.int64)
+    dq = np.zeros((len(q_rows), n_heads, d_qk), np.float64)
+    dk = np.zeros((len(k_rows), n_kv_heads, d_qk), np.float64)
+    dv = np.zeros((len(k_rows), n_kv_heads, d_v), np.float64)
+    rc = _load().ssa_oracle_backward_rows(q, k, v, dout, cu, len(cu) - 1, n_heads,
+                                          n_kv_heads, d_qk, d_v, block_size, n_sink,
+                                          n_local, float(scale), q_rows, len(q_rows),
+                                          k_rows, len(k_rows), dq, dk, dv)
+    if rc != 0:
+        raise ValueError("oracle backward rejected its arguments")
+    return dq, dk, dv
+
+
+def visible_count(i, block_size=128, n_sink=1, n_local=7) -> int:
+    """|A(i)| under the oracle's block-index map."""
+    return int(_load().ssa_oracle_visible_count(int(i), block_size, n_sink, n_local))
