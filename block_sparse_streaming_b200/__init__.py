@@ -1,0 +1,206 @@
+"""B200 (sm_100a) streaming sparse attention of LongCat ZigZag Attention.
+
+Python binding of the C ABI in ``include/loza_ssa.h``: argument marshalling
+only. Every step of the computation runs in the CUDA kernels of
+``libloza_ssa.so``; there is no CPU path. If the library is missing or cannot
+be loaded, every call raises.
+
+Tensors are torch CUDA tensors (PyTorch provides device memory and streams):
+  q [T, H, d_qk], k [T, Hkv, d_qk], v [T, Hkv, d_v] bf16 (rows may be strided,
+  heads and head dims contiguous); for the absorbed MLA layout pass the latent
+  [T, 1, 576] as k and its first 512 columns (a view of the same storage) as v.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from ._build import LIB_PATH, build  # noqa: F401  (build is re-exported)
+
+LOZA_UNBOUNDED = -1
+LOZA_OP_PREFILL, LOZA_OP_DECODE, LOZA_OP_BACKWARD = 0, 1, 2
+
+_STATUS = {
+    0: "LOZA_OK",
+    -1: "LOZA_ERR_INVALID_ARG",
+    -2: "LOZA_ERR_UNSUPPORTED",
+    -3: "LOZA_ERR_WORKSPACE",
+    -4: "LOZA_ERR_CUDA",
+    -5: "LOZA_ERR_TIMEOUT",
+}
+
+# Every symbol include/loza_ssa.h declares.
+EXPORTED = [
+    "loza_ssa_workspace_size",
+    "loza_ssa_prefill",
+    "loza_ssa_decode",
+    "loza_ssa_backward",
+    "loza_status_string",
+    "loza_device_status",
+    "loza_launch_count",
+]
+
+
+class LozaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+class Params(ctypes.Structure):
+    """loza_ssa_params {block_size, n_sink, n_local, scale}."""
+    _fields_ = [("block_size", ctypes.c_int32), ("n_sink", ctypes.c_int32),
+                ("n_local", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+    def __init__(self, scale: float, block_size: int = 128, n_sink: int = 1, n_local: int = 7):
+        super().__init__(block_size, n_sink, n_local, scale)
+
+
+_lib = None
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libloza_ssa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run block_sparse_streaming_b200.build() "
+                               "(nvcc, sm_100a); there is no fallback path")
+        L = ctypes.CDLL(LIB_PATH)
+        L.loza_ssa_workspace_size.restype = _sz
+        L.loza_ssa_workspace_size.argtypes = [ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _i32, Params]
+        L.loza_ssa_prefill.restype = ctypes.c_int
+        L.loza_ssa_prefill.argtypes = [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
+                                       _i64, _i64, _i64, Params, _vp, _vp, _vp, _sz, _vp]
+        L.loza_ssa_decode.restype = ctypes.c_int
+        L.loza_ssa_decode.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i64, _i64, _i32, _i32, _i32, _i32,
+                                      Params, _vp, _vp, _vp, _sz, _vp]
+        L.loza_ssa_backward.restype = ctypes.c_int
+        L.loza_ssa_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
+                                        _i32, _i32, Params, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.loza_status_string.restype = ctypes.c_char_p
+        L.loza_status_string.argtypes = [ctypes.c_int]
+        L.loza_device_status.restype = ctypes.c_int
+        L.loza_device_status.argtypes = [_vp]
+        L.loza_launch_count.restype = ctypes.c_uint64
+        L.loza_launch_count.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise LozaError(rc, what)
+
+
+def _stream_ptr(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _require(t, name, dtype=None, ndim=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+
+
+def _row_tensor(t, name):
+    """[rows, heads, dim] with heads/dim contiguous; returns its row stride."""
+    if t.stride(2) != 1 or (t.shape[1] > 1 and t.stride(1) != t.shape[2]):
+        raise ValueError(f"{name}: heads and head dim must be contiguous within a row")
+    return t.stride(0)
+
+
+def workspace_size(op, batch, total_tokens, max_seqlen, n_heads, n_kv_heads, d_qk, d_v, params: Params) -> int:
+    return int(lib().loza_ssa_workspace_size(op, batch, total_tokens, max_seqlen, n_heads, n_kv_heads,
+                                             d_qk, d_v, params))
+
+
+def loza_ssa_prefill(q, k, v, cu_seqlens, max_seqlen: int, params: Params, out=None, lse=None,
+                     workspace=None, stream=None):
+    """SSA forward over a packed batch. Returns (out [T,H,d_v] bf16, lse [T,H] fp32)."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, torch.bfloat16, 3)
+    _require(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, H, d_qk = q.shape
+    Hkv, d_v = k.shape[1], v.shape[2]
+    if out is None:
+        out = torch.empty((T, H, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib().loza_ssa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T,
+                                int(max_seqlen), H, Hkv, d_qk, d_v, _row_tensor(q, "q"), _row_tensor(k, "k"),
+                                _row_tensor(v, "v"), params, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+                                _stream_ptr(stream))
+    _check(rc, "loza_ssa_prefill")
+    return out, lse
+
+
+def loza_ssa_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, params: Params, out=None, lse=None,
+                    workspace=None, stream=None):
+    """SSA decode. q [B,H,d_qk]; k_cache [B,Lcap,Hkv,d_qk] (row/batch strides taken from the
+    tensor); v_cache None for the absorbed latent cache. Returns (out [B,H,d_v], lse [B,H])."""
+    import torch
+    _require(q, "q", torch.bfloat16, 3)
+    _require(k_cache, "k_cache", torch.bfloat16, 4)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B, H, d_qk = q.shape
+    Hkv = k_cache.shape[2]
+    d_v = v_cache.shape[3] if v_cache is not None else 512
+    if k_cache.stride(3) != 1 or (Hkv > 1 and k_cache.stride(2) != d_qk):
+        raise ValueError("k_cache: heads and head dim must be contiguous within a row")
+    if out is None:
+        out = torch.empty((B, H, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = workspace_size(LOZA_OP_DECODE, B, 0, int(max_seqlen), H, Hkv, d_qk, d_v, params)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().loza_ssa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, int(max_seqlen),
+                               k_cache.stride(0), k_cache.stride(1), H, Hkv, d_qk, d_v, params, _ptr(out),
+                               _ptr(lse), _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check(rc, "loza_ssa_decode")
+    return out, lse
+
+
+def loza_ssa_backward(q, k, v, out, dout, lse, cu_seqlens, max_seqlen: int, params: Params, dq=None, dk=None,
+                      dv=None, workspace=None, stream=None):
+    """SSA backward. All of q, k, v, out, dout contiguous [T, heads, dim]. Returns (dq, dk, dv)."""
+    import torch
+    T, H, d_qk = q.shape
+    Hkv, d_v = k.shape[1], v.shape[2]
+    B = cu_seqlens.numel() - 1
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        n = workspace_size(LOZA_OP_BACKWARD, B, T, int(max_seqlen), H, Hkv, d_qk, d_v, params)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().loza_ssa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(cu_seqlens),
+                                 B, T, int(max_seqlen), H, Hkv, d_qk, d_v, params, _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check(rc, "loza_ssa_backward")
+    return dq, dk, dv
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and return the kernels' device status (0, or -5 after a timed-out wait)."""
+    return int(lib().loza_device_status(_stream_ptr(stream)))
+
+
+def launch_count() -> int:
+    return int(lib().loza_launch_count())

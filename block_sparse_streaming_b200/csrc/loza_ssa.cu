@@ -1,0 +1,193 @@
+// loza_ssa.cu - host side of the C ABI declared in include/loza_ssa.h:
+// argument validation, TMA descriptor construction, kernel selection and
+// launch on the caller's stream. All arithmetic runs in the kernels included
+// below; nothing here touches tensor data.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "loza_ssa.h"
+#include "prefill.cuh"
+
+namespace loza {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+// cuTensorMapEncodeTiled, fetched from the driver at first use (no libcuda link).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D bf16 map over [rows, heads, dim] with 128-byte swizzle and a
+// {64, 1, 128} box: one [128 rows x 64 columns] tile of one head per load.
+bool make_map_3d(CUtensorMap* m, const void* base, int64_t dim, int64_t heads, int64_t rows,
+                 int64_t head_stride_elems, int64_t row_stride_elems) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)(head_stride_elems * 2), (cuuint64_t)(row_stride_elems * 2)};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride_ok(int64_t s) { return s > 0 && (s * 2) % 16 == 0 && s * 2 < (int64_t(1) << 40); }
+
+bool window_ok(const loza_ssa_params& p) {
+  if (p.block_size != kTile) return false;
+  if (p.n_local != LOZA_UNBOUNDED && (p.n_local < 1 || p.n_sink < 0)) return false;
+  return true;
+}
+
+template <int DQK, int DVT, int NSTAGE>
+loza_status launch_prefill(const PrefillParams& prm, int max_seqlen, int batch, cudaStream_t stream) {
+  using LY = PrefillLayout<DQK, DVT, NSTAGE>;
+  auto kern = ssa_prefill_kernel<DQK, DVT, NSTAGE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM_BYTES) != cudaSuccess)
+    return LOZA_ERR_CUDA;
+  dim3 grid((max_seqlen + kTile - 1) / kTile, prm.n_heads * prm.dv_slices, batch);
+  kern<<<grid, kPrefillThreads, LY::SMEM_BYTES, stream>>>(prm);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace loza
+
+using namespace loza;
+
+extern "C" {
+
+const char* loza_status_string(loza_status s) {
+  switch (s) {
+    case LOZA_OK: return "ok";
+    case LOZA_ERR_INVALID_ARG: return "invalid argument";
+    case LOZA_ERR_UNSUPPORTED: return "unsupported shape or window";
+    case LOZA_ERR_WORKSPACE: return "workspace too small";
+    case LOZA_ERR_CUDA: return "CUDA error";
+    case LOZA_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+uint64_t loza_launch_count(void) { return g_launches.load(); }
+
+loza_status loza_device_status(loza_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return LOZA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return LOZA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return LOZA_ERR_CUDA;
+    return LOZA_ERR_TIMEOUT;
+  }
+  return LOZA_OK;
+}
+
+size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int32_t max_seqlen,
+                               int32_t n_heads, int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
+                               loza_ssa_params p) {
+  (void)total_tokens; (void)max_seqlen; (void)n_kv_heads; (void)d_qk; (void)d_v; (void)p;
+  (void)batch; (void)n_heads;
+  if (op == LOZA_OP_PREFILL) return 0;
+  return 0;
+}
+
+loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                             int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t n_heads,
+                             int32_t n_kv_heads, int32_t d_qk, int32_t d_v, int64_t q_row_stride,
+                             int64_t k_row_stride, int64_t v_row_stride, loza_ssa_params p, void* out,
+                             float* lse, void* workspace, size_t workspace_bytes, loza_stream_t stream) {
+  (void)workspace; (void)workspace_bytes;
+  if (!q || !k || !v || !cu_seqlens || !out || !lse) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || total_tokens < 1 || total_tokens > INT32_MAX || max_seqlen < 1 ||
+      max_seqlen > total_tokens)
+    return LOZA_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
+  if (!stride_ok(q_row_stride) || !stride_ok(k_row_stride) || !stride_ok(v_row_stride))
+    return LOZA_ERR_INVALID_ARG;
+  if (q_row_stride < (int64_t)n_heads * d_qk || k_row_stride < (int64_t)n_kv_heads * d_qk)
+    return LOZA_ERR_INVALID_ARG;
+  const bool latent_v = (v == k);
+  if (latent_v ? (d_v > d_qk || v_row_stride != k_row_stride) : v_row_stride < (int64_t)n_kv_heads * d_v)
+    return LOZA_ERR_INVALID_ARG;
+  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (!(n_kv_heads == 1 || n_kv_heads == n_heads)) return LOZA_ERR_UNSUPPORTED;
+
+  PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.cu_seqlens = cu_seqlens;
+  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.n_heads = n_heads;
+  prm.n_kv_heads = n_kv_heads;
+  prm.d_v = d_v;
+  prm.n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
+  prm.n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
+  prm.scale_log2 = p.scale * 1.4426950408889634f;
+
+  int dvt;
+  if (d_qk == 64 && d_v == 64) dvt = 64;
+  else if (d_qk == 192 && d_v == 128) dvt = 128;
+  else if (d_qk == 576 && d_v == 512) dvt = 256;
+  else return LOZA_ERR_UNSUPPORTED;
+  prm.dv_slices = d_v / dvt;
+  if ((int64_t)n_heads * prm.dv_slices > 65535) return LOZA_ERR_UNSUPPORTED;
+
+  const int64_t v_head_stride = latent_v ? d_qk : d_v;
+  if (!make_map_3d(&prm.tm_q, q, d_qk, n_heads, total_tokens, d_qk, q_row_stride) ||
+      !make_map_3d(&prm.tm_k, k, d_qk, n_kv_heads, total_tokens, d_qk, k_row_stride) ||
+      !make_map_3d(&prm.tm_v, v, d_v, n_kv_heads, total_tokens, v_head_stride, v_row_stride))
+    return LOZA_ERR_CUDA;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  switch (dvt) {
+    case 64: return launch_prefill<64, 64, 8>(prm, max_seqlen, batch, st);
+    case 128: return launch_prefill<192, 128, 8>(prm, max_seqlen, batch, st);
+    default: return launch_prefill<576, 256, 5>(prm, max_seqlen, batch, st);
+  }
+}
+
+loza_status loza_ssa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                            int32_t batch, int32_t max_seqlen, int64_t cache_batch_stride,
+                            int64_t cache_row_stride, int32_t n_heads, int32_t n_kv_heads, int32_t d_qk,
+                            int32_t d_v, loza_ssa_params p, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, loza_stream_t stream) {
+  (void)q; (void)k_cache; (void)v_cache; (void)seqlens; (void)batch; (void)max_seqlen;
+  (void)cache_batch_stride; (void)cache_row_stride; (void)n_heads; (void)n_kv_heads; (void)d_qk; (void)d_v;
+  (void)p; (void)out; (void)lse; (void)workspace; (void)workspace_bytes; (void)stream;
+  return LOZA_ERR_UNSUPPORTED;
+}
+
+loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                              const float* lse, const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
+                              int32_t max_seqlen, int32_t n_heads, int32_t n_kv_heads, int32_t d_qk,
+                              int32_t d_v, loza_ssa_params p, void* dq, void* dk, void* dv, void* workspace,
+                              size_t workspace_bytes, loza_stream_t stream) {
+  (void)q; (void)k; (void)v; (void)out; (void)dout; (void)lse; (void)cu_seqlens; (void)batch;
+  (void)total_tokens; (void)max_seqlen; (void)n_heads; (void)n_kv_heads; (void)d_qk; (void)d_v; (void)p;
+  (void)dq; (void)dk; (void)dv; (void)workspace; (void)workspace_bytes; (void)stream;
+  return LOZA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,335 @@
+// prefill.cuh - SSA prefill / training forward on sm_100a (tcgen05 + TMA).
+//
+// One CTA computes a 128-query tile (128 consecutive tokens of one sequence,
+// one head) against the key blocks the window selects, for one slice of the
+// value dimension:
+//   key blocks of query block j:  sink blocks 0 .. min(s, j+1)-1, then local
+//   blocks max(s, j-l+1) .. j (page 1 section 01 (1)-(2) of the LoZA pages:
+//   sink + local blocks of b = 128 tokens, s = 1, l = 7), diagonal block last;
+//   token-causal inside block j.
+//
+// Pipeline (warp-specialised, 6 warps):
+//   warp 0      TMA producer: Q tile once, then K chunks / V chunks of every
+//               selected block into a ring of 16 KB [128 x 64] bf16 tiles
+//               (128-byte swizzle), in exactly the order the MMA consumes them.
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
+//                 S_b  = Q K_b^T      (A = Q smem, B = K smem, both K-major)
+//                 O   += P_b V_b      (A = P in TMEM, B = V smem, MN-major)
+//               S is double-buffered in TMEM so S_{b+1} runs while the
+//               softmax works on S_b; P_b overwrites the first half of S_b.
+//   warps 2..5  softmax / correction / epilogue, one query row per thread
+//               (thread <-> TMEM lane). Online softmax in base 2; O is
+//               rescaled in TMEM only when the running max grows by more than
+//               2^8 (otherwise the stale max is kept, which is exact).
+//
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+DVT).
+// The value dimension is split into slices of DVT <= 256 columns so that O
+// fits next to the two S buffers; the d_v = 512 (absorbed MLA) case runs two
+// slices, each recomputing S.
+#pragma once
+
+#include <cuda.h>
+
+#include "sm100.cuh"
+
+namespace loza {
+
+struct PrefillParams {
+  CUtensorMap tm_q;   // [T, H, DQK]   box {64, 1, 128}
+  CUtensorMap tm_k;   // [T, Hkv, DQK] box {64, 1, 128}
+  CUtensorMap tm_v;   // [T, Hkv, DV]  box {64, 1, 128}
+  const int32_t* cu_seqlens;
+  __nv_bfloat16* out;  // [T, H, DV]
+  float* lse;          // [T, H]
+  int n_heads;
+  int n_kv_heads;
+  int d_v;             // full value width (row length of out)
+  int dv_slices;       // d_v / DVT
+  int n_sink;          // already 0 for the unbounded window
+  int n_local;         // < 0: unbounded (full causal)
+  float scale_log2;    // scale * log2(e)
+};
+
+constexpr int kTile = 128;               // queries per tile == keys per block
+constexpr int kChunkBytes = 128 * 64 * 2;  // one [128 x 64] bf16 tile
+constexpr int kPrefillThreads = 192;
+constexpr uint32_t kRescaleThreshold = 8;  // log2 units
+
+template <int DQK, int DVT, int NSTAGE>
+struct PrefillLayout {
+  static constexpr int NQC = DQK / 64;
+  static constexpr int NVC = DVT / 64;
+  static constexpr int Q_OFF = 0;
+  static constexpr int RING_OFF = NQC * kChunkBytes;
+  static constexpr int BAR_OFF = RING_OFF + NSTAGE * kChunkBytes;
+  // barriers: q_full, ring_full[NSTAGE], ring_empty[NSTAGE], s_full[2], p_full, pv_done
+  static constexpr int BAR_Q = 0;
+  static constexpr int BAR_FULL = 1;
+  static constexpr int BAR_EMPTY = 1 + NSTAGE;
+  static constexpr int BAR_S = 1 + 2 * NSTAGE;
+  static constexpr int BAR_P = BAR_S + 2;
+  static constexpr int BAR_PV = BAR_P + 1;
+  static constexpr int NBAR = BAR_PV + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base (u32), abort (int)
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+  static_assert(DQK % 64 == 0 && DVT % 64 == 0 && DVT <= 256, "tile shape");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Key block visited at step `it` of query block qb (sinks first, diagonal last).
+struct BlockWalk {
+  int sinks, local_lo, count;
+  __device__ __forceinline__ BlockWalk(int qb, int n_sink, int n_local) {
+    sinks = min(n_sink, qb + 1);
+    local_lo = n_local < 0 ? sinks : max(n_sink, qb - n_local + 1);
+    count = sinks + max(0, qb - local_lo + 1);
+  }
+  __device__ __forceinline__ int block(int it) const { return it < sinks ? it : local_lo + (it - sinks); }
+};
+
+template <int DQK, int DVT, int NSTAGE>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
+  using LY = PrefillLayout<DQK, DVT, NSTAGE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int qb = blockIdx.x;
+  const int head = blockIdx.y / p.dv_slices;
+  const int slice = blockIdx.y % p.dv_slices;
+  const int seq = blockIdx.z;
+  const int seq_start = p.cu_seqlens[seq];
+  const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
+  if (qb * kTile >= seq_len) return;  // whole CTA leaves before any setup
+  const int hk = head / (p.n_heads / p.n_kv_heads);
+  const BlockWalk walk(qb, p.n_sink, p.n_local);
+  const int nb = walk.count;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + LY::BAR_OFF;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(LY::BAR_Q), 1);
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(bar(LY::BAR_FULL + i), 1);
+      mbar_init(bar(LY::BAR_EMPTY + i), 1);
+    }
+    mbar_init(bar(LY::BAR_S + 0), 1);
+    mbar_init(bar(LY::BAR_S + 1), 1);
+    mbar_init(bar(LY::BAR_P), 128);
+    mbar_init(bar(LY::BAR_PV), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      const int row0 = seq_start + qb * kTile;
+      mbar_arrive_expect_tx(bar(LY::BAR_Q), LY::NQC * kChunkBytes);
+      for (int c = 0; c < LY::NQC; ++c)
+        tma_load_3d(sbase + LY::Q_OFF + c * kChunkBytes, &p.tm_q, bar(LY::BAR_Q), c * 64, head, row0);
+      int slot = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int it = 0; it <= nb && ok; ++it) {
+        if (it < nb) {
+          const int krow = seq_start + walk.block(it) * kTile;
+          for (int c = 0; c < LY::NQC && ok; ++c) {
+            ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
+            tma_load_3d(sbase + LY::RING_OFF + slot * kChunkBytes, &p.tm_k, bar(LY::BAR_FULL + slot),
+                        c * 64, hk, krow);
+            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
+          }
+        }
+        if (it >= 1) {
+          const int vrow = seq_start + walk.block(it - 1) * kTile;
+          for (int c = 0; c < LY::NVC && ok; ++c) {
+            ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
+            tma_load_3d(sbase + LY::RING_OFF + slot * kChunkBytes, &p.tm_v, bar(LY::BAR_FULL + slot),
+                        slice * DVT + c * 64, hk, vrow);
+            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, 64, false, true);
+      const uint32_t tmem_o = tmem + 256;
+      int slot = 0;
+      uint32_t phase = 0;
+      bool ok = mbar_wait(bar(LY::BAR_Q), 0, abort_flag);
+      tc_fence_after();
+      for (int it = 0; it <= nb && ok; ++it) {
+        if (it < nb) {
+          const uint32_t tmem_s = tmem + (it & 1) * 128;
+          for (int c = 0; c < LY::NQC; ++c) {
+            ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t qa = sbase + LY::Q_OFF + c * kChunkBytes;
+            const uint32_t kbuf = sbase + LY::RING_OFF + slot * kChunkBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem_s, sdesc_sw128(qa + 32 * kk, 16, 1024), sdesc_sw128(kbuf + 32 * kk, 16, 1024),
+                     idesc_s, (c | kk) != 0);
+            mma_commit(bar(LY::BAR_EMPTY + slot));
+            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
+          }
+          if (!ok) break;
+          mma_commit(bar(LY::BAR_S + (it & 1)));
+        }
+        if (it >= 1) {
+          const int b = it - 1;
+          ok = mbar_wait(bar(LY::BAR_P), b & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t tmem_p = tmem + (b & 1) * 128;
+          for (int c = 0; c < LY::NVC; ++c) {
+            ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t vbuf = sbase + LY::RING_OFF + slot * kChunkBytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem_o + c * 64, tmem_p + kk * 8, sdesc_sw128(vbuf + 2048 * kk, 8192, 1024), idesc_pv,
+                     (b > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar(LY::BAR_EMPTY + slot));
+            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
+          }
+          if (!ok) break;
+          mma_commit(bar(LY::BAR_PV));
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;               // row of the tile == TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int qpos = qb * kTile + row;                  // position inside the sequence
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int b = 0; b < nb && ok; ++b) {
+      ok = mbar_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      float s[128];
+      {
+        float t[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tmem_ld32(lane_addr + (b & 1) * 128 + 32 * j, t);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * j + i] = t[i];
+        }
+      }
+      const bool diag = walk.block(b) == qb;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 128; ++j) {
+        float x = s[j] * p.scale_log2;
+        if (diag && j > row) x = -INFINITY;
+        s[j] = x;
+        mx = fmaxf(mx, x);
+      }
+      if (b > 0) {
+        ok = mbar_wait(bar(LY::BAR_PV), (b - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      float alpha = 1.f;
+      if (b == 0) {
+        m_run = mx;
+      } else if (mx > m_run + (float)kRescaleThreshold) {
+        alpha = exp2f(m_run - mx);
+        m_run = mx;
+      }
+      // O rescale (warp-uniform decision so the TMEM accesses stay converged)
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < DVT / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + 256 + 32 * c, o);
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+          tmem_st32(lane_addr + 256 + 32 * c, w);
+        }
+        tmem_st_wait();
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = exp2f(s[64 * h + 2 * i] - m_run);
+          const float p1 = exp2f(s[64 * h + 2 * i + 1] - m_run);
+          sum += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st32(lane_addr + (b & 1) * 128 + 32 * h, pk);
+      }
+      l_run = l_run * alpha + sum;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(LY::BAR_P));
+    }
+    if (ok) ok = mbar_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      const bool valid = qpos < seq_len;
+      const int64_t grow = (int64_t)seq_start + qpos;
+      __nv_bfloat16* orow = p.out + (grow * p.n_heads + head) * (int64_t)p.d_v + slice * DVT;
+#pragma unroll 1
+      for (int c = 0; c < DVT / 32; ++c) {
+        float o[32];
+        tmem_ld32(lane_addr + 256 + 32 * c, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * inv, o[2 * i + 1] * inv);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (valid && slice == 0)
+        p.lse[grow * p.n_heads + head] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace loza

@@ -1,0 +1,175 @@
+/*
+ * loza_ssa.h - C ABI of the B200 (sm_100a) streaming sparse attention library.
+ *
+ * Streaming sparse attention (SSA) is the sparse branch of LongCat ZigZag
+ * Attention (Efficient Context Scaling with LongCat ZigZag Attention, page 1,
+ * section 01 (1) "calibration"): every query token attends, by softmax
+ * attention, only to selected and blocked keys/values K*, V*, defined by the
+ * block size b, the number of sink blocks s and the number of local blocks l.
+ * Page 1 section 01 (2) fixes b = 128, s = 1, l = 7, a 1,024-token window;
+ * page 5 (QbitAI article) describes it as one global block and seven local
+ * blocks of 128 tokens. With query position i in block j = floor(i/b), the keys
+ * of a query are
+ *     t <= i  with  floor(t/b) in {0 .. s-1} U {j-l+1 .. j}
+ * i.e. the sink blocks, the l most recent blocks including its own, and
+ * token-causal inside its own block (the "streaming" pattern). Blocks restart
+ * at every sequence start of a packed batch; a sequence's last block may be
+ * short.
+ *
+ * The operator runs inside MLA modules (page 1 section 01 (1); page 2 section
+ * 1.2). Two layouts are supported:
+ *   - per-head K/V ("non-absorbed" MLA, MHA): n_kv_heads == n_heads,
+ *     (d_qk, d_v) in {(64, 64), (192, 128)};
+ *   - one latent KV row shared by all heads ("absorbed" MLA): n_kv_heads == 1,
+ *     d_qk = 576 (512 latent + 64 rope) and d_v = 512, where V is the first 512
+ *     columns of the latent row (pass v == k).
+ *
+ * Conventions for every entry point:
+ *   - All pointers named q, k, v, out, dout, dq, dk, dv, lse, workspace,
+ *     cu_seqlens and seqlens are DEVICE pointers. bf16 tensors are raw bf16
+ *     bit patterns. The caller owns and allocates every buffer; the library
+ *     never allocates, frees or synchronises.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream).
+ *   - Validation errors return a negative status BEFORE anything is launched.
+ *     A launch failure returns LOZA_ERR_CUDA. Kernels never trap; a kernel
+ *     that gives up on a bounded wait records LOZA_ERR_TIMEOUT, which
+ *     loza_device_status() reports.
+ *   - Strides are in elements. Rows (tokens) may be strided; within a row,
+ *     heads are contiguous with head stride = head dim.
+ *   - Every row stride times 2 bytes and every base pointer must be 16-byte
+ *     aligned (TMA requirement); otherwise LOZA_ERR_INVALID_ARG.
+ *   - Only block_size == 128 is compiled; n_sink >= 0, n_local >= 1, or
+ *     n_local == LOZA_UNBOUNDED for full causal attention (n_sink ignored).
+ */
+#ifndef LOZA_SSA_H
+#define LOZA_SSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without the CUDA headers: the same opaque pointer. */
+typedef struct CUstream_st *loza_stream_t;
+
+/* Window parameters {b, s, l, scale}; the pages' configuration is
+ * {128, 1, 7, scale}. scale multiplies q.k before the softmax. */
+typedef struct {
+    int32_t block_size;
+    int32_t n_sink;
+    int32_t n_local;
+    float scale;
+} loza_ssa_params;
+
+/* n_local value selecting full causal attention (the dense baseline). */
+#define LOZA_UNBOUNDED (-1)
+
+typedef enum {
+    LOZA_OK = 0,
+    LOZA_ERR_INVALID_ARG = -1,
+    LOZA_ERR_UNSUPPORTED = -2,
+    LOZA_ERR_WORKSPACE = -3,
+    LOZA_ERR_CUDA = -4,
+    LOZA_ERR_TIMEOUT = -5
+} loza_status;
+
+/* Operation codes for loza_ssa_workspace_size. */
+#define LOZA_OP_PREFILL 0
+#define LOZA_OP_DECODE 1
+#define LOZA_OP_BACKWARD 2
+
+/*
+ * Bytes of device workspace the operation needs for this shape (0 if none).
+ * batch: number of sequences; total_tokens: packed tokens (prefill/backward);
+ * max_seqlen: longest sequence (decode: longest context). Returns 0 for an
+ * unsupported shape as well; the entry point then reports the error.
+ */
+size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int32_t max_seqlen,
+                               int32_t n_heads, int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
+                               loza_ssa_params p);
+
+/*
+ * Prefill / training forward over a packed variable-length batch.
+ *   q   [T, n_heads, d_qk]     bf16, token stride q_row_stride (>= n_heads*d_qk)
+ *   k   [T, n_kv_heads, d_qk]  bf16, token stride k_row_stride
+ *   v   [T, n_kv_heads, d_v]   bf16, token stride v_row_stride (absorbed: v == k,
+ *                              v_row_stride == k_row_stride, V = first d_v columns)
+ *   cu_seqlens int32 [batch+1], cu_seqlens[0] = 0, non-decreasing,
+ *               cu_seqlens[batch] == total_tokens (T)
+ *   total_tokens T, the packed row count of q, k, v, out and lse (the bound the
+ *               TMA descriptors are built with; rows past T read as zero)
+ *   max_seqlen  >= every sequence length (sizes the launch grid)
+ *   out [T, n_heads, d_v] bf16 contiguous; lse [T, n_heads] fp32, natural log of
+ *   the sum of exp(scale * q.k) over the visible keys.
+ * Definition: page 1 section 01 (1) and (2) of the LoZA pages (see above).
+ */
+loza_status loza_ssa_prefill(const void *q, const void *k, const void *v,
+                             const int32_t *cu_seqlens, int32_t batch, int64_t total_tokens,
+                             int32_t max_seqlen,
+                             int32_t n_heads, int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
+                             int64_t q_row_stride, int64_t k_row_stride, int64_t v_row_stride,
+                             loza_ssa_params p, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, loza_stream_t stream);
+
+/*
+ * Decode: one new query token per sequence against its KV cache.
+ *   q        [batch, n_heads, d_qk] bf16 contiguous; the query of sequence n is
+ *            its last token, position seqlens[n]-1, whose KV row is already in
+ *            the cache (page 1 section 02: the streaming kernel in decode)
+ *   k_cache  sequence n's row t at k_cache + (n*cache_batch_stride + t*cache_row_stride)
+ *            elements, [n_kv_heads, d_qk] bf16 per row
+ *   v_cache  same layout with d_v; NULL means the first d_v columns of k_cache
+ *            (absorbed MLA latent cache)
+ *   seqlens  int32 [batch], 1 <= seqlens[n] <= max_seqlen
+ *   out [batch, n_heads, d_v] bf16; lse [batch, n_heads] fp32
+ *   workspace: loza_ssa_workspace_size(LOZA_OP_DECODE, ...) bytes (split-KV
+ *   partial results); contents on entry are ignored.
+ * Only n_kv_heads == 1 with (d_qk, d_v) == (576, 512) is compiled for decode.
+ */
+loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                            int64_t cache_batch_stride, int64_t cache_row_stride,
+                            int32_t n_heads, int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
+                            loza_ssa_params p, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, loza_stream_t stream);
+
+/*
+ * Training backward of loza_ssa_prefill (page 1 section 01 "training": the
+ * model is mid-trained with SSA in place). Given q, k, v, the forward out and
+ * lse, and the upstream gradient dout [T, n_heads, d_v] (bf16, contiguous),
+ * writes dq [T, n_heads, d_qk], dk [T, n_kv_heads, d_qk], dv [T, n_kv_heads, d_v]
+ * (bf16, contiguous); q, k, v, out and dout are contiguous [T, heads, dim]
+ * tensors here. Gradients of a key block are owned by one CTA (no
+ * atomics); the sink block, which every query block reads, is reduced from
+ * fp32 partials in the workspace in a fixed order.
+ * Only per-head K/V (n_kv_heads == n_heads) with (d_qk, d_v) in
+ * {(64,64), (192,128)} is compiled for the backward.
+ */
+loza_status loza_ssa_backward(const void *q, const void *k, const void *v, const void *out,
+                              const void *dout, const float *lse, const int32_t *cu_seqlens,
+                              int32_t batch, int64_t total_tokens, int32_t max_seqlen,
+                              int32_t n_heads,
+                              int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
+                              loza_ssa_params p, void *dq, void *dk, void *dv,
+                              void *workspace, size_t workspace_bytes, loza_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *loza_status_string(loza_status s);
+
+/*
+ * Synchronises `stream`, then returns and clears the library's device-side
+ * status word: LOZA_OK, or LOZA_ERR_TIMEOUT if a kernel gave up on a bounded
+ * wait since the last call. LOZA_ERR_CUDA if the synchronisation failed.
+ */
+loza_status loza_device_status(loza_stream_t stream);
+
+/* Number of kernel launches the library issued since load (all entry points). */
+uint64_t loza_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOZA_SSA_H */
