@@ -11,6 +11,7 @@
 
 #include "loza_ssa.h"
 #include "prefill.cuh"
+#include "decode.cuh"
 
 namespace loza {
 namespace {
@@ -56,6 +57,36 @@ bool window_ok(const loza_ssa_params& p) {
   if (p.block_size != kTile) return false;
   if (p.n_local != LOZA_UNBOUNDED && (p.n_local < 1 || p.n_sink < 0)) return false;
   return true;
+}
+
+// Split-KV plan of the absorbed decode: selected blocks per CTA and CTAs per
+// sequence. A bounded window has at most s + l blocks (one per CTA); the
+// unbounded (dense) window spreads up to ceil(max_seqlen / 128) blocks over at
+// most 32 CTAs per sequence.
+struct DecodePlan {
+  int bps, nsplit;
+};
+DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen) {
+  const int max_blocks = (max_seqlen + kTile - 1) / kTile;
+  if (p.n_local == LOZA_UNBOUNDED) {
+    const int bps = (max_blocks + 31) / 32;
+    return {bps, (max_blocks + bps - 1) / bps};
+  }
+  const int nb = p.n_sink + p.n_local;
+  return {1, nb < max_blocks ? nb : max_blocks};
+}
+
+struct DecodeWorkspace {
+  size_t o_off, ml_off, ticket_off, total;
+};
+DecodeWorkspace decode_workspace(int32_t batch, int nsplit) {
+  DecodeWorkspace w;
+  const size_t parts = (size_t)batch * nsplit * kDecHeads;
+  w.o_off = 0;
+  w.ml_off = parts * 512 * sizeof(float);
+  w.ticket_off = w.ml_off + parts * sizeof(float2);
+  w.total = w.ticket_off + ((size_t)batch * sizeof(int) + 255) / 256 * 256;
+  return w;
 }
 
 template <int DQK, int DVT, int NSTAGE>
@@ -106,9 +137,13 @@ loza_status loza_device_status(loza_stream_t stream) {
 size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int32_t max_seqlen,
                                int32_t n_heads, int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
                                loza_ssa_params p) {
-  (void)total_tokens; (void)max_seqlen; (void)n_kv_heads; (void)d_qk; (void)d_v; (void)p;
-  (void)batch; (void)n_heads;
-  if (op == LOZA_OP_PREFILL) return 0;
+  (void)total_tokens;
+  if (batch < 1 || max_seqlen < 1 || !window_ok(p)) return 0;
+  if (op == LOZA_OP_DECODE) {
+    if (n_kv_heads == 1 && n_heads == kDecHeads && d_qk == 576 && d_v == 512)
+      return decode_workspace(batch, decode_plan(p, max_seqlen).nsplit).total;
+    return 0;
+  }
   return 0;
 }
 
@@ -173,10 +208,100 @@ loza_status loza_ssa_decode(const void* q, const void* k_cache, const void* v_ca
                             int64_t cache_row_stride, int32_t n_heads, int32_t n_kv_heads, int32_t d_qk,
                             int32_t d_v, loza_ssa_params p, void* out, float* lse, void* workspace,
                             size_t workspace_bytes, loza_stream_t stream) {
-  (void)q; (void)k_cache; (void)v_cache; (void)seqlens; (void)batch; (void)max_seqlen;
-  (void)cache_batch_stride; (void)cache_row_stride; (void)n_heads; (void)n_kv_heads; (void)d_qk; (void)d_v;
-  (void)p; (void)out; (void)lse; (void)workspace; (void)workspace_bytes; (void)stream;
-  return LOZA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !seqlens || !out || !lse) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(out) || (v_cache && !aligned16(v_cache)))
+    return LOZA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || max_seqlen < 1) return LOZA_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
+  if (!stride_ok(cache_row_stride) || !stride_ok(cache_batch_stride) ||
+      cache_batch_stride < (int64_t)max_seqlen * cache_row_stride || cache_row_stride < (int64_t)n_kv_heads * d_qk)
+    return LOZA_ERR_INVALID_ARG;
+  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
+  const int n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
+  const float scale_log2 = p.scale * 1.4426950408889634f;
+
+  if (n_kv_heads == 1 && d_qk == 576 && d_v == 512) {
+    // absorbed MLA: shared latent cache, V = first 512 columns
+    if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
+    if (v_cache && v_cache != k_cache) return LOZA_ERR_UNSUPPORTED;
+    const DecodePlan plan = decode_plan(p, max_seqlen);
+    const DecodeWorkspace wl = decode_workspace(batch, plan.nsplit);
+    if (!workspace || !aligned16(workspace)) return LOZA_ERR_INVALID_ARG;
+    if (workspace_bytes < wl.total) return LOZA_ERR_WORKSPACE;
+    DecodeParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return LOZA_ERR_CUDA;
+    {
+      cuuint64_t dims[3] = {576, (cuuint64_t)n_heads, (cuuint64_t)batch};
+      cuuint64_t strides[2] = {576 * 2, (cuuint64_t)n_heads * 576 * 2};
+      cuuint32_t box[3] = {64, 64, 1};
+      cuuint32_t estr[3] = {1, 1, 1};
+      if (fn(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LOZA_ERR_CUDA;
+    }
+    {
+      cuuint64_t dims[3] = {576, (cuuint64_t)max_seqlen, (cuuint64_t)batch};
+      cuuint64_t strides[2] = {(cuuint64_t)cache_row_stride * 2, (cuuint64_t)cache_batch_stride * 2};
+      cuuint32_t box[3] = {64, 128, 1};
+      cuuint32_t estr[3] = {1, 1, 1};
+      if (fn(&prm.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LOZA_ERR_CUDA;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    prm.seqlens = seqlens;
+    prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+    prm.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
+    prm.ws_ticket = reinterpret_cast<int*>(ws + wl.ticket_off);
+    prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+    prm.lse = lse;
+    prm.nsplit = plan.nsplit;
+    prm.bps = plan.bps;
+    prm.n_sink = n_sink;
+    prm.n_local = n_local;
+    prm.scale_log2 = scale_log2;
+    if (cudaMemsetAsync(prm.ws_ticket, 0, (size_t)batch * sizeof(int), st) != cudaSuccess) return LOZA_ERR_CUDA;
+    if (cudaFuncSetAttribute(ssa_decode_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeLayout::SMEM_BYTES) != cudaSuccess)
+      return LOZA_ERR_CUDA;
+    ssa_decode_mla_kernel<<<dim3(plan.nsplit, batch), kDecThreads, DecodeLayout::SMEM_BYTES, st>>>(prm);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+  }
+
+  // per-head K/V on CUDA cores
+  if (!(n_kv_heads == n_heads || n_kv_heads == 1)) return LOZA_ERR_UNSUPPORTED;
+  if (!v_cache) return LOZA_ERR_INVALID_ARG;
+  if (n_heads > 65535) return LOZA_ERR_UNSUPPORTED;
+  DecodeMhaParams prm;
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k_cache);
+  prm.v = static_cast<const __nv_bfloat16*>(v_cache);
+  prm.k_batch_stride = cache_batch_stride;
+  prm.k_row_stride = cache_row_stride;
+  prm.v_batch_stride = cache_batch_stride / d_qk * d_v;
+  prm.v_row_stride = cache_row_stride / d_qk * d_v;
+  prm.seqlens = seqlens;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.n_heads = n_heads;
+  prm.n_kv_heads = n_kv_heads;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  prm.scale_log2 = scale_log2;
+  if (cache_batch_stride % d_qk != 0 || cache_row_stride % d_qk != 0) return LOZA_ERR_INVALID_ARG;
+  const dim3 grid(n_heads, batch);
+  if (d_qk == 64 && d_v == 64) ssa_decode_mha_kernel<64, 64><<<grid, 128, 0, st>>>(prm);
+  else if (d_qk == 192 && d_v == 128) ssa_decode_mha_kernel<192, 128><<<grid, 128, 0, st>>>(prm);
+  else return LOZA_ERR_UNSUPPORTED;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
 loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,

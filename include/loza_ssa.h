@@ -120,13 +120,20 @@ loza_status loza_ssa_prefill(const void *q, const void *k, const void *v,
  *            the cache (page 1 section 02: the streaming kernel in decode)
  *   k_cache  sequence n's row t at k_cache + (n*cache_batch_stride + t*cache_row_stride)
  *            elements, [n_kv_heads, d_qk] bf16 per row
- *   v_cache  same layout with d_v; NULL means the first d_v columns of k_cache
- *            (absorbed MLA latent cache)
+ *   v_cache  absorbed MLA: NULL (or == k_cache): V is the first d_v columns of
+ *            the latent row. Per-head K/V: a second cache whose strides are the
+ *            K strides scaled by d_v / d_qk (both caches are [batch, Lcap,
+ *            n_kv_heads, d] arrays with the same Lcap).
+ *   The cache must hold at least max_seqlen rows per sequence
+ *   (cache_batch_stride >= max_seqlen * cache_row_stride); rows at or past
+ *   seqlens[n] are never used, whatever they contain.
  *   seqlens  int32 [batch], 1 <= seqlens[n] <= max_seqlen
  *   out [batch, n_heads, d_v] bf16; lse [batch, n_heads] fp32
  *   workspace: loza_ssa_workspace_size(LOZA_OP_DECODE, ...) bytes (split-KV
  *   partial results); contents on entry are ignored.
- * Only n_kv_heads == 1 with (d_qk, d_v) == (576, 512) is compiled for decode.
+ * Compiled shapes: absorbed MLA (n_kv_heads == 1, 64 heads, (576, 512)) on
+ * tensor cores, with split-KV partials merged in-kernel; per-head K/V
+ * ((64, 64) or (192, 128)) on CUDA cores, which needs no workspace.
  */
 loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_cache,
                             const int32_t *seqlens, int32_t batch, int32_t max_seqlen,

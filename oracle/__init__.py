@@ -57,7 +57,7 @@ def _load():
             _i64p, ctypes.c_int64, _f64p, _f64p]
         lib.ssa_oracle_decode.restype = ctypes.c_int
         lib.ssa_oracle_decode.argtypes = [
-            _u16p, _u16p, _u16p, ctypes.c_int64, _i32p, ctypes.c_int,
+            _u16p, _u16p, _u16p, ctypes.c_int64, ctypes.c_int64, _i32p, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
             _f64p, _f64p]
@@ -103,16 +103,25 @@ def forward(q, k, v, cu_seqlens, n_heads, n_kv_heads, block_size=128, n_sink=1,
 
 
 def decode(q, k_cache, v_cache, seqlens, n_heads, n_kv_heads, block_size=128,
-           n_sink=1, n_local=7, scale=1.0):
+           n_sink=1, n_local=7, scale=1.0, d_v=None):
     """O [B,H,d_v], LSE [B,H] for one query per sequence (position L_n - 1).
-    q [B,H,d_qk]; k_cache [B,Lcap,Hkv,d_qk]; v_cache [B,Lcap,Hkv,d_v]."""
-    q, kc, vc = _u16(q), _u16(k_cache), _u16(v_cache)
+    q [B,H,d_qk]; k_cache [B,Lcap,Hkv,d_qk]; v_cache [B,Lcap,Hkv,d_v], or None
+    for an absorbed latent cache whose first ``d_v`` columns are V (the cache
+    is then read in place, so a large, sparsely filled array is never copied)."""
+    q, kc = _u16(q), _u16(k_cache)
+    if v_cache is None:
+        if d_v is None or n_kv_heads != 1:
+            raise ValueError("a latent cache needs d_v and one kv head")
+        vc, v_row = kc, kc.shape[-1]
+    else:
+        vc = _u16(v_cache)
+        d_v, v_row = vc.shape[-1], vc.shape[-1] * n_kv_heads
     sl = np.ascontiguousarray(seqlens, dtype=np.int32)
     B = q.shape[0]
-    d_qk, d_v = q.shape[-1], vc.shape[-1]
+    d_qk = q.shape[-1]
     o = np.zeros((B, n_heads, d_v), np.float64)
     lse = np.zeros((B, n_heads), np.float64)
-    rc = _load().ssa_oracle_decode(q, kc, vc, kc.shape[1], sl, B, n_heads, n_kv_heads,
+    rc = _load().ssa_oracle_decode(q, kc, vc, kc.shape[1], v_row, sl, B, n_heads, n_kv_heads,
                                    d_qk, d_v, block_size, n_sink, n_local, float(scale),
                                    o, lse)
     if rc != 0:

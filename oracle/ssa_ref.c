@@ -175,11 +175,14 @@ int ssa_oracle_forward_rows(const uint16_t *q, const uint16_t *k, const uint16_t
  * Decode: sequence n's query q[n] (its last token, position L_n - 1) against
  * cache rows 0 .. L_n - 1 of that sequence (step 6 of the definition).
  * q [B,H,d_qk]; sequence n's cache row t lives at
- *   k_cache + ((n*cache_batch_rows + t)*Hkv + hk)*d_qk  (v_cache likewise, d_v).
+ *   k_cache + ((n*cache_batch_rows + t)*Hkv + hk)*d_qk, and its value row at
+ *   v_cache + (n*cache_batch_rows + t)*v_row_elems + hk*d_v
+ * (v_row_elems = Hkv*d_v for a separate V cache; for an absorbed latent cache
+ * v_cache = k_cache and v_row_elems = d_qk, so V is the first d_v columns).
  * o_out [B,H,d_v], lse_out [B,H].
  */
 int ssa_oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-                      int64_t cache_batch_rows, const int32_t *seqlens, int batch,
+                      int64_t cache_batch_rows, int64_t v_row_elems, const int32_t *seqlens, int batch,
                       int n_heads, int n_kv_heads, int d_qk, int d_v,
                       int block_size, int n_sink, int n_local, double scale,
                       double *o_out, double *lse_out) {
@@ -197,7 +200,7 @@ int ssa_oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
         const int64_t i = L - 1;
         const uint16_t *qi = q + ((int64_t)n * n_heads + h) * d_qk;
         const uint16_t *kc = k_cache + (int64_t)n * cache_batch_rows * n_kv_heads * d_qk;
-        const uint16_t *vc = v_cache + (int64_t)n * cache_batch_rows * n_kv_heads * d_v;
+        const uint16_t *vc = v_cache + (int64_t)n * cache_batch_rows * v_row_elems;
         int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (size_t)L);
         double *z = (double *)malloc(sizeof(double) * (size_t)L);
         const int64_t c = visible_keys(i, block_size, n_sink, n_local, keys);
@@ -216,7 +219,7 @@ int ssa_oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
         for (int d = 0; d < d_v; ++d) o[d] = 0.0;
         for (int64_t a = 0; a < c; ++a) {
             const double pt = exp(z[a] - lse);
-            const uint16_t *vt = vc + (keys[a] * n_kv_heads + hk) * (int64_t)d_v;
+            const uint16_t *vt = vc + keys[a] * v_row_elems + (int64_t)hk * d_v;
             for (int d = 0; d < d_v; ++d) o[d] += pt * widen(vt[d]);
         }
         lse_out[r] = lse;

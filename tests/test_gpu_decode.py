@@ -1,0 +1,129 @@
+"""GPU parity of SSA decode against the fp64 oracle.
+
+Decode runs the last token of each sequence against its KV cache. Cache rows
+the window does not select are filled with NaN, so any out-of-window read
+shows up as a non-finite or different output (the bounds check); the same call
+with those rows zeroed must give bit-identical results.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import synth
+from helpers import assert_close_lse, assert_close_o, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+NAN_BF16 = np.uint16(0x7FC0)
+
+
+@pytest.fixture(scope="module")
+def bss():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import block_sparse_streaming_b200 as m
+    m.build()
+    return m
+
+
+def selected_rows(L, b=128, s=1, l=7):
+    """Cache rows the decode query (position L-1) may read: whole selected blocks."""
+    j = (L - 1) // b
+    if l < 0:
+        blocks = range(j + 1)
+    else:
+        blocks = sorted(set(range(min(s, j + 1))) | set(range(max(0, j - l + 1), j + 1)))
+    return np.concatenate([np.arange(kb * b, min((kb + 1) * b, L)) for kb in blocks])
+
+
+def absorbed_case(bss, oracle_mod, seed, lens, Lcap, n_sink=1, n_local=7, poison=True, compare=True):
+    """Absorbed MLA decode: 64 heads, latent cache [B, Lcap, 1, 576]. Only the rows
+    the window selects carry seeded values; every other row is NaN (or zero)."""
+    import torch
+    H, D = 64, 576
+    B = len(lens)
+    g = synth.rng(seed)
+    q = synth.normal_bits(g, (B, H, D))
+    cache_dev = torch.full((B, Lcap, 1, D), float("nan") if poison else 0.0, dtype=torch.bfloat16, device="cuda")
+    host = np.empty((B, Lcap, 1, D), np.uint16)          # lazily backed: only touched rows materialise
+    for n, L in enumerate(lens):
+        rows = selected_rows(L, 128, n_sink, n_local)
+        vals = synth.normal_bits(g, (len(rows), 1, D))
+        host[n, rows] = vals
+        cache_dev[n, torch.from_numpy(rows).cuda()] = to_dev(vals)
+    seqlens = np.array(lens, np.int32)
+    scale = 1.0 / math.sqrt(192.0)
+    params = bss.Params(scale, 128, n_sink, n_local)
+    out, lse = bss.loza_ssa_decode(to_dev(q), cache_dev, None, torch.from_numpy(seqlens).cuda(), Lcap, params)
+    torch.cuda.synchronize()
+    assert bss.device_status() == 0
+    res = (out.clone(), lse.clone())
+    if compare:
+        o_ref, lse_ref = oracle_mod.decode(q, host, None, seqlens, H, 1, 128, n_sink, n_local, scale, d_v=512)
+        assert_close_o(from_dev(out), o_ref, "absorbed decode O")
+        assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, "absorbed decode LSE")
+    del cache_dev
+    return res
+
+
+def test_absorbed_decode_small(bss, oracle_mod):
+    absorbed_case(bss, oracle_mod, 61, [1, 127, 128, 129, 1000, 1024, 1025, 3000], 3072)
+
+
+def test_absorbed_decode_nan_bounds_bitwise(bss, oracle_mod):
+    lens = [5, 300, 2049, 4000]
+    o1, l1 = absorbed_case(bss, oracle_mod, 62, lens, 4096, poison=True, compare=False)
+    o2, l2 = absorbed_case(bss, oracle_mod, 62, lens, 4096, poison=False, compare=False)
+    import torch
+    assert torch.isfinite(o1.float()).all()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_absorbed_dense_decode(bss, oracle_mod):
+    absorbed_case(bss, oracle_mod, 63, [1, 700, 5000, 9000], 9216, n_sink=0, n_local=-1)
+
+
+def test_absorbed_decode_workload3_full_size(bss, oracle_mod):
+    """64 sequences, contexts uniform in [65536, 131072], cache [64, 131072, 576]."""
+    w = synth.WORKLOADS[3]
+    g = synth.rng(synth.workload_seed(3))
+    lens = synth.uniform_lengths(g, w["batch"], w["ctx_lo"], w["ctx_hi"]).tolist()
+    absorbed_case(bss, oracle_mod, synth.workload_seed(3) + 1, lens, w["ctx_hi"])
+
+
+def test_absorbed_decode_1m_context(bss, oracle_mod):
+    """Contexts of 1,048,576 tokens (4 sequences here; the workload has 32)."""
+    absorbed_case(bss, oracle_mod, synth.workload_seed(4) + 2, [1 << 20] * 4, 1 << 20)
+
+
+@pytest.mark.parametrize("dqk,dv", [(64, 64), (192, 128)])
+def test_mha_decode_matches_oracle_and_prefill(bss, oracle_mod, dqk, dv):
+    """Per-head K/V decode; workload 1 shape for d = 64 (L = 2048, 4 heads, scale 1/8).
+    Decode of the last token must also equal the last row of the prefill."""
+    import torch
+    H = 4
+    lens = [2048] if dqk == 64 else [2048, 900, 1]
+    B, Lcap = len(lens), max(lens)
+    g = synth.rng(synth.workload_seed(1) + dqk)
+    kc = synth.normal_bits(g, (B, Lcap, H, dqk))
+    vc = synth.normal_bits(g, (B, Lcap, H, dv))
+    qd = synth.normal_bits(g, (B, H, dqk))
+    scale = 1 / 8 if dqk == 64 else 1 / math.sqrt(192)
+    params = bss.Params(scale)
+    seqlens = np.array(lens, np.int32)
+    out, lse = bss.loza_ssa_decode(to_dev(qd), to_dev(kc), to_dev(vc), torch.from_numpy(seqlens).cuda(), Lcap,
+                                   params)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle_mod.decode(qd, kc, vc, seqlens, H, H, 128, 1, 7, scale)
+    assert_close_o(from_dev(out), o_ref, "mha decode O")
+    assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, "mha decode LSE")
+    # phase equivalence on the GPU: prefill with the decode query as the last row
+    for n, L in enumerate(lens):
+        q = np.zeros((L, H, dqk), np.uint16)
+        q[L - 1] = qd[n]
+        cu = torch.tensor([0, L], dtype=torch.int32, device="cuda")
+        po, pl = bss.loza_ssa_prefill(to_dev(q), to_dev(kc[n, :L]), to_dev(vc[n, :L]), cu, L, params)
+        torch.cuda.synchronize()
+        assert_close_o(from_dev(po[L - 1]), from_dev(out[n]), "decode vs prefill row")
+        assert abs(float(pl[L - 1, 0] - lse[n, 0])) <= 1e-3

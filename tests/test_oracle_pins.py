@@ -336,3 +336,17 @@ def test_oracle_rejects_bad_arguments(oracle_mod):
         oracle_mod.forward(q, k, v, cu, 3, 3, 4, 1, 1, 1.0, rows=np.array([10]))
     with pytest.raises(TypeError):
         oracle_mod.forward(q.astype(np.float32), k, v, cu, 3, 3, 4, 1, 1, 1.0)
+
+
+def test_latent_decode_reads_cache_in_place(oracle_mod):
+    """A latent cache passed once (V = its first d_v columns) gives the same result
+    as a separate, copied V cache."""
+    g = synth.rng(91)
+    B, Lcap, H, D, DV = 3, 700, 4, 24, 16
+    kc = synth.normal_bits(g, (B, Lcap, 1, D))
+    qd = synth.normal_bits(g, (B, H, D))
+    lens = np.array([1, 300, 700], np.int32)
+    o1, l1 = oracle_mod.decode(qd, kc, np.ascontiguousarray(kc[..., :DV]), lens, H, 1, 128, 1, 7, 0.3)
+    o2, l2 = oracle_mod.decode(qd, kc, None, lens, H, 1, 128, 1, 7, 0.3, d_v=DV)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
