@@ -34,6 +34,7 @@ EXPORTED = [
     "loza_ssa_workspace_size",
     "loza_ssa_prefill",
     "loza_ssa_decode",
+    "loza_ssa_decode_noalloc",
     "loza_ssa_backward",
     "loza_status_string",
     "loza_device_status",
@@ -76,6 +77,9 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_decode.restype = ctypes.c_int
         L.loza_ssa_decode.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i64, _i64, _i32, _i32, _i32, _i32,
                                       Params, _vp, _vp, _vp, _sz, _vp]
+        L.loza_ssa_decode_noalloc.restype = ctypes.c_int
+        L.loza_ssa_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i64, _i64, _i32, _i32, _i32, _i32,
+                                              Params, _vp, _vp, _vp]
         L.loza_ssa_backward.restype = ctypes.c_int
         L.loza_ssa_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
                                         _i32, _i32, Params, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -173,6 +177,28 @@ def loza_ssa_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, params: Param
                                k_cache.stride(0), k_cache.stride(1), H, Hkv, d_qk, d_v, params, _ptr(out),
                                _ptr(lse), _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check(rc, "loza_ssa_decode")
+    return out, lse
+
+
+def loza_ssa_decode_noalloc(q, k_cache, v_cache, seqlens, max_seqlen: int, params: Params, out, lse,
+                            stream=None):
+    """Decode for callers that cannot allocate device memory: like loza_ssa_decode,
+    but the split-KV partials live in a fixed 16 MiB array inside the library, so
+    nothing is allocated here either (out and lse must be given). Calls that can
+    overlap on the GPU share that array and must not run concurrently."""
+    import torch
+    _require(q, "q", torch.bfloat16, 3)
+    _require(k_cache, "k_cache", torch.bfloat16, 4)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    _require(out, "out", torch.bfloat16, 3)
+    _require(lse, "lse", torch.float32, 2)
+    B, H, d_qk = q.shape
+    Hkv = k_cache.shape[2]
+    d_v = v_cache.shape[3] if v_cache is not None else 512
+    rc = lib().loza_ssa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, int(max_seqlen),
+                                       k_cache.stride(0), k_cache.stride(1), H, Hkv, d_qk, d_v, params, _ptr(out),
+                                       _ptr(lse), _stream_ptr(stream))
+    _check(rc, "loza_ssa_decode_noalloc")
     return out, lse
 
 

@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "loza_ssa.h"
 #include "prefill.cuh"
@@ -99,6 +100,38 @@ loza_status launch_prefill(const PrefillParams& prm, int max_seqlen, int batch, 
   kern<<<grid, kPrefillThreads, LY::SMEM_BYTES, stream>>>(prm);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Built-in scratch for loza_ssa_decode_noalloc.
+//
+// The absorbed decode keeps one partial result per (sequence, split, head)
+// between its split CTAs and the CTA that merges them. Callers that cannot
+// allocate device memory get this fixed array instead of a caller-provided
+// workspace. It is ordinary device memory of this module: every GPU that loads
+// the library reserves kNoAllocScratchBytes for it until the process exits.
+// Host code must not use the name g_decode_scratch as a pointer; the device
+// address comes from cudaGetSymbolAddress, once per device.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) uint8_t g_decode_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device (looked up on the
+// first call per device). Returns nullptr if the lookup fails.
+void* decode_scratch_address() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_addr[dev] = p;
+  }
+  return g_scratch_addr[dev];
 }
 
 }  // namespace
@@ -313,6 +346,76 @@ loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const
   (void)total_tokens; (void)max_seqlen; (void)n_heads; (void)n_kv_heads; (void)d_qk; (void)d_v; (void)p;
   (void)dq; (void)dk; (void)dv; (void)workspace; (void)workspace_bytes; (void)stream;
   return LOZA_ERR_UNSUPPORTED;
+}
+
+loza_status loza_ssa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* seqlens, int32_t batch, int32_t max_seqlen,
+                                    int64_t cache_batch_stride, int64_t cache_row_stride, int32_t n_heads,
+                                    int32_t n_kv_heads, int32_t d_qk, int32_t d_v, loza_ssa_params p, void* out,
+                                    float* lse, loza_stream_t stream) {
+  // Per-head K/V decode needs no scratch at all: same call, no workspace.
+  if (!(n_kv_heads == 1 && d_qk == 576 && d_v == 512))
+    return loza_ssa_decode(q, k_cache, v_cache, seqlens, batch, max_seqlen, cache_batch_stride, cache_row_stride,
+                           n_heads, n_kv_heads, d_qk, d_v, p, out, lse, nullptr, 0, stream);
+  if (!q || !k_cache || !seqlens || !out || !lse) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || max_seqlen < 1) return LOZA_ERR_INVALID_ARG;
+  if (!stride_ok(cache_row_stride) || !stride_ok(cache_batch_stride) ||
+      cache_batch_stride < (int64_t)max_seqlen * cache_row_stride || cache_row_stride < d_qk)
+    return LOZA_ERR_INVALID_ARG;
+  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
+  if (v_cache && v_cache != k_cache) return LOZA_ERR_UNSUPPORTED;
+  const DecodePlan plan = decode_plan(p, max_seqlen);
+  const DecodeWorkspace wl = decode_workspace(batch, plan.nsplit);
+  if (wl.total > kNoAllocScratchBytes) return LOZA_ERR_WORKSPACE;  // batch too large for the built-in scratch
+
+  uint8_t* ws = static_cast<uint8_t*>(decode_scratch_address());
+  if (!ws) return LOZA_ERR_CUDA;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return LOZA_ERR_CUDA;
+  DecodeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  {
+    cuuint64_t dims[3] = {576, (cuuint64_t)n_heads, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {576 * 2, (cuuint64_t)n_heads * 576 * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return LOZA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {576, (cuuint64_t)max_seqlen, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {(cuuint64_t)cache_row_stride * 2, (cuuint64_t)cache_batch_stride * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&prm.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return LOZA_ERR_CUDA;
+  }
+  prm.seqlens = seqlens;
+  prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+  prm.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
+  prm.ws_ticket = reinterpret_cast<int*>(ws + wl.ticket_off);
+  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.nsplit = plan.nsplit;
+  prm.bps = plan.bps;
+  prm.n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
+  prm.n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
+  prm.scale_log2 = p.scale * 1.4426950408889634f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The arrival counters must start at zero; the partials are fully rewritten.
+  if (cudaMemsetAsync(prm.ws_ticket, 0, (size_t)batch * sizeof(int), st) != cudaSuccess) return LOZA_ERR_CUDA;
+  if (cudaFuncSetAttribute(ssa_decode_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           DecodeLayout::SMEM_BYTES) != cudaSuccess)
+    return LOZA_ERR_CUDA;
+  ssa_decode_mla_kernel<<<dim3(plan.nsplit, batch), kDecThreads, DecodeLayout::SMEM_BYTES, st>>>(prm);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
 }  // extern "C"

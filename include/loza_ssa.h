@@ -143,6 +143,41 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
                             void *workspace, size_t workspace_bytes, loza_stream_t stream);
 
 /*
+ * Decode without any caller-provided device memory. (The LoZA pages have no
+ * counterpart to this entry point; it exists for callers of this library.)
+ *
+ * Some callers cannot allocate device memory at the point where they decode:
+ * a host application that owns the device allocator and gives plug-ins no
+ * access to it, a serving runtime that has reserved all device memory for its
+ * own KV-cache pool up front, or a latency-critical loop that must not pay
+ * for cudaMalloc/cudaFree. For them this entry point takes the same arguments
+ * as loza_ssa_decode minus the workspace, and keeps the split-KV partial
+ * results in a fixed 16 MiB array that is part of the library itself.
+ *   - The library never allocates: every GPU that loads the library holds the
+ *     16 MiB array until the process exits.
+ *   - Limit: the absorbed MLA shape needs batch * nsplit * 131,584 bytes plus
+ *     256 for the counters, where nsplit = n_sink + n_local (8 for the pages'
+ *     1 + 7 window) or min(32, number of 128-token blocks) for the unbounded
+ *     window. With the pages' window at most 15 sequences fit. A larger batch
+ *     returns LOZA_ERR_WORKSPACE before anything is launched; call
+ *     loza_ssa_decode with a workspace instead, or split the batch.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture on that device.
+ *   - Every call uses the same array and leaves its last contents there; the
+ *     arrival counters are cleared on the caller's stream at the start of each
+ *     call. Two calls whose kernels can overlap on the GPU (different streams
+ *     without ordering between them) race on the array and give wrong results.
+ *   - Per-head K/V shapes need no scratch and behave exactly like
+ *     loza_ssa_decode.
+ */
+loza_status loza_ssa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                    const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                                    int64_t cache_batch_stride, int64_t cache_row_stride,
+                                    int32_t n_heads, int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
+                                    loza_ssa_params p, void *out, float *lse, loza_stream_t stream);
+
+/*
  * Training backward of loza_ssa_prefill (page 1 section 01 "training": the
  * model is mid-trained with SSA in place). Given q, k, v, the forward out and
  * lse, and the upstream gradient dout [T, n_heads, d_v] (bf16, contiguous),
