@@ -1,0 +1,612 @@
+// backward.cuh - SSA training backward on sm_100a (tcgen05 + TMA).
+//
+// The model is mid-trained with SSA in place (page 1 section 01 "training" of
+// the LoZA pages), so the operator needs dQ, dK, dV. With P = softmax over the
+// selected keys (recomputed from the forward LSE), D_i = dO_i . O_i,
+// dP = dO V^T, dS = P o (dP - D):
+//     dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO.
+// Gradients are written by exactly one owner CTA per output tile (no atomics):
+//   ssa_bwd_dq_kernel     owner of a 128-query tile; walks the <= s+l key
+//                         blocks its window selects (S, dP, dQ += dS K).
+//   ssa_bwd_dkdv_kernel   owner of a 128-key block; walks the query blocks
+//                         that select it: j = k .. k+l-1 ("local" part). A sink
+//                         block (k < s) is also selected by every later query
+//                         block; those "far" query blocks are handled by extra
+//                         CTAs in fixed chunks, and every contribution to a
+//                         sink block goes to an fp32 partial in the workspace.
+//   ssa_bwd_sink_reduce   adds a sink block's partials in a fixed order
+//                         (deterministic) and writes its dK, dV.
+//   ssa_bwd_preprocess    D = rowsum(dO o O), bandwidth bound.
+#pragma once
+
+#include <cuda.h>
+
+#include "sm100.cuh"
+
+namespace loza {
+
+constexpr int kBwdThreads = 192;
+constexpr int kSinkChunk = 256;  // far query blocks per sink-partial CTA
+
+struct BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // [T, H, d] maps, box {64, 1, 128}
+  const int32_t* cu_seqlens;
+  const float* lse;    // [T, H] natural log
+  const float* dvec;   // [T, H] D = rowsum(dO o O)
+  __nv_bfloat16* dq;   // [T, H, DQK]
+  __nv_bfloat16* dk;   // [T, H, DQK]
+  __nv_bfloat16* dv;   // [T, H, DV]
+  float* partial;      // sink partials [B][s][H][nslots][128][DQK + DV]
+  int n_heads;
+  int n_sink, n_local;
+  int nslots;          // partial slots per (sequence, sink block, head)
+  int far_mode;        // dK/dV kernel: 0 = owners, 1 = far sink chunks
+  float scale;         // softmax scale
+  float scale_log2;    // scale * log2(e)
+};
+
+// ---------------------------------------------------------------------------
+// D = rowsum(dO o O) over DV columns; one half-warp per (token, head) row.
+// ---------------------------------------------------------------------------
+template <int DV>
+__global__ void __launch_bounds__(256) ssa_bwd_preprocess(const __nv_bfloat16* __restrict__ out,
+                                                          const __nv_bfloat16* __restrict__ dout,
+                                                          float* __restrict__ dvec, int64_t rows) {
+  constexpr int LANES = DV / 8;  // 16-byte vectors per row
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gid / LANES;
+  const int l = (int)(gid % LANES);
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = reinterpret_cast<const uint4*>(out + row * DV)[l];
+    const uint4 b = reinterpret_cast<const uint4*>(dout + row * DV)[l];
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(pa[i]);
+      const float2 y = __bfloat1622float2(pb[i]);
+      acc += x.x * y.x + x.y * y.y;
+    }
+  }
+#pragma unroll
+  for (int o = LANES / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o, LANES);
+  if (row < rows && l == 0) dvec[row] = acc;
+}
+
+// ---------------------------------------------------------------------------
+// dQ: one CTA per (query tile, head, sequence).
+// TMEM: S [0,128) (dS packed into [0,64)), dP [128,256), dQ [256, 256+DQK).
+// Ring order per key block: K (DQK/64 tiles, for S), V (DV/64, for dP), K again (for dQ).
+// ---------------------------------------------------------------------------
+template <int DQK, int DV>
+struct BwdDqLayout {
+  static constexpr int NQC = DQK / 64, NVC = DV / 64, NSTAGE = 8;
+  static constexpr int Q_OFF = 0;
+  static constexpr int DO_OFF = NQC * kChunkBytes;
+  static constexpr int RING_OFF = DO_OFF + NVC * kChunkBytes;
+  static constexpr int BAR_OFF = RING_OFF + NSTAGE * kChunkBytes;
+  static constexpr int BAR_IN = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NSTAGE, BAR_DP = 1 + 2 * NSTAGE,
+                       BAR_DS = BAR_DP + 1, BAR_DQ = BAR_DS + 1, NBAR = BAR_DQ + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(256 + DQK <= 512, "TMEM budget");
+};
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  using LY = BwdDqLayout<DQK, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int qb = blockIdx.x, head = blockIdx.y, seq = blockIdx.z;
+  const int seq_start = p.cu_seqlens[seq];
+  const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
+  if (qb * kTile >= seq_len) return;
+  const BlockWalk walk(qb, p.n_sink, p.n_local);
+  const int nb = walk.count;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + LY::BAR_OFF;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(LY::BAR_IN), 1);
+    for (int i = 0; i < LY::NSTAGE; ++i) {
+      mbar_init(bar(LY::BAR_FULL + i), 1);
+      mbar_init(bar(LY::BAR_EMPTY + i), 1);
+    }
+    mbar_init(bar(LY::BAR_DP), 1);
+    mbar_init(bar(LY::BAR_DS), 128);
+    mbar_init(bar(LY::BAR_DQ), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int row0 = seq_start + qb * kTile;
+      mbar_arrive_expect_tx(bar(LY::BAR_IN), (LY::NQC + LY::NVC) * kChunkBytes);
+      for (int c = 0; c < LY::NQC; ++c)
+        tma_load_3d(sbase + LY::Q_OFF + c * kChunkBytes, &p.tm_q, bar(LY::BAR_IN), c * 64, head, row0);
+      for (int c = 0; c < LY::NVC; ++c)
+        tma_load_3d(sbase + LY::DO_OFF + c * kChunkBytes, &p.tm_do, bar(LY::BAR_IN), c * 64, head, row0);
+      int slot = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int b = 0; b < nb && ok; ++b) {
+        const int krow = seq_start + walk.block(b) * kTile;
+        for (int t = 0; t < 2 * LY::NQC + LY::NVC && ok; ++t) {
+          ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
+          const uint32_t dst = sbase + LY::RING_OFF + slot * kChunkBytes;
+          if (t < LY::NQC)
+            tma_load_3d(dst, &p.tm_k, bar(LY::BAR_FULL + slot), t * 64, head, krow);
+          else if (t < LY::NQC + LY::NVC)
+            tma_load_3d(dst, &p.tm_v, bar(LY::BAR_FULL + slot), (t - LY::NQC) * 64, head, krow);
+          else
+            tma_load_3d(dst, &p.tm_k, bar(LY::BAR_FULL + slot), (t - LY::NQC - LY::NVC) * 64, head, krow);
+          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_dq = idesc_bf16(128, 64, false, true);
+      const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+      int slot = 0;
+      uint32_t phase = 0;
+      bool ok = mbar_wait(bar(LY::BAR_IN), 0, abort_flag);
+      tc_fence_after();
+      for (int b = 0; b < nb && ok; ++b) {
+        // S = Q K^T
+        for (int c = 0; c < LY::NQC && ok; ++c) {
+          ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a = sbase + LY::Q_OFF + c * kChunkBytes, bb = sbase + LY::RING_OFF + slot * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(t_s, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
+                   (c | kk) != 0);
+          mma_commit(bar(LY::BAR_EMPTY + slot));
+          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+        }
+        // dP = dO V^T
+        for (int c = 0; c < LY::NVC && ok; ++c) {
+          ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a = sbase + LY::DO_OFF + c * kChunkBytes, bb = sbase + LY::RING_OFF + slot * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(t_dp, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
+                   (c | kk) != 0);
+          mma_commit(bar(LY::BAR_EMPTY + slot));
+          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(bar(LY::BAR_DP));
+        ok = mbar_wait(bar(LY::BAR_DS), b & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // dQ += dS K  (A = dS in TMEM, B = K tiles MN-major)
+        for (int c = 0; c < LY::NQC && ok; ++c) {
+          ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t bb = sbase + LY::RING_OFF + slot * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(t_dq + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_dq,
+                   (b > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(LY::BAR_EMPTY + slot));
+          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(bar(LY::BAR_DQ));
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int qpos = qb * kTile + row;
+    const bool valid = qpos < seq_len;
+    const int64_t grow = (int64_t)seq_start + qpos;
+    const float lse2 = valid ? p.lse[grow * p.n_heads + head] * 1.4426950408889634f : 0.f;
+    const float dd = valid ? p.dvec[grow * p.n_heads + head] : 0.f;
+    bool ok = true;
+    for (int b = 0; b < nb && ok; ++b) {
+      ok = mbar_wait(bar(LY::BAR_DP), b & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = walk.block(b) == qb;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float s[32], dp[32];
+        tmem_ld32(lane_addr + 32 * c, s);
+        tmem_ld32(lane_addr + 128 + 32 * c, dp);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float ds2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = 32 * c + 2 * i + e;
+            float pr = exp2f(s[2 * i + e] * p.scale_log2 - lse2);
+            if (diag && key > row) pr = 0.f;
+            ds2[e] = pr * (dp[2 * i + e] - dd);
+          }
+          pk[i] = pack_bf16(ds2[0], ds2[1]);
+        }
+        tmem_st16(lane_addr + 16 * c, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(LY::BAR_DS));
+    }
+    if (ok) ok = mbar_wait(bar(LY::BAR_DQ), (nb - 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + (grow * p.n_heads + head) * (int64_t)DQK;
+#pragma unroll 1
+      for (int c = 0; c < DQK / 32; ++c) {
+        float o[32];
+        tmem_ld32(lane_addr + 256 + 32 * c, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * p.scale, o[2 * i + 1] * p.scale);
+        if (valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK / dV: one CTA per (key block, head, sequence) in owner mode, or per
+// (far chunk, sink block x head, sequence) in far mode.
+// TMEM: S^T [0,128) (P^T and later dS^T packed into [0,64)), dP^T [64,192),
+//       dV [192, 192+DV), dK [192+DV, 192+DV+DQK).
+// ---------------------------------------------------------------------------
+template <int DQK, int DV>
+struct BwdDkvLayout {
+  static constexpr int NQC = DQK / 64, NVC = DV / 64;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = NQC * kChunkBytes;
+  static constexpr int Q_OFF = V_OFF + NVC * kChunkBytes;
+  static constexpr int DO_OFF = Q_OFF + NQC * kChunkBytes;
+  static constexpr int STAT_OFF = DO_OFF + NVC * kChunkBytes;  // lse2[128], d[128]
+  static constexpr int BAR_OFF = STAT_OFF + 2 * 128 * 4;
+  static constexpr int BAR_KV = 0, BAR_QD = 1, BAR_QD_EMPTY = 2, BAR_S = 3, BAR_P = 4, BAR_DP = 5, BAR_DS = 6,
+                       NBAR = 7;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr int T_DV = 192, T_DK = 192 + DV;
+  static_assert(T_DK + DQK <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+  using LY = BwdDkvLayout<DQK, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int seq = blockIdx.z;
+  const int seq_start = p.cu_seqlens[seq];
+  const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
+  const int nq = (seq_len + kTile - 1) / kTile;
+  int kblk, head, j_lo, j_hi, slot = -1;
+  if (!p.far_mode) {
+    kblk = blockIdx.x;
+    head = blockIdx.y;
+    if (kblk >= nq) return;
+    j_lo = kblk;
+    j_hi = min(nq, kblk + p.n_local);
+    if (kblk < p.n_sink) slot = 0;
+  } else {
+    kblk = blockIdx.y % p.n_sink;
+    head = blockIdx.y / p.n_sink;
+    if (kblk >= nq) return;  // no such sink block: its partial slots are never read
+    j_lo = kblk + p.n_local + blockIdx.x * kSinkChunk;
+    j_hi = min(nq, j_lo + kSinkChunk);
+    slot = 1 + blockIdx.x;
+  }
+  const int nj = max(0, j_hi - j_lo);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // sink partial destination: [seq][kblk][head][slot][128][DQK+DV]
+  float* part = nullptr;
+  if (slot >= 0)
+    part = p.partial + ((((int64_t)seq * p.n_sink + kblk) * p.n_heads + head) * p.nslots + slot) *
+                           (int64_t)(kTile * (DQK + DV));
+  if (nj == 0) {
+    // empty far chunk: its partial contributes zero
+    for (int i = threadIdx.x; i < kTile * (DQK + DV) / 4; i += blockDim.x)
+      reinterpret_cast<float4*>(part)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + LY::BAR_OFF;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::MISC_OFF + 4);
+  float* s_lse2 = reinterpret_cast<float*>(smem + LY::STAT_OFF);
+  float* s_d = s_lse2 + 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(LY::BAR_KV), 1);
+    mbar_init(bar(LY::BAR_QD), 1);
+    mbar_init(bar(LY::BAR_QD_EMPTY), 1);
+    mbar_init(bar(LY::BAR_S), 1);
+    mbar_init(bar(LY::BAR_P), 128);
+    mbar_init(bar(LY::BAR_DP), 1);
+    mbar_init(bar(LY::BAR_DS), 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int krow = seq_start + kblk * kTile;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(LY::BAR_KV), (LY::NQC + LY::NVC) * kChunkBytes);
+      for (int c = 0; c < LY::NQC; ++c)
+        tma_load_3d(sbase + LY::K_OFF + c * kChunkBytes, &p.tm_k, bar(LY::BAR_KV), c * 64, head, krow);
+      for (int c = 0; c < LY::NVC; ++c)
+        tma_load_3d(sbase + LY::V_OFF + c * kChunkBytes, &p.tm_v, bar(LY::BAR_KV), c * 64, head, krow);
+      bool ok = true;
+      for (int jj = 0; jj < nj && ok; ++jj) {
+        ok = mbar_wait(bar(LY::BAR_QD_EMPTY), (jj & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        const int qrow = seq_start + (j_lo + jj) * kTile;
+        mbar_arrive_expect_tx(bar(LY::BAR_QD), (LY::NQC + LY::NVC) * kChunkBytes);
+        for (int c = 0; c < LY::NQC; ++c)
+          tma_load_3d(sbase + LY::Q_OFF + c * kChunkBytes, &p.tm_q, bar(LY::BAR_QD), c * 64, head, qrow);
+        for (int c = 0; c < LY::NVC; ++c)
+          tma_load_3d(sbase + LY::DO_OFF + c * kChunkBytes, &p.tm_do, bar(LY::BAR_QD), c * 64, head, qrow);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_ts = idesc_bf16(128, 64, false, true);
+      const uint32_t t_s = tmem, t_dp = tmem + 64, t_dv = tmem + LY::T_DV, t_dk = tmem + LY::T_DK;
+      bool ok = mbar_wait(bar(LY::BAR_KV), 0, abort_flag);
+      for (int jj = 0; jj < nj && ok; ++jj) {
+        ok = mbar_wait(bar(LY::BAR_QD), jj & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // S^T = K Q^T
+        for (int c = 0; c < LY::NQC; ++c) {
+          const uint32_t a = sbase + LY::K_OFF + c * kChunkBytes, bb = sbase + LY::Q_OFF + c * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(t_s, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
+                   (c | kk) != 0);
+        }
+        mma_commit(bar(LY::BAR_S));
+        ok = mbar_wait(bar(LY::BAR_P), jj & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // dV += P^T dO   (A = P^T in TMEM, B = dO tiles MN-major)
+        for (int c = 0; c < LY::NVC; ++c) {
+          const uint32_t bb = sbase + LY::DO_OFF + c * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(t_dv + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_ts,
+                   (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        // dP^T = V dO^T
+        for (int c = 0; c < LY::NVC; ++c) {
+          const uint32_t a = sbase + LY::V_OFF + c * kChunkBytes, bb = sbase + LY::DO_OFF + c * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(t_dp, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
+                   (c | kk) != 0);
+        }
+        mma_commit(bar(LY::BAR_DP));
+        ok = mbar_wait(bar(LY::BAR_DS), jj & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // dK += dS^T Q   (A = dS^T in TMEM, B = Q tiles MN-major)
+        for (int c = 0; c < LY::NQC; ++c) {
+          const uint32_t bb = sbase + LY::Q_OFF + c * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(t_dk + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_ts,
+                   (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(LY::BAR_QD_EMPTY));
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int tid = threadIdx.x - 64;
+    const int key = quarter * 32 + lane;  // TMEM lane == key row of the block
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    for (int jj = 0; jj < nj && ok; ++jj) {
+      const int j = j_lo + jj;
+      {
+        // per-query statistics of block j (invalid rows: P = 0, D = 0)
+        const int qpos = j * kTile + tid;
+        const bool v = qpos < seq_len;
+        const int64_t g = (int64_t)seq_start + qpos;
+        s_lse2[tid] = v ? p.lse[g * p.n_heads + head] * 1.4426950408889634f : INFINITY;
+        s_d[tid] = v ? p.dvec[g * p.n_heads + head] : 0.f;
+      }
+      named_barrier_sync(1, 128);
+      ok = mbar_wait(bar(LY::BAR_S), jj & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = (j == kblk);
+      float pr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float s[32];
+        tmem_ld32(lane_addr + 32 * c, s);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = 32 * c + i;  // query row of block j
+          float v = exp2f(s[i] * p.scale_log2 - s_lse2[col]);
+          if (diag && col < key) v = 0.f;
+          pr[col] = v;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(pr[64 * c + 2 * i], pr[64 * c + 2 * i + 1]);
+        tmem_st32(lane_addr + 32 * c, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(LY::BAR_P));
+      ok = mbar_wait(bar(LY::BAR_DP), jj & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float dp[32];
+        tmem_ld32(lane_addr + 64 + 32 * c, dp);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pr[32 * c + i] = pr[32 * c + i] * (dp[i] - s_d[32 * c + i]);
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(pr[64 * c + 2 * i], pr[64 * c + 2 * i + 1]);
+        tmem_st32(lane_addr + 32 * c, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(LY::BAR_DS));
+      named_barrier_sync(1, 128);  // statistics of block j no longer read
+    }
+    if (ok) ok = mbar_wait(bar(LY::BAR_QD_EMPTY), (nj - 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const int kpos = kblk * kTile + key;
+      const bool valid = kpos < seq_len;
+      const int64_t g = (int64_t)seq_start + kpos;
+      if (part) {
+        float* prow = part + (int64_t)key * (DQK + DV);
+#pragma unroll 1
+        for (int c = 0; c < DQK / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + LY::T_DK + 32 * c, o);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(prow + 32 * c + i) =
+                make_float4(o[i] * p.scale, o[i + 1] * p.scale, o[i + 2] * p.scale, o[i + 3] * p.scale);
+        }
+#pragma unroll 1
+        for (int c = 0; c < DV / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + LY::T_DV + 32 * c, o);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(prow + DQK + 32 * c + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        }
+      } else {
+        __nv_bfloat16* dkr = p.dk + (g * p.n_heads + head) * (int64_t)DQK;
+        __nv_bfloat16* dvr = p.dv + (g * p.n_heads + head) * (int64_t)DV;
+#pragma unroll 1
+        for (int c = 0; c < DQK / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + LY::T_DK + 32 * c, o);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * p.scale, o[2 * i + 1] * p.scale);
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dkr + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+#pragma unroll 1
+        for (int c = 0; c < DV / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + LY::T_DV + 32 * c, o);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i], o[2 * i + 1]);
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dvr + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Sink blocks: dK, dV = sum of the partial slots, in slot order.
+// grid (128 key rows, s * H, B); thread = column of [DQK | DV].
+// ---------------------------------------------------------------------------
+template <int DQK, int DV>
+__global__ void __launch_bounds__(DQK + DV) ssa_bwd_sink_reduce(const BwdParams p) {
+  const int key = blockIdx.x;
+  const int kblk = blockIdx.y % p.n_sink, head = blockIdx.y / p.n_sink, seq = blockIdx.z;
+  const int seq_start = p.cu_seqlens[seq];
+  const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
+  const int nq = (seq_len + kTile - 1) / kTile;
+  const int kpos = kblk * kTile + key;
+  if (kblk >= nq || kpos >= seq_len) return;
+  const int col = threadIdx.x;
+  // slots that received work: 0 (local) and the far chunks that start inside the sequence
+  const int far = max(0, nq - (kblk + p.n_local));
+  const int used = min(p.nslots, 1 + (far + kSinkChunk - 1) / kSinkChunk);
+  const float* base = p.partial + (((int64_t)seq * p.n_sink + kblk) * p.n_heads + head) * p.nslots *
+                                      (int64_t)(kTile * (DQK + DV));
+  float acc = 0.f;
+  for (int s = 0; s < used; ++s) acc += base[(int64_t)s * kTile * (DQK + DV) + (int64_t)key * (DQK + DV) + col];
+  const int64_t g = (int64_t)seq_start + kpos;
+  if (col < DQK)
+    p.dk[(g * p.n_heads + head) * DQK + col] = __float2bfloat16_rn(acc);
+  else
+    p.dv[(g * p.n_heads + head) * DV + (col - DQK)] = __float2bfloat16_rn(acc);
+}
+
+}  // namespace loza

@@ -13,6 +13,7 @@
 #include "loza_ssa.h"
 #include "prefill.cuh"
 #include "decode.cuh"
+#include "backward.cuh"
 
 namespace loza {
 namespace {
@@ -88,6 +89,59 @@ DecodeWorkspace decode_workspace(int32_t batch, int nsplit) {
   w.ticket_off = w.ml_off + parts * sizeof(float2);
   w.total = w.ticket_off + ((size_t)batch * sizeof(int) + 255) / 256 * 256;
   return w;
+}
+
+// Backward workspace: D [T*H] fp32, then the sink partials
+// [B][s][H][nslots][128][DQK+DV] fp32.
+struct BwdWorkspace {
+  size_t d_off, part_off, total;
+  int nslots;
+};
+BwdWorkspace bwd_workspace(int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t n_heads, int d_qk,
+                           int d_v, const loza_ssa_params& p) {
+  BwdWorkspace w;
+  const int nq_max = (max_seqlen + kTile - 1) / kTile;
+  // sink block 0 has the most "far" query blocks: those at or after block l
+  const int far = nq_max > p.n_local ? nq_max - p.n_local : 0;
+  w.nslots = 1 + (far + kSinkChunk - 1) / kSinkChunk;
+  w.d_off = 0;
+  w.part_off = ((size_t)total_tokens * n_heads * sizeof(float) + 255) / 256 * 256;
+  w.total = w.part_off + (size_t)batch * p.n_sink * n_heads * w.nslots * kTile * (d_qk + d_v) * sizeof(float);
+  return w;
+}
+
+template <int DQK, int DV>
+loza_status launch_backward(BwdParams& prm, const void* out, const void* dout, int64_t rows, int nq_max, int batch,
+                            cudaStream_t st) {
+  {
+    const int64_t threads = rows * (DV / 8);
+    ssa_bwd_preprocess<DV><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), const_cast<float*>(prm.dvec),
+        rows);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  using LQ = BwdDqLayout<DQK, DV>;
+  using LK = BwdDkvLayout<DQK, DV>;
+  if (cudaFuncSetAttribute(ssa_bwd_dq_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           LQ::SMEM_BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(ssa_bwd_dkdv_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           LK::SMEM_BYTES) != cudaSuccess)
+    return LOZA_ERR_CUDA;
+  prm.far_mode = 0;
+  ssa_bwd_dq_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdThreads, LQ::SMEM_BYTES, st>>>(prm);
+  ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdThreads, LK::SMEM_BYTES, st>>>(prm);
+  g_launches.fetch_add(2, std::memory_order_relaxed);
+  if (prm.n_sink > 0) {
+    if (prm.nslots > 1) {
+      prm.far_mode = 1;
+      ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(prm.nslots - 1, prm.n_heads * prm.n_sink, batch), kBwdThreads,
+                                     LK::SMEM_BYTES, st>>>(prm);
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+    ssa_bwd_sink_reduce<DQK, DV><<<dim3(kTile, prm.n_heads * prm.n_sink, batch), DQK + DV, 0, st>>>(prm);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
 template <int DQK, int DVT, int NSTAGE>
@@ -176,6 +230,11 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
     if (n_kv_heads == 1 && n_heads == kDecHeads && d_qk == 576 && d_v == 512)
       return decode_workspace(batch, decode_plan(p, max_seqlen).nsplit).total;
     return 0;
+  }
+  if (op == LOZA_OP_BACKWARD) {
+    if (n_kv_heads != n_heads || p.n_local == LOZA_UNBOUNDED || total_tokens < 1) return 0;
+    if (!((d_qk == 64 && d_v == 64) || (d_qk == 192 && d_v == 128))) return 0;
+    return bwd_workspace(batch, total_tokens, max_seqlen, n_heads, d_qk, d_v, p).total;
   }
   return 0;
 }
@@ -342,10 +401,49 @@ loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const
                               int32_t max_seqlen, int32_t n_heads, int32_t n_kv_heads, int32_t d_qk,
                               int32_t d_v, loza_ssa_params p, void* dq, void* dk, void* dv, void* workspace,
                               size_t workspace_bytes, loza_stream_t stream) {
-  (void)q; (void)k; (void)v; (void)out; (void)dout; (void)lse; (void)cu_seqlens; (void)batch;
-  (void)total_tokens; (void)max_seqlen; (void)n_heads; (void)n_kv_heads; (void)d_qk; (void)d_v; (void)p;
-  (void)dq; (void)dk; (void)dv; (void)workspace; (void)workspace_bytes; (void)stream;
-  return LOZA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out || !dout || !lse || !cu_seqlens || !dq || !dk || !dv) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return LOZA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || total_tokens < 1 || total_tokens > INT32_MAX || max_seqlen < 1 ||
+      max_seqlen > total_tokens)
+    return LOZA_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
+  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (p.n_local == LOZA_UNBOUNDED) return LOZA_ERR_UNSUPPORTED;
+  if (n_kv_heads != n_heads || n_heads > 65535 / (p.n_sink > 0 ? p.n_sink : 1)) return LOZA_ERR_UNSUPPORTED;
+  const bool d64 = (d_qk == 64 && d_v == 64), d192 = (d_qk == 192 && d_v == 128);
+  if (!d64 && !d192) return LOZA_ERR_UNSUPPORTED;
+  const BwdWorkspace wl = bwd_workspace(batch, total_tokens, max_seqlen, n_heads, d_qk, d_v, p);
+  if (!workspace || !aligned16(workspace)) return LOZA_ERR_INVALID_ARG;
+  if (workspace_bytes < wl.total) return LOZA_ERR_WORKSPACE;
+
+  BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  const int64_t T = total_tokens;
+  if (!make_map_3d(&prm.tm_q, q, d_qk, n_heads, T, d_qk, (int64_t)n_heads * d_qk) ||
+      !make_map_3d(&prm.tm_k, k, d_qk, n_heads, T, d_qk, (int64_t)n_heads * d_qk) ||
+      !make_map_3d(&prm.tm_v, v, d_v, n_heads, T, d_v, (int64_t)n_heads * d_v) ||
+      !make_map_3d(&prm.tm_do, dout, d_v, n_heads, T, d_v, (int64_t)n_heads * d_v))
+    return LOZA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  prm.cu_seqlens = cu_seqlens;
+  prm.lse = lse;
+  prm.dvec = reinterpret_cast<float*>(ws + wl.d_off);
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.partial = reinterpret_cast<float*>(ws + wl.part_off);
+  prm.n_heads = n_heads;
+  prm.n_sink = p.n_sink;
+  prm.n_local = p.n_local;
+  prm.nslots = wl.nslots;
+  prm.scale = p.scale;
+  prm.scale_log2 = p.scale * 1.4426950408889634f;
+  const int nq_max = (max_seqlen + kTile - 1) / kTile;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d64) return launch_backward<64, 64>(prm, out, dout, T * n_heads, nq_max, batch, st);
+  return launch_backward<192, 128>(prm, out, dout, T * n_heads, nq_max, batch, st);
 }
 
 loza_status loza_ssa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

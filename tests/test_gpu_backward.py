@@ -1,0 +1,102 @@
+"""GPU parity of the SSA backward (dQ, dK, dV) against the fp64 oracle.
+
+Tolerance per tensor (the pages fix none for gradients; see the design notes):
+max-abs <= 1e-2 * max(1, max|ref|) and mean-abs <= 1e-3 * max(1, mean|ref|).
+The forward O and LSE fed to the backward come from the GPU forward, as in
+training; the oracle recomputes everything in fp64 from the inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import synth
+from helpers import from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def assert_close_grad(got, ref, what):
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), f"{what}: non-finite"
+    tol_max = 1e-2 * max(1.0, float(np.abs(ref).max()))
+    tol_mean = 1e-3 * max(1.0, float(np.abs(ref).mean()))
+    assert err.max() <= tol_max, f"{what}: max-abs {err.max():.3e} > {tol_max:.3e}"
+    assert err.mean() <= tol_mean, f"{what}: mean-abs {err.mean():.3e} > {tol_mean:.3e}"
+
+
+@pytest.fixture(scope="module")
+def bss():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import block_sparse_streaming_b200 as m
+    m.build()
+    return m
+
+
+def run_bwd(bss, seed, lens, H, dqk, dv, scale, n_sink=1, n_local=7):
+    import torch
+    g = synth.rng(seed)
+    T = int(sum(lens))
+    cu = synth.cu_seqlens(lens)
+    q = synth.normal_bits(g, (T, H, dqk))
+    k = synth.normal_bits(g, (T, H, dqk))
+    v = synth.normal_bits(g, (T, H, dv))
+    do = synth.normal_bits(g, (T, H, dv))
+    params = bss.Params(scale, 128, n_sink, n_local)
+    cu_d = torch.from_numpy(cu).cuda()
+    qd, kd, vd, dod = to_dev(q), to_dev(k), to_dev(v), to_dev(do)
+    out, lse = bss.loza_ssa_prefill(qd, kd, vd, cu_d, max(lens), params)
+    dq, dk, dvv = bss.loza_ssa_backward(qd, kd, vd, out, dod, lse, cu_d, max(lens), params)
+    torch.cuda.synchronize()
+    assert bss.device_status() == 0
+    return (q, k, v, do, cu), (from_dev(dq), from_dev(dk), from_dev(dvv))
+
+
+@pytest.mark.parametrize("dqk,dv,lens", [
+    (64, 64, [1000, 300, 129]),
+    (64, 64, [1]),
+    (192, 128, [2100, 700, 1]),
+])
+def test_backward_full_oracle(bss, oracle_mod, dqk, dv, lens):
+    H = 2
+    scale = 1 / 8 if dqk == 64 else 1 / math.sqrt(192)
+    (q, k, v, do, cu), (dq, dk, dvv) = run_bwd(bss, 101 + dqk, lens, H, dqk, dv, scale)
+    rq, rk, rv = oracle_mod.backward(q, k, v, do, cu, H, H, 128, 1, 7, scale)
+    assert_close_grad(dq, rq, "dQ")
+    assert_close_grad(dk, rk, "dK")
+    assert_close_grad(dvv, rv, "dV")
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(2, 3), (0, 2)])
+def test_backward_other_windows(bss, oracle_mod, n_sink, n_local):
+    lens = [1500, 260]
+    (q, k, v, do, cu), (dq, dk, dvv) = run_bwd(bss, 107, lens, 2, 64, 64, 0.125, n_sink, n_local)
+    rq, rk, rv = oracle_mod.backward(q, k, v, do, cu, 2, 2, 128, n_sink, n_local, 0.125)
+    assert_close_grad(dq, rq, "dQ")
+    assert_close_grad(dk, rk, "dK")
+    assert_close_grad(dvv, rv, "dV")
+
+
+def test_backward_long_sequence_sampled(bss, oracle_mod):
+    """40,000 tokens (313 query blocks): the sink block's far part spans two
+    partial chunks. dQ on 64 sampled rows; dK/dV on the sink rows and on rows of
+    ordinary blocks."""
+    L, H, dqk, dv = 40000, 1, 192, 128
+    scale = 1 / math.sqrt(192)
+    (q, k, v, do, cu), (dq, dk, dvv) = run_bwd(bss, 109, [L], H, dqk, dv, scale)
+    rs = np.random.default_rng(5)
+    qr = np.sort(rs.choice(L, 64, replace=False))
+    kr = np.array([0, 77, 127, 128, 5000, 20000, 39999] + list(rs.choice(L, 5, replace=False)))
+    rq, rk, rv = oracle_mod.backward(q, k, v, do, cu, H, H, 128, 1, 7, scale, q_rows=qr, k_rows=kr)
+    assert_close_grad(dq[qr], rq, "dQ rows")
+    assert_close_grad(dk[kr], rk, "dK rows")
+    assert_close_grad(dvv[kr], rv, "dV rows")
+
+
+def test_backward_is_deterministic(bss):
+    lens = [3000, 500]
+    _, a = run_bwd(bss, 111, lens, 2, 192, 128, 0.07)
+    _, b = run_bwd(bss, 111, lens, 2, 192, 128, 0.07)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
