@@ -152,16 +152,21 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- oracle (CPU) leg
 
-def oracle_sample(n_rows_target_s=15.0, rank_seed=0):
+_LATENT_CACHE = {}
+
+
+def oracle_sample(n_rows_target_s=15.0, rank_seed=0, seq_len=SEQLEN):
     """Time the fp64 oracle on a bounded sample of the prefill workload: query rows
-    spread over the sequence (all 64 heads of each). Returns (TFLOP/s, desc, cores)."""
+    spread over the sequence (all 64 heads of each). Returns (TFLOP/s, desc, cores, s)."""
     import oracle
     oracle.build()
     g = synth.rng(synth.workload_seed(2))
-    L = SEQLEN
+    L = seq_len
     # the latent KV in full (37.7 MB); Q only for the sampled rows
-    lat = synth.normal_bits(g, (L, 1, DQK))
-    vlat = np.ascontiguousarray(lat[:, :, :DV])
+    if L not in _LATENT_CACHE:
+        lat0 = synth.normal_bits(g, (L, 1, DQK))
+        _LATENT_CACHE[L] = (lat0, np.ascontiguousarray(lat0[:, :, :DV]))
+    lat, vlat = _LATENT_CACHE[L]
     cu = synth.cu_seqlens([L])
     q = np.zeros((L, H, DQK), np.uint16)
     rs = np.random.default_rng(12345 + rank_seed)
@@ -189,8 +194,9 @@ def run_reference(args, rank, world):
         return
     per = []
     desc = cores = None
+    per_step_s = max(0.5, 150.0 / (args.warmup + args.steps))   # whole run within a few minutes
     for i in range(args.warmup + args.steps):
-        v, desc, cores, dt = oracle_sample(n_rows_target_s=8.0, rank_seed=i)
+        v, desc, cores, dt = oracle_sample(n_rows_target_s=per_step_s, rank_seed=i)
         if i >= args.warmup:
             per.append((v, dt))
     value = statistics.mean(v for v, _ in per)
@@ -209,13 +215,188 @@ def run_reference(args, rank, world):
 
 # --------------------------------------------------------------------------- GPU leg
 
-def make_inputs(device, seed_offset=0):
+def make_inputs(device, seq_len, seed_offset=0):
     import torch
     seed = synth.workload_seed(2) * 1000 + seed_offset
-    q = synth.torch_normal_bf16((SEQLEN, H, DQK), seed, device)
-    lat = synth.torch_normal_bf16((SEQLEN, 1, DQK), seed + 1, device)
-    cu = torch.tensor([0, SEQLEN], dtype=torch.int32, device=device)
+    q = synth.torch_normal_bf16((seq_len, H, DQK), seed, device)
+    lat = synth.torch_normal_bf16((seq_len, 1, DQK), seed + 1, device)
+    cu = torch.tensor([0, seq_len], dtype=torch.int32, device=device)
     return q, lat, cu
+
+
+def time_launches(fn, stream, n, flush=None):
+    """Mean device time (ms) of n calls of fn, CUDA events on `stream` around each
+    call only; `flush` (if given) runs before every call, outside the events."""
+    import torch
+    ts = []
+    for _ in range(n):
+        if flush is not None:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.mean(ts), ts
+
+
+def decode_bytes(lens, n_local=LW):
+    """Algorithmic bytes of one absorbed decode call: every selected latent row once
+    (576 bf16; K and V share it), q, out and lse."""
+    rows = 0
+    for L in lens:
+        if n_local < 0:
+            rows += L
+        else:
+            j = (L - 1) // B
+            sel = set(range(min(S, j + 1))) | set(range(max(0, j - n_local + 1), j + 1))
+            rows += sum(min(B, L - kb * B) for kb in sel)
+    n = len(lens)
+    return rows * DQK * 2 + n * H * (DQK * 2 + DV * 2 + 4)
+
+
+def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20):
+    """SSA decode (and the dense full-context decode) on a latent cache
+    [len(lens), cap, 576]; L2 flushed (256 MB write) before every timed call."""
+    import torch
+    Bn = len(lens)
+    q = synth.torch_normal_bf16((Bn, H, DQK), synth.workload_seed(3) * 1000 + 1, device)
+    cache = synth.torch_normal_bf16((Bn, cap, 1, DQK), synth.workload_seed(3) * 1000 + 2, device)
+    seqlens = torch.tensor(lens, dtype=torch.int32, device=device)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    out = torch.empty((Bn, H, DV), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((Bn, H), dtype=torch.float32, device=device)
+    res = {}
+    for name, nl, n in (("ssa", LW, steps), ("dense", -1, 3)):
+        if name == "dense" and not with_dense:
+            continue
+        params = bss.Params(SCALE, B, S if nl > 0 else 0, nl)
+        ws = torch.empty(max(16, bss.workspace_size(bss.LOZA_OP_DECODE, Bn, 0, cap, H, 1, DQK, DV, params)),
+                         dtype=torch.uint8, device=device)
+
+        def call():
+            bss.loza_ssa_decode(q, cache, None, seqlens, cap, params, out=out, lse=lse, workspace=ws, stream=stream)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        ms, _ = time_launches(call, stream, n, flush=lambda: flush_buf.zero_())
+        nbytes = decode_bytes(lens, nl)
+        res[name] = {"ms": ms, "bytes": nbytes, "GB/s": nbytes / (ms / 1000.0) / 1e9, "launches_timed": n}
+        if bss.device_status() != 0:
+            raise RuntimeError("device status reports a timed-out wait in decode")
+    del cache
+    torch.cuda.empty_cache()
+    return res
+
+
+def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None):
+    w = synth.WORKLOADS[3]
+    g = synth.rng(synth.workload_seed(3))
+    lens = synth.uniform_lengths(g, w["batch"], w["ctx_lo"], w["ctx_hi"]).tolist()
+    if batch is not None:
+        lens = lens[:batch]
+    r = run_decode(bss, device, stream, lens, w["ctx_hi"])
+    hbm = float(peaks["hbm_gbs"])
+    ssa = r["ssa"]
+    out = {"workload": w["name"] if len(lens) == w["batch"] else f"{w['name']} (first {len(lens)} sequences)",
+           "metric": "SSA decode GB/s (bytes touched)", "value": ssa["GB/s"], "unit": "GB/s",
+           "ms_per_call": ssa["ms"], "bytes_per_call": ssa["bytes"],
+           "roofline": {"bound": "hbm", "achieved": ssa["GB/s"], "peak": hbm, "unit": "GB/s",
+                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic("ssa_decode_mla_kernel"),
+                        "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
+                        "kernel": "ssa_decode_mla_kernel"},
+           "timing": "mean of per-call CUDA events, L2 flushed (256 MB write) before each call"}
+    if "dense" in r:
+        d = r["dense"]
+        out["dense"] = {"ms_per_call": d["ms"], "bytes_per_call": d["bytes"], "GB/s": d["GB/s"],
+                        "frac_of_hbm": d["GB/s"] / hbm, "ssa_speedup": d["ms"] / ssa["ms"]}
+    return out
+
+
+def long_secondary(bss, device, stream, peaks):
+    """Workload 4: L = 262144 absorbed prefill, SSA next to full causal attention;
+    then SSA and dense decode of 32 sequences of 1,048,576 tokens."""
+    import torch
+    w = synth.WORKLOADS[4]
+    L = w["seqlen"]
+    q, lat, cu = make_inputs(device, L, seed_offset=40)
+    out = torch.empty((L, H, DV), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((L, H), dtype=torch.float32, device=device)
+    res = {"workload": w["name"]}
+    for name, nl, n in (("ssa", LW, 5), ("dense", -1, 1)):
+        params = bss.Params(SCALE, B, S if nl > 0 else 0, nl)
+
+        def call():
+            bss.loza_ssa_prefill(q, lat, lat[:, :, :DV], cu, L, params, out=out, lse=lse, stream=stream)
+
+        call()
+        torch.cuda.synchronize()
+        ms, _ = time_launches(call, stream, n)
+        fl = prefill_flops(L) if nl > 0 else 2.0 * (DQK + DV) * H * L * (L + 1) / 2
+        res[f"prefill_{name}"] = {"ms": ms, "algorithmic_tflop": fl / 1e12, "TFLOP/s": fl / (ms / 1000) / 1e12,
+                                  "frac_of_peak": fl / (ms / 1000) / 1e12 / float(peaks["bf16_tflops"])}
+    res["prefill_dense_over_ssa_time"] = res["prefill_dense"]["ms"] / res["prefill_ssa"]["ms"]
+    del q, lat, out, lse
+    torch.cuda.empty_cache()
+    r = run_decode(bss, device, stream, [w["decode_ctx"]] * w["decode_batch"], w["decode_ctx"])
+    hbm = float(peaks["hbm_gbs"])
+    res["decode_1m"] = {"ssa": dict(r["ssa"], frac_of_hbm=r["ssa"]["GB/s"] / hbm),
+                        "dense": dict(r["dense"], frac_of_hbm=r["dense"]["GB/s"] / hbm),
+                        "dense_over_ssa_time": r["dense"]["ms"] / r["ssa"]["ms"]}
+    return res
+
+
+def train_secondary(bss, device, stream, peaks):
+    """Workload 5: varlen forward + backward, per-head 192/128 dims, 64 heads."""
+    import torch
+    w = synth.WORKLOADS[5]
+    g = synth.rng(synth.workload_seed(5))
+    lens = synth.loguniform_lengths(g, w["batch"], w["len_lo"], w["len_hi"], w["total_cap"])
+    T = int(lens.sum())
+    Hh, dqk, dv = w["n_heads"], w["d_qk"], w["d_v"]
+    base = synth.workload_seed(5) * 1000
+    q = synth.torch_normal_bf16((T, Hh, dqk), base + 1, device)
+    k = synth.torch_normal_bf16((T, Hh, dqk), base + 2, device)
+    v = synth.torch_normal_bf16((T, Hh, dv), base + 3, device)
+    do = synth.torch_normal_bf16((T, Hh, dv), base + 4, device)
+    cu = torch.from_numpy(synth.cu_seqlens(lens)).to(device)
+    params = bss.Params(w["scale"], B, S, LW)
+    out = torch.empty((T, Hh, dv), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((T, Hh), dtype=torch.float32, device=device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dvv = torch.empty_like(v)
+    ws = torch.empty(bss.workspace_size(bss.LOZA_OP_BACKWARD, len(lens), T, int(lens.max()), Hh, Hh, dqk, dv, params),
+                     dtype=torch.uint8, device=device)
+    pairs = sum(visible_pairs(int(L)) for L in lens)
+    f_fwd = 2.0 * (dqk + dv) * Hh * pairs
+    f_bwd = 2.0 * (3 * dqk + 2 * dv) * Hh * pairs
+
+    def fwd():
+        bss.loza_ssa_prefill(q, k, v, cu, int(lens.max()), params, out=out, lse=lse, stream=stream)
+
+    def bwd():
+        bss.loza_ssa_backward(q, k, v, out, do, lse, cu, int(lens.max()), params, dq=dq, dk=dk, dv=dvv,
+                              workspace=ws, stream=stream)
+
+    fwd(); bwd()
+    torch.cuda.synchronize()
+    mf, _ = time_launches(fwd, stream, 3)
+    mb, _ = time_launches(bwd, stream, 3)
+    if bss.device_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait in training")
+    pk = float(peaks["bf16_tflops"])
+    res = {"workload": w["name"], "lengths": lens.tolist(), "total_tokens": T,
+           "forward": {"ms": mf, "TFLOP/s": f_fwd / (mf / 1000) / 1e12, "frac_of_peak": f_fwd / (mf / 1000) / 1e12 / pk,
+                       "algorithmic_tflop": f_fwd / 1e12},
+           "backward": {"ms": mb, "TFLOP/s": f_bwd / (mb / 1000) / 1e12, "frac_of_peak": f_bwd / (mb / 1000) / 1e12 / pk,
+                        "algorithmic_tflop": f_bwd / 1e12}}
+    del q, k, v, do, out, lse, dq, dk, dvv, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args, rank, world, local_rank):
@@ -226,15 +407,17 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     bss.lib()
-    params = bss.Params(SCALE, B, S, LW)
-    q, lat, cu = make_inputs(device, seed_offset=rank)
-    v = lat[:, :, :DV]
-    out = torch.empty((SEQLEN, H, DV), dtype=torch.bfloat16, device=device)
-    lse = torch.empty((SEQLEN, H), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream()
+    peaks, peak_kind = measured_peaks()
+    L = args.seq_len
+    params = bss.Params(SCALE, B, S, LW)
+    q, lat, cu = make_inputs(device, L, seed_offset=rank)
+    v = lat[:, :, :DV]
+    out = torch.empty((L, H, DV), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((L, H), dtype=torch.float32, device=device)
 
     def step():
-        bss.loza_ssa_prefill(q, lat, v, cu, SEQLEN, params, out=out, lse=lse, stream=stream)
+        bss.loza_ssa_prefill(q, lat, v, cu, L, params, out=out, lse=lse, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -264,74 +447,83 @@ def run_ours(args, rank, world, local_rank):
     launches = bss.launch_count() - launches0
     total_ms = t_all0.elapsed_time(t_all1)
     per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    status = bss.device_status()
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
+    if bss.device_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait after the timed region")
+    del q, lat, out, lse
+    torch.cuda.empty_cache()
 
     t = torch.tensor([total_ms], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     total_ms = float(t.item())
-    flops = prefill_flops()
+    flops = prefill_flops(L)
     value = world * args.steps * flops / (total_ms / 1000.0) / 1e12
 
-    # ---- end to end through the public API with host buffers
-    e2e = run_e2e(bss, params, device, stream, steps=max(1, min(args.steps, 3)))
+    e2e = None if args.no_e2e else run_e2e(bss, params, device, stream, L, steps=max(1, min(args.steps, 3)))
 
-    peaks, peak_kind = measured_peaks()
     avg_launch_ms = statistics.mean(per_launch_ms)
     achieved = flops / (avg_launch_ms / 1000.0) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = profiled_traffic("ssa_prefill_kernel<576,256,5>")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
+                "frac": achieved / peak, "traffic": profiled_traffic("ssa_prefill_kernel<576,256,5>"),
                 "peak_kind": f"{peak_kind} bf16 dense burst (MEASURED_PEAKS.json bf16_tflops)",
                 "kernel": "ssa_prefill_kernel<576,256,5>",
-                "algorithmic_flop_per_launch": flops}
+                "algorithmic_flop_per_launch": flops,
+                "avg_launch_ms": avg_launch_ms}
+
+    secondary = {}
+    if args.workload in ("default", "all"):
+        secondary["decode"] = decode_secondary(bss, device, stream, peaks, peak_kind, args.decode_batch)
+    if args.workload in ("long", "all"):
+        secondary["long"] = long_secondary(bss, device, stream, peaks)
+    if args.workload in ("train", "all"):
+        secondary["train"] = train_secondary(bss, device, stream, peaks)
 
     line = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            v_cpu, desc, cores, _ = oracle_sample()
+            v_cpu, desc, cores, _ = oracle_sample(seq_len=L)
             cpu = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD["name"], "batch": 1, "seq_len": SEQLEN, "n_heads": H,
+            "config": {"workload": WORKLOAD["name"] if L == SEQLEN else f"MLA-absorbed SSA prefill L={L}",
+                       "batch": 1, "seq_len": L, "n_heads": H,
                        "kv": "shared latent 576 (V = first 512)", "d_qk": DQK, "d_v": DV,
                        "block": [B, S, LW], "parallelism": f"replica x{world}",
-                       "l2": "inputs larger than L2 (Q is 2.4 GB per step)"},
+                       "l2": f"inputs larger than L2 (Q is {L * H * DQK * 2 / 1e9:.2f} GB per step)"},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk.summary(),
+            "secondary": secondary,
         }
     return line
 
 
-def run_e2e(bss, params, device, stream, steps):
+def run_e2e(bss, params, device, stream, L, steps):
     """Same metric through the public API with the inputs in pinned host memory:
     each step copies Q and the latent host->device, runs the prefill, copies O and
     LSE device->host; timed with CUDA events on the stream."""
     import torch
-    q_d, lat_d, cu = make_inputs(device, seed_offset=7)
+    q_d, lat_d, cu = make_inputs(device, L, seed_offset=7)
     q_h = torch.empty(q_d.shape, dtype=q_d.dtype, pin_memory=True)
     lat_h = torch.empty(lat_d.shape, dtype=lat_d.dtype, pin_memory=True)
     q_h.copy_(q_d)
     lat_h.copy_(lat_d)
-    out_h = torch.empty((SEQLEN, H, DV), dtype=torch.bfloat16, pin_memory=True)
-    lse_h = torch.empty((SEQLEN, H), dtype=torch.float32, pin_memory=True)
-    out_d = torch.empty((SEQLEN, H, DV), dtype=torch.bfloat16, device=device)
-    lse_d = torch.empty((SEQLEN, H), dtype=torch.float32, device=device)
+    out_h = torch.empty((L, H, DV), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = torch.empty((L, H), dtype=torch.float32, pin_memory=True)
+    out_d = torch.empty((L, H, DV), dtype=torch.bfloat16, device=device)
+    lse_d = torch.empty((L, H), dtype=torch.float32, device=device)
     torch.cuda.synchronize()
 
     def one():
         q_d.copy_(q_h, non_blocking=True)
         lat_d.copy_(lat_h, non_blocking=True)
-        bss.loza_ssa_prefill(q_d, lat_d, lat_d[:, :, :DV], cu, SEQLEN, params, out=out_d, lse=lse_d, stream=stream)
+        bss.loza_ssa_prefill(q_d, lat_d, lat_d[:, :, :DV], cu, L, params, out=out_d, lse=lse_d, stream=stream)
         out_h.copy_(out_d, non_blocking=True)
         lse_h.copy_(lse_d, non_blocking=True)
 
@@ -348,7 +540,8 @@ def run_e2e(bss, params, device, stream, steps):
     h2d = q_h.numel() * 2 + lat_h.numel() * 2
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
     del q_h, lat_h, out_h, lse_h, q_d, lat_d, out_d, lse_d
-    return {"value": prefill_flops() / (ms / 1000.0) / 1e12, "unit": UNIT, "ms_per_step": ms,
+    torch.cuda.empty_cache()
+    return {"value": prefill_flops(L) / (ms / 1000.0) / 1e12, "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 
@@ -359,6 +552,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=SEQLEN,
+                    help="prefill length (default: the 32,768-token workload; smaller values serve profiling)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="use only the first N sequences of the decode workload (profiling)")
+    ap.add_argument("--workload", choices=["default", "prefill", "long", "train", "all"], default="default",
+                    help="default: prefill line plus the 64-sequence decode; long/train/all add workloads 4/5")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

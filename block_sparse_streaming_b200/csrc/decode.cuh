@@ -15,9 +15,16 @@
 //     each block is loaded whole into shared memory (9 TMA tiles), S^T is
 //     computed as the tiles land, the softmax over keys is a column reduction
 //     (shuffle reduce-scatter + a 4-warp combine in shared memory), P^T goes to
-//     shared memory and O^T stays in TMEM. Each CTA writes its unnormalised
-//     partial (O, m, l) to the workspace; the last CTA of a sequence (atomic
-//     ticket, no waiting) merges the partials with the log-sum-exp rule.
+//     shared memory and O^T stays in TMEM. The partials (O, m, l) of a
+//     sequence's splits are merged with the log-sum-exp rule:
+//       - sink + local window (<= 8 blocks, one per CTA): the 8 CTAs of a
+//         sequence form a thread-block cluster; each stages its partial O in
+//         its own shared memory and then merges one 64-column slice of the
+//         output by reading all 8 partials over distributed shared memory, so
+//         no partial ever leaves the chip;
+//       - unbounded window (dense baseline, up to 32 splits of many blocks):
+//         partials go to the workspace and the last CTA of a sequence (atomic
+//         ticket, no waiting) merges them.
 // (2) ssa_decode_mha_kernel - per-head K/V (d = 64 or 192/128): one query
 //     vector per head against <= 1024 keys is a matrix-vector product, so it
 //     runs on CUDA cores: 4 warps per (sequence, head), online softmax per
@@ -56,8 +63,8 @@ struct DecodeLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = kDecQBytes;                 // 73728, 1024-aligned
   static constexpr int P_OFF = KV_OFF + 8 * kChunkBytes;    // P^T reuses the rope tile
-  static constexpr int RED_OFF = KV_OFF + kDecKvBytes;      // [4 warps][64] floats
-  static constexpr int STAT_OFF = RED_OFF + 4 * 64 * 4;     // m_run[64], l_run[64], alpha[64]
+  static constexpr int RED_OFF = KV_OFF + kDecKvBytes;      // [8][64] floats (reductions, merge weights)
+  static constexpr int STAT_OFF = RED_OFF + 8 * 64 * 4;     // m_run[64], l_run[64], alpha[64]
   static constexpr int BAR_OFF = STAT_OFF + 3 * 64 * 4;
   // barriers: q_full, kv_full[9], s_full, p_ready, pv_done
   static constexpr int BAR_Q = 0, BAR_KV = 1, BAR_S = 10, BAR_P = 11, BAR_PV = 12, NBAR = 13;
@@ -133,6 +140,7 @@ __device__ __forceinline__ void warp_reduce_scatter64(const float (&v)[64], floa
          (lane & 1) * 2;
 }
 
+template <bool CLUSTER>
 __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __grid_constant__ DecodeParams p) {
   using LY = DecodeLayout;
   extern __shared__ uint8_t smem_raw[];
@@ -356,6 +364,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       if (ok) {
         tc_fence_after();
         named_barrier_sync(1, 128);  // l_run complete
+        // CLUSTER: stage O^T as [head][512] fp32 over the (now idle) K/V tiles;
+        // otherwise write it to this split's workspace slot.
+        float* so = reinterpret_cast<float*>(smem + LY::KV_OFF);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           const int dv = 128 * c + key;
@@ -364,16 +375,92 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
             float o[32];
             tmem_ld32(lane_addr + 64 + 64 * c + 32 * hh, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              p.ws_o[(part * kDecHeads + 32 * hh + i) * 512 + dv] = o[i];
+            for (int i = 0; i < 32; ++i) {
+              if (CLUSTER)
+                so[(32 * hh + i) * 512 + dv] = o[i];
+              else
+                p.ws_o[(part * kDecHeads + 32 * hh + i) * 512 + dv] = o[i];
+            }
           }
         }
-        if (tid < 64) p.ws_ml[part * kDecHeads + tid] = make_float2(m_run[tid], l_run[tid]);
+        if (!CLUSTER && tid < 64) p.ws_ml[part * kDecHeads + tid] = make_float2(m_run[tid], l_run[tid]);
       }
     }
-  } else if (threadIdx.x < 64) {
+  } else if (!CLUSTER && threadIdx.x < 64) {
     // no block for this split: an empty partial
     p.ws_ml[part * kDecHeads + threadIdx.x] = make_float2(-INFINITY, 0.f);
+  }
+
+  if (CLUSTER) {
+    // ---------------------------------------------------------- on-chip merge
+    // Split r of the cluster merges output columns [r*W, (r+1)*W) of every head,
+    // W = 512 / nsplit, reading the partials of all splits over DSMEM. Splits
+    // without a block have l = 0 and weight 0 (their staging area is not read).
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    const int r = (int)cluster_rank();
+    constexpr int NS = 8;  // splits per cluster (== cluster size)
+    float* wgt = red;      // [NS][64] merge weights
+    float* mls = reinterpret_cast<float*>(smem + LY::Q_OFF);  // [2][NS][64] peers' m, l (Q tiles are idle now)
+    for (int idx = threadIdx.x; idx < NS * 64; idx += blockDim.x) {
+      const int s2 = idx >> 6, h = idx & 63;
+      const float* pm = static_cast<const float*>(__cluster_map_shared_rank(m_run + h, s2));
+      const float* pl = static_cast<const float*>(__cluster_map_shared_rank(l_run + h, s2));
+      mls[idx] = *pm;
+      mls[NS * 64 + idx] = *pl;
+    }
+    __syncthreads();
+    if (threadIdx.x < 64) {
+      const int h = threadIdx.x;
+      float M = -INFINITY;
+#pragma unroll
+      for (int s2 = 0; s2 < NS; ++s2)
+        if (mls[NS * 64 + s2 * 64 + h] > 0.f) M = fmaxf(M, mls[s2 * 64 + h]);
+      float Ls = 0.f, w[NS];
+#pragma unroll
+      for (int s2 = 0; s2 < NS; ++s2) {
+        const float l = mls[NS * 64 + s2 * 64 + h];
+        w[s2] = l > 0.f ? exp2f(mls[s2 * 64 + h] - M) : 0.f;
+        Ls += l * w[s2];
+      }
+      const float inv = 1.f / Ls;
+#pragma unroll
+      for (int s2 = 0; s2 < NS; ++s2) wgt[s2 * 64 + h] = w[s2] * inv;
+      if (r == 0) p.lse[(int64_t)seq * kDecHeads + h] = (M + log2f(Ls)) * 0.69314718055994530942f;
+    }
+    __syncthreads();
+    constexpr int W = 512 / NS;  // output columns this split merges
+    const float* so = reinterpret_cast<const float*>(smem + LY::KV_OFF);
+    for (int idx = threadIdx.x; idx < kDecHeads * (W / 4); idx += blockDim.x) {
+      const int h = idx / (W / 4);
+      const int d = r * W + (idx % (W / 4)) * 4;
+      float4 o[NS];
+#pragma unroll
+      for (int s2 = 0; s2 < NS; ++s2) {
+        // a split without a block has weight 0 and an unwritten staging area: do not read it
+        o[s2] = wgt[s2 * 64 + h] != 0.f
+                    ? *static_cast<const float4*>(__cluster_map_shared_rank(so + h * 512 + d, s2))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s2 = 0; s2 < NS; ++s2) {
+        const float w = wgt[s2 * 64 + h];
+        acc.x += o[s2].x * w;
+        acc.y += o[s2].y * w;
+        acc.z += o[s2].z * w;
+        acc.w += o[s2].w * w;
+      }
+      __nv_bfloat16* dst = p.out + ((int64_t)seq * kDecHeads + h) * 512 + d;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+    }
+    cluster_sync_all();  // peers may still read this CTA's shared memory until here
+    if (warp == 1 && nb > 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+    return;
   }
 
   // ------------------------------------------------------------ last CTA merges
@@ -384,30 +471,44 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
   __syncthreads();
   if (*last_flag) {
     __threadfence();
-    // 192 threads: head h = t / 3 ... use a strided loop over (head, dv) pairs
+    // merge weights per (split, head) once, then stream the partials
+    float* wgt = reinterpret_cast<float*>(smem + LY::KV_OFF);  // [nsplit][64], K/V tiles are idle now
+    if (threadIdx.x < 64) {
+      const int h = threadIdx.x;
+      float M = -INFINITY;
+      for (int s2 = 0; s2 < p.nsplit; ++s2) {
+        const float2 ml = p.ws_ml[((int64_t)seq * p.nsplit + s2) * kDecHeads + h];
+        if (ml.y > 0.f) M = fmaxf(M, ml.x);
+      }
+      float Ls = 0.f;
+      for (int s2 = 0; s2 < p.nsplit; ++s2) {
+        const float2 ml = p.ws_ml[((int64_t)seq * p.nsplit + s2) * kDecHeads + h];
+        const float w = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;
+        wgt[s2 * 64 + h] = w;
+        Ls += ml.y * w;
+      }
+      const float inv = 1.f / Ls;
+      for (int s2 = 0; s2 < p.nsplit; ++s2) wgt[s2 * 64 + h] *= inv;
+      p.lse[(int64_t)seq * kDecHeads + h] = (M + log2f(Ls)) * 0.69314718055994530942f;
+    }
+    __syncthreads();
     for (int idx = threadIdx.x; idx < kDecHeads * 128; idx += blockDim.x) {
       const int h = idx >> 7;
       const int d4 = (idx & 127) * 4;
-      float mmax = -INFINITY;
-      for (int s = 0; s < p.nsplit; ++s) mmax = fmaxf(mmax, p.ws_ml[((int64_t)seq * p.nsplit + s) * kDecHeads + h].x);
-      float lsum = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s = 0; s < p.nsplit; ++s) {
-        const int64_t ps = (int64_t)seq * p.nsplit + s;
-        const float2 ml = p.ws_ml[ps * kDecHeads + h];
-        if (ml.y == 0.f) continue;
-        const float w = exp2f(ml.x - mmax);
-        lsum += ml.y * w;
-        const float4 o = *reinterpret_cast<const float4*>(p.ws_o + (ps * kDecHeads + h) * 512 + d4);
-        acc.x += o.x * w;
-        acc.y += o.y * w;
-        acc.z += o.z * w;
-        acc.w += o.w * w;
+#pragma unroll 8
+      for (int s2 = 0; s2 < p.nsplit; ++s2) {
+        const float w = wgt[s2 * 64 + h];
+        const float4 o = *reinterpret_cast<const float4*>(p.ws_o + (((int64_t)seq * p.nsplit + s2) * kDecHeads + h) * 512 + d4);
+        if (w != 0.f) {
+          acc.x += o.x * w;
+          acc.y += o.y * w;
+          acc.z += o.z * w;
+          acc.w += o.w * w;
+        }
       }
-      const float inv = 1.f / lsum;
       __nv_bfloat16* dst = p.out + ((int64_t)seq * kDecHeads + h) * 512 + d4;
-      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
-      if ((idx & 127) == 0) p.lse[(int64_t)seq * kDecHeads + h] = (mmax + log2f(lsum)) * 0.69314718055994530942f;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
     }
     if (threadIdx.x == 0) p.ws_ticket[seq] = 0;  // ready for the next call
   }

@@ -62,33 +62,123 @@ bool window_ok(const loza_ssa_params& p) {
 }
 
 // Split-KV plan of the absorbed decode: selected blocks per CTA and CTAs per
-// sequence. A bounded window has at most s + l blocks (one per CTA); the
-// unbounded (dense) window spreads up to ceil(max_seqlen / 128) blocks over at
-// most 32 CTAs per sequence.
+// sequence. A sink + local window of at most 8 blocks runs one block per CTA,
+// 8 CTAs per sequence in one thread-block cluster that merges on chip (no
+// workspace). Larger windows and the unbounded (dense) window spread the
+// blocks over at most 32 CTAs per sequence and merge through the workspace.
 struct DecodePlan {
   int bps, nsplit;
+  bool cluster;
 };
+constexpr int kDecClusterSplits = 8;
 DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen) {
   const int max_blocks = (max_seqlen + kTile - 1) / kTile;
-  if (p.n_local == LOZA_UNBOUNDED) {
-    const int bps = (max_blocks + 31) / 32;
-    return {bps, (max_blocks + bps - 1) / bps};
-  }
-  const int nb = p.n_sink + p.n_local;
-  return {1, nb < max_blocks ? nb : max_blocks};
+  if (p.n_local != LOZA_UNBOUNDED && p.n_sink + p.n_local <= kDecClusterSplits)
+    return {1, kDecClusterSplits, true};
+  const int nb = p.n_local == LOZA_UNBOUNDED ? max_blocks
+                                             : (p.n_sink + p.n_local < max_blocks ? p.n_sink + p.n_local : max_blocks);
+  const int bps = (nb + 31) / 32;
+  return {bps, (nb + bps - 1) / bps, false};
 }
 
 struct DecodeWorkspace {
   size_t o_off, ml_off, ticket_off, total;
 };
-DecodeWorkspace decode_workspace(int32_t batch, int nsplit) {
-  DecodeWorkspace w;
-  const size_t parts = (size_t)batch * nsplit * kDecHeads;
+DecodeWorkspace decode_workspace(int32_t batch, const DecodePlan& plan) {
+  DecodeWorkspace w{0, 0, 0, 0};
+  if (plan.cluster) return w;
+  const size_t parts = (size_t)batch * plan.nsplit * kDecHeads;
   w.o_off = 0;
   w.ml_off = parts * 512 * sizeof(float);
   w.ticket_off = w.ml_off + parts * sizeof(float2);
   w.total = w.ticket_off + ((size_t)batch * sizeof(int) + 255) / 256 * 256;
   return w;
+}
+
+// Validate an absorbed-MLA decode call and build its kernel parameters
+// (everything except the workspace pointers).
+loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                             int32_t batch, int32_t max_seqlen, int64_t cache_batch_stride,
+                             int64_t cache_row_stride, int32_t n_heads, const loza_ssa_params& p, void* out,
+                             float* lse, DecodeParams* prm, DecodePlan* plan) {
+  if (!q || !k_cache || !seqlens || !out || !lse) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || max_seqlen < 1) return LOZA_ERR_INVALID_ARG;
+  if (!stride_ok(cache_row_stride) || !stride_ok(cache_batch_stride) ||
+      cache_batch_stride < (int64_t)max_seqlen * cache_row_stride || cache_row_stride < 576)
+    return LOZA_ERR_INVALID_ARG;
+  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
+  if (v_cache && v_cache != k_cache) return LOZA_ERR_UNSUPPORTED;
+  *plan = decode_plan(p, max_seqlen);
+  std::memset(prm, 0, sizeof(*prm));
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return LOZA_ERR_CUDA;
+  {
+    cuuint64_t dims[3] = {576, (cuuint64_t)n_heads, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {576 * 2, (cuuint64_t)n_heads * 576 * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&prm->tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return LOZA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {576, (cuuint64_t)max_seqlen, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {(cuuint64_t)cache_row_stride * 2, (cuuint64_t)cache_batch_stride * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&prm->tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return LOZA_ERR_CUDA;
+  }
+  prm->seqlens = seqlens;
+  prm->out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm->lse = lse;
+  prm->nsplit = plan->nsplit;
+  prm->bps = plan->bps;
+  prm->n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
+  prm->n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
+  prm->scale_log2 = p.scale * 1.4426950408889634f;
+  return LOZA_OK;
+}
+
+// Point the kernel at its workspace (unless the plan merges on chip) and launch.
+loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t batch, uint8_t* ws,
+                              cudaStream_t st) {
+  if (!plan.cluster) {
+    const DecodeWorkspace wl = decode_workspace(batch, plan);
+    prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+    prm.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
+    prm.ws_ticket = reinterpret_cast<int*>(ws + wl.ticket_off);
+    // the arrival counters must start at zero; the partials are fully rewritten
+    if (cudaMemsetAsync(prm.ws_ticket, 0, (size_t)batch * sizeof(int), st) != cudaSuccess) return LOZA_ERR_CUDA;
+    if (cudaFuncSetAttribute(ssa_decode_mla_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeLayout::SMEM_BYTES) != cudaSuccess)
+      return LOZA_ERR_CUDA;
+    ssa_decode_mla_kernel<false><<<dim3(plan.nsplit, batch), kDecThreads, DecodeLayout::SMEM_BYTES, st>>>(prm);
+  } else {
+    if (cudaFuncSetAttribute(ssa_decode_mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeLayout::SMEM_BYTES) != cudaSuccess)
+      return LOZA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.nsplit, batch, 1);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = DecodeLayout::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = plan.nsplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, ssa_decode_mla_kernel<true>, prm) != cudaSuccess) return LOZA_ERR_CUDA;
+  }
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
 // Backward workspace: D [T*H] fp32, then the sink partials
@@ -228,7 +318,7 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
   if (batch < 1 || max_seqlen < 1 || !window_ok(p)) return 0;
   if (op == LOZA_OP_DECODE) {
     if (n_kv_heads == 1 && n_heads == kDecHeads && d_qk == 576 && d_v == 512)
-      return decode_workspace(batch, decode_plan(p, max_seqlen).nsplit).total;
+      return decode_workspace(batch, decode_plan(p, max_seqlen)).total;
     return 0;
   }
   if (op == LOZA_OP_BACKWARD) {
@@ -316,55 +406,17 @@ loza_status loza_ssa_decode(const void* q, const void* k_cache, const void* v_ca
 
   if (n_kv_heads == 1 && d_qk == 576 && d_v == 512) {
     // absorbed MLA: shared latent cache, V = first 512 columns
-    if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
-    if (v_cache && v_cache != k_cache) return LOZA_ERR_UNSUPPORTED;
-    const DecodePlan plan = decode_plan(p, max_seqlen);
-    const DecodeWorkspace wl = decode_workspace(batch, plan.nsplit);
-    if (!workspace || !aligned16(workspace)) return LOZA_ERR_INVALID_ARG;
-    if (workspace_bytes < wl.total) return LOZA_ERR_WORKSPACE;
     DecodeParams prm;
-    std::memset(&prm, 0, sizeof(prm));
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return LOZA_ERR_CUDA;
-    {
-      cuuint64_t dims[3] = {576, (cuuint64_t)n_heads, (cuuint64_t)batch};
-      cuuint64_t strides[2] = {576 * 2, (cuuint64_t)n_heads * 576 * 2};
-      cuuint32_t box[3] = {64, 64, 1};
-      cuuint32_t estr[3] = {1, 1, 1};
-      if (fn(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return LOZA_ERR_CUDA;
+    DecodePlan plan;
+    const loza_status rc = setup_decode_mla(q, k_cache, v_cache, seqlens, batch, max_seqlen, cache_batch_stride,
+                                            cache_row_stride, n_heads, p, out, lse, &prm, &plan);
+    if (rc != LOZA_OK) return rc;
+    const DecodeWorkspace wl = decode_workspace(batch, plan);
+    if (wl.total > 0) {
+      if (!workspace || !aligned16(workspace)) return LOZA_ERR_INVALID_ARG;
+      if (workspace_bytes < wl.total) return LOZA_ERR_WORKSPACE;
     }
-    {
-      cuuint64_t dims[3] = {576, (cuuint64_t)max_seqlen, (cuuint64_t)batch};
-      cuuint64_t strides[2] = {(cuuint64_t)cache_row_stride * 2, (cuuint64_t)cache_batch_stride * 2};
-      cuuint32_t box[3] = {64, 128, 1};
-      cuuint32_t estr[3] = {1, 1, 1};
-      if (fn(&prm.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return LOZA_ERR_CUDA;
-    }
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    prm.seqlens = seqlens;
-    prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
-    prm.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
-    prm.ws_ticket = reinterpret_cast<int*>(ws + wl.ticket_off);
-    prm.out = reinterpret_cast<__nv_bfloat16*>(out);
-    prm.lse = lse;
-    prm.nsplit = plan.nsplit;
-    prm.bps = plan.bps;
-    prm.n_sink = n_sink;
-    prm.n_local = n_local;
-    prm.scale_log2 = scale_log2;
-    if (cudaMemsetAsync(prm.ws_ticket, 0, (size_t)batch * sizeof(int), st) != cudaSuccess) return LOZA_ERR_CUDA;
-    if (cudaFuncSetAttribute(ssa_decode_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DecodeLayout::SMEM_BYTES) != cudaSuccess)
-      return LOZA_ERR_CUDA;
-    ssa_decode_mla_kernel<<<dim3(plan.nsplit, batch), kDecThreads, DecodeLayout::SMEM_BYTES, st>>>(prm);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+    return launch_decode_mla(prm, plan, batch, static_cast<uint8_t*>(workspace), st);
   }
 
   // per-head K/V on CUDA cores
@@ -455,65 +507,22 @@ loza_status loza_ssa_decode_noalloc(const void* q, const void* k_cache, const vo
   if (!(n_kv_heads == 1 && d_qk == 576 && d_v == 512))
     return loza_ssa_decode(q, k_cache, v_cache, seqlens, batch, max_seqlen, cache_batch_stride, cache_row_stride,
                            n_heads, n_kv_heads, d_qk, d_v, p, out, lse, nullptr, 0, stream);
-  if (!q || !k_cache || !seqlens || !out || !lse) return LOZA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
-  if (batch < 1 || batch > 65535 || max_seqlen < 1) return LOZA_ERR_INVALID_ARG;
-  if (!stride_ok(cache_row_stride) || !stride_ok(cache_batch_stride) ||
-      cache_batch_stride < (int64_t)max_seqlen * cache_row_stride || cache_row_stride < d_qk)
-    return LOZA_ERR_INVALID_ARG;
-  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
-  if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
-  if (v_cache && v_cache != k_cache) return LOZA_ERR_UNSUPPORTED;
-  const DecodePlan plan = decode_plan(p, max_seqlen);
-  const DecodeWorkspace wl = decode_workspace(batch, plan.nsplit);
-  if (wl.total > kNoAllocScratchBytes) return LOZA_ERR_WORKSPACE;  // batch too large for the built-in scratch
-
-  uint8_t* ws = static_cast<uint8_t*>(decode_scratch_address());
-  if (!ws) return LOZA_ERR_CUDA;
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return LOZA_ERR_CUDA;
+  // batch too large for the built-in scratch: refuse before touching the driver
+  if (batch >= 1 && max_seqlen >= 1 && window_ok(p) &&
+      decode_workspace(batch, decode_plan(p, max_seqlen)).total > kNoAllocScratchBytes)
+    return LOZA_ERR_WORKSPACE;
   DecodeParams prm;
-  std::memset(&prm, 0, sizeof(prm));
-  {
-    cuuint64_t dims[3] = {576, (cuuint64_t)n_heads, (cuuint64_t)batch};
-    cuuint64_t strides[2] = {576 * 2, (cuuint64_t)n_heads * 576 * 2};
-    cuuint32_t box[3] = {64, 64, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    if (fn(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return LOZA_ERR_CUDA;
+  DecodePlan plan;
+  const loza_status rc = setup_decode_mla(q, k_cache, v_cache, seqlens, batch, max_seqlen, cache_batch_stride,
+                                          cache_row_stride, n_heads, p, out, lse, &prm, &plan);
+  if (rc != LOZA_OK) return rc;
+  const DecodeWorkspace wl = decode_workspace(batch, plan);
+  uint8_t* ws = nullptr;
+  if (wl.total > 0) {
+    ws = static_cast<uint8_t*>(decode_scratch_address());
+    if (!ws) return LOZA_ERR_CUDA;
   }
-  {
-    cuuint64_t dims[3] = {576, (cuuint64_t)max_seqlen, (cuuint64_t)batch};
-    cuuint64_t strides[2] = {(cuuint64_t)cache_row_stride * 2, (cuuint64_t)cache_batch_stride * 2};
-    cuuint32_t box[3] = {64, 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    if (fn(&prm.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return LOZA_ERR_CUDA;
-  }
-  prm.seqlens = seqlens;
-  prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
-  prm.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
-  prm.ws_ticket = reinterpret_cast<int*>(ws + wl.ticket_off);
-  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
-  prm.lse = lse;
-  prm.nsplit = plan.nsplit;
-  prm.bps = plan.bps;
-  prm.n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
-  prm.n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
-  prm.scale_log2 = p.scale * 1.4426950408889634f;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // The arrival counters must start at zero; the partials are fully rewritten.
-  if (cudaMemsetAsync(prm.ws_ticket, 0, (size_t)batch * sizeof(int), st) != cudaSuccess) return LOZA_ERR_CUDA;
-  if (cudaFuncSetAttribute(ssa_decode_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           DecodeLayout::SMEM_BYTES) != cudaSuccess)
-    return LOZA_ERR_CUDA;
-  ssa_decode_mla_kernel<<<dim3(plan.nsplit, batch), kDecThreads, DecodeLayout::SMEM_BYTES, st>>>(prm);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+  return launch_decode_mla(prm, plan, batch, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -231,69 +231,80 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     const int row = quarter * 32 + lane;               // row of the tile == TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int qpos = qb * kTile + row;                  // position inside the sequence
+    // m_run: running row maximum of scale*log2(e)*s (the reference of P);
+    // l_run: running sum of 2^(x - m_run).
     float m_run = -INFINITY, l_run = 0.f;
+    const float c = p.scale_log2;  // > 0, so max(c*s) = c*max(s)
     bool ok = true;
     for (int b = 0; b < nb && ok; ++b) {
       ok = mbar_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       float s[128];
+      tmem_ld128(lane_addr + (b & 1) * 128, s);
+      // the diagonal block is token-causal: keys after this row's query do not exist
+      if (walk.block(b) == qb) {
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          if (j > row) s[j] = -INFINITY;
+      }
+      float mx;
       {
-        float t[32];
+        float m8[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          tmem_ld32(lane_addr + (b & 1) * 128 + 32 * j, t);
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s[32 * j + i] = t[i];
-        }
+        for (int j = 8; j < 128; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        mx *= c;
       }
-      const bool diag = walk.block(b) == qb;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 128; ++j) {
-        float x = s[j] * p.scale_log2;
-        if (diag && j > row) x = -INFINITY;
-        s[j] = x;
-        mx = fmaxf(mx, x);
-      }
+      // Wait for PV(b-1) every block (it has normally long finished by now).
+      // Phases of this barrier must be waited in order: a parity wait is only
+      // exact while the waiter is at most one phase behind.
       if (b > 0) {
         ok = mbar_wait(bar(LY::BAR_PV), (b - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
       }
+      // keep the stale maximum unless this block raises it by more than 2^8;
+      // only then is O (in TMEM) rescaled
       float alpha = 1.f;
       if (b == 0) {
         m_run = mx;
       } else if (mx > m_run + (float)kRescaleThreshold) {
-        alpha = exp2f(m_run - mx);
+        alpha = ex2_approx(m_run - mx);
         m_run = mx;
       }
-      // O rescale (warp-uniform decision so the TMEM accesses stay converged)
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-        for (int c = 0; c < DVT / 32; ++c) {
+        for (int cc = 0; cc < DVT / 32; ++cc) {
           float o[32];
-          tmem_ld32(lane_addr + 256 + 32 * c, o);
+          tmem_ld32(lane_addr + 256 + 32 * cc, o);
           uint32_t w[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
-          tmem_st32(lane_addr + 256 + 32 * c, w);
+          tmem_st32(lane_addr + 256 + 32 * cc, w);
         }
         tmem_st_wait();
       }
-      float sum = 0.f;
+      const float neg_m = -m_run;
+      float sum8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = exp2f(s[64 * h + 2 * i] - m_run);
-          const float p1 = exp2f(s[64 * h + 2 * i + 1] - m_run);
-          sum += p0 + p1;
+          const float p0 = ex2_approx(fmaf(s[64 * h + 2 * i], c, neg_m));
+          const float p1 = ex2_approx(fmaf(s[64 * h + 2 * i + 1], c, neg_m));
+          sum8[(2 * i) & 7] += p0;
+          sum8[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16(p0, p1);
         }
         tmem_st32(lane_addr + (b & 1) * 128 + 32 * h, pk);
       }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * alpha + sum;
       tmem_st_wait();
       tc_fence_before();
@@ -307,16 +318,20 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       const int64_t grow = (int64_t)seq_start + qpos;
       __nv_bfloat16* orow = p.out + (grow * p.n_heads + head) * (int64_t)p.d_v + slice * DVT;
 #pragma unroll 1
-      for (int c = 0; c < DVT / 32; ++c) {
-        float o[32];
-        tmem_ld32(lane_addr + 256 + 32 * c, o);
-        uint32_t w[16];
+      for (int cc = 0; cc < DVT / 64; ++cc) {
+        float o[32], o2[32];
+        tmem_ld32(lane_addr + 256 + 64 * cc, o);
+        tmem_ld32(lane_addr + 256 + 64 * cc + 32, o2);
+        uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * inv, o[2 * i + 1] * inv);
+        for (int i = 0; i < 16; ++i) {
+          w[i] = pack_bf16(o[2 * i] * inv, o[2 * i + 1] * inv);
+          w[16 + i] = pack_bf16(o2[2 * i] * inv, o2[2 * i + 1] * inv);
+        }
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(orow + 64 * cc);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
       if (valid && slice == 0)

@@ -151,19 +151,21 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  * access to it, a serving runtime that has reserved all device memory for its
  * own KV-cache pool up front, or a latency-critical loop that must not pay
  * for cudaMalloc/cudaFree. For them this entry point takes the same arguments
- * as loza_ssa_decode minus the workspace, and keeps the split-KV partial
- * results in a fixed 16 MiB array that is part of the library itself.
+ * as loza_ssa_decode minus the workspace. Where the absorbed decode needs
+ * scratch for its split-KV partial results (windows of more than 8 blocks and
+ * the unbounded window), they go to a fixed 16 MiB array that is part of the
+ * library itself; the 1 + 7 window merges its partials on chip and needs none.
  *   - The library never allocates: every GPU that loads the library holds the
  *     16 MiB array until the process exits.
- *   - Limit: the absorbed MLA shape needs batch * nsplit * 131,584 bytes plus
- *     256 for the counters, where nsplit = n_sink + n_local (8 for the pages'
- *     1 + 7 window) or min(32, number of 128-token blocks) for the unbounded
- *     window. With the pages' window at most 15 sequences fit. A larger batch
- *     returns LOZA_ERR_WORKSPACE before anything is launched; call
- *     loza_ssa_decode with a workspace instead, or split the batch.
- *   - The first call on each device looks up the array's device address
- *     (with that device current); make that first call before any stream
- *     capture on that device.
+ *   - Limit: a call that needs scratch needs batch * nsplit * 131,584 bytes
+ *     plus 256 for the counters, with nsplit = min(32, number of selected
+ *     128-token blocks); e.g. at most 3 sequences of 4,096+ tokens with the
+ *     unbounded window. A larger call returns LOZA_ERR_WORKSPACE before
+ *     anything is launched; use loza_ssa_decode with a workspace instead, or
+ *     split the batch.
+ *   - The first call on each device that needs scratch looks up the array's
+ *     device address (with that device current); make that first call before
+ *     any stream capture on that device.
  *   - Every call uses the same array and leaves its last contents there; the
  *     arrival counters are cleared on the caller's stream at the start of each
  *     call. Two calls whose kernels can overlap on the GPU (different streams

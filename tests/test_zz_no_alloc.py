@@ -3,10 +3,12 @@
 loza_ssa_decode_noalloc serves callers such as a plug-in whose host
 application owns the device allocator, or a serving runtime that reserved all
 device memory for its own pool: it takes no workspace and keeps its split-KV
-partials in a fixed array inside the library. These tests call it through the
-C ABI and check it against loza_ssa_decode (which uses a caller-provided
-workspace) on two calls in a row, so the second call also shows that the
-shared array is correctly reused. This file is collected last on purpose.
+partials in a fixed array inside the library (the unbounded window is the
+decode that needs such scratch; the 1 + 7 window merges on chip). These tests
+call it through the C ABI and check it against loza_ssa_decode (which uses a
+caller-provided workspace) on two calls in a row per window, so the second
+call also shows that the shared array is correctly reused. This file is
+collected last on purpose.
 """
 import ctypes
 import math
@@ -33,9 +35,10 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     import torch
     import block_sparse_streaming_b200 as bss
     bss.build()
-    params = bss.Params(1.0 / math.sqrt(192.0))
-    cases = [(71, [1, 130, 1025, 3000, 4096], 4096), (72, [4096, 7, 2000], 4096)]
-    for seed, lens, Lcap in cases:                    # two calls in a row
+    windows = [bss.Params(1.0 / math.sqrt(192.0)),                          # 1 + 7 window
+               bss.Params(1.0 / math.sqrt(192.0), 128, 0, bss.LOZA_UNBOUNDED)]  # needs the scratch array
+    cases = [(71, [1, 130, 1025, 3000], 3072), (72, [3072, 7, 2000], 3072)]
+    for params, (seed, lens, Lcap) in [(w, c) for w in windows for c in cases]:  # two calls in a row each
         q, cache, seqlens = _inputs(seed, lens, Lcap)
         ref_o, ref_l = bss.loza_ssa_decode(q, cache, None, seqlens, Lcap, params)
         out = torch.empty_like(ref_o)
@@ -51,14 +54,16 @@ def test_noalloc_decode_matches_workspace_decode_twice():
 
 
 def test_noalloc_decode_rejects_batch_beyond_builtin_scratch():
-    """16 sequences with the 1 + 7 window need more than the 16 MiB built in:
-    rejected with LOZA_ERR_WORKSPACE before anything runs (no GPU needed)."""
+    """4 sequences of up to 4,096 tokens with the unbounded window need more than
+    the 16 MiB built in: rejected with LOZA_ERR_WORKSPACE before anything runs
+    (no GPU needed)."""
     import block_sparse_streaming_b200 as bss
     bss.build()
     L = bss.lib()
     vp = ctypes.c_void_p
     count = L.loza_launch_count()
-    rc = L.loza_ssa_decode_noalloc(vp(1 << 20), vp(1 << 21), vp(0), vp(1 << 22), 16, 4096, 4096 * 576, 576,
-                                   64, 1, 576, 512, bss.Params(0.07), vp(1 << 23), vp(1 << 24), vp(0))
+    rc = L.loza_ssa_decode_noalloc(vp(1 << 20), vp(1 << 21), vp(0), vp(1 << 22), 4, 4096, 4096 * 576, 576,
+                                   64, 1, 576, 512, bss.Params(0.07, 128, 0, bss.LOZA_UNBOUNDED), vp(1 << 23),
+                                   vp(1 << 24), vp(0))
     assert rc == -3
     assert L.loza_launch_count() == count
