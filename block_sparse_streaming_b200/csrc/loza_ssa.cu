@@ -13,6 +13,7 @@
 #include "loza_ssa.h"
 #include "prefill.cuh"
 #include "decode.cuh"
+#include "decode_mla.cuh"
 #include "backward.cuh"
 
 namespace loza {
@@ -61,24 +62,41 @@ bool window_ok(const loza_ssa_params& p) {
   return true;
 }
 
-// Split-KV plan of the absorbed decode: selected blocks per CTA and CTAs per
-// sequence. A sink + local window of at most 8 blocks runs one block per CTA,
-// 8 CTAs per sequence in one thread-block cluster that merges on chip (no
-// workspace). Larger windows and the unbounded (dense) window spread the
-// blocks over at most 32 CTAs per sequence and merge through the workspace.
+int sm_count() {
+  static const int n = [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      return v;
+    return 148;
+  }();
+  return n;
+}
+
+// Split-KV plan of the absorbed decode: CTAs per sequence (nsplit) and selected
+// blocks per CTA (bps), sized so that batch * nsplit CTAs fill the GPU in one
+// wave. Up to 8 splits form one thread-block cluster per sequence and merge
+// on chip (no workspace). Only when a few sequences have long windows (more
+// than 8 splits pay off) do the splits merge through the workspace.
 struct DecodePlan {
   int bps, nsplit;
   bool cluster;
 };
-constexpr int kDecClusterSplits = 8;
-DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen) {
+DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t batch) {
   const int max_blocks = (max_seqlen + kTile - 1) / kTile;
-  if (p.n_local != LOZA_UNBOUNDED && p.n_sink + p.n_local <= kDecClusterSplits)
-    return {1, kDecClusterSplits, true};
-  const int nb = p.n_local == LOZA_UNBOUNDED ? max_blocks
-                                             : (p.n_sink + p.n_local < max_blocks ? p.n_sink + p.n_local : max_blocks);
-  const int bps = (nb + 31) / 32;
-  return {bps, (nb + bps - 1) / bps, false};
+  const int count = p.n_local == LOZA_UNBOUNDED
+                        ? max_blocks
+                        : (p.n_sink + p.n_local < max_blocks ? p.n_sink + p.n_local : max_blocks);
+  const int sms = sm_count();
+  if (count > 8 && (int64_t)batch * 16 <= sms) {
+    int ns = (sms + batch - 1) / batch;
+    if (ns > count) ns = count;
+    const int bps = (count + ns - 1) / ns;
+    return {bps, (count + bps - 1) / bps, false};
+  }
+  int ns = 1;
+  while (ns < 8 && ns * 2 <= count && (int64_t)batch * ns * 2 <= sms) ns *= 2;
+  return {(count + ns - 1) / ns, ns, true};
 }
 
 struct DecodeWorkspace {
@@ -110,7 +128,7 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
   if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
   if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
   if (v_cache && v_cache != k_cache) return LOZA_ERR_UNSUPPORTED;
-  *plan = decode_plan(p, max_seqlen);
+  *plan = decode_plan(p, max_seqlen, batch);
   std::memset(prm, 0, sizeof(*prm));
   EncodeTiledFn fn = encode_fn();
   if (!fn) return LOZA_ERR_CUDA;
@@ -318,7 +336,7 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
   if (batch < 1 || max_seqlen < 1 || !window_ok(p)) return 0;
   if (op == LOZA_OP_DECODE) {
     if (n_kv_heads == 1 && n_heads == kDecHeads && d_qk == 576 && d_v == 512)
-      return decode_workspace(batch, decode_plan(p, max_seqlen)).total;
+      return decode_workspace(batch, decode_plan(p, max_seqlen, batch)).total;
     return 0;
   }
   if (op == LOZA_OP_BACKWARD) {
@@ -509,7 +527,7 @@ loza_status loza_ssa_decode_noalloc(const void* q, const void* k_cache, const vo
                            n_heads, n_kv_heads, d_qk, d_v, p, out, lse, nullptr, 0, stream);
   // batch too large for the built-in scratch: refuse before touching the driver
   if (batch >= 1 && max_seqlen >= 1 && window_ok(p) &&
-      decode_workspace(batch, decode_plan(p, max_seqlen)).total > kNoAllocScratchBytes)
+      decode_workspace(batch, decode_plan(p, max_seqlen, batch)).total > kNoAllocScratchBytes)
     return LOZA_ERR_WORKSPACE;
   DecodeParams prm;
   DecodePlan plan;

@@ -151,18 +151,19 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  * access to it, a serving runtime that has reserved all device memory for its
  * own KV-cache pool up front, or a latency-critical loop that must not pay
  * for cudaMalloc/cudaFree. For them this entry point takes the same arguments
- * as loza_ssa_decode minus the workspace. Where the absorbed decode needs
- * scratch for its split-KV partial results (windows of more than 8 blocks and
- * the unbounded window), they go to a fixed 16 MiB array that is part of the
- * library itself; the 1 + 7 window merges its partials on chip and needs none.
+ * as loza_ssa_decode minus the workspace. The absorbed decode needs scratch
+ * only when a few sequences have long windows (more than 8 selected blocks
+ * and batch * 16 <= number of SMs): its split-KV partial results then go to a
+ * fixed 16 MiB array that is part of the library itself. Every other call
+ * merges its partials on chip and needs none.
  *   - The library never allocates: every GPU that loads the library holds the
  *     16 MiB array until the process exits.
  *   - Limit: a call that needs scratch needs batch * nsplit * 131,584 bytes
- *     plus 256 for the counters, with nsplit = min(32, number of selected
- *     128-token blocks); e.g. at most 3 sequences of 4,096+ tokens with the
- *     unbounded window. A larger call returns LOZA_ERR_WORKSPACE before
- *     anything is launched; use loza_ssa_decode with a workspace instead, or
- *     split the batch.
+ *     plus 256 for the counters, with nsplit = min(selected blocks,
+ *     ceil(SMs / batch)); e.g. at most 3 sequences of 4,096+ tokens with the
+ *     unbounded window on a 148-SM B200. A larger call returns
+ *     LOZA_ERR_WORKSPACE before anything is launched; use loza_ssa_decode with
+ *     a workspace instead, or split the batch.
  *   - The first call on each device that needs scratch looks up the array's
  *     device address (with that device current); make that first call before
  *     any stream capture on that device.
