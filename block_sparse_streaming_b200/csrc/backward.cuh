@@ -162,62 +162,72 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_dq = idesc_bf16(128, 64, false, true);
-      const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
-      int slot = 0;
-      uint32_t phase = 0;
-      bool ok = mbar_wait(bar(LY::BAR_IN), 0, abort_flag);
-      tc_fence_after();
-      for (int b = 0; b < nb && ok; ++b) {
-        // S = Q K^T
-        for (int c = 0; c < LY::NQC && ok; ++c) {
-          ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
+    // whole warp walks the schedule; one elected lane issues each tcgen05 instruction
+    constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_dq = idesc_bf16(128, 64, false, true);
+    const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = warp_wait(bar(LY::BAR_IN), 0, abort_flag);
+    tc_fence_after();
+    for (int b = 0; b < nb && ok; ++b) {
+      // S = Q K^T
+      for (int c = 0; c < LY::NQC && ok; ++c) {
+        ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
           const uint32_t a = sbase + LY::Q_OFF + c * kChunkBytes, bb = sbase + LY::RING_OFF + slot * kChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(t_s, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
                    (c | kk) != 0);
           mma_commit(bar(LY::BAR_EMPTY + slot));
-          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
         }
-        // dP = dO V^T
-        for (int c = 0; c < LY::NVC && ok; ++c) {
-          ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
+        __syncwarp();
+        if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+      }
+      // dP = dO V^T
+      for (int c = 0; c < LY::NVC && ok; ++c) {
+        ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
           const uint32_t a = sbase + LY::DO_OFF + c * kChunkBytes, bb = sbase + LY::RING_OFF + slot * kChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(t_dp, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
                    (c | kk) != 0);
           mma_commit(bar(LY::BAR_EMPTY + slot));
-          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
         }
-        if (!ok) break;
-        mma_commit(bar(LY::BAR_DP));
-        ok = mbar_wait(bar(LY::BAR_DS), b & 1, abort_flag);
+        __syncwarp();
+        if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      if (elect_one()) mma_commit(bar(LY::BAR_DP));
+      __syncwarp();
+      ok = warp_wait(bar(LY::BAR_DS), b & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      // dQ += dS K  (A = dS in TMEM, B = K tiles MN-major)
+      for (int c = 0; c < LY::NQC && ok; ++c) {
+        ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        // dQ += dS K  (A = dS in TMEM, B = K tiles MN-major)
-        for (int c = 0; c < LY::NQC && ok; ++c) {
-          ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
+        if (elect_one()) {
           const uint32_t bb = sbase + LY::RING_OFF + slot * kChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(t_dq + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_dq,
                    (b > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(LY::BAR_EMPTY + slot));
-          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
         }
-        if (!ok) break;
-        mma_commit(bar(LY::BAR_DQ));
+        __syncwarp();
+        if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
       }
+      if (!ok) break;
+      if (elect_one()) mma_commit(bar(LY::BAR_DQ));
+      __syncwarp();
     }
   } else {
     const int quarter = warp & 3;
@@ -398,57 +408,65 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_ts = idesc_bf16(128, 64, false, true);
-      const uint32_t t_s = tmem, t_dp = tmem + 64, t_dv = tmem + LY::T_DV, t_dk = tmem + LY::T_DK;
-      bool ok = mbar_wait(bar(LY::BAR_KV), 0, abort_flag);
-      for (int jj = 0; jj < nj && ok; ++jj) {
-        ok = mbar_wait(bar(LY::BAR_QD), jj & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        // S^T = K Q^T
-        for (int c = 0; c < LY::NQC; ++c) {
-          const uint32_t a = sbase + LY::K_OFF + c * kChunkBytes, bb = sbase + LY::Q_OFF + c * kChunkBytes;
+    // whole warp walks the schedule; one elected lane issues each tcgen05 instruction
+    constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_ts = idesc_bf16(128, 64, false, true);
+    const uint32_t t_s = tmem, t_dp = tmem + 64, t_dv = tmem + LY::T_DV, t_dk = tmem + LY::T_DK;
+    bool ok = warp_wait(bar(LY::BAR_KV), 0, abort_flag);
+    for (int jj = 0; jj < nj && ok; ++jj) {
+      ok = warp_wait(bar(LY::BAR_QD), jj & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      // S^T = K Q^T
+      if (elect_one()) {
+      for (int c = 0; c < LY::NQC; ++c) {
+        const uint32_t a = sbase + LY::K_OFF + c * kChunkBytes, bb = sbase + LY::Q_OFF + c * kChunkBytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(t_s, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
-                   (c | kk) != 0);
-        }
-        mma_commit(bar(LY::BAR_S));
-        ok = mbar_wait(bar(LY::BAR_P), jj & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        // dV += P^T dO   (A = P^T in TMEM, B = dO tiles MN-major)
-        for (int c = 0; c < LY::NVC; ++c) {
-          const uint32_t bb = sbase + LY::DO_OFF + c * kChunkBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(t_dv + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_ts,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        // dP^T = V dO^T
-        for (int c = 0; c < LY::NVC; ++c) {
-          const uint32_t a = sbase + LY::V_OFF + c * kChunkBytes, bb = sbase + LY::DO_OFF + c * kChunkBytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(t_dp, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
-                   (c | kk) != 0);
-        }
-        mma_commit(bar(LY::BAR_DP));
-        ok = mbar_wait(bar(LY::BAR_DS), jj & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        // dK += dS^T Q   (A = dS^T in TMEM, B = Q tiles MN-major)
-        for (int c = 0; c < LY::NQC; ++c) {
-          const uint32_t bb = sbase + LY::Q_OFF + c * kChunkBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(t_dk + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_ts,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(LY::BAR_QD_EMPTY));
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(t_s, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
+                 (c | kk) != 0);
       }
+      mma_commit(bar(LY::BAR_S));
+      }
+      __syncwarp();
+      ok = warp_wait(bar(LY::BAR_P), jj & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      // dV += P^T dO   (A = P^T in TMEM, B = dO tiles MN-major)
+      if (elect_one()) {
+      for (int c = 0; c < LY::NVC; ++c) {
+        const uint32_t bb = sbase + LY::DO_OFF + c * kChunkBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(t_dv + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_ts,
+                 (jj > 0 || kk > 0) ? 1u : 0u);
+      }
+      // dP^T = V dO^T
+      for (int c = 0; c < LY::NVC; ++c) {
+        const uint32_t a = sbase + LY::V_OFF + c * kChunkBytes, bb = sbase + LY::DO_OFF + c * kChunkBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(t_dp, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
+                 (c | kk) != 0);
+      }
+      mma_commit(bar(LY::BAR_DP));
+      }
+      __syncwarp();
+      ok = warp_wait(bar(LY::BAR_DS), jj & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      // dK += dS^T Q   (A = dS^T in TMEM, B = Q tiles MN-major)
+      if (elect_one()) {
+      for (int c = 0; c < LY::NQC; ++c) {
+        const uint32_t bb = sbase + LY::Q_OFF + c * kChunkBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(t_dk + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_ts,
+                 (jj > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(bar(LY::BAR_QD_EMPTY));
+      }
+      __syncwarp();
     }
   } else {
     const int quarter = warp & 3;

@@ -25,9 +25,10 @@
 //
 // Merge of the splits of a sequence (log-sum-exp rule):
 //   CLUSTER  = true : the nsplit (<= 8) CTAs of a sequence form a thread-block
-//                     cluster; each stages its partial O in its own shared
-//                     memory and merges 512/nsplit output columns by reading
-//                     every partial over distributed shared memory.
+//                     cluster; after exchanging (m, l), each pushes its
+//                     weighted partial O from TMEM into the shared memory of
+//                     the CTA that owns those output columns (DSMEM stores),
+//                     and each CTA sums its 512/nsplit columns locally.
 //   CLUSTER  = false: partials go to the workspace and the last CTA of the
 //                     sequence (atomic ticket, no waiting) merges them; used
 //                     when a few long sequences need more than 8 splits.
@@ -201,103 +202,116 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
   if (nb > 0) {
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      if (lane == 0) {
+      // whole warp walks the schedule; one elected lane issues the TMA loads
+      if (elect_one()) {
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_kv);
         mbar_arrive_expect_tx(bar(LY::BAR_Q), 9 * kDecQTile);
         for (int c = 0; c < 9; ++c)
           tma_load_3d(sbase + LY::Q_OFF + c * kDecQTile, &p.tm_q, bar(LY::BAR_Q), c * 64, 0, seq);
-        int slot = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        auto load_unit = [&](int row, int u) {
-          ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
-          if (!ok) return;
+      }
+      __syncwarp();
+      int slot = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      auto load_unit = [&](int row, int u) {
+        ok = warp_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
+        if (!ok) return;
+        if (elect_one()) {
           const uint32_t dst = sbase + LY::RING_OFF + slot * kDecUnit;
           const int ntile = (u < 4) ? 2 : 1;
           mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), ntile * kChunkBytes);
           for (int t = 0; t < ntile; ++t)
             tma_load_3d(dst + t * kChunkBytes, &p.tm_kv, bar(LY::BAR_FULL + slot), 128 * u + 64 * t, row, seq);
-          if (++slot == kDecStages) { slot = 0; phase ^= 1; }
-        };
-        for (int it = 0; it <= nb && ok; ++it) {
-          if (it < nb) {
-            const int krow = walk.block(b_lo + it) * kTile;
-            for (int u = 0; u < kDecKUnits && ok; ++u) load_unit(krow, u);
-          }
-          if (it >= 1) {
-            const int vrow = walk.block(b_lo + it - 1) * kTile;
-            for (int u = 0; u < kDecVUnits && ok; ++u) load_unit(vrow, u);
-          }
+        }
+        __syncwarp();
+        if (++slot == kDecStages) { slot = 0; phase ^= 1; }
+      };
+      for (int it = 0; it <= nb && ok; ++it) {
+        if (it < nb) {
+          const int krow = walk.block(b_lo + it) * kTile;
+          for (int u = 0; u < kDecKUnits && ok; ++u) load_unit(krow, u);
+        }
+        if (it >= 1) {
+          const int vrow = walk.block(b_lo + it - 1) * kTile;
+          for (int u = 0; u < kDecVUnits && ok; ++u) load_unit(vrow, u);
         }
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
-      if (lane == 0) {
-        constexpr uint32_t idesc_s = idesc_bf16(128, kDecHeads, false, false);
-        constexpr uint32_t idesc_o = idesc_bf16(128, kDecHeads, true, false);
-        const uint32_t tmem_o = tmem + 128;  // O^T: 4 x 64 columns after the two S^T buffers
-        int slot = 0;
-        uint32_t phase = 0;
-        bool ok = mbar_wait(bar(LY::BAR_Q), 0, abort_flag);
-        for (int it = 0; it <= nb && ok; ++it) {
-          if (it < nb) {
-            // S^T(it) = K . Q^T over 9 column tiles
-            const uint32_t tmem_s = tmem + 64 * (it & 1);
-            for (int u = 0; u < kDecKUnits && ok; ++u) {
-              ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-              if (!ok) break;
-              tc_fence_after();
-              const uint32_t unit = sbase + LY::RING_OFF + slot * kDecUnit;
-              for (int t = 0; t < ((u < 4) ? 2 : 1); ++t) {
-                const int c = 2 * u + t;
-                const uint32_t ka = unit + t * kChunkBytes;
-                const uint32_t qb = sbase + LY::Q_OFF + c * kDecQTile;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_ss(tmem_s, sdesc_sw128(ka + 32 * kk, 16, 1024), sdesc_sw128(qb + 32 * kk, 16, 1024), idesc_s,
-                         (c | kk) != 0);
-              }
-              mma_commit(bar(LY::BAR_EMPTY + slot));
-              if (++slot == kDecStages) { slot = 0; phase ^= 1; }
-            }
-            if (!ok) break;
-            mma_commit(bar(LY::BAR_S + (it & 1)));
-          }
-          if (it >= 1) {
-            // O^T += V^T . P^T(b), V unit u = latent columns 128u .. 128u+127
-            const int b = it - 1;
-            if (walk.block(b_lo + b) == jq) {
-              // the query's own block may end inside the block: once its V units
-              // are resident, let the softmax warps zero the rows past the end
-              for (int u = 0; u < kDecVUnits && ok; ++u) {
-                const int su = slot + u;
-                ok = mbar_wait(bar(LY::BAR_FULL + su % kDecStages), phase ^ (su >= kDecStages ? 1u : 0u),
-                               abort_flag);
-              }
-              if (!ok) break;
-              mbar_arrive(bar(LY::BAR_VT));
-            }
-            ok = mbar_wait(bar(LY::BAR_P), b & 1, abort_flag);
+      // whole warp walks the schedule with warp-uniform descriptors; one
+      // elected lane issues each tcgen05 instruction
+      constexpr uint32_t idesc_s = idesc_bf16(128, kDecHeads, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(128, kDecHeads, true, false);
+      const uint32_t tmem_o = tmem + 128;  // O^T: 4 x 64 columns after the two S^T buffers
+      const uint64_t dk0 = sdesc_sw128(sbase + LY::RING_OFF, 16, 1024);           // K tiles, K-major
+      const uint64_t dq0 = sdesc_sw128(sbase + LY::Q_OFF, 16, 1024);              // Q tiles, K-major
+      const uint64_t dv0 = sdesc_sw128(sbase + LY::RING_OFF, kChunkBytes, 1024);  // V unit, MN-major
+      const uint64_t dp0 = sdesc_sw128(sbase + LY::P_OFF, 16, 1024);              // P^T tiles, K-major
+      int slot = 0;
+      uint32_t phase = 0;
+      bool ok = warp_wait(bar(LY::BAR_Q), 0, abort_flag);
+      for (int it = 0; it <= nb && ok; ++it) {
+        if (it < nb) {
+          // S^T(it) = K . Q^T over 9 column tiles
+          const uint32_t tmem_s = tmem + 64 * (it & 1);
+          for (int u = 0; u < kDecKUnits && ok; ++u) {
+            ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            for (int u = 0; u < kDecVUnits && ok; ++u) {
-              ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-              if (!ok) break;
-              tc_fence_after();
-              const uint32_t va = sbase + LY::RING_OFF + slot * kDecUnit;
+            if (elect_one()) {
+              for (int t = 0; t < ((u < 4) ? 2 : 1); ++t) {
+                const int c = 2 * u + t;
+                const uint64_t da = desc_add(dk0, slot * kDecUnit + t * kChunkBytes);
+                const uint64_t db = desc_add(dq0, c * kDecQTile);
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t pb = sbase + LY::P_OFF + (kk >> 2) * kDecQTile + (kk & 3) * 32;
-                mma_ss(tmem_o + 64 * u, sdesc_sw128(va + 2048 * kk, kChunkBytes, 1024), sdesc_sw128(pb, 16, 1024),
-                       idesc_o, (b > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_ss(tmem_s, desc_add(da, 32 * kk), desc_add(db, 32 * kk), idesc_s, (c | kk) != 0);
               }
               mma_commit(bar(LY::BAR_EMPTY + slot));
-              if (++slot == kDecStages) { slot = 0; phase ^= 1; }
+            }
+            __syncwarp();
+            if (++slot == kDecStages) { slot = 0; phase ^= 1; }
+          }
+          if (!ok) break;
+          if (elect_one()) mma_commit(bar(LY::BAR_S + (it & 1)));
+          __syncwarp();
+        }
+        if (it >= 1) {
+          // O^T += V^T . P^T(b), V unit u = latent columns 128u .. 128u+127
+          const int b = it - 1;
+          if (walk.block(b_lo + b) == jq) {
+            // the query's own block may end inside the block: once its V units
+            // are resident, let the softmax warps zero the rows past the end
+            for (int u = 0; u < kDecVUnits && ok; ++u) {
+              const int su = slot + u;
+              ok = warp_wait(bar(LY::BAR_FULL + su % kDecStages), phase ^ (su >= kDecStages ? 1u : 0u), abort_flag);
             }
             if (!ok) break;
-            mma_commit(bar(LY::BAR_PV));
+            if (elect_one()) mbar_arrive(bar(LY::BAR_VT));
+            __syncwarp();
           }
+          ok = warp_wait(bar(LY::BAR_P), b & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          for (int u = 0; u < kDecVUnits && ok; ++u) {
+            ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            if (elect_one()) {
+              const uint64_t da = desc_add(dv0, slot * kDecUnit);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem_o + 64 * u, desc_add(da, 2048 * kk), desc_add(dp0, (kk >> 2) * kDecQTile + (kk & 3) * 32),
+                       idesc_o, (b > 0 || kk > 0) ? 1u : 0u);
+              mma_commit(bar(LY::BAR_EMPTY + slot));
+            }
+            __syncwarp();
+            if (++slot == kDecStages) { slot = 0; phase ^= 1; }
+          }
+          if (!ok) break;
+          if (elect_one()) mma_commit(bar(LY::BAR_PV));
+          __syncwarp();
         }
       }
     } else {
@@ -399,19 +413,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       if (ok) {
         tc_fence_after();
         named_barrier_sync(1, 256);  // l_run complete
-        float* so = reinterpret_cast<float*>(smem + LY::RING_OFF);  // ring is idle now
+        if (!CLUSTER) {
 #pragma unroll 1
-        for (int u = 0; u < 4; ++u) {
-          const int dv = 128 * u + key;
-          float o[32];
-          tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
+          for (int u = 0; u < 4; ++u) {
+            const int dv = 128 * u + key;
+            float o[32];
+            tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int h = 32 * grp + i;
-            if (CLUSTER)
-              so[h * 512 + dv] = o[i];
-            else
-              p.ws_o[(part * kDecHeads + h) * 512 + dv] = o[i];
+            for (int i = 0; i < 32; ++i) p.ws_o[(part * kDecHeads + 32 * grp + i) * 512 + dv] = o[i];
           }
         }
         if (!CLUSTER && tid < 64) p.ws_ml[part * kDecHeads + tid] = make_float2(m_run[tid], l_run[tid]);
@@ -423,16 +432,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
 
   if (CLUSTER) {
     // ---------------------------------------------------------- on-chip merge
-    // Split r of the cluster merges output columns [r*W, (r+1)*W) of every head,
-    // W = 512 / nsplit, reading every split's staged partial over DSMEM. Splits
-    // without blocks have l = 0 and weight 0; their staging area is not read.
+    // 1. every CTA reads all splits' (m, l) over DSMEM and computes the same
+    //    merge weights; 2. each thread scales its O^T values (read from TMEM)
+    //    by its split's weight and pushes them, with plain DSMEM stores, into
+    //    the receive buffer of the CTA that owns those output columns
+    //    (split r owns columns [r*W, (r+1)*W), W = 512 / nsplit);
+    // 3. after one cluster barrier every CTA sums its buffer locally.
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();
+    cluster_sync_all();  // (m, l) of every split visible
     const int r = (int)cluster_rank();
     const int ns = p.nsplit;
+    const int W = 512 / ns;
     float* wgt = reinterpret_cast<float*>(smem + LY::Q_OFF);  // [8][64]; Q tiles are idle now
-    float* mls = wgt + 8 * 64;                                 // [2][8][64] peers' m, l
+    float* mls = wgt + 8 * 64;                                 // [2][8][64] all splits' m, l
+    float* recv = reinterpret_cast<float*>(smem + LY::RING_OFF);  // [ns][64][W]; the ring is idle now
     for (int idx = threadIdx.x; idx < ns * 64; idx += blockDim.x) {
       const int s2 = idx >> 6, h = idx & 63;
       mls[idx] = *static_cast<const float*>(__cluster_map_shared_rank(m_run + h, s2));
@@ -456,30 +470,42 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       if (r == 0) p.lse[(int64_t)seq * kDecHeads + h] = (M + log2f(Ls)) * 0.69314718055994530942f;
     }
     __syncthreads();
-    const int W4 = (512 / ns) / 4;  // float4 groups per head this split merges
-    const float* so = reinterpret_cast<const float*>(smem + LY::RING_OFF);
+    if (nb > 0 && warp >= 2) {
+      const int quarter = warp & 3, grp = (warp - 2) >> 2, key = quarter * 32 + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {
+        const int d = 128 * u + key;  // latent column of this lane
+        const int owner = d / W;
+        float* dst = static_cast<float*>(__cluster_map_shared_rank(recv, owner)) + (size_t)r * 64 * W + (d - owner * W);
+        float o[32];
+        tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int h = 32 * grp + i;
+          dst[(size_t)h * W] = o[i] * wgt[r * 64 + h];
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // every push landed; no CTA touches another's memory after this
+    const int W4 = W / 4;
     for (int idx = threadIdx.x; idx < kDecHeads * W4; idx += blockDim.x) {
       const int h = idx / W4;
-      const int d = r * (512 / ns) + (idx % W4) * 4;
-      float4 o[8];
-#pragma unroll
-      for (int s2 = 0; s2 < 8; ++s2)
-        o[s2] = (s2 < ns && wgt[s2 * 64 + h] != 0.f)
-                    ? *static_cast<const float4*>(__cluster_map_shared_rank(so + h * 512 + d, s2))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int j = (idx % W4) * 4;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int s2 = 0; s2 < 8; ++s2) {
-        const float w = s2 < ns ? wgt[s2 * 64 + h] : 0.f;
-        acc.x += o[s2].x * w;
-        acc.y += o[s2].y * w;
-        acc.z += o[s2].z * w;
-        acc.w += o[s2].w * w;
+      for (int s2 = 0; s2 < ns; ++s2) {
+        if (wgt[s2 * 64 + h] == 0.f) continue;  // a split without blocks pushed nothing
+        const float4 o = *reinterpret_cast<const float4*>(recv + ((size_t)s2 * 64 + h) * W + j);
+        acc.x += o.x;
+        acc.y += o.y;
+        acc.z += o.z;
+        acc.w += o.w;
       }
-      __nv_bfloat16* dst = p.out + ((int64_t)seq * kDecHeads + h) * 512 + d;
+      __nv_bfloat16* dst = p.out + ((int64_t)seq * kDecHeads + h) * 512 + r * W + j;
       *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
     }
-    cluster_sync_all();  // peers may read this CTA's shared memory until here
   } else {
     // ---------------------------------------------------------- last CTA merges
     __threadfence();

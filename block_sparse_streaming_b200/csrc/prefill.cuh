@@ -137,7 +137,8 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // whole warp walks the schedule; one elected lane issues the TMA loads
+    if (elect_one()) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
@@ -145,84 +146,90 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       mbar_arrive_expect_tx(bar(LY::BAR_Q), LY::NQC * kChunkBytes);
       for (int c = 0; c < LY::NQC; ++c)
         tma_load_3d(sbase + LY::Q_OFF + c * kChunkBytes, &p.tm_q, bar(LY::BAR_Q), c * 64, head, row0);
-      int slot = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int it = 0; it <= nb && ok; ++it) {
-        if (it < nb) {
-          const int krow = seq_start + walk.block(it) * kTile;
-          for (int c = 0; c < LY::NQC && ok; ++c) {
-            ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
-            if (!ok) break;
-            mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
-            tma_load_3d(sbase + LY::RING_OFF + slot * kChunkBytes, &p.tm_k, bar(LY::BAR_FULL + slot),
-                        c * 64, hk, krow);
-            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
-          }
-        }
-        if (it >= 1) {
-          const int vrow = seq_start + walk.block(it - 1) * kTile;
-          for (int c = 0; c < LY::NVC && ok; ++c) {
-            ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
-            if (!ok) break;
-            mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
-            tma_load_3d(sbase + LY::RING_OFF + slot * kChunkBytes, &p.tm_v, bar(LY::BAR_FULL + slot),
-                        slice * DVT + c * 64, hk, vrow);
-            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
-          }
-        }
+    }
+    __syncwarp();
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    auto load_tile = [&](const CUtensorMap* map, int col, int row) {
+      ok = warp_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
+      if (!ok) return;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
+        tma_load_3d(sbase + LY::RING_OFF + slot * kChunkBytes, map, bar(LY::BAR_FULL + slot), col, hk, row);
+      }
+      __syncwarp();
+      if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
+    };
+    for (int it = 0; it <= nb && ok; ++it) {
+      if (it < nb) {
+        const int krow = seq_start + walk.block(it) * kTile;
+        for (int c = 0; c < LY::NQC && ok; ++c) load_tile(&p.tm_k, c * 64, krow);
+      }
+      if (it >= 1) {
+        const int vrow = seq_start + walk.block(it - 1) * kTile;
+        for (int c = 0; c < LY::NVC && ok; ++c) load_tile(&p.tm_v, slice * DVT + c * 64, vrow);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, 64, false, true);
-      const uint32_t tmem_o = tmem + 256;
-      int slot = 0;
-      uint32_t phase = 0;
-      bool ok = mbar_wait(bar(LY::BAR_Q), 0, abort_flag);
-      tc_fence_after();
-      for (int it = 0; it <= nb && ok; ++it) {
-        if (it < nb) {
-          const uint32_t tmem_s = tmem + (it & 1) * 128;
-          for (int c = 0; c < LY::NQC; ++c) {
-            ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t qa = sbase + LY::Q_OFF + c * kChunkBytes;
-            const uint32_t kbuf = sbase + LY::RING_OFF + slot * kChunkBytes;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ss(tmem_s, sdesc_sw128(qa + 32 * kk, 16, 1024), sdesc_sw128(kbuf + 32 * kk, 16, 1024),
-                     idesc_s, (c | kk) != 0);
-            mma_commit(bar(LY::BAR_EMPTY + slot));
-            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
-          }
-          if (!ok) break;
-          mma_commit(bar(LY::BAR_S + (it & 1)));
-        }
-        if (it >= 1) {
-          const int b = it - 1;
-          ok = mbar_wait(bar(LY::BAR_P), b & 1, abort_flag);
+    // The whole warp walks the schedule (warp-uniform descriptors); one
+    // elected lane issues each tcgen05 instruction.
+    constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_pv = idesc_bf16(128, 64, false, true);
+    const uint32_t tmem_o = tmem + 256;
+    const uint64_t dq0 = sdesc_sw128(sbase + LY::Q_OFF, 16, 1024);       // Q tile 0 (K-major)
+    const uint64_t dk0 = sdesc_sw128(sbase + LY::RING_OFF, 16, 1024);    // ring slot 0 read K-major
+    const uint64_t dv0 = sdesc_sw128(sbase + LY::RING_OFF, 8192, 1024);  // ring slot 0 read MN-major
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = warp_wait(bar(LY::BAR_Q), 0, abort_flag);
+    tc_fence_after();
+    for (int it = 0; it <= nb && ok; ++it) {
+      if (it < nb) {
+        const uint32_t tmem_s = tmem + (it & 1) * 128;
+        for (int c = 0; c < LY::NQC; ++c) {
+          ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t tmem_p = tmem + (b & 1) * 128;
-          for (int c = 0; c < LY::NVC; ++c) {
-            ok = mbar_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t vbuf = sbase + LY::RING_OFF + slot * kChunkBytes;
+          if (elect_one()) {
+            const uint64_t da = desc_add(dq0, c * kChunkBytes);
+            const uint64_t db = desc_add(dk0, slot * kChunkBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem_s, desc_add(da, 32 * kk), desc_add(db, 32 * kk), idesc_s, (c | kk) != 0);
+            mma_commit(bar(LY::BAR_EMPTY + slot));
+          }
+          __syncwarp();
+          if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (elect_one()) mma_commit(bar(LY::BAR_S + (it & 1)));
+        __syncwarp();
+      }
+      if (it >= 1) {
+        const int b = it - 1;
+        ok = warp_wait(bar(LY::BAR_P), b & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tmem_p = tmem + (b & 1) * 128;
+        for (int c = 0; c < LY::NVC; ++c) {
+          ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          if (elect_one()) {
+            const uint64_t dv = desc_add(dv0, slot * kChunkBytes);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem_o + c * 64, tmem_p + kk * 8, sdesc_sw128(vbuf + 2048 * kk, 8192, 1024), idesc_pv,
-                     (b > 0 || kk > 0) ? 1u : 0u);
+              mma_ts(tmem_o + c * 64, tmem_p + kk * 8, desc_add(dv, 2048 * kk), idesc_pv, (b > 0 || kk > 0) ? 1u : 0u);
             mma_commit(bar(LY::BAR_EMPTY + slot));
-            if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
           }
-          if (!ok) break;
-          mma_commit(bar(LY::BAR_PV));
+          __syncwarp();
+          if (++slot == NSTAGE) { slot = 0; phase ^= 1; }
         }
+        if (!ok) break;
+        if (elect_one()) mma_commit(bar(LY::BAR_PV));
+        __syncwarp();
       }
     }
   } else {

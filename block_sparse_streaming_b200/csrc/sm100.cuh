@@ -33,6 +33,20 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
+// One lane of a converged warp (elect.sync). Issue loops run on the whole warp
+// so that loop state and descriptors stay warp-uniform, and only the elected
+// lane issues the tcgen05 / TMA instruction.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{ .reg .pred p; .reg .b32 r; elect.sync r|p, 0xffffffff; selp.u32 %0, 1, 0, p; }" : "=r"(pred));
+  return pred != 0;
+}
+
+// Advance a shared-memory matrix descriptor by `bytes` (a multiple of 16)
+// within the same 256 KB window: only the start-address field changes.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
@@ -78,6 +92,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
+}
+
+// mbar_wait executed by a whole warp, with a warp-uniform result (if any lane
+// gave up, every lane reports failure), so issue loops stay converged.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA,
