@@ -349,12 +349,15 @@ def long_secondary(bss, device, stream, peaks):
     return res
 
 
-def train_secondary(bss, device, stream, peaks):
-    """Workload 5: varlen forward + backward, per-head 192/128 dims, 64 heads."""
+def train_secondary(bss, device, stream, peaks, train_len=None):
+    """Workload 5: varlen forward + backward, per-head 192/128 dims, 64 heads
+    (train_len: one sequence of that many tokens instead, for profiling)."""
     import torch
     w = synth.WORKLOADS[5]
     g = synth.rng(synth.workload_seed(5))
     lens = synth.loguniform_lengths(g, w["batch"], w["len_lo"], w["len_hi"], w["total_cap"])
+    if train_len:
+        lens = np.array([train_len], dtype=np.int64)
     T = int(lens.sum())
     Hh, dqk, dv = w["n_heads"], w["d_qk"], w["d_v"]
     base = synth.workload_seed(5) * 1000
@@ -389,7 +392,8 @@ def train_secondary(bss, device, stream, peaks):
     if bss.device_status() != 0:
         raise RuntimeError("device status reports a timed-out wait in training")
     pk = float(peaks["bf16_tflops"])
-    res = {"workload": w["name"], "lengths": lens.tolist(), "total_tokens": T,
+    res = {"workload": w["name"] if not train_len else f"training fwd+bwd, one sequence of {train_len} tokens",
+           "lengths": lens.tolist(), "total_tokens": T,
            "forward": {"ms": mf, "TFLOP/s": f_fwd / (mf / 1000) / 1e12, "frac_of_peak": f_fwd / (mf / 1000) / 1e12 / pk,
                        "algorithmic_tflop": f_fwd / 1e12},
            "backward": {"ms": mb, "TFLOP/s": f_bwd / (mb / 1000) / 1e12, "frac_of_peak": f_bwd / (mb / 1000) / 1e12 / pk,
@@ -477,7 +481,7 @@ def run_ours(args, rank, world, local_rank):
     if args.workload in ("long", "all"):
         secondary["long"] = long_secondary(bss, device, stream, peaks)
     if args.workload in ("train", "all"):
-        secondary["train"] = train_secondary(bss, device, stream, peaks)
+        secondary["train"] = train_secondary(bss, device, stream, peaks, args.train_len)
 
     line = None
     if rank == 0:
@@ -557,6 +561,8 @@ def main():
                     help="prefill length (default: the 32,768-token workload; smaller values serve profiling)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="use only the first N sequences of the decode workload (profiling)")
+    ap.add_argument("--train-len", type=int, default=None,
+                    help="training workload as one sequence of this length (profiling)")
     ap.add_argument("--workload", choices=["default", "prefill", "long", "train", "all"], default="default",
                     help="default: prefill line plus the 64-sequence decode; long/train/all add workloads 4/5")
     args = ap.parse_args()
