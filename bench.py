@@ -213,6 +213,24 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- multi-rank helpers
+
+def max_over_ranks(x: float, device) -> float:
+    """Maximum of a per-rank number over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, steps: int, work_per_step: float, max_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks' replicas over the slowest rank's time."""
+    return world * steps * work_per_step / (max_ms / 1000.0)
+
+
 # --------------------------------------------------------------------------- GPU leg
 
 def make_inputs(device, seq_len, seed_offset=0):
@@ -456,12 +474,9 @@ def run_ours(args, rank, world, local_rank):
     del q, lat, out, lse
     torch.cuda.empty_cache()
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, device)
     flops = prefill_flops(L)
-    value = world * args.steps * flops / (total_ms / 1000.0) / 1e12
+    value = job_value(world, args.steps, flops, total_ms) / 1e12
 
     e2e = None if args.no_e2e else run_e2e(bss, params, device, stream, L, steps=max(1, min(args.steps, 3)))
 

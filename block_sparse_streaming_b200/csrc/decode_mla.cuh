@@ -53,7 +53,7 @@ struct DecodeParams {
   CUtensorMap tm_kv;   // cache [B, rows, 576] box {64, 128, 1}
   const int32_t* seqlens;
   float* ws_o;         // workspace mode: [B, nsplit, H, 512] partial O (unnormalised)
-  float2* ws_ml;       // workspace mode: [B, nsplit, H] partial (m in log2 units, l)
+  float4* ws_ml;       // workspace mode: [B, nsplit, H] partial (m in log2 units, l exact, l of bf16 P, -)
   int* ws_ticket;      // workspace mode: [B] arrival counters (zero on entry)
   __nv_bfloat16* out;  // [B, H, 512]
   float* lse;          // [B, H]
@@ -68,9 +68,9 @@ struct DecodeLayout {
   static constexpr int Q_OFF = 0;                                   // 9 Q tiles, 72 KB
   static constexpr int RING_OFF = 9 * kDecQTile;                    // 73728 (1024-aligned)
   static constexpr int P_OFF = RING_OFF + kDecStages * kDecUnit;    // P^T: 2 tiles [64 heads x 64 keys]
-  static constexpr int RED_OFF = P_OFF + 2 * kDecQTile;             // redmax[4][64], redsum[4][64]
-  static constexpr int STAT_OFF = RED_OFF + 2 * 4 * 64 * 4;         // m_run[64], l_run[64], alpha[64]
-  static constexpr int BAR_OFF = STAT_OFF + 3 * 64 * 4;
+  static constexpr int RED_OFF = P_OFF + 2 * kDecQTile;             // redmax, redsum, redrsum [4][64] each
+  static constexpr int STAT_OFF = RED_OFF + 3 * 4 * 64 * 4;         // m_run, l_run, alpha, r_run [64] each
+  static constexpr int BAR_OFF = STAT_OFF + 4 * 64 * 4;
   // barriers: q_full, full[4], empty[4], s_full[2], p_ready, pv_done, vtail (the block holding
   // the query's own, possibly partial, block has all its V units resident)
   static constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = 1 + kDecStages, BAR_S = 1 + 2 * kDecStages,
@@ -166,9 +166,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::MISC_OFF + 4);
   int* last_flag = reinterpret_cast<int*>(smem + LY::MISC_OFF + 8);
   float* redmax = reinterpret_cast<float*>(smem + LY::RED_OFF);  // [4 quarters][64]
-  float* redsum = redmax + 4 * 64;
+  float* redsum = redmax + 4 * 64;   // sums of exact P (for the LSE)
+  float* redrsum = redsum + 4 * 64;  // sums of bf16-rounded P (for normalising O)
   float* m_run = reinterpret_cast<float*>(smem + LY::STAT_OFF);
   float* l_run = m_run + 64;
+  float* r_run = m_run + 192;
   float* alpha = m_run + 128;
   const int64_t part = (int64_t)seq * p.nsplit + split;
 
@@ -189,6 +191,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
   if (threadIdx.x < 64) {
     m_run[threadIdx.x] = -INFINITY;
     l_run[threadIdx.x] = 0.f;
+    r_run[threadIdx.x] = 0.f;
   }
   if (warp == 1 && nb > 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -356,6 +359,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
         }
         named_barrier_sync(1, 256);
         // P^T = 2^(cs*s - m) as the K-major B operand [64 heads x 128 keys]
+        float xr[32];
         {
           uint8_t* pbase = smem + LY::P_OFF + (key >> 6) * kDecQTile;
           const uint32_t col = key & 63;
@@ -363,10 +367,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
           for (int i = 0; i < 32; ++i) {
             const int h = 32 * grp + i;
             x[i] = ex2_approx(fmaf(x[i], cs, -m_run[h]));
-            *reinterpret_cast<__nv_bfloat16*>(pbase + sw128_offset(h, col)) = __float2bfloat16_rn(x[i]);
+            const __nv_bfloat16 pb16 = __float2bfloat16_rn(x[i]);
+            *reinterpret_cast<__nv_bfloat16*>(pbase + sw128_offset(h, col)) = pb16;
+            xr[i] = __bfloat162float(pb16);
           }
         }
         redsum[quarter * 64 + grp * 32 + lane] = warp_reduce_scatter32<false>(x);
+        redrsum[quarter * 64 + grp * 32 + lane] = warp_reduce_scatter32<false>(xr);
         // O^T rescale where a head's running maximum moved (lane = latent column)
         bool any_rescale = false;
 #pragma unroll 1
@@ -384,8 +391,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
           tmem_st_wait();
         }
         named_barrier_sync(1, 256);
-        if (tid < 64)
+        if (tid < 64) {
           l_run[tid] = l_run[tid] * alpha[tid] + ((redsum[tid] + redsum[64 + tid]) + (redsum[128 + tid] + redsum[192 + tid]));
+          r_run[tid] = r_run[tid] * alpha[tid] + ((redrsum[tid] + redrsum[64 + tid]) + (redrsum[128 + tid] + redrsum[192 + tid]));
+        }
         if (kb == jq) {
           // rows past the sequence end: zero them in the V units (the cache may
           // hold anything there) so that 0 * garbage cannot reach O
@@ -423,11 +432,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
             for (int i = 0; i < 32; ++i) p.ws_o[(part * kDecHeads + 32 * grp + i) * 512 + dv] = o[i];
           }
         }
-        if (!CLUSTER && tid < 64) p.ws_ml[part * kDecHeads + tid] = make_float2(m_run[tid], l_run[tid]);
+        if (!CLUSTER && tid < 64) p.ws_ml[part * kDecHeads + tid] = make_float4(m_run[tid], l_run[tid], r_run[tid], 0.f);
       }
     }
   } else if (!CLUSTER && threadIdx.x < 64) {
-    p.ws_ml[part * kDecHeads + threadIdx.x] = make_float2(-INFINITY, 0.f);  // a split without blocks
+    p.ws_ml[part * kDecHeads + threadIdx.x] = make_float4(-INFINITY, 0.f, 0.f, 0.f);  // a split without blocks
   }
 
   if (CLUSTER) {
@@ -445,12 +454,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
     const int ns = p.nsplit;
     const int W = 512 / ns;
     float* wgt = reinterpret_cast<float*>(smem + LY::Q_OFF);  // [8][64]; Q tiles are idle now
-    float* mls = wgt + 8 * 64;                                 // [2][8][64] all splits' m, l
+    float* mls = wgt + 8 * 64;                                 // [3][8][64] all splits' m, l, r
     float* recv = reinterpret_cast<float*>(smem + LY::RING_OFF);  // [ns][64][W]; the ring is idle now
     for (int idx = threadIdx.x; idx < ns * 64; idx += blockDim.x) {
       const int s2 = idx >> 6, h = idx & 63;
       mls[idx] = *static_cast<const float*>(__cluster_map_shared_rank(m_run + h, s2));
       mls[8 * 64 + idx] = *static_cast<const float*>(__cluster_map_shared_rank(l_run + h, s2));
+      mls[16 * 64 + idx] = *static_cast<const float*>(__cluster_map_shared_rank(r_run + h, s2));
     }
     __syncthreads();
     if (threadIdx.x < 64) {
@@ -458,14 +468,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       float M = -INFINITY;
       for (int s2 = 0; s2 < ns; ++s2)
         if (mls[8 * 64 + s2 * 64 + h] > 0.f) M = fmaxf(M, mls[s2 * 64 + h]);
-      float Ls = 0.f;
+      // O is normalised by the merged sum of the bf16 P that multiplied V,
+      // the LSE by the merged exact sum
+      float Ls = 0.f, Rs = 0.f;
       for (int s2 = 0; s2 < ns; ++s2) {
         const float l = mls[8 * 64 + s2 * 64 + h];
         const float w = l > 0.f ? ex2_approx(mls[s2 * 64 + h] - M) : 0.f;
         wgt[s2 * 64 + h] = w;
         Ls += l * w;
+        Rs += mls[16 * 64 + s2 * 64 + h] * w;
       }
-      const float inv = 1.f / Ls;
+      const float inv = 1.f / Rs;
       for (int s2 = 0; s2 < ns; ++s2) wgt[s2 * 64 + h] *= inv;
       if (r == 0) p.lse[(int64_t)seq * kDecHeads + h] = (M + log2f(Ls)) * 0.69314718055994530942f;
     }
@@ -520,17 +533,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
         const int h = threadIdx.x;
         float M = -INFINITY;
         for (int s2 = 0; s2 < p.nsplit; ++s2) {
-          const float2 ml = p.ws_ml[((int64_t)seq * p.nsplit + s2) * kDecHeads + h];
+          const float4 ml = p.ws_ml[((int64_t)seq * p.nsplit + s2) * kDecHeads + h];
           if (ml.y > 0.f) M = fmaxf(M, ml.x);
         }
-        float Ls = 0.f;
+        float Ls = 0.f, Rs = 0.f;
         for (int s2 = 0; s2 < p.nsplit; ++s2) {
-          const float2 ml = p.ws_ml[((int64_t)seq * p.nsplit + s2) * kDecHeads + h];
+          const float4 ml = p.ws_ml[((int64_t)seq * p.nsplit + s2) * kDecHeads + h];
           const float w = ml.y > 0.f ? ex2_approx(ml.x - M) : 0.f;
           wgt[s2 * 64 + h] = w;
           Ls += ml.y * w;
+          Rs += ml.z * w;
         }
-        const float inv = 1.f / Ls;
+        const float inv = 1.f / Rs;
         for (int s2 = 0; s2 < p.nsplit; ++s2) wgt[s2 * 64 + h] *= inv;
         p.lse[(int64_t)seq * kDecHeads + h] = (M + log2f(Ls)) * 0.69314718055994530942f;
       }

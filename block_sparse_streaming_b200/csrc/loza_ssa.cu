@@ -108,7 +108,7 @@ DecodeWorkspace decode_workspace(int32_t batch, const DecodePlan& plan) {
   const size_t parts = (size_t)batch * plan.nsplit * kDecHeads;
   w.o_off = 0;
   w.ml_off = parts * 512 * sizeof(float);
-  w.ticket_off = w.ml_off + parts * sizeof(float2);
+  w.ticket_off = w.ml_off + parts * sizeof(float4);
   w.total = w.ticket_off + ((size_t)batch * sizeof(int) + 255) / 256 * 256;
   return w;
 }
@@ -169,7 +169,7 @@ loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t
   if (!plan.cluster) {
     const DecodeWorkspace wl = decode_workspace(batch, plan);
     prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
-    prm.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
+    prm.ws_ml = reinterpret_cast<float4*>(ws + wl.ml_off);
     prm.ws_ticket = reinterpret_cast<int*>(ws + wl.ticket_off);
     // the arrival counters must start at zero; the partials are fully rewritten
     if (cudaMemsetAsync(prm.ws_ticket, 0, (size_t)batch * sizeof(int), st) != cudaSuccess) return LOZA_ERR_CUDA;

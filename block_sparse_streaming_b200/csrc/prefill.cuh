@@ -239,8 +239,10 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int qpos = qb * kTile + row;                  // position inside the sequence
     // m_run: running row maximum of scale*log2(e)*s (the reference of P);
-    // l_run: running sum of 2^(x - m_run).
-    float m_run = -INFINITY, l_run = 0.f;
+    // l_run: running sum of 2^(x - m_run) (exact, for the LSE);
+    // r_run: running sum of the bf16-rounded P values that enter P.V, so that
+    //        O is normalised by exactly the weights it was accumulated with.
+    float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float c = p.scale_log2;  // > 0, so max(c*s) = c*max(s)
     bool ok = true;
     for (int b = 0; b < nb && ok; ++b) {
@@ -295,9 +297,9 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
         tmem_st_wait();
       }
       const float neg_m = -m_run;
-      float sum8[8];
+      float sum8[8], rs8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
+      for (int i = 0; i < 8; ++i) sum8[i] = rs8[i] = 0.f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
@@ -308,11 +310,15 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
           sum8[(2 * i) & 7] += p0;
           sum8[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16(p0, p1);
+          rs8[(2 * i) & 7] += __uint_as_float(pk[i] << 16);
+          rs8[(2 * i + 1) & 7] += __uint_as_float(pk[i] & 0xFFFF0000u);
         }
         tmem_st32(lane_addr + (b & 1) * 128 + 32 * h, pk);
       }
       const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      const float rsum = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l_run = l_run * alpha + sum;
+      r_run = r_run * alpha + rsum;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(LY::BAR_P));
@@ -320,7 +326,7 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     if (ok) ok = mbar_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l_run;
+      const float inv = 1.f / r_run;
       const bool valid = qpos < seq_len;
       const int64_t grow = (int64_t)seq_start + qpos;
       __nv_bfloat16* orow = p.out + (grow * p.n_heads + head) * (int64_t)p.d_v + slice * DVT;

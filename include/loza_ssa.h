@@ -158,10 +158,11 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  * merges its partials on chip and needs none.
  *   - The library never allocates: every GPU that loads the library holds the
  *     16 MiB array until the process exits.
- *   - Limit: a call that needs scratch needs batch * nsplit * 131,584 bytes
+ *   - Limit: a call that needs scratch needs batch * nsplit * 132,096 bytes
  *     plus 256 for the counters, with nsplit = min(selected blocks,
- *     ceil(SMs / batch)); e.g. at most 3 sequences of 4,096+ tokens with the
- *     unbounded window on a 148-SM B200. A larger call returns
+ *     ceil(SMs / batch)), so it fits when batch * nsplit <= 127; e.g. with
+ *     the unbounded window on a 148-SM B200, one sequence of up to 16,256
+ *     tokens or four of up to 3,968 tokens. A larger call returns
  *     LOZA_ERR_WORKSPACE before anything is launched; use loza_ssa_decode with
  *     a workspace instead, or split the batch.
  *   - The first call on each device that needs scratch looks up the array's
