@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
       mbar_init(bar(LY::BAR_EMPTY + i), 1);
     }
     mbar_init(bar(LY::BAR_DP), 1);
-    mbar_init(bar(LY::BAR_DS), 128);
+    mbar_init(bar(LY::BAR_DS), 4);  // one arrival per softmax warp
     mbar_init(bar(LY::BAR_DQ), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
     const float dd = valid ? p.dvec[grow * p.n_heads + head] : 0.f;
     bool ok = true;
     for (int b = 0; b < nb && ok; ++b) {
-      ok = mbar_wait(bar(LY::BAR_DP), b & 1, abort_flag);
+      ok = warp_wait(bar(LY::BAR_DP), b & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const bool diag = walk.block(b) == qb;
@@ -266,9 +266,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(LY::BAR_DS));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(LY::BAR_DS));  // one arrival per warp
     }
-    if (ok) ok = mbar_wait(bar(LY::BAR_DQ), (nb - 1) & 1, abort_flag);
+    if (ok) ok = warp_wait(bar(LY::BAR_DQ), (nb - 1) & 1, abort_flag);
     if (ok) {
       tc_fence_after();
       __nv_bfloat16* dst = p.dq + (grow * p.n_heads + head) * (int64_t)DQK;
@@ -372,9 +373,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
     mbar_init(bar(LY::BAR_QD), 1);
     mbar_init(bar(LY::BAR_QD_EMPTY), 1);
     mbar_init(bar(LY::BAR_S), 1);
-    mbar_init(bar(LY::BAR_P), 128);
+    mbar_init(bar(LY::BAR_P), 4);  // one arrival per softmax warp
     mbar_init(bar(LY::BAR_DP), 1);
-    mbar_init(bar(LY::BAR_DS), 128);
+    mbar_init(bar(LY::BAR_DS), 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -485,7 +486,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
         s_d[tid] = v ? p.dvec[g * p.n_heads + head] : 0.f;
       }
       named_barrier_sync(1, 128);
-      ok = mbar_wait(bar(LY::BAR_S), jj & 1, abort_flag);
+      ok = warp_wait(bar(LY::BAR_S), jj & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const bool diag = (j == kblk);
@@ -511,8 +512,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(LY::BAR_P));
-      ok = mbar_wait(bar(LY::BAR_DP), jj & 1, abort_flag);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(LY::BAR_P));  // one arrival per warp
+      ok = warp_wait(bar(LY::BAR_DP), jj & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -531,10 +533,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(LY::BAR_DS));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(LY::BAR_DS));  // one arrival per warp
       named_barrier_sync(1, 128);  // statistics of block j no longer read
     }
-    if (ok) ok = mbar_wait(bar(LY::BAR_QD_EMPTY), (nj - 1) & 1, abort_flag);
+    if (ok) ok = warp_wait(bar(LY::BAR_QD_EMPTY), (nj - 1) & 1, abort_flag);
     if (ok) {
       tc_fence_after();
       const int kpos = kblk * kTile + key;

@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
     }
     mbar_init(bar(LY::BAR_S + 0), 1);
     mbar_init(bar(LY::BAR_S + 1), 1);
-    mbar_init(bar(LY::BAR_P), 256);
+    mbar_init(bar(LY::BAR_P), 8);  // one arrival per softmax warp
     mbar_init(bar(LY::BAR_PV), 1);
     mbar_init(bar(LY::BAR_VT), 1);
     *abort_flag = 0;
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       const float cs = p.scale_log2;
       bool ok = true;
       for (int b = 0; b < nb && ok; ++b) {
-        ok = mbar_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
+        ok = warp_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         float x[32];
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
         named_barrier_sync(1, 256);
         if (b > 0) {
           // PV(b-1) done: P^T buffer free and O^T stable (phases waited in order)
-          ok = mbar_wait(bar(LY::BAR_PV), (b - 1) & 1, abort_flag);
+          ok = warp_wait(bar(LY::BAR_PV), (b - 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
         }
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
         if (kb == jq) {
           // rows past the sequence end: zero them in the V units (the cache may
           // hold anything there) so that 0 * garbage cannot reach O
-          ok = mbar_wait(bar(LY::BAR_VT), 0, abort_flag);
+          ok = warp_wait(bar(LY::BAR_VT), 0, abort_flag);
           if (!ok) break;
           if (!valid) {
             const uint4 z = make_uint4(0, 0, 0, 0);
@@ -413,12 +413,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
             }
           }
         }
+        // one arrival per warp, after every lane's shared-memory writes are
+        // made visible to the tensor core
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(LY::BAR_P));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(LY::BAR_P));
       }
       // ---------------------------------------------------------- partial epilogue
-      if (ok) ok = mbar_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
+      if (ok) ok = warp_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
       if (ok) {
         tc_fence_after();
         named_barrier_sync(1, 256);  // l_run complete

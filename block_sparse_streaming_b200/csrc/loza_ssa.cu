@@ -12,6 +12,7 @@
 
 #include "loza_ssa.h"
 #include "prefill.cuh"
+#include "prefill_pair.cuh"
 #include "decode.cuh"
 #include "decode_mla.cuh"
 #include "backward.cuh"
@@ -39,14 +40,14 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D bf16 map over [rows, heads, dim] with 128-byte swizzle and a
-// {64, 1, 128} box: one [128 rows x 64 columns] tile of one head per load.
+// {64, 1, box_rows} box: one [box_rows x 64 columns] tile of one head per load.
 bool make_map_3d(CUtensorMap* m, const void* base, int64_t dim, int64_t heads, int64_t rows,
-                 int64_t head_stride_elems, int64_t row_stride_elems) {
+                 int64_t head_stride_elems, int64_t row_stride_elems, uint32_t box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)(head_stride_elems * 2), (cuuint64_t)(row_stride_elems * 2)};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -264,6 +265,31 @@ loza_status launch_prefill(const PrefillParams& prm, int max_seqlen, int batch, 
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
+// Absorbed-MLA prefill on CTA pairs: grid x = (head pair, value slice, CTA of
+// the pair), y = query tile, z = sequence; clusters of 2 along x.
+loza_status launch_prefill_pair(const PrefillPairParams& prm, int max_seqlen, int batch, cudaStream_t stream) {
+  using LY = PrefillPairLayout;
+  if (cudaFuncSetAttribute(ssa_prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM_BYTES) !=
+      cudaSuccess)
+    return LOZA_ERR_CUDA;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * prm.n_heads, (max_seqlen + kTile - 1) / kTile, batch);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = LY::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, ssa_prefill_pair_kernel, prm) != cudaSuccess) return LOZA_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Built-in scratch for loza_ssa_decode_noalloc.
 //
@@ -390,12 +416,29 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
   if ((int64_t)n_heads * prm.dv_slices > 65535) return LOZA_ERR_UNSUPPORTED;
 
   const int64_t v_head_stride = latent_v ? d_qk : d_v;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0 && (max_seqlen + kTile - 1) / kTile <= 65535) {
+    // absorbed MLA: two heads share every key block, so pairs of CTAs split the B operands
+    PrefillPairParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.cu_seqlens = cu_seqlens;
+    pp.out = prm.out;
+    pp.lse = lse;
+    pp.n_heads = n_heads;
+    pp.n_sink = prm.n_sink;
+    pp.n_local = prm.n_local;
+    pp.scale_log2 = prm.scale_log2;
+    if (!make_map_3d(&pp.tm_q, q, d_qk, n_heads, total_tokens, d_qk, q_row_stride) ||
+        !make_map_3d(&pp.tm_k, k, d_qk, 1, total_tokens, d_qk, k_row_stride, 64) ||
+        !make_map_3d(&pp.tm_v, v, d_v, 1, total_tokens, v_head_stride, v_row_stride))
+      return LOZA_ERR_CUDA;
+    return launch_prefill_pair(pp, max_seqlen, batch, st);
+  }
   if (!make_map_3d(&prm.tm_q, q, d_qk, n_heads, total_tokens, d_qk, q_row_stride) ||
       !make_map_3d(&prm.tm_k, k, d_qk, n_kv_heads, total_tokens, d_qk, k_row_stride) ||
       !make_map_3d(&prm.tm_v, v, d_v, n_kv_heads, total_tokens, v_head_stride, v_row_stride))
     return LOZA_ERR_CUDA;
 
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (dvt) {
     case 64: return launch_prefill<64, 64, 8>(prm, max_seqlen, batch, st);
     case 128: return launch_prefill<192, 128, 8>(prm, max_seqlen, batch, st);

@@ -121,7 +121,7 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     }
     mbar_init(bar(LY::BAR_S + 0), 1);
     mbar_init(bar(LY::BAR_S + 1), 1);
-    mbar_init(bar(LY::BAR_P), 128);
+    mbar_init(bar(LY::BAR_P), 4);  // one arrival per softmax warp
     mbar_init(bar(LY::BAR_PV), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -246,7 +246,7 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     const float c = p.scale_log2;  // > 0, so max(c*s) = c*max(s)
     bool ok = true;
     for (int b = 0; b < nb && ok; ++b) {
-      ok = mbar_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
+      ok = warp_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       float s[128];
@@ -267,34 +267,13 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
         mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         mx *= c;
       }
-      // Wait for PV(b-1) every block (it has normally long finished by now).
-      // Phases of this barrier must be waited in order: a parity wait is only
-      // exact while the waiter is at most one phase behind.
-      if (b > 0) {
-        ok = mbar_wait(bar(LY::BAR_PV), (b - 1) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-      }
-      // keep the stale maximum unless this block raises it by more than 2^8;
-      // only then is O (in TMEM) rescaled
+      // keep the stale maximum unless this block raises it by more than 2^8
       float alpha = 1.f;
       if (b == 0) {
         m_run = mx;
       } else if (mx > m_run + (float)kRescaleThreshold) {
         alpha = ex2_approx(m_run - mx);
         m_run = mx;
-      }
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-        for (int cc = 0; cc < DVT / 32; ++cc) {
-          float o[32];
-          tmem_ld32(lane_addr + 256 + 32 * cc, o);
-          uint32_t w[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
-          tmem_st32(lane_addr + 256 + 32 * cc, w);
-        }
-        tmem_st_wait();
       }
       const float neg_m = -m_run;
       float sum8[8], rs8[8];
@@ -320,10 +299,38 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       l_run = l_run * alpha + sum;
       r_run = r_run * alpha + rsum;
       tmem_st_wait();
+      // O must be rescaled (when the maximum moved) before PV(b) runs, and
+      // PV(b-1) must have finished writing it first. S(b) completing implies
+      // PV(b-2) completed (the MMA thread issues PV(b-2) before S(b)), and
+      // PV(b) cannot complete before this thread's P(b) arrival, so here the
+      // PV barrier is at most one phase behind PV(b-1) and its parity wait is
+      // exact. The last block always waits, which keeps the epilogue's wait
+      // for PV(nb-1) exact as well.
+      const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
+      if (b > 0 && (rescale || b == nb - 1)) {
+        ok = warp_wait(bar(LY::BAR_PV), (b - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        if (rescale) {
+#pragma unroll 1
+          for (int cc = 0; cc < DVT / 32; ++cc) {
+            float o[32];
+            tmem_ld32(lane_addr + 256 + 32 * cc, o);
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+            tmem_st32(lane_addr + 256 + 32 * cc, w);
+          }
+          tmem_st_wait();
+        }
+      }
+      // one arrival per warp: every lane's TMEM stores have completed
+      // (tcgen05.wait::st) and are ordered before lane 0's release-arrive
       tc_fence_before();
-      mbar_arrive(bar(LY::BAR_P));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(LY::BAR_P));
     }
-    if (ok) ok = mbar_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
+    if (ok) ok = warp_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / r_run;

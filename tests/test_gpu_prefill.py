@@ -86,3 +86,20 @@ def test_other_windows(bss, oracle_mod, n_sink, n_local):
     o, o_ref, l, l_ref = run_case(bss, oracle_mod, 31, [1200, 500], 2, 2, 64, 64, 0.125, n_sink, n_local)
     assert_close_o(o, o_ref, f"s={n_sink} l={n_local}")
     assert_close_lse(l, l_ref, f"s={n_sink} l={n_local}")
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(0, -1), (2, 3)])
+def test_absorbed_other_windows(bss, oracle_mod, n_sink, n_local):
+    """Absorbed shapes (CTA-pair kernel: even head count) with the unbounded and a (2, 3) window."""
+    o, o_ref, l, l_ref = run_case(bss, oracle_mod, 37, [1100, 300], 2, 1, 576, 512, 1 / math.sqrt(192),
+                                  n_sink, n_local, latent=True)
+    assert_close_o(o, o_ref, f"absorbed s={n_sink} l={n_local}")
+    assert_close_lse(l, l_ref, f"absorbed s={n_sink} l={n_local}")
+
+
+def test_absorbed_odd_heads(bss, oracle_mod):
+    """An odd head count runs the absorbed shapes on single CTAs."""
+    o, o_ref, l, l_ref = run_case(bss, oracle_mod, 41, [700, 129], 3, 1, 576, 512, 1 / math.sqrt(192),
+                                  latent=True)
+    assert_close_o(o, o_ref, "absorbed, 3 heads")
+    assert_close_lse(l, l_ref, "absorbed, 3 heads")
