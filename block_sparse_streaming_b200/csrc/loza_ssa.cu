@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -274,7 +275,8 @@ loza_status launch_prefill_pair(const PrefillPairParams& prm, int max_seqlen, in
     return LOZA_ERR_CUDA;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(2 * prm.n_heads, (max_seqlen + kTile - 1) / kTile, batch);
+  const int pairs = std::max(1, std::min(sm_count() / 2, prm.total_tiles));
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kPairThreads, 1, 1);
   cfg.dynamicSmemBytes = LY::SMEM_BYTES;
   cfg.stream = stream;
@@ -417,7 +419,7 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
 
   const int64_t v_head_stride = latent_v ? d_qk : d_v;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0 && (max_seqlen + kTile - 1) / kTile <= 65535) {
+  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0) {
     // absorbed MLA: two heads share every key block, so pairs of CTAs split the B operands
     PrefillPairParams pp;
     std::memset(&pp, 0, sizeof(pp));
@@ -425,6 +427,9 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
     pp.out = prm.out;
     pp.lse = lse;
     pp.n_heads = n_heads;
+    pp.n_qtiles = (max_seqlen + kTile - 1) / kTile;
+    if ((int64_t)batch * pp.n_qtiles * n_heads > INT32_MAX) return LOZA_ERR_UNSUPPORTED;
+    pp.total_tiles = batch * pp.n_qtiles * n_heads;
     pp.n_sink = prm.n_sink;
     pp.n_local = prm.n_local;
     pp.scale_log2 = prm.scale_log2;

@@ -62,13 +62,15 @@ struct PrefillLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQC * kChunkBytes;
   static constexpr int BAR_OFF = RING_OFF + NSTAGE * kChunkBytes;
-  // barriers: q_full, ring_full[NSTAGE], ring_empty[NSTAGE], s_full[2], p_full, pv_done
+  // barriers: q_full, ring_full[NSTAGE], ring_empty[NSTAGE], s_full[2], p_full[2], pv_done
+  // (P-ready alternates between two barriers by block parity: a warp that has
+  // already finished block b+1 must not count towards block b)
   static constexpr int BAR_Q = 0;
   static constexpr int BAR_FULL = 1;
   static constexpr int BAR_EMPTY = 1 + NSTAGE;
   static constexpr int BAR_S = 1 + 2 * NSTAGE;
   static constexpr int BAR_P = BAR_S + 2;
-  static constexpr int BAR_PV = BAR_P + 1;
+  static constexpr int BAR_PV = BAR_P + 2;
   static constexpr int NBAR = BAR_PV + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base (u32), abort (int)
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
@@ -121,7 +123,8 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     }
     mbar_init(bar(LY::BAR_S + 0), 1);
     mbar_init(bar(LY::BAR_S + 1), 1);
-    mbar_init(bar(LY::BAR_P), 4);  // one arrival per softmax warp
+    mbar_init(bar(LY::BAR_P + 0), 4);  // one arrival per softmax warp
+    mbar_init(bar(LY::BAR_P + 1), 4);
     mbar_init(bar(LY::BAR_PV), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -209,7 +212,7 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       }
       if (it >= 1) {
         const int b = it - 1;
-        ok = warp_wait(bar(LY::BAR_P), b & 1, abort_flag);
+        ok = warp_wait(bar(LY::BAR_P + (b & 1)), (b >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t tmem_p = tmem + (b & 1) * 128;
@@ -299,15 +302,12 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       l_run = l_run * alpha + sum;
       r_run = r_run * alpha + rsum;
       tmem_st_wait();
-      // O must be rescaled (when the maximum moved) before PV(b) runs, and
-      // PV(b-1) must have finished writing it first. S(b) completing implies
-      // PV(b-2) completed (the MMA thread issues PV(b-2) before S(b)), and
-      // PV(b) cannot complete before this thread's P(b) arrival, so here the
-      // PV barrier is at most one phase behind PV(b-1) and its parity wait is
-      // exact. The last block always waits, which keeps the epilogue's wait
-      // for PV(nb-1) exact as well.
+      // PV(b-1) is waited every block, after the exponentials (by then it has
+      // normally finished): O may then be rescaled before PV(b) runs. The
+      // waits are taken in order and PV(b) cannot complete before this warp's
+      // P(b) arrival, so each parity wait is exact.
       const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
-      if (b > 0 && (rescale || b == nb - 1)) {
+      if (b > 0) {
         ok = warp_wait(bar(LY::BAR_PV), (b - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
@@ -328,7 +328,7 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       // (tcgen05.wait::st) and are ordered before lane 0's release-arrive
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(LY::BAR_P));
+      if (lane == 0) mbar_arrive(bar(LY::BAR_P + (b & 1)));
     }
     if (ok) ok = warp_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
     if (ok) {

@@ -106,3 +106,26 @@ def test_training_workload_lengths(bss, oracle_mod):
         assert np.isfinite(got).all(), name
         assert err.max() <= 1e-2 * max(1.0, float(np.abs(ref).max())), f"{name}: max-abs {err.max():.3e}"
         assert err.mean() <= 1e-3 * max(1.0, float(np.abs(ref).mean())), f"{name}: mean-abs {err.mean():.3e}"
+
+
+def test_absorbed_prefill_bitwise_repeatable(bss):
+    """Workload 4's prefill length run three times: every output bit equal.
+    The kernel keeps no atomics in its arithmetic, so any difference between
+    runs exposes a synchronisation race between its pipeline roles."""
+    import torch
+    L, H, D, DV = 262144, 64, 576, 512
+    dev = torch.device("cuda")
+    seed = synth.workload_seed(4) * 1000 + 3
+    q = synth.torch_normal_bf16((L, H, D), seed, dev)
+    lat = synth.torch_normal_bf16((L, 1, D), seed + 1, dev)
+    cu = torch.tensor([0, L], dtype=torch.int32, device=dev)
+    p = bss.Params(1.0 / math.sqrt(192.0))
+    o0, l0 = bss.loza_ssa_prefill(q, lat, lat[:, :, :DV], cu, L, p)
+    for _ in range(2):
+        o1, l1 = bss.loza_ssa_prefill(q, lat, lat[:, :, :DV], cu, L, p)
+        torch.cuda.synchronize()
+        assert bss.device_status() == 0
+        bad_o = int((o1.view(torch.int16) != o0.view(torch.int16)).sum())
+        bad_l = int((l1.view(torch.int32) != l0.view(torch.int32)).sum())
+        assert bad_o == 0 and bad_l == 0, f"runs differ: {bad_o} O elements, {bad_l} LSE entries"
+        del o1, l1
