@@ -67,7 +67,7 @@ struct DecodeParams {
 struct DecodeLayout {
   static constexpr int Q_OFF = 0;                                   // 9 Q tiles, 72 KB
   static constexpr int RING_OFF = 9 * kDecQTile;                    // 73728 (1024-aligned)
-  static constexpr int P_OFF = RING_OFF + kDecStages * kDecUnit;    // P^T: 2 tiles [64 heads x 64 keys]
+  static constexpr int P_OFF = RING_OFF + kDecStages * kDecUnit;    // P^T: [128 keys x 64 heads], heads contiguous
   static constexpr int RED_OFF = P_OFF + 2 * kDecQTile;             // redmax, redsum, redrsum [4][64] each
   static constexpr int STAT_OFF = RED_OFF + 3 * 4 * 64 * 4;         // m_run, l_run, alpha, r_run [64] each
   static constexpr int BAR_OFF = STAT_OFF + 4 * 64 * 4;
@@ -245,12 +245,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       // whole warp walks the schedule with warp-uniform descriptors; one
       // elected lane issues each tcgen05 instruction
       constexpr uint32_t idesc_s = idesc_bf16(128, kDecHeads, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16(128, kDecHeads, true, false);
+      constexpr uint32_t idesc_o = idesc_bf16(128, kDecHeads, true, true);
       const uint32_t tmem_o = tmem + 128;  // O^T: 4 x 64 columns after the two S^T buffers
       const uint64_t dk0 = sdesc_sw128(sbase + LY::RING_OFF, 16, 1024);           // K tiles, K-major
       const uint64_t dq0 = sdesc_sw128(sbase + LY::Q_OFF, 16, 1024);              // Q tiles, K-major
       const uint64_t dv0 = sdesc_sw128(sbase + LY::RING_OFF, kChunkBytes, 1024);  // V unit, MN-major
-      const uint64_t dp0 = sdesc_sw128(sbase + LY::P_OFF, 16, 1024);              // P^T tiles, K-major
+      const uint64_t dp0 = sdesc_sw128(sbase + LY::P_OFF, 8192, 1024);            // P^T, MN-major (heads contiguous)
       int slot = 0;
       uint32_t phase = 0;
       bool ok = warp_wait(bar(LY::BAR_Q), 0, abort_flag);
@@ -305,8 +305,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
               const uint64_t da = desc_add(dv0, slot * kDecUnit);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem_o + 64 * u, desc_add(da, 2048 * kk), desc_add(dp0, (kk >> 2) * kDecQTile + (kk & 3) * 32),
-                       idesc_o, (b > 0 || kk > 0) ? 1u : 0u);
+                mma_ss(tmem_o + 64 * u, desc_add(da, 2048 * kk), desc_add(dp0, 2048 * kk), idesc_o,
+                       (b > 0 || kk > 0) ? 1u : 0u);
               mma_commit(bar(LY::BAR_EMPTY + slot));
             }
             __syncwarp();
@@ -326,10 +326,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
       const float cs = p.scale_log2;
       bool ok = true;
+      volatile int* rescale_flag = reinterpret_cast<volatile int*>(smem + LY::MISC_OFF + 12);
       for (int b = 0; b < nb && ok; ++b) {
         ok = warp_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
+        if (tid == 0) *rescale_flag = 0;  // read by all only after the next two barriers
         float x[32];
         tmem_ld32(lane_addr + 64 * (b & 1) + 32 * grp, x);
         const int kb = walk.block(b_lo + b);
@@ -356,36 +358,55 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
           }
           m_run[tid] = mn;
           alpha[tid] = a;
+          if (a != 1.f) *rescale_flag = 1;
         }
         named_barrier_sync(1, 256);
-        // P^T = 2^(cs*s - m) as the K-major B operand [64 heads x 128 keys]
+        // P^T = 2^(cs*s - m) as the MN-major B operand: row = key, its 64
+        // heads contiguous (128-byte swizzled rows); this thread writes the
+        // 32 heads of its group as four 16-byte chunks
         float xr[32];
         {
-          uint8_t* pbase = smem + LY::P_OFF + (key >> 6) * kDecQTile;
-          const uint32_t col = key & 63;
+          const float4* m4 = reinterpret_cast<const float4*>(m_run + 32 * grp);
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int h = 32 * grp + i;
-            x[i] = ex2_approx(fmaf(x[i], cs, -m_run[h]));
-            const __nv_bfloat16 pb16 = __float2bfloat16_rn(x[i]);
-            *reinterpret_cast<__nv_bfloat16*>(pbase + sw128_offset(h, col)) = pb16;
-            xr[i] = __bfloat162float(pb16);
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 mm = m4[i4];
+            const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[4 * i4 + j] = ex2_approx(fmaf(x[4 * i4 + j], cs, -mv[j]));
           }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
+            xr[2 * i] = __uint_as_float(pk[i] << 16);
+            xr[2 * i + 1] = __uint_as_float(pk[i] & 0xFFFF0000u);
+          }
+          uint8_t* prow = smem + LY::P_OFF + key * 128;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(prow + (((4 * grp + j) ^ (key & 7)) << 4)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
         }
         redsum[quarter * 64 + grp * 32 + lane] = warp_reduce_scatter32<false>(x);
         redrsum[quarter * 64 + grp * 32 + lane] = warp_reduce_scatter32<false>(xr);
         // O^T rescale where a head's running maximum moved (lane = latent column)
-        bool any_rescale = false;
-#pragma unroll 1
-        for (int h = 0; h < 64; ++h) any_rescale |= (alpha[h] != 1.f);
-        if (b > 0 && any_rescale) {
+        if (b > 0 && *rescale_flag) {
+          float av[32];
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 a4 = reinterpret_cast<const float4*>(alpha + 32 * grp)[i4];
+            av[4 * i4] = a4.x;
+            av[4 * i4 + 1] = a4.y;
+            av[4 * i4 + 2] = a4.z;
+            av[4 * i4 + 3] = a4.w;
+          }
 #pragma unroll 1
           for (int u = 0; u < 4; ++u) {
             float o[32];
             tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
             uint32_t w[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha[32 * grp + i]);
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * av[i]);
             tmem_st32(lane_addr + 128 + 64 * u + 32 * grp, w);
           }
           tmem_st_wait();
