@@ -446,7 +446,7 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
 
   switch (dvt) {
     case 64: return launch_prefill<64, 64, 8>(prm, max_seqlen, batch, st);
-    case 128: return launch_prefill<192, 128, 8>(prm, max_seqlen, batch, st);
+    case 128: return launch_prefill<192, 128, 11>(prm, max_seqlen, batch, st);
     default: return launch_prefill<576, 256, 5>(prm, max_seqlen, batch, st);
   }
 }

@@ -262,13 +262,10 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       }
       float mx;
       {
-        float m8[8];
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-        for (int j = 8; j < 128; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        mx *= c;
+        for (int j = 0; j < 64; ++j) m4[j & 3] = fmax3(m4[j & 3], s[2 * j], s[2 * j + 1]);
+        mx = c * fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
       // keep the stale maximum unless this block raises it by more than 2^8
       float alpha = 1.f;
@@ -278,27 +275,27 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
         alpha = ex2_approx(m_run - mx);
         m_run = mx;
       }
-      const float neg_m = -m_run;
-      float sum8[8], rs8[8];
+      const float2 c2 = make_float2(c, c);
+      const float2 nm2 = make_float2(-m_run, -m_run);
+      float2 l2[4], r2[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = rs8[i] = 0.f;
+      for (int i = 0; i < 4; ++i) l2[i] = r2[i] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(s[64 * h + 2 * i], c, neg_m));
-          const float p1 = ex2_approx(fmaf(s[64 * h + 2 * i + 1], c, neg_m));
-          sum8[(2 * i) & 7] += p0;
-          sum8[(2 * i + 1) & 7] += p1;
+          const float2 x = ffma2(make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), c2, nm2);
+          const float p0 = ex2_approx(x.x);
+          const float p1 = ex2_approx(x.y);
           pk[i] = pack_bf16(p0, p1);
-          rs8[(2 * i) & 7] += __uint_as_float(pk[i] << 16);
-          rs8[(2 * i + 1) & 7] += __uint_as_float(pk[i] & 0xFFFF0000u);
+          l2[i & 3] = fadd2(l2[i & 3], make_float2(p0, p1));
+          r2[i & 3] = fadd2(r2[i & 3], make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u)));
         }
         tmem_st32(lane_addr + (b & 1) * 128 + 32 * h, pk);
       }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-      const float rsum = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      const float sum = ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
+      const float rsum = ((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y)) + ((r2[2].x + r2[2].y) + (r2[3].x + r2[3].y));
       l_run = l_run * alpha + sum;
       r_run = r_run * alpha + rsum;
       tmem_st_wait();
