@@ -334,6 +334,14 @@ def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None):
     return out
 
 
+def prefill_workspace(bss, device, batch, T, L, params, H_=None, Hkv=1, dqk=None, dv=None):
+    """Device workspace for loza_ssa_prefill, allocated once outside the timed
+    region (None when the shape needs none)."""
+    import torch
+    n = bss.workspace_size(bss.LOZA_OP_PREFILL, batch, T, L, H_ or H, Hkv, dqk or DQK, dv or DV, params)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
 def long_secondary(bss, device, stream, peaks):
     """Workload 4: L = 262144 absorbed prefill, SSA next to full causal attention;
     then SSA and dense decode of 32 sequences of 1,048,576 tokens."""
@@ -346,9 +354,10 @@ def long_secondary(bss, device, stream, peaks):
     res = {"workload": w["name"]}
     for name, nl, n in (("ssa", LW, 5), ("dense", -1, 1)):
         params = bss.Params(SCALE, B, S if nl > 0 else 0, nl)
+        ws = prefill_workspace(bss, device, 1, L, L, params)
 
         def call():
-            bss.loza_ssa_prefill(q, lat, lat[:, :, :DV], cu, L, params, out=out, lse=lse, stream=stream)
+            bss.loza_ssa_prefill(q, lat, lat[:, :, :DV], cu, L, params, out=out, lse=lse, workspace=ws, stream=stream)
 
         call()
         torch.cuda.synchronize()
@@ -437,9 +446,10 @@ def run_ours(args, rank, world, local_rank):
     v = lat[:, :, :DV]
     out = torch.empty((L, H, DV), dtype=torch.bfloat16, device=device)
     lse = torch.empty((L, H), dtype=torch.float32, device=device)
+    ws = prefill_workspace(bss, device, 1, L, L, params)
 
     def step():
-        bss.loza_ssa_prefill(q, lat, v, cu, L, params, out=out, lse=lse, stream=stream)
+        bss.loza_ssa_prefill(q, lat, v, cu, L, params, out=out, lse=lse, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -537,12 +547,14 @@ def run_e2e(bss, params, device, stream, L, steps):
     lse_h = torch.empty((L, H), dtype=torch.float32, pin_memory=True)
     out_d = torch.empty((L, H, DV), dtype=torch.bfloat16, device=device)
     lse_d = torch.empty((L, H), dtype=torch.float32, device=device)
+    ws = prefill_workspace(bss, device, 1, L, L, params)
     torch.cuda.synchronize()
 
     def one():
         q_d.copy_(q_h, non_blocking=True)
         lat_d.copy_(lat_h, non_blocking=True)
-        bss.loza_ssa_prefill(q_d, lat_d, lat_d[:, :, :DV], cu, L, params, out=out_d, lse=lse_d, stream=stream)
+        bss.loza_ssa_prefill(q_d, lat_d, lat_d[:, :, :DV], cu, L, params, out=out_d, lse=lse_d, workspace=ws,
+                             stream=stream)
         out_h.copy_(out_d, non_blocking=True)
         lse_h.copy_(lse_d, non_blocking=True)
 

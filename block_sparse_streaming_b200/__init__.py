@@ -143,6 +143,10 @@ def loza_ssa_prefill(q, k, v, cu_seqlens, max_seqlen: int, params: Params, out=N
         out = torch.empty((T, H, d_v), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = workspace_size(LOZA_OP_PREFILL, cu_seqlens.numel() - 1, T, int(max_seqlen), H, Hkv, d_qk, d_v, params)
+        if n:
+            workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     rc = lib().loza_ssa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T,
                                 int(max_seqlen), H, Hkv, d_qk, d_v, _row_tensor(q, "q"), _row_tensor(k, "k"),

@@ -14,6 +14,7 @@
 #include "loza_ssa.h"
 #include "prefill.cuh"
 #include "prefill_pair.cuh"
+#include "prefill_mla.cuh"
 #include "decode.cuh"
 #include "decode_mla.cuh"
 #include "backward.cuh"
@@ -292,6 +293,54 @@ loza_status launch_prefill_pair(const PrefillPairParams& prm, int max_seqlen, in
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
+// Two-pass absorbed prefill: scratch per CTA of the persistent grid (at most
+// one CTA per SM): P of every key block of a tile, and the rescale factors.
+size_t mla_scratch_per_cta(int max_blocks) {
+  return (size_t)max_blocks * (kTile * kTile * 2 + 256 * 4);
+}
+size_t mla_workspace_bytes(int max_blocks) { return (size_t)sm_count() * mla_scratch_per_cta(max_blocks); }
+
+loza_status launch_prefill_mla(PrefillMlaParams& prm, void* workspace, cudaStream_t stream) {
+  using LY = PrefillMlaLayout;
+  if (cudaFuncSetAttribute(ssa_prefill_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM_BYTES) !=
+      cudaSuccess)
+    return LOZA_ERR_CUDA;
+  const int pairs = std::max(1, std::min(sm_count() / 2, prm.total_tiles));
+  const int ctas = 2 * pairs;
+  // scratch: P rows [ctas * max_blocks * 128][128] bf16, then the factors
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  prm.p_ws = reinterpret_cast<__nv_bfloat16*>(ws);
+  prm.a_ws = reinterpret_cast<float*>(ws + (size_t)sm_count() * prm.max_blocks * kTile * kTile * 2);
+  {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return LOZA_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)kTile, (cuuint64_t)ctas * prm.max_blocks * kTile};
+    cuuint64_t strides[1] = {(cuuint64_t)kTile * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&prm.tm_p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, prm.p_ws, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return LOZA_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(ctas, 1, 1);
+  cfg.blockDim = dim3(kMlaThreads, 1, 1);
+  cfg.dynamicSmemBytes = LY::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, ssa_prefill_mla_kernel, prm) != cudaSuccess) return LOZA_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Built-in scratch for loza_ssa_decode_noalloc.
 //
@@ -367,6 +416,11 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
       return decode_workspace(batch, decode_plan(p, max_seqlen, batch)).total;
     return 0;
   }
+  if (op == LOZA_OP_PREFILL) {
+    if (n_kv_heads == 1 && d_qk == 576 && d_v == 512 && n_heads % 2 == 0 && p.n_local != LOZA_UNBOUNDED)
+      return mla_workspace_bytes(p.n_sink + p.n_local);
+    return 0;
+  }
   if (op == LOZA_OP_BACKWARD) {
     if (n_kv_heads != n_heads || p.n_local == LOZA_UNBOUNDED || total_tokens < 1) return 0;
     if (!((d_qk == 64 && d_v == 64) || (d_qk == 192 && d_v == 128))) return 0;
@@ -380,7 +434,6 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
                              int32_t n_kv_heads, int32_t d_qk, int32_t d_v, int64_t q_row_stride,
                              int64_t k_row_stride, int64_t v_row_stride, loza_ssa_params p, void* out,
                              float* lse, void* workspace, size_t workspace_bytes, loza_stream_t stream) {
-  (void)workspace; (void)workspace_bytes;
   if (!q || !k || !v || !cu_seqlens || !out || !lse) return LOZA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
   if (batch < 1 || batch > 65535 || total_tokens < 1 || total_tokens > INT32_MAX || max_seqlen < 1 ||
@@ -419,6 +472,29 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
 
   const int64_t v_head_stride = latent_v ? d_qk : d_v;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0 && prm.n_local >= 0 && workspace != nullptr &&
+      aligned16(workspace) && workspace_bytes >= mla_workspace_bytes(prm.n_sink + prm.n_local)) {
+    // absorbed MLA, bounded window: S once, the value dimension in two passes
+    PrefillMlaParams mp;
+    std::memset(&mp, 0, sizeof(mp));
+    mp.cu_seqlens = cu_seqlens;
+    mp.out = prm.out;
+    mp.lse = lse;
+    mp.max_blocks = prm.n_sink + prm.n_local;
+    mp.n_heads = n_heads;
+    mp.n_qtiles = (max_seqlen + kTile - 1) / kTile;
+    if ((int64_t)batch * mp.n_qtiles * (n_heads / 2) > INT32_MAX) return LOZA_ERR_UNSUPPORTED;
+    mp.total_tiles = batch * mp.n_qtiles * (n_heads / 2);
+    mp.n_sink = prm.n_sink;
+    mp.n_local = prm.n_local;
+    mp.scale_log2 = prm.scale_log2;
+    if (!make_map_3d(&mp.tm_q, q, d_qk, n_heads, total_tokens, d_qk, q_row_stride) ||
+        !make_map_3d(&mp.tm_k, k, d_qk, 1, total_tokens, d_qk, k_row_stride, 64) ||
+        !make_map_3d(&mp.tm_v, v, d_v, 1, total_tokens, v_head_stride, v_row_stride) ||
+        !make_map_3d(&mp.tm_v64, v, d_v, 1, total_tokens, v_head_stride, v_row_stride, 64))
+      return LOZA_ERR_CUDA;
+    return launch_prefill_mla(mp, workspace, st);
+  }
   if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0) {
     // absorbed MLA: two heads share every key block, so pairs of CTAs split the B operands
     PrefillPairParams pp;

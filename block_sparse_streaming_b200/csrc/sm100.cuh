@@ -281,6 +281,21 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* desc,
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* desc, uint32_t bar, int32_t c0,
+                                                 int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// Make this thread's global-memory writes visible to later reads of that
+// memory through the async proxy (TMA loads).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster (`bar` is a
 // shared::cluster address), with the default release.cta semantics: what the
 // waiter consumes was completed before the arrive (TMEM stores waited with

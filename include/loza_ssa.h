@@ -103,6 +103,14 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
  *   max_seqlen  >= every sequence length (sizes the launch grid)
  *   out [T, n_heads, d_v] bf16 contiguous; lse [T, n_heads] fp32, natural log of
  *   the sum of exp(scale * q.k) over the visible keys.
+ *   workspace: optional. For the absorbed shapes (n_kv_heads 1, 576 / 512,
+ *               even n_heads) with a bounded window, a workspace of at least
+ *               loza_ssa_workspace_size(LOZA_OP_PREFILL, ...) bytes lets the
+ *               kernel compute S once for both halves of the value dimension
+ *               (it keeps P there between the two halves); with NULL or fewer
+ *               bytes it recomputes S per half. Same results either way up to
+ *               rounding order; the workspace is scratch owned by the caller
+ *               and must not be used by other work running at the same time.
  * Definition: page 1 section 01 (1) and (2) of the LoZA pages (see above).
  */
 loza_status loza_ssa_prefill(const void *q, const void *k, const void *v,

@@ -103,3 +103,24 @@ def test_absorbed_odd_heads(bss, oracle_mod):
                                   latent=True)
     assert_close_o(o, o_ref, "absorbed, 3 heads")
     assert_close_lse(l, l_ref, "absorbed, 3 heads")
+
+
+def test_absorbed_without_workspace(bss, oracle_mod):
+    """Absorbed shapes with no prefill workspace: the kernel recomputes S for
+    each half of the value dimension instead of keeping P between them."""
+    import torch
+    g = synth.rng(43)
+    lens = [900, 260]
+    T, H = sum(lens), 4
+    cu = synth.cu_seqlens(lens)
+    q = synth.normal_bits(g, (T, H, 576))
+    kv = synth.normal_bits(g, (T, 1, 576))
+    k_dev = to_dev(kv)
+    scale = 1 / math.sqrt(192)
+    out, lse = bss.loza_ssa_prefill(to_dev(q), k_dev, k_dev[:, :, :512], torch.from_numpy(cu).cuda(), max(lens),
+                                    bss.Params(scale), workspace=torch.empty(0, dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+    assert bss.device_status() == 0
+    o_ref, lse_ref = oracle_mod.forward(q, kv, np.ascontiguousarray(kv[:, :, :512]), cu, H, 1, 128, 1, 7, scale)
+    assert_close_o(from_dev(out), o_ref, "absorbed, no workspace")
+    assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, "absorbed, no workspace")
