@@ -494,9 +494,9 @@ def run_ours(args, rank, world, local_rank):
     achieved = flops / (avg_launch_ms / 1000.0) / 1e12
     peak = float(peaks["bf16_tflops"])
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profiled_traffic("ssa_prefill_pair_kernel"),
+                "frac": achieved / peak, "traffic": profiled_traffic("ssa_prefill_mla_kernel"),
                 "peak_kind": f"{peak_kind} bf16 dense burst (MEASURED_PEAKS.json bf16_tflops)",
-                "kernel": "ssa_prefill_pair_kernel",
+                "kernel": "ssa_prefill_mla_kernel",
                 "algorithmic_flop_per_launch": flops,
                 "avg_launch_ms": avg_launch_ms}
 

@@ -307,19 +307,21 @@ loza_status launch_prefill_mla(PrefillMlaParams& prm, void* workspace, cudaStrea
     return LOZA_ERR_CUDA;
   const int pairs = std::max(1, std::min(sm_count() / 2, prm.total_tiles));
   const int ctas = 2 * pairs;
-  // scratch: P rows [ctas * max_blocks * 128][128] bf16, then the factors
+  // scratch: P as 16 KB images of [8 key chunks][128 rows][8 keys] bf16, two
+  // per key block (keys 0-63, 64-127), max_blocks blocks per CTA; then the factors.
+  // The map reads one image as 128 lines of 128 bytes, copied unswizzled.
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   prm.p_ws = reinterpret_cast<__nv_bfloat16*>(ws);
   prm.a_ws = reinterpret_cast<float*>(ws + (size_t)sm_count() * prm.max_blocks * kTile * kTile * 2);
   {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return LOZA_ERR_CUDA;
-    cuuint64_t dims[2] = {(cuuint64_t)kTile, (cuuint64_t)ctas * prm.max_blocks * kTile};
-    cuuint64_t strides[1] = {(cuuint64_t)kTile * 2};
+    cuuint64_t dims[2] = {64, (cuuint64_t)ctas * prm.max_blocks * 2 * kTile};
+    cuuint64_t strides[1] = {128};
     cuuint32_t box[2] = {64, (cuuint32_t)kTile};
     cuuint32_t estr[2] = {1, 1};
     if (fn(&prm.tm_p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, prm.p_ws, dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return LOZA_ERR_CUDA;
   }

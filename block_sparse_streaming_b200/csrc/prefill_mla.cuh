@@ -37,11 +37,11 @@ struct PrefillMlaParams {
   CUtensorMap tm_k;    // latent [T, 1, 576]         box {64, 1, 64}
   CUtensorMap tm_v;    // value [T, 1, 512]          box {64, 1, 128}
   CUtensorMap tm_v64;  // value [T, 1, 512]          box {64, 1, 64}
-  CUtensorMap tm_p;    // P scratch [rows, 128] bf16 box {64, 128}
+  CUtensorMap tm_p;    // P scratch as lines of 64 bf16  box {64, 128}, unswizzled
   const int32_t* cu_seqlens;
   __nv_bfloat16* out;  // [T, H, 512]
   float* lse;          // [T, H]
-  __nv_bfloat16* p_ws; // [grid CTAs][max_blocks][128 rows][128 keys]
+  __nv_bfloat16* p_ws; // [grid CTAs][max_blocks][2 key halves][8 key chunks][128 rows][8 keys]
   float* a_ws;         // [grid CTAs][max_blocks][2 halves][128 rows] rescale factors
   int max_blocks;      // key blocks per tile at most (the window's s + l)
   int n_heads;         // even
@@ -218,8 +218,8 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
         for (int kh = 0; kh < 2 && ok; ++kh) {
           if (!acquire(kChunkBytes)) break;
           if (elect_one())
-            tma_load_2d_pair(sbase + LY::RING_OFF + slot * kChunkBytes, &p.tm_p, lead_bar(LY::BAR_FULL + slot),
-                             64 * kh, p_row0 + b * kTile);
+            tma_load_2d_pair(sbase + LY::RING_OFF + slot * kChunkBytes, &p.tm_p, lead_bar(LY::BAR_FULL + slot), 0,
+                             2 * p_row0 + (2 * b + kh) * kTile);
           __syncwarp();
           advance();
           if (!acquire(kChunkBytes)) break;
@@ -243,7 +243,8 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       constexpr uint16_t kBoth = 0x3;
       const uint32_t tmem_o = tmem + 256;
       const uint64_t dq0 = sdesc_sw128(sbase + LY::Q_OFF, 16, 1024);       // Q column tile (K-major)
-      const uint64_t dk0 = sdesc_sw128(sbase + LY::RING_OFF, 16, 1024);    // [64 keys x 64] K-major; P [128 x 64 keys]
+      const uint64_t dk0 = sdesc_sw128(sbase + LY::RING_OFF, 16, 1024);    // [64 keys x 64] K-major
+      const uint64_t dp0 = sdesc_interleave(sbase + LY::RING_OFF, 2048, 128);  // P [128 x 64 keys] K-major, unswizzled
       const uint64_t dv0 = sdesc_sw128(sbase + LY::RING_OFF, 8192, 1024);  // [128 or 64 keys x 64 values] MN-major
       int slot = 0;
       uint32_t phase = 0;
@@ -330,12 +331,12 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
             advance();
             if (!next_full()) break;
             if (elect_one()) {
-              const uint64_t da = desc_add(dk0, pslot * kChunkBytes);
+              const uint64_t da = desc_add(dp0, pslot * kChunkBytes);
               const uint64_t dv = desc_add(dv0, slot * kChunkBytes);
               for (int m = 0; m < 2; ++m) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                  mma_ss_pair(tmem_o + 128 * m, desc_add(da, 32 * kk), desc_add(dv, m * kMlaHalfK + 2048 * kk), idesc_pv,
+                  mma_ss_pair(tmem_o + 128 * m, desc_add(da, 4096 * kk), desc_add(dv, m * kMlaHalfK + 2048 * kk), idesc_pv,
                               (b > 0 || kh > 0 || kk > 0) ? 1u : 0u);
               }
               mma_commit_pair(bar(LY::BAR_EMPTY + pslot), kBoth);
@@ -389,9 +390,13 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       }
       tmem_st_wait();
     };
-    // write this warp's 128 O columns, normalised, to value columns col0 ..
-    auto store_o = [&](float inv, bool valid, int64_t grow, int head, int col0) {
-      __nv_bfloat16* orow = p.out + (grow * p.n_heads + head) * (int64_t)512 + col0 + 128 * half;
+    // write this warp's 128 O columns, normalised, to value columns col0 ..;
+    // rows [0, n_valid) of the tile exist. Each 8-lane group transposes its
+    // 8 rows x 8 chunks of 16 bytes, so that every store of the warp writes
+    // four whole 128-byte row segments.
+    const int j8 = lane & 7;
+    const int r8 = quarter * 32 + (lane & ~7);  // first row of this lane's group
+    auto store_o = [&](float inv, int64_t grow0, int n_valid, int head, int col0) {
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         float o[32], o2[32];
@@ -403,10 +408,14 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
           w[i] = pack_bf16(o[2 * i] * inv, o[2 * i + 1] * inv);
           w[16 + i] = pack_bf16(o2[2 * i] * inv, o2[2 * i + 1] * inv);
         }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 64 * cc);
+        transpose8x8_u4(w, lane);  // now chunk j8 of rows r8 .. r8 + 7
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int k = 0; k < 8; ++k) {
+          if (r8 + k < n_valid) {
+            __nv_bfloat16* dst =
+                p.out + ((grow0 + r8 + k) * p.n_heads + head) * (int64_t)512 + col0 + 128 * half + 64 * cc + 8 * j8;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
         }
       }
     };
@@ -472,10 +481,11 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
         }
         tmem_st32(s_addr + 32 * half, pk);  // P for pass 1's P.V, over the first 64 columns of S
         {
-          // the same P and the rescale factor, for pass 2 (row-major rows of 128 keys)
-          uint4* dst = reinterpret_cast<uint4*>(p_mine + ((size_t)b * kTile + row) * kTile + 64 * half);
+          // the same P and the rescale factor, for pass 2: chunk i of 8 keys of
+          // every row is contiguous, so each store of a warp fills 512 bytes
+          uint4* dst = reinterpret_cast<uint4*>(p_mine + (size_t)(b * 2 + half) * (8 * kTile * 8)) + row;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 8; ++i) dst[i * kTile] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           a_mine[(b * 2 + half) * 128 + row] = alpha;
         }
         l_run = l_run * alpha + (((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y)));
@@ -511,9 +521,11 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       const int qpos = tl.qb * kTile + row;
       const bool valid = qpos < tl.seq_len;
       const int64_t grow = (int64_t)tl.seq_start + qpos;
+      const int64_t grow0 = (int64_t)tl.seq_start + tl.qb * kTile;
+      const int n_valid = min(kTile, tl.seq_len - tl.qb * kTile);
       if (ok) {
         tc_fence_after();
-        store_o(inv, valid, grow, head, 0);
+        store_o(inv, grow0, n_valid, head, 0);
         if (valid && half == 0) p.lse[grow * p.n_heads + head] = (m_run + log2f(l_tot)) * 0.69314718055994530942f;
       }
       // ---------------- pass 2: follow pass 1's rescales for value columns [256, 512)
@@ -535,7 +547,7 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       if (ok) ok = warp_wait(bar(LY::BAR_PV2), (g + nb - 1) & 1, abort_flag);
       if (ok) {
         tc_fence_after();
-        store_o(inv, valid, grow, head, 256);
+        store_o(inv, grow0, n_valid, head, 256);
       }
       // the sums buffer is rewritten only after every warp has read it, and
       // all softmax warps leave together once any role gave up

@@ -332,6 +332,44 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t start, uint32_t lbo, ui
   return d;
 }
 
+// Transpose, inside each group of 8 lanes, an 8 x 8 matrix of 16-byte
+// elements: on entry lane j of the group holds row j (element k in
+// w[4k .. 4k+3]); on return it holds column j (element k = row k's element j).
+// Three exchange stages over lane distances 4, 2, 1; at each stage a lane
+// swaps with its partner the four elements whose index differs from its own
+// lane index in that bit.
+__device__ __forceinline__ void transpose8x8_u4(uint32_t (&w)[32], int lane) {
+#pragma unroll
+  for (int m = 4; m >= 1; m >>= 1) {
+    const bool hi = (lane & m) != 0;
+#pragma unroll
+    for (int base = 0; base < 8; ++base) {
+      if (base & m) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t send = hi ? w[4 * base + e] : w[4 * (base | m) + e];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+        if (hi)
+          w[4 * base + e] = recv;
+        else
+          w[4 * (base | m) + e] = recv;
+      }
+    }
+  }
+}
+
+// Unswizzled (interleaved) K-major operand: 8-row x 16-byte core matrices of
+// 128 contiguous bytes; lbo = bytes between core matrices adjacent along K,
+// sbo = bytes between core matrices adjacent along M/N; layout type 0.
+__device__ __forceinline__ uint64_t sdesc_interleave(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= 1ull << 46;
+  return d;
+}
+
 // ---------------------------------------------------------------------------
 // TMEM <-> registers. Warp w may touch TMEM lanes 32*(w%4) .. 32*(w%4)+31;
 // thread i of the warp reads/writes lane 32*(w%4)+i. taddr = base + (lane<<16) + col.
