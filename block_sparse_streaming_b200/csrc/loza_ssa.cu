@@ -299,6 +299,8 @@ size_t mla_scratch_per_cta(int max_blocks) {
   return (size_t)max_blocks * (kTile * kTile * 2 + 256 * 4);
 }
 size_t mla_workspace_bytes(int max_blocks) { return (size_t)sm_count() * mla_scratch_per_cta(max_blocks); }
+// The two-pass kernel keeps one bit per key block of a query tile.
+bool mla_window_ok(int n_sink, int n_local) { return n_local >= 0 && n_sink + n_local <= 32; }
 
 loza_status launch_prefill_mla(PrefillMlaParams& prm, void* workspace, cudaStream_t stream) {
   using LY = PrefillMlaLayout;
@@ -419,7 +421,7 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
     return 0;
   }
   if (op == LOZA_OP_PREFILL) {
-    if (n_kv_heads == 1 && d_qk == 576 && d_v == 512 && n_heads % 2 == 0 && p.n_local != LOZA_UNBOUNDED)
+    if (n_kv_heads == 1 && d_qk == 576 && d_v == 512 && n_heads % 2 == 0 && mla_window_ok(p.n_sink, p.n_local))
       return mla_workspace_bytes(p.n_sink + p.n_local);
     return 0;
   }
@@ -474,7 +476,7 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
 
   const int64_t v_head_stride = latent_v ? d_qk : d_v;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0 && prm.n_local >= 0 && workspace != nullptr &&
+  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0 && mla_window_ok(prm.n_sink, prm.n_local) && workspace != nullptr &&
       aligned16(workspace) && workspace_bytes >= mla_workspace_bytes(prm.n_sink + prm.n_local)) {
     // absorbed MLA, bounded window: S once, the value dimension in two passes
     PrefillMlaParams mp;

@@ -66,11 +66,17 @@ struct PrefillMlaLayout {
                        BAR_P = BAR_S + 2,           // [2] pass-1 P ready, by block parity (even CTA)
                        BAR_PV = BAR_P + 2,          // pass-1 P.V done (both)
                        BAR_PG = BAR_PV + 1,         // this tile's P all stored to global (this CTA)
-                       BAR_R2 = BAR_PG + 1,         // [2] pass-2 block ready (even CTA)
+                       BAR_E1 = BAR_PG + 1,         // pass-1 O read out by both CTAs (even CTA)
+                       BAR_RS = BAR_E1 + 1,         // pass-2 O ready for a rescale (this CTA)
+                       BAR_R2 = BAR_RS + 1,         // [2] pass-2 rescale done, per CTA rank (even CTA)
                        BAR_PV2 = BAR_R2 + 2,        // pass-2 P.V done (both)
                        BAR_ROW = BAR_PV2 + 1,       // [4] the two softmax warps of a lane quarter
                        NBAR = BAR_ROW + 4;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  // rescale masks: bit b set if block b rescaled O in some row of a warp;
+  // [2 ranks][8 warps] in the even CTA (for the MMA issuer), then [8 warps]
+  // of this CTA (for its own softmax warps)
+  static constexpr int MASK_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int MISC_OFF = MASK_OFF + 24 * 4;
   static constexpr int SMEM_BYTES = MISC_OFF + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -124,11 +130,13 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(LY::BAR_S + i), 1);
       mbar_init(bar(LY::BAR_P + i), 16);   // one arrival per softmax warp of each CTA
-      mbar_init(bar(LY::BAR_R2 + i), 16);
+      mbar_init(bar(LY::BAR_R2 + i), 8);   // the softmax warps of CTA rank i
     }
     mbar_init(bar(LY::BAR_PV), 1);
     mbar_init(bar(LY::BAR_PV2), 1);
     mbar_init(bar(LY::BAR_PG), 8);         // this CTA's softmax warps
+    mbar_init(bar(LY::BAR_E1), 16);
+    mbar_init(bar(LY::BAR_RS), 1);
     for (int i = 0; i < 4; ++i) mbar_init(bar(LY::BAR_ROW + i), 2);
     *abort_flag = 0;
     fence_barrier_init();
@@ -166,20 +174,25 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
     };
     int ntile = 0;
     MlaTile tl;
-    for (int t = pair; t < p.total_tiles && ok; t += npairs) {
-      if (!tl.load(p, t)) continue;
-      const BlockWalk walk(tl.qb, p.n_sink, p.n_local);
-      const int nb = walk.count;
-      const int head = 2 * tl.hp + (int)rank;
-      if (ntile > 0) ok = warp_wait(bar(LY::BAR_QE), (ntile - 1) & 1, abort_flag);
-      if (!ok) break;
+    auto next_tile = [&](int t, MlaTile& x) {
+      while (t < p.total_tiles && !x.load(p, t)) t += npairs;
+      return t;
+    };
+    auto load_q = [&](const MlaTile& x) {
       if (elect_one()) {
         if (rank == 0) mbar_arrive_expect_tx(bar(LY::BAR_Q), 2u * 9 * kChunkBytes);
-        const int row0 = tl.seq_start + tl.qb * kTile;
+        const int row0 = x.seq_start + x.qb * kTile;
         for (int c = 0; c < 9; ++c)
-          tma_load_3d_pair(sbase + LY::Q_OFF + c * kChunkBytes, &p.tm_q, lead_bar(LY::BAR_Q), c * 64, head, row0);
+          tma_load_3d_pair(sbase + LY::Q_OFF + c * kChunkBytes, &p.tm_q, lead_bar(LY::BAR_Q), c * 64,
+                           2 * x.hp + (int)rank, row0);
       }
       __syncwarp();
+    };
+    int t = next_tile(pair, tl);
+    if (t < p.total_tiles) load_q(tl);
+    while (t < p.total_tiles && ok) {
+      const BlockWalk walk(tl.qb, p.n_sink, p.n_local);
+      const int nb = walk.count;
       // pass 1: K halves of every block, value columns [0, 256)
       for (int it = 0; it <= nb && ok; ++it) {
         if (it < nb) {
@@ -208,6 +221,13 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
           }
         }
       }
+      // the next tile's Q, as soon as this tile's S no longer read Q
+      MlaTile tn;
+      const int t_next = next_tile(t + npairs, tn);
+      if (ok && t_next < p.total_tiles) {
+        ok = warp_wait(bar(LY::BAR_QE), ntile & 1, abort_flag);
+        if (ok) load_q(tn);
+      }
       // pass 2: the stored P of every block (once all of it is in global
       // memory) and value columns [256, 512)
       if (ok) ok = warp_wait(bar(LY::BAR_PG), ntile & 1, abort_flag);
@@ -234,22 +254,29 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
         }
       }
       ++ntile;
+      t = t_next;
+      tl = tn;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
+    // TMEM columns: the tile's S double buffer and later its pass-2 O share
+    // one half (ra); its pass-1 O is the other half. ra alternates between
+    // tiles, so pass 2 runs while the softmax warps read out pass-1 O, and the
+    // next tile's first S while they read out pass-2 O.
     if (rank == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(256, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(256, 128, false, true);
       constexpr uint16_t kBoth = 0x3;
-      const uint32_t tmem_o = tmem + 256;
       const uint64_t dq0 = sdesc_sw128(sbase + LY::Q_OFF, 16, 1024);       // Q column tile (K-major)
       const uint64_t dk0 = sdesc_sw128(sbase + LY::RING_OFF, 16, 1024);    // [64 keys x 64] K-major
       const uint64_t dp0 = sdesc_interleave(sbase + LY::RING_OFF, 2048, 128);  // P [128 x 64 keys] K-major, unswizzled
       const uint64_t dv0 = sdesc_sw128(sbase + LY::RING_OFF, 8192, 1024);  // [128 or 64 keys x 64 values] MN-major
+      const volatile uint32_t* masks = reinterpret_cast<const volatile uint32_t*>(smem + LY::MASK_OFF);
       int slot = 0;
       uint32_t phase = 0;
       bool ok = true;
       int ntile = 0, g = 0;
+      int ev[2] = {0, 0};  // rescale events so far, per CTA rank
       MlaTile tl;
       auto next_full = [&]() {
         ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
@@ -262,14 +289,19 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       for (int t = pair; t < p.total_tiles && ok; t += npairs) {
         if (!tl.load(p, t)) continue;
         const int nb = BlockWalk(tl.qb, p.n_sink, p.n_local).count;
+        const uint32_t ra = (uint32_t)(ntile & 1) * 256;
+        const uint32_t tmem_o1 = tmem + (256 - ra);
+        const uint32_t tmem_o2 = tmem + ra;
         ok = warp_wait(bar(LY::BAR_Q), ntile & 1, abort_flag);
+        // S overwrites the columns of the previous tile's pass-1 O
+        if (ok && ntile > 0) ok = warp_wait(bar(LY::BAR_E1), (ntile - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         // ---------------- pass 1: S and the first 256 value columns
         for (int it = 0; it <= nb && ok; ++it) {
           if (it < nb) {
             const int gs = g + it;
-            const uint32_t tmem_s = tmem + (gs & 1) * 128;
+            const uint32_t tmem_s = tmem + ra + (gs & 1) * 128;
             for (int k = 0; k < 5; ++k) {
               if (!next_full()) break;
               if (elect_one()) {
@@ -297,17 +329,19 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
           if (it >= 1) {
             const int b = it - 1;
             const int gb = g + b;
-            ok = warp_wait(bar(LY::BAR_P + (gb & 1)), (gb >> 1) & 1, abort_flag);
+            // the last block's arrivals also publish the warps' rescale masks
+            ok = b == nb - 1 ? warp_wait_cluster(bar(LY::BAR_P + (gb & 1)), (gb >> 1) & 1, abort_flag)
+                             : warp_wait(bar(LY::BAR_P + (gb & 1)), (gb >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tmem_p = tmem + (gb & 1) * 128;
+            const uint32_t tmem_p = tmem + ra + (gb & 1) * 128;
             for (int m = 0; m < 2; ++m) {
               if (!next_full()) break;
               if (elect_one()) {
                 const uint64_t dv = desc_add(dv0, slot * kChunkBytes);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                  mma_ts_pair(tmem_o + 128 * m, tmem_p + kk * 8, desc_add(dv, 2048 * kk), idesc_pv,
+                  mma_ts_pair(tmem_o1 + 128 * m, tmem_p + kk * 8, desc_add(dv, 2048 * kk), idesc_pv,
                               (b > 0 || kk > 0) ? 1u : 0u);
                 mma_commit_pair(bar(LY::BAR_EMPTY + slot), kBoth);
               }
@@ -319,10 +353,21 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
             __syncwarp();
           }
         }
-        // ---------------- pass 2: the stored P against value columns [256, 512)
+        if (!ok) break;
+        // ---------------- pass 2: the stored P against value columns [256, 512);
+        // O is rescaled only at the blocks where some row of a CTA rescaled in pass 1
+        uint32_t rmask[2] = {0u, 0u};
+        for (int w = 0; w < 8; ++w) {
+          rmask[0] |= masks[w];
+          rmask[1] |= masks[8 + w];
+        }
         for (int b = 0; b < nb && ok; ++b) {
-          const int gb = g + b;
-          ok = warp_wait(bar(LY::BAR_R2 + (gb & 1)), (gb >> 1) & 1, abort_flag);
+          for (int c = 0; c < 2 && ok; ++c) {
+            if ((rmask[c] >> b) & 1u) {
+              ok = warp_wait(bar(LY::BAR_R2 + c), ev[c] & 1, abort_flag);
+              ++ev[c];
+            }
+          }
           if (!ok) break;
           tc_fence_after();
           for (int kh = 0; kh < 2; ++kh) {
@@ -336,8 +381,8 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
               for (int m = 0; m < 2; ++m) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                  mma_ss_pair(tmem_o + 128 * m, desc_add(da, 4096 * kk), desc_add(dv, m * kMlaHalfK + 2048 * kk), idesc_pv,
-                              (b > 0 || kh > 0 || kk > 0) ? 1u : 0u);
+                  mma_ss_pair(tmem_o2 + 128 * m, desc_add(da, 4096 * kk), desc_add(dv, m * kMlaHalfK + 2048 * kk),
+                              idesc_pv, (b > 0 || kh > 0 || kk > 0) ? 1u : 0u);
               }
               mma_commit_pair(bar(LY::BAR_EMPTY + pslot), kBoth);
               mma_commit_pair(bar(LY::BAR_EMPTY + slot), kBoth);
@@ -346,9 +391,16 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
             advance();
           }
           if (!ok) break;
-          if (elect_one()) mma_commit_pair(bar(LY::BAR_PV2), kBoth);
+          // O holds blocks 0 .. b once these complete: a CTA that rescales at b + 1 may start
+          if (elect_one()) {
+            for (int c = 0; c < 2; ++c)
+              if (b + 1 < nb && ((rmask[c] >> (b + 1)) & 1u)) mma_commit_pair(bar(LY::BAR_RS), (uint16_t)(1u << c));
+          }
           __syncwarp();
         }
+        if (!ok) break;
+        if (elect_one()) mma_commit_pair(bar(LY::BAR_PV2), kBoth);
+        __syncwarp();
         g += nb;
         ++ntile;
       }
@@ -367,8 +419,11 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
     __nv_bfloat16* p_mine = p.p_ws + (size_t)p_row0 * kTile;    // this CTA's stored P
     float* a_mine = p.a_ws + (size_t)blockIdx.x * p.max_blocks * 256;  // this CTA's rescale factors
     const float c = p.scale_log2;
+    // this warp's rescale mask: its slot in the even CTA, and in this CTA
+    const uint32_t mask_lead = peer_addr(sbase + LY::MASK_OFF, 0) + 4u * (rank * 8 + (warp - 2));
+    volatile uint32_t* mask_own = reinterpret_cast<volatile uint32_t*>(smem + LY::MASK_OFF + 64);
     bool ok = true;
-    int g = 0, n_row = 0;
+    int g = 0, n_row = 0, ntile = 0, n_ev = 0;
     MlaTile tl;
     auto arrive_lead = [&](int i) {
       if (rank == 0)
@@ -376,11 +431,11 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       else
         mbar_arrive_cluster(lead_bar(i));
     };
-    // multiply this warp's 128 O columns by alpha (per row)
-    auto rescale_o = [&](float alpha) {
+    // multiply this warp's 128 columns of the O at TMEM column o_col by alpha (per row)
+    auto rescale_o = [&](uint32_t o_col, float alpha) {
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
-        const uint32_t o_addr = lane_addr + 256 + 128 * half + 32 * cc;
+        const uint32_t o_addr = lane_addr + o_col + 128 * half + 32 * cc;
         float o[32];
         tmem_ld32(o_addr, o);
         uint32_t w[32];
@@ -396,12 +451,12 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
     // four whole 128-byte row segments.
     const int j8 = lane & 7;
     const int r8 = quarter * 32 + (lane & ~7);  // first row of this lane's group
-    auto store_o = [&](float inv, int64_t grow0, int n_valid, int head, int col0) {
+    auto store_o = [&](uint32_t o_col, float inv, int64_t grow0, int n_valid, int head, int col0) {
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         float o[32], o2[32];
-        tmem_ld32(lane_addr + 256 + 128 * half + 64 * cc, o);
-        tmem_ld32(lane_addr + 256 + 128 * half + 64 * cc + 32, o2);
+        tmem_ld32(lane_addr + o_col + 128 * half + 64 * cc, o);
+        tmem_ld32(lane_addr + o_col + 128 * half + 64 * cc + 32, o2);
         uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -427,13 +482,15 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       // m_run: running row maximum of scale*log2(e)*s (the reference of P);
       // l_run / r_run: this warp's share of the exact / bf16-rounded sums of P
       float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
+      const uint32_t ra = (uint32_t)(ntile & 1) * 256;  // S and pass-2 O; pass-1 O at 256 - ra
+      uint32_t wmask = 0;  // blocks at which some row of this warp rescaled O
       // ---------------- pass 1
       for (int b = 0; b < nb && ok; ++b) {
         const int gb = g + b;
         ok = warp_wait(bar(LY::BAR_S + (gb & 1)), (gb >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t s_addr = lane_addr + (gb & 1) * 128;
+        const uint32_t s_addr = lane_addr + ra + (gb & 1) * 128;
         float so[64], s[64];  // the other warp's keys (maximum only) and this warp's keys
         tmem_ld64x2(s_addr + 64 * (half ^ 1), s_addr + 64 * half, so, s);
         // P is stored over S columns holding keys of both warps of the row:
@@ -493,16 +550,33 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
         tmem_st_wait();
         // PV(b-1) is waited every block (parity waits in order); O is then
         // rescaled, if the maximum moved, before PV(b) runs
-        const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
+        const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);  // never at b == 0
         if (b > 0) {
           ok = warp_wait(bar(LY::BAR_PV), (gb - 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          if (rescale) rescale_o(alpha);
+          if (rescale) {
+            rescale_o(256 - ra, alpha);
+            wmask |= 1u << b;
+          }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_lead(LY::BAR_P + (gb & 1));
+        if (lane == 0) {
+          if (b == nb - 1) {
+            // publish the mask: to the MMA issuer with this arrival, and to this CTA's warps
+            mask_own[warp - 2] = wmask;
+            if (rank == 0) {
+              *reinterpret_cast<volatile uint32_t*>(smem + LY::MASK_OFF + 4 * (warp - 2)) = wmask;
+              mbar_arrive(bar(LY::BAR_P + (gb & 1)));
+            } else {
+              st_cluster_u32(mask_lead, wmask);
+              mbar_arrive_cluster_release(lead_bar(LY::BAR_P + (gb & 1)));
+            }
+          } else {
+            arrive_lead(LY::BAR_P + (gb & 1));
+          }
+        }
       }
       // every P of this tile is in global memory: visible to the TMA loads of pass 2
       fence_proxy_async_global();
@@ -518,6 +592,8 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       const float l_tot = xl[row] + xl[128 + row];
       const float r_tot = xr[row] + xr[128 + row];
       const float inv = 1.f / r_tot;
+      uint32_t cmask = 0;  // blocks at which some row of this CTA rescaled O
+      for (int w = 0; w < 8; ++w) cmask |= mask_own[w];
       const int qpos = tl.qb * kTile + row;
       const bool valid = qpos < tl.seq_len;
       const int64_t grow = (int64_t)tl.seq_start + qpos;
@@ -525,35 +601,39 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       const int n_valid = min(kTile, tl.seq_len - tl.qb * kTile);
       if (ok) {
         tc_fence_after();
-        store_o(inv, grow0, n_valid, head, 0);
+        store_o(256 - ra, inv, grow0, n_valid, head, 0);
         if (valid && half == 0) p.lse[grow * p.n_heads + head] = (m_run + log2f(l_tot)) * 0.69314718055994530942f;
       }
-      // ---------------- pass 2: follow pass 1's rescales for value columns [256, 512)
-      for (int b = 0; b < nb && ok; ++b) {
-        const int gb = g + b;
+      // pass-1 O has been read: the next tile's S may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_lead(LY::BAR_E1);
+      // ---------------- pass 2: repeat pass 1's rescales on value columns [256, 512),
+      // at the blocks where some row of this CTA rescaled
+      for (int b = 1; b < nb && ok; ++b) {
+        if (!((cmask >> b) & 1u)) continue;
         const float alpha = a_mine[(b * 2 + half) * 128 + row];  // this thread's own pass-1 write
-        const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
-        if (b > 0) {
-          ok = warp_wait(bar(LY::BAR_PV2), (gb - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          if (rescale) rescale_o(alpha);
-        }
+        ok = warp_wait(bar(LY::BAR_RS), n_ev & 1, abort_flag);
+        ++n_ev;
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o(ra, alpha);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_lead(LY::BAR_R2 + (gb & 1));
+        if (lane == 0) arrive_lead(LY::BAR_R2 + (int)rank);
       }
       // ---------------- epilogue 2: value columns [256, 512)
-      if (ok) ok = warp_wait(bar(LY::BAR_PV2), (g + nb - 1) & 1, abort_flag);
+      if (ok) ok = warp_wait(bar(LY::BAR_PV2), ntile & 1, abort_flag);
       if (ok) {
         tc_fence_after();
-        store_o(inv, grow0, n_valid, head, 256);
+        store_o(ra, inv, grow0, n_valid, head, 256);
       }
       // the sums buffer is rewritten only after every warp has read it, and
       // all softmax warps leave together once any role gave up
       named_barrier_sync(1, 256);
       ok = ok && *abort_flag == 0;
       g += nb;
+      ++ntile;
     }
   }
 

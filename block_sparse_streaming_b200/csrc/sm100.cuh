@@ -305,6 +305,46 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// The same with release semantics at cluster scope: plain shared-memory
+// writes this thread made to another CTA before it are visible to a thread
+// that observes the phase with mbar_wait_cluster.
+__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// warp_wait with acquire semantics at cluster scope (pairs with
+// mbar_arrive_cluster_release); bounded like mbar_wait.
+__device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
+  bool ok = mbar_try_wait_cluster(bar, parity);
+  if (!ok) {
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try_wait_cluster(bar, parity)) { ok = true; break; }
+      if ((it & 255) == 0) {
+        if (abort && *abort) break;
+        if (global_ns() - t0 > kWaitLimitNs) {
+          atomicOr(&g_device_status, kErrTimeout);
+          if (abort) *abort = 1;
+          break;
+        }
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Instruction descriptor: bf16 x bf16 -> fp32, M x N, operand majors.
 // Bit layout (tcgen05 instruction descriptor for kind::f16): [4,6) D format
 // (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),

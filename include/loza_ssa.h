@@ -104,7 +104,8 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
  *   out [T, n_heads, d_v] bf16 contiguous; lse [T, n_heads] fp32, natural log of
  *   the sum of exp(scale * q.k) over the visible keys.
  *   workspace: optional. For the absorbed shapes (n_kv_heads 1, 576 / 512,
- *               even n_heads) with a bounded window, a workspace of at least
+ *               even n_heads) with a bounded window of at most 32 blocks
+ *               (n_sink + n_local <= 32), a workspace of at least
  *               loza_ssa_workspace_size(LOZA_OP_PREFILL, ...) bytes lets the
  *               kernel compute S once for both halves of the value dimension
  *               (it keeps P there between the two halves); with NULL or fewer

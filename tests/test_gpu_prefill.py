@@ -124,3 +124,36 @@ def test_absorbed_without_workspace(bss, oracle_mod):
     o_ref, lse_ref = oracle_mod.forward(q, kv, np.ascontiguousarray(kv[:, :, :512]), cu, H, 1, 128, 1, 7, scale)
     assert_close_o(from_dev(out), o_ref, "absorbed, no workspace")
     assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, "absorbed, no workspace")
+
+
+@pytest.mark.parametrize("seed", [47, 53])
+def test_absorbed_rescales(bss, oracle_mod, seed):
+    """Absorbed shapes where the running row maximum jumps by far more than
+    the lazy-rescale threshold at scattered key blocks: the 64 rotary columns
+    of each key block carry a factor from {0.5, 1, 4, 8} and each head's
+    queries another, so the two heads of a CTA pair rescale at different
+    blocks (the quietest head rarely). The 512 value columns are halved, so
+    that O stays where bf16 output rounding is below the O tolerance. Pass 2
+    of the two-pass kernel must repeat exactly pass 1's rescales."""
+    import torch
+    g = synth.rng(seed)
+    lens = [1500, 700]
+    T, H = sum(lens), 4
+    cu = synth.cu_seqlens(lens)
+    q = synth.bits_to_f32(synth.normal_bits(g, (T, H, 576)))
+    kv = synth.bits_to_f32(synth.normal_bits(g, (T, 1, 576)))
+    q *= np.array([0.2, 1.0, 1.5, 0.7], np.float32)[None, :, None]
+    block_f = g.choice(np.array([0.5, 1.0, 4.0, 8.0], np.float32), size=(T + 127) // 128)
+    kv[:, :, 512:] *= np.repeat(block_f, 128)[:T, None, None]
+    kv[:, :, :512] *= np.float32(0.5)
+    q_bits, kv_bits = synth.bf16_bits(q), synth.bf16_bits(kv)
+    k_dev = to_dev(kv_bits)
+    scale = 1 / math.sqrt(192)
+    out, lse = bss.loza_ssa_prefill(to_dev(q_bits), k_dev, k_dev[:, :, :512], torch.from_numpy(cu).cuda(),
+                                    max(lens), bss.Params(scale))
+    torch.cuda.synchronize()
+    assert bss.device_status() == 0
+    o_ref, lse_ref = oracle_mod.forward(q_bits, kv_bits, np.ascontiguousarray(kv_bits[:, :, :512]), cu, H, 1, 128,
+                                        1, 7, scale)
+    assert_close_o(from_dev(out), o_ref, f"absorbed rescales seed={seed}")
+    assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, f"absorbed rescales seed={seed}")
