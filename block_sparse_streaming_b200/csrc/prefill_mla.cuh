@@ -53,6 +53,7 @@ struct PrefillMlaParams {
 };
 
 constexpr int kMlaStages = 5;
+constexpr int kMlaMaxBlocks = 32;  // key blocks per query tile
 constexpr int kMlaThreads = 320;
 constexpr int kMlaHalfK = 64 * 64 * 2;  // [64 keys x 64 dims]
 
@@ -65,8 +66,8 @@ struct PrefillMlaLayout {
                        BAR_S = 2 + 2 * kMlaStages,  // [2]
                        BAR_P = BAR_S + 2,           // [2] pass-1 P ready, by block parity (even CTA)
                        BAR_PV = BAR_P + 2,          // pass-1 P.V done (both)
-                       BAR_PG = BAR_PV + 1,         // this tile's P all stored to global (this CTA)
-                       BAR_E1 = BAR_PG + 1,         // pass-1 O read out by both CTAs (even CTA)
+                       BAR_PG = BAR_PV + 1,         // [kMlaMaxBlocks] P of block b stored to global (this CTA)
+                       BAR_E1 = BAR_PG + kMlaMaxBlocks,  // pass-1 O read out by both CTAs (even CTA)
                        BAR_RS = BAR_E1 + 1,         // pass-2 O ready for a rescale (this CTA)
                        BAR_R2 = BAR_RS + 1,         // [2] pass-2 rescale done, per CTA rank (even CTA)
                        BAR_PV2 = BAR_R2 + 2,        // pass-2 P.V done (both)
@@ -134,7 +135,7 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
     }
     mbar_init(bar(LY::BAR_PV), 1);
     mbar_init(bar(LY::BAR_PV2), 1);
-    mbar_init(bar(LY::BAR_PG), 8);         // this CTA's softmax warps
+    for (int i = 0; i < kMlaMaxBlocks; ++i) mbar_init(bar(LY::BAR_PG + i), 8);  // this CTA's softmax warps
     mbar_init(bar(LY::BAR_E1), 16);
     mbar_init(bar(LY::BAR_RS), 1);
     for (int i = 0; i < 4; ++i) mbar_init(bar(LY::BAR_ROW + i), 2);
@@ -188,6 +189,7 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       }
       __syncwarp();
     };
+    uint32_t pg_parity = 0;  // bit b: parity of the next phase of PG[b]
     int t = next_tile(pair, tl);
     if (t < p.total_tiles) load_q(tl);
     while (t < p.total_tiles && ok) {
@@ -228,12 +230,15 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
         ok = warp_wait(bar(LY::BAR_QE), ntile & 1, abort_flag);
         if (ok) load_q(tn);
       }
-      // pass 2: the stored P of every block (once all of it is in global
-      // memory) and value columns [256, 512)
-      if (ok) ok = warp_wait(bar(LY::BAR_PG), ntile & 1, abort_flag);
-      // per block and key half kh: P[:, 64kh .. +64] (one slot), then this
-      // CTA's value columns of both 128-column groups for those keys (one slot)
+      // pass 2: the stored P of every block (once it is in global memory) and
+      // value columns [256, 512); per block and key half kh: P[:, 64kh .. +64]
+      // (one slot), then this CTA's value columns of both 128-column groups
+      // for those keys (one slot)
       for (int b = 0; b < nb && ok; ++b) {
+        // PG[b] completes once per tile that has a block b
+        ok = warp_wait(bar(LY::BAR_PG + b), (pg_parity >> b) & 1u, abort_flag);
+        pg_parity ^= 1u << b;
+        if (!ok) break;
         const int vrow = tl.seq_start + walk.block(b) * kTile;
         for (int kh = 0; kh < 2 && ok; ++kh) {
           if (!acquire(kChunkBytes)) break;
@@ -489,6 +494,12 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
         const int gb = g + b;
         ok = warp_wait(bar(LY::BAR_S + (gb & 1)), (gb >> 1) & 1, abort_flag);
         if (!ok) break;
+        if (b > 0) {
+          // the previous block's P (stored a block ago) is visible to the TMA loads of pass 2
+          fence_proxy_async_global();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(LY::BAR_PG + b - 1));
+        }
         tc_fence_after();
         const uint32_t s_addr = lane_addr + ra + (gb & 1) * 128;
         float so[64], s[64];  // the other warp's keys (maximum only) and this warp's keys
@@ -578,10 +589,10 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
           }
         }
       }
-      // every P of this tile is in global memory: visible to the TMA loads of pass 2
+      // the last block's P
       fence_proxy_async_global();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(LY::BAR_PG));
+      if (lane == 0) mbar_arrive(bar(LY::BAR_PG + nb - 1));
       // ---------------- epilogue 1: value columns [0, 256)
       if (ok) ok = warp_wait(bar(LY::BAR_PV), (g + nb - 1) & 1, abort_flag);
       if (ok) {
