@@ -74,7 +74,9 @@ struct DecodeLayout {
   // barriers: q_full, full[4], empty[4], s_full[2], p_ready, pv_done, vtail (the block holding
   // the query's own, possibly partial, block has all its V units resident)
   static constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = 1 + kDecStages, BAR_S = 1 + 2 * kDecStages,
-                       BAR_P = BAR_S + 2, BAR_PV = BAR_P + 1, BAR_VT = BAR_PV + 1, NBAR = BAR_VT + 1;
+                       BAR_P = BAR_S + 2, BAR_PV = BAR_P + 1, BAR_VT = BAR_PV + 1,
+                       BAR_MRG = BAR_VT + 1,  // on-chip merge: the other splits' parts have arrived
+                       NBAR = BAR_MRG + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, abort, last-CTA flag
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -185,6 +187,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
     mbar_init(bar(LY::BAR_P), 8);  // one arrival per softmax warp
     mbar_init(bar(LY::BAR_PV), 1);
     mbar_init(bar(LY::BAR_VT), 1);
+    mbar_init(bar(LY::BAR_MRG), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
               for (int t = 0; t < 2; ++t) {
                 uint4* row = reinterpret_cast<uint4*>(smem + LY::RING_OFF + slot_u * kDecUnit + t * kChunkBytes + key * 128);
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) row[q8] = z;
+                for (int q8 = 0; q8 < 8; ++q8) row[(q8 + lane) & 7] = z;  // lanes spread over the banks
               }
             }
           }
@@ -463,8 +466,119 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
     p.ws_ml[part * kDecHeads + threadIdx.x] = make_float4(-INFINITY, 0.f, 0.f, 0.f);  // a split without blocks
   }
 
-  if (CLUSTER) {
+  if (CLUSTER && p.nsplit <= 4) {
     // ---------------------------------------------------------- on-chip merge
+    // Split r owns output columns [r*W, (r+1)*W), W = 512 / nsplit.
+    // 1. every CTA reads all splits' (m, l) over DSMEM and computes the same
+    //    merge weights; 2. each thread scales the O^T values it holds in TMEM
+    //    that belong to other splits' columns and stores them to a staging
+    //    area in this CTA's shared memory, laid out as the owner's receive
+    //    slot; 3. one bulk copy per owner moves the slot into the owner's
+    //    shared memory; 4. each CTA adds its own scaled part (from TMEM) and
+    //    the received parts and writes its columns.
+    const int r = (int)cluster_rank();
+    const int ns = p.nsplit;
+    const int W = 512 / ns;
+    const uint32_t part_bytes = 64u * (uint32_t)W * 4u;
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && ns > 1) mbar_arrive_expect_tx(bar(LY::BAR_MRG), (uint32_t)(ns - 1) * part_bytes);
+    cluster_sync_all();  // (m, l) of every split visible; every receive barrier armed
+    // staging [ns-1][64][W] and receive [ns-1][64][W] buffers over the idle Q
+    // tiles and ring; slot of split s in either: s < r ? s : s - 1
+    float* stg = reinterpret_cast<float*>(smem + LY::Q_OFF);
+    float* recv = stg + (size_t)(ns - 1) * 64 * W;
+    float* wgt = reinterpret_cast<float*>(smem + LY::P_OFF);  // [8][64]; P^T is idle now
+    float* mls = wgt + 8 * 64;                                 // [3][8][64] all splits' m, l, r
+    for (int idx = threadIdx.x; idx < ns * 64; idx += blockDim.x) {
+      const int s2 = idx >> 6, h = idx & 63;
+      mls[idx] = *static_cast<const float*>(__cluster_map_shared_rank(m_run + h, s2));
+      mls[8 * 64 + idx] = *static_cast<const float*>(__cluster_map_shared_rank(l_run + h, s2));
+      mls[16 * 64 + idx] = *static_cast<const float*>(__cluster_map_shared_rank(r_run + h, s2));
+    }
+    __syncthreads();
+    if (threadIdx.x < 64) {
+      const int h = threadIdx.x;
+      float M = -INFINITY;
+      for (int s2 = 0; s2 < ns; ++s2)
+        if (mls[8 * 64 + s2 * 64 + h] > 0.f) M = fmaxf(M, mls[s2 * 64 + h]);
+      // O is normalised by the merged sum of the bf16 P that multiplied V,
+      // the LSE by the merged exact sum
+      float Ls = 0.f, Rs = 0.f;
+      for (int s2 = 0; s2 < ns; ++s2) {
+        const float l = mls[8 * 64 + s2 * 64 + h];
+        const float w = l > 0.f ? ex2_approx(mls[s2 * 64 + h] - M) : 0.f;
+        wgt[s2 * 64 + h] = w;
+        Ls += l * w;
+        Rs += mls[16 * 64 + s2 * 64 + h] * w;
+      }
+      const float inv = 1.f / Rs;
+      for (int s2 = 0; s2 < ns; ++s2) wgt[s2 * 64 + h] *= inv;
+      if (r == 0) p.lse[(int64_t)seq * kDecHeads + h] = (M + log2f(Ls)) * 0.69314718055994530942f;
+    }
+    __syncthreads();
+    const int quarter = warp & 3, grp = (warp - 2) >> 2, key = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    if (nb > 0 && warp >= 2) {
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {
+        const int d = 128 * u + key;  // latent column of this lane
+        const int owner = d / W;
+        if (owner == r) continue;
+        float* dst = stg + (size_t)(owner < r ? owner : owner - 1) * 64 * W + (d - owner * W);
+        float o[32];
+        tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int h = 32 * grp + i;
+          dst[(size_t)h * W] = o[i] * wgt[r * 64 + h];
+        }
+      }
+    }
+    fence_proxy_async_smem();  // staging written by threads, read by the bulk copies
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int s2 = 0; s2 < ns; ++s2) {
+        if (s2 == r) continue;
+        const uint32_t src = smem_u32(stg + (size_t)(s2 < r ? s2 : s2 - 1) * 64 * W);
+        const uint32_t dst = peer_addr(smem_u32(recv + (size_t)(r < s2 ? r : r - 1) * 64 * W), (uint32_t)s2);
+        bulk_copy_to_peer(dst, src, part_bytes, peer_addr(bar(LY::BAR_MRG), (uint32_t)s2));
+      }
+    }
+    const bool arrived = ns == 1 || mbar_wait(bar(LY::BAR_MRG), 0, nullptr);
+    if (arrived && warp >= 2) {
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {
+        const int d = 128 * u + key;
+        if (d / W != r) continue;
+        float acc[32];
+        if (nb > 0) {
+          tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, acc);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] *= wgt[r * 64 + 32 * grp + i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+        }
+        for (int s2 = 0; s2 < ns; ++s2) {
+          if (s2 == r) continue;
+          const float* src = recv + (size_t)(s2 < r ? s2 : s2 - 1) * 64 * W + (d - r * W);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int h = 32 * grp + i;
+            if (wgt[s2 * 64 + h] != 0.f) acc[i] += src[(size_t)h * W];  // a split without blocks sent no data
+          }
+        }
+        __nv_bfloat16* dst = p.out + (int64_t)seq * kDecHeads * 512 + d;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dst[(int64_t)(32 * grp + i) * 512] = __float2bfloat16_rn(acc[i]);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // every bulk copy has finished reading its source before any CTA exits
+  } else if (CLUSTER) {
+    // ---------------------------------------------------------- on-chip merge, 8 splits
     // 1. every CTA reads all splits' (m, l) over DSMEM and computes the same
     //    merge weights; 2. each thread scales its O^T values (read from TMEM)
     //    by its split's weight and pushes them, with plain DSMEM stores, into

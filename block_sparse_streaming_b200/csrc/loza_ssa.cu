@@ -17,6 +17,7 @@
 #include "prefill_mla.cuh"
 #include "decode.cuh"
 #include "decode_mla.cuh"
+#include "decode_mla_hs.cuh"
 #include "backward.cuh"
 
 namespace loza {
@@ -84,6 +85,7 @@ int sm_count() {
 struct DecodePlan {
   int bps, nsplit;
   bool cluster;
+  bool head_split;  // kHsHeads heads per CTA, every CTA walks all of its sequence's blocks
 };
 DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t batch) {
   const int max_blocks = (max_seqlen + kTile - 1) / kTile;
@@ -95,11 +97,17 @@ DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t bat
     int ns = (sms + batch - 1) / batch;
     if (ns > count) ns = count;
     const int bps = (count + ns - 1) / ns;
-    return {bps, (count + bps - 1) / bps, false};
+    return {bps, (count + bps - 1) / bps, false, false};
   }
+  // a window of at most 16 blocks and a batch that fills half the GPU or
+  // more with two CTAs per sequence: split the heads, not the blocks, so no
+  // partial results need merging
+  const int per_seq = kDecHeads / kHsHeads;
+  if (count <= 16 && (int64_t)batch * per_seq <= sms && (int64_t)batch * per_seq * 2 > sms)
+    return {count, 1, false, true};
   int ns = 1;
   while (ns < 8 && ns * 2 <= count && (int64_t)batch * ns * 2 <= sms) ns *= 2;
-  return {(count + ns - 1) / ns, ns, true};
+  return {(count + ns - 1) / ns, ns, true, false};
 }
 
 struct DecodeWorkspace {
@@ -107,7 +115,7 @@ struct DecodeWorkspace {
 };
 DecodeWorkspace decode_workspace(int32_t batch, const DecodePlan& plan) {
   DecodeWorkspace w{0, 0, 0, 0};
-  if (plan.cluster) return w;
+  if (plan.cluster || plan.head_split) return w;
   const size_t parts = (size_t)batch * plan.nsplit * kDecHeads;
   w.o_off = 0;
   w.ml_off = parts * 512 * sizeof(float);
@@ -138,7 +146,7 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
   {
     cuuint64_t dims[3] = {576, (cuuint64_t)n_heads, (cuuint64_t)batch};
     cuuint64_t strides[2] = {576 * 2, (cuuint64_t)n_heads * 576 * 2};
-    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)(plan->head_split ? kHsHeads : kDecHeads), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     if (fn(&prm->tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -169,7 +177,12 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
 // Point the kernel at its workspace (unless the plan merges on chip) and launch.
 loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t batch, uint8_t* ws,
                               cudaStream_t st) {
-  if (!plan.cluster) {
+  if (plan.head_split) {
+    if (cudaFuncSetAttribute(ssa_decode_mla_hs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeHsLayout::SMEM_BYTES) != cudaSuccess)
+      return LOZA_ERR_CUDA;
+    ssa_decode_mla_hs_kernel<<<dim3(kDecHeads / kHsHeads, batch), kHsThreads, DecodeHsLayout::SMEM_BYTES, st>>>(prm);
+  } else if (!plan.cluster) {
     const DecodeWorkspace wl = decode_workspace(batch, plan);
     prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
     prm.ws_ml = reinterpret_cast<float4*>(ws + wl.ml_off);

@@ -80,6 +80,27 @@ def test_absorbed_decode_nan_bounds_bitwise(bss, oracle_mod):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("batch", [20, 40, 80])
+def test_absorbed_decode_split_plans(bss, oracle_mod, batch):
+    """Batches whose plans are: 4 CTAs per sequence splitting its blocks (a
+    cluster merging on chip by bulk copies), 2 CTAs splitting its heads (no
+    merge), and 1 CTA per sequence. Some sequences are shorter than the
+    window, so some block splits have no key block at all."""
+    g = synth.rng(70 + batch)
+    lens = g.integers(1, 6000, size=batch)
+    lens[:4] = [1, 129, 700, 2049]
+    absorbed_case(bss, oracle_mod, 71 + batch, lens.tolist(), 6144)
+
+
+def test_absorbed_decode_wide_window_two_splits(bss, oracle_mod):
+    """A 22-block window (s=2, l=20) on 40 sequences: two CTAs of a cluster
+    split each sequence's blocks and merge on chip."""
+    g = synth.rng(90)
+    lens = g.integers(1, 4000, size=40)
+    lens[:3] = [1, 300, 2817]
+    absorbed_case(bss, oracle_mod, 91, lens.tolist(), 4096, n_sink=2, n_local=20)
+
+
 def test_absorbed_dense_decode(bss, oracle_mod):
     absorbed_case(bss, oracle_mod, 63, [1, 700, 5000, 9000], 9216, n_sink=0, n_local=-1)
 
