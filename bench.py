@@ -310,22 +310,26 @@ def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20):
     return res
 
 
-def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None):
+def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None, ctx=None):
     w = synth.WORKLOADS[3]
     g = synth.rng(synth.workload_seed(3))
-    lens = synth.uniform_lengths(g, w["batch"], w["ctx_lo"], w["ctx_hi"]).tolist()
+    lo, hi = (w["ctx_lo"], w["ctx_hi"]) if ctx is None else (ctx // 2, ctx)
+    lens = synth.uniform_lengths(g, w["batch"], lo, hi).tolist()
     if batch is not None:
         lens = lens[:batch]
-    r = run_decode(bss, device, stream, lens, w["ctx_hi"])
+    r = run_decode(bss, device, stream, lens, hi)
     hbm = float(peaks["hbm_gbs"])
     ssa = r["ssa"]
-    out = {"workload": w["name"] if len(lens) == w["batch"] else f"{w['name']} (first {len(lens)} sequences)",
+    name = w["name"] if len(lens) == w["batch"] else f"{w['name']} (first {len(lens)} sequences)"
+    if ctx is not None:
+        name += f" (contexts in [{lo}, {hi}])"
+    out = {"workload": name,
            "metric": "SSA decode GB/s (bytes touched)", "value": ssa["GB/s"], "unit": "GB/s",
            "ms_per_call": ssa["ms"], "bytes_per_call": ssa["bytes"],
            "roofline": {"bound": "hbm", "achieved": ssa["GB/s"], "peak": hbm, "unit": "GB/s",
-                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic("ssa_decode_mla_kernel"),
+                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic("ssa_decode_mla_hs_kernel"),
                         "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
-                        "kernel": "ssa_decode_mla_kernel"},
+                        "kernel": "ssa_decode_mla_hs_kernel"},
            "timing": "mean of per-call CUDA events, L2 flushed (256 MB write) before each call"}
     if "dense" in r:
         d = r["dense"]
@@ -502,7 +506,8 @@ def run_ours(args, rank, world, local_rank):
 
     secondary = {}
     if args.workload in ("default", "all"):
-        secondary["decode"] = decode_secondary(bss, device, stream, peaks, peak_kind, args.decode_batch)
+        secondary["decode"] = decode_secondary(bss, device, stream, peaks, peak_kind, args.decode_batch,
+                                               args.decode_ctx)
     if args.workload in ("long", "all"):
         secondary["long"] = long_secondary(bss, device, stream, peaks)
     if args.workload in ("train", "all"):
@@ -588,6 +593,9 @@ def main():
                     help="prefill length (default: the 32,768-token workload; smaller values serve profiling)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="use only the first N sequences of the decode workload (profiling)")
+    ap.add_argument("--decode-ctx", type=int, default=None,
+                    help="decode contexts in [N/2, N] instead of the workload's (profiling: same bytes per "
+                         "sequence, a smaller cache)")
     ap.add_argument("--train-len", type=int, default=None,
                     help="training workload as one sequence of this length (profiling)")
     ap.add_argument("--workload", choices=["default", "prefill", "long", "train", "all"], default="default",
