@@ -14,6 +14,7 @@
 #include "loza_ssa.h"
 #include "prefill.cuh"
 #include "prefill_pair.cuh"
+#include "prefill_mha2.cuh"
 #include "prefill_mla.cuh"
 #include "decode.cuh"
 #include "decode_mla.cuh"
@@ -280,6 +281,19 @@ loza_status launch_prefill(const PrefillParams& prm, int max_seqlen, int batch, 
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
+// Per-head 192 / 128 prefill, two query tiles per CTA: grid (tile pairs, heads, sequences).
+loza_status launch_prefill_mha2(const PrefillParams& prm, int max_seqlen, int batch, cudaStream_t stream) {
+  using LY = PrefillMha2Layout<192, 128>;
+  auto kern = ssa_prefill_mha2_kernel<192, 128>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM_BYTES) != cudaSuccess)
+    return LOZA_ERR_CUDA;
+  const int tiles = (max_seqlen + kTile - 1) / kTile;
+  dim3 grid((tiles + 1) / 2, prm.n_heads, batch);
+  kern<<<grid, kMha2Threads, LY::SMEM_BYTES, stream>>>(prm);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
 // Absorbed-MLA prefill on CTA pairs: grid x = (head pair, value slice, CTA of
 // the pair), y = query tile, z = sequence; clusters of 2 along x.
 loza_status launch_prefill_pair(const PrefillPairParams& prm, int max_seqlen, int batch, cudaStream_t stream) {
@@ -539,7 +553,7 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
 
   switch (dvt) {
     case 64: return launch_prefill<64, 64, 8>(prm, max_seqlen, batch, st);
-    case 128: return launch_prefill<192, 128, 11>(prm, max_seqlen, batch, st);
+    case 128: return launch_prefill_mha2(prm, max_seqlen, batch, st);
     default: return launch_prefill<576, 256, 5>(prm, max_seqlen, batch, st);
   }
 }

@@ -17,10 +17,14 @@
 //                 O   += P_b V_b      (A = P in TMEM, B = V smem, MN-major)
 //               S is double-buffered in TMEM so S_{b+1} runs while the
 //               softmax works on S_b; P_b overwrites the first half of S_b.
-//   warps 2..5  softmax / correction / epilogue, one query row per thread
-//               (thread <-> TMEM lane). Online softmax in base 2; O is
-//               rescaled in TMEM only when the running max grows by more than
-//               2^8 (otherwise the stale max is kept, which is exact).
+//   warps 2..9  softmax / correction / epilogue, two warps per TMEM lane
+//               quarter (one query row per lane): warp half h computes the
+//               exponentials of keys [64h, 64h+64) and rescales / writes half of
+//               the O columns; both read the whole row of S for the maximum, so
+//               only the row sums are combined (once, at the end). Online
+//               softmax in base 2; O is rescaled in TMEM only when the running
+//               max grows by more than 2^8 (otherwise the stale max is kept,
+//               which is exact).
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+DVT).
 // The value dimension is split into slices of DVT <= 256 columns so that O
@@ -52,7 +56,7 @@ struct PrefillParams {
 
 constexpr int kTile = 128;               // queries per tile == keys per block
 constexpr int kChunkBytes = 128 * 64 * 2;  // one [128 x 64] bf16 tile
-constexpr int kPrefillThreads = 192;
+constexpr int kPrefillThreads = 320;
 constexpr uint32_t kRescaleThreshold = 8;  // log2 units
 
 template <int DQK, int DVT, int NSTAGE>
@@ -61,8 +65,10 @@ struct PrefillLayout {
   static constexpr int NVC = DVT / 64;
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQC * kChunkBytes;
-  static constexpr int BAR_OFF = RING_OFF + NSTAGE * kChunkBytes;
-  // barriers: q_full, ring_full[NSTAGE], ring_empty[NSTAGE], s_full[2], p_full[2], pv_done
+  static constexpr int XCH_OFF = RING_OFF + NSTAGE * kChunkBytes;  // [2][2][128] f32 row sums
+  static constexpr int BAR_OFF = XCH_OFF + 2 * 2 * 128 * 4;
+  // barriers: q_full, ring_full[NSTAGE], ring_empty[NSTAGE], s_full[2], p_full[2], pv_done,
+  // row[4] (the two softmax warps of a lane quarter)
   // (P-ready alternates between two barriers by block parity: a warp that has
   // already finished block b+1 must not count towards block b)
   static constexpr int BAR_Q = 0;
@@ -71,9 +77,10 @@ struct PrefillLayout {
   static constexpr int BAR_S = 1 + 2 * NSTAGE;
   static constexpr int BAR_P = BAR_S + 2;
   static constexpr int BAR_PV = BAR_P + 2;
-  static constexpr int NBAR = BAR_PV + 1;
+  static constexpr int BAR_ROW = BAR_PV + 1;
+  static constexpr int NBAR = BAR_ROW + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base (u32), abort (int)
-  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+  static constexpr int SMEM_BYTES = MISC_OFF + 16;
   static_assert(DQK % 64 == 0 && DVT % 64 == 0 && DVT <= 256, "tile shape");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -93,8 +100,11 @@ template <int DQK, int DVT, int NSTAGE>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
   using LY = PrefillLayout<DQK, DVT, NSTAGE>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(&g_device_status, kErrLayout);
+    return;
+  }
 
   const int qb = blockIdx.x;
   const int head = blockIdx.y / p.dv_slices;
@@ -123,9 +133,10 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     }
     mbar_init(bar(LY::BAR_S + 0), 1);
     mbar_init(bar(LY::BAR_S + 1), 1);
-    mbar_init(bar(LY::BAR_P + 0), 4);  // one arrival per softmax warp
-    mbar_init(bar(LY::BAR_P + 1), 4);
+    mbar_init(bar(LY::BAR_P + 0), 8);  // one arrival per softmax warp
+    mbar_init(bar(LY::BAR_P + 1), 8);
     mbar_init(bar(LY::BAR_PV), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(LY::BAR_ROW + i), 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -238,13 +249,16 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
   } else {
     // ------------------------------------------------------------ softmax / epilogue
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;                  // keys [64*half, +64) of every block
     const int row = quarter * 32 + lane;               // row of the tile == TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int qpos = qb * kTile + row;                  // position inside the sequence
+    float* xl = reinterpret_cast<float*>(smem + LY::XCH_OFF);  // [2][128] exact row sums
+    float* xr = xl + 256;                                       // [2][128] sums of bf16 P
     // m_run: running row maximum of scale*log2(e)*s (the reference of P);
-    // l_run: running sum of 2^(x - m_run) (exact, for the LSE);
-    // r_run: running sum of the bf16-rounded P values that enter P.V, so that
-    //        O is normalised by exactly the weights it was accumulated with.
+    // l_run: this warp's share of the running sum of 2^(x - m_run) (exact, for the LSE);
+    // r_run: its share of the running sum of the bf16-rounded P values that enter
+    //        P.V, so that O is normalised by exactly the weights it was accumulated with.
     float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float c = p.scale_log2;  // > 0, so max(c*s) = c*max(s)
     bool ok = true;
@@ -252,19 +266,30 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       ok = warp_wait(bar(LY::BAR_S + (b & 1)), (b >> 1) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
-      float s[128];
-      tmem_ld128(lane_addr + (b & 1) * 128, s);
+      const uint32_t s_addr = lane_addr + (b & 1) * 128;
+      float so[64], s[64];  // the other warp's keys (maximum only) and this warp's keys
+      tmem_ld64x2(s_addr + 64 * (half ^ 1), s_addr + 64 * half, so, s);
+      // P is stored over S columns holding keys of both warps of the row:
+      // neither stores before its partner warp has loaded S
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(LY::BAR_ROW + quarter));
+      ok = warp_wait(bar(LY::BAR_ROW + quarter), b & 1, abort_flag);
+      if (!ok) break;
       // the diagonal block is token-causal: keys after this row's query do not exist
       if (walk.block(b) == qb) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
-          if (j > row) s[j] = -INFINITY;
+        for (int j = 0; j < 64; ++j) {
+          if (64 * (half ^ 1) + j > row) so[j] = -INFINITY;
+          if (64 * half + j > row) s[j] = -INFINITY;
+        }
       }
       float mx;
       {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int j = 0; j < 64; ++j) m4[j & 3] = fmax3(m4[j & 3], s[2 * j], s[2 * j + 1]);
+        for (int j = 0; j < 32; ++j) m4[j & 3] = fmax3(m4[j & 3], so[2 * j], so[2 * j + 1]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m4[j & 3] = fmax3(m4[j & 3], s[2 * j], s[2 * j + 1]);
         mx = c * fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
       // keep the stale maximum unless this block raises it by more than 2^8
@@ -280,24 +305,19 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       float2 l2[4], r2[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) l2[i] = r2[i] = make_float2(0.f, 0.f);
+      uint32_t pk[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 x = ffma2(make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), c2, nm2);
-          const float p0 = ex2_approx(x.x);
-          const float p1 = ex2_approx(x.y);
-          pk[i] = pack_bf16(p0, p1);
-          l2[i & 3] = fadd2(l2[i & 3], make_float2(p0, p1));
-          r2[i & 3] = fadd2(r2[i & 3], make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u)));
-        }
-        tmem_st32(lane_addr + (b & 1) * 128 + 32 * h, pk);
+      for (int i = 0; i < 32; ++i) {
+        const float2 x = ffma2(make_float2(s[2 * i], s[2 * i + 1]), c2, nm2);
+        const float p0 = ex2_approx(x.x);
+        const float p1 = ex2_approx(x.y);
+        pk[i] = pack_bf16(p0, p1);
+        l2[i & 3] = fadd2(l2[i & 3], make_float2(p0, p1));
+        r2[i & 3] = fadd2(r2[i & 3], make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u)));
       }
-      const float sum = ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
-      const float rsum = ((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y)) + ((r2[2].x + r2[2].y) + (r2[3].x + r2[3].y));
-      l_run = l_run * alpha + sum;
-      r_run = r_run * alpha + rsum;
+      tmem_st32(s_addr + 32 * half, pk);  // P over the first 64 columns of S
+      l_run = l_run * alpha + (((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y)));
+      r_run = r_run * alpha + (((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y)) + ((r2[2].x + r2[2].y) + (r2[3].x + r2[3].y)));
       tmem_st_wait();
       // PV(b-1) is waited every block, after the exponentials (by then it has
       // normally finished): O may then be rescaled before PV(b) runs. The
@@ -309,8 +329,9 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
         if (!ok) break;
         tc_fence_after();
         if (rescale) {
+          // this warp's 32-column units of O: u = half, half + 2, ...
 #pragma unroll 1
-          for (int cc = 0; cc < DVT / 32; ++cc) {
+          for (int cc = half; cc < DVT / 32; cc += 2) {
             float o[32];
             tmem_ld32(lane_addr + 256 + 32 * cc, o);
             uint32_t w[32];
@@ -329,30 +350,43 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     }
     if (ok) ok = warp_wait(bar(LY::BAR_PV), (nb - 1) & 1, abort_flag);
     if (ok) {
+      xl[half * 128 + row] = l_run;
+      xr[half * 128 + row] = r_run;
+    }
+    named_barrier_sync(1, 256);
+    if (ok) {
       tc_fence_after();
-      const float inv = 1.f / r_run;
-      const bool valid = qpos < seq_len;
-      const int64_t grow = (int64_t)seq_start + qpos;
-      __nv_bfloat16* orow = p.out + (grow * p.n_heads + head) * (int64_t)p.d_v + slice * DVT;
+      const float inv = 1.f / (xr[row] + xr[128 + row]);
+      const int64_t grow0 = (int64_t)seq_start + qb * kTile;
+      const int n_valid = min(kTile, seq_len - qb * kTile);
+      // O in 64-column groups g = half, half + 2, ...: each 8-lane group
+      // transposes its 8 rows x 8 chunks of 16 bytes so that every store of
+      // the warp writes four whole 128-byte row segments
+      const int j8 = lane & 7;
+      const int r8 = quarter * 32 + (lane & ~7);  // first row of this lane's group
 #pragma unroll 1
-      for (int cc = 0; cc < DVT / 64; ++cc) {
+      for (int g = half; g < DVT / 64; g += 2) {
         float o[32], o2[32];
-        tmem_ld32(lane_addr + 256 + 64 * cc, o);
-        tmem_ld32(lane_addr + 256 + 64 * cc + 32, o2);
+        tmem_ld32(lane_addr + 256 + 64 * g, o);
+        tmem_ld32(lane_addr + 256 + 64 * g + 32, o2);
         uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           w[i] = pack_bf16(o[2 * i] * inv, o[2 * i + 1] * inv);
           w[16 + i] = pack_bf16(o2[2 * i] * inv, o2[2 * i + 1] * inv);
         }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 64 * cc);
+        transpose8x8_u4(w, lane);  // now chunk j8 of rows r8 .. r8 + 7
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int k = 0; k < 8; ++k) {
+          if (r8 + k < n_valid) {
+            __nv_bfloat16* dst = p.out + ((grow0 + r8 + k) * p.n_heads + head) * (int64_t)p.d_v + slice * DVT +
+                                 64 * g + 8 * j8;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
         }
       }
-      if (valid && slice == 0)
-        p.lse[grow * p.n_heads + head] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      if (half == 0 && qpos < seq_len && slice == 0)
+        p.lse[(grow0 + row) * p.n_heads + head] = (m_run + log2f(xl[row] + xl[128 + row])) * 0.69314718055994530942f;
     }
   }
 

@@ -88,6 +88,17 @@ def test_other_windows(bss, oracle_mod, n_sink, n_local):
     assert_close_lse(l, l_ref, f"s={n_sink} l={n_local}")
 
 
+@pytest.mark.parametrize("n_sink,n_local", [(0, -1), (2, 3), (1, 1), (0, 2)])
+def test_nonabsorbed_192_128_windows(bss, oracle_mod, n_sink, n_local):
+    """192 / 128 (two query tiles per CTA over the union of their windows)
+    with the unbounded window, several sinks, a window of one block and no
+    sink; odd and even tile counts, a 1-row last tile."""
+    o, o_ref, l, l_ref = run_case(bss, oracle_mod, 39, [1665, 257, 900], 2, 2, 192, 128, 1 / math.sqrt(192),
+                                  n_sink, n_local)
+    assert_close_o(o, o_ref, f"192/128 s={n_sink} l={n_local}")
+    assert_close_lse(l, l_ref, f"192/128 s={n_sink} l={n_local}")
+
+
 @pytest.mark.parametrize("n_sink,n_local", [(0, -1), (2, 3)])
 def test_absorbed_other_windows(bss, oracle_mod, n_sink, n_local):
     """Absorbed shapes (CTA-pair kernel: even head count) with the unbounded and a (2, 3) window."""
