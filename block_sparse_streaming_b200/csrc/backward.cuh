@@ -76,9 +76,16 @@ __global__ void __launch_bounds__(256) ssa_bwd_preprocess(const __nv_bfloat16* _
 
 // ---------------------------------------------------------------------------
 // dQ: one CTA per (query tile, head, sequence).
-// TMEM: S [0,128) (dS packed into [0,64)), dP [128,256), dQ [256, 256+DQK).
-// Ring order per key block: K (DQK/64 tiles, for S), V (DV/64, for dP), K again (for dQ).
+// TMEM: S [0,128), dP [128,256), dQ [256, 256+DQK), dS (bf16, packed) [448,512).
+// dS has columns of its own, so the MMAs of block b+1 (S, dP) are issued as
+// soon as the elementwise warps have read S(b) and dP(b), and run while they
+// compute dS(b); dQ(b) follows. Ring order: K(0) V(0), then per block b:
+// K(b+1) V(b+1) (for S, dP) and K(b) again (for dQ), as the MMAs consume them.
+// Warps: 0 TMA producer, 1 TMEM allocation + MMA issuer, 2-9 elementwise
+// (two per TMEM lane quarter, 64 keys each).
 // ---------------------------------------------------------------------------
+constexpr int kBwdDqThreads = 320;
+
 template <int DQK, int DV>
 struct BwdDqLayout {
   static constexpr int NQC = DQK / 64, NVC = DV / 64, NSTAGE = 8;
@@ -87,18 +94,22 @@ struct BwdDqLayout {
   static constexpr int RING_OFF = DO_OFF + NVC * kChunkBytes;
   static constexpr int BAR_OFF = RING_OFF + NSTAGE * kChunkBytes;
   static constexpr int BAR_IN = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NSTAGE, BAR_DP = 1 + 2 * NSTAGE,
-                       BAR_DS = BAR_DP + 1, BAR_DQ = BAR_DS + 1, NBAR = BAR_DQ + 1;
+                       BAR_FREE = BAR_DP + 1, BAR_DS = BAR_FREE + 1, BAR_DQ = BAR_DS + 1, NBAR = BAR_DQ + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16;
+  static constexpr int T_DS = 448;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(256 + DQK <= 512, "TMEM budget");
+  static_assert(256 + DQK <= T_DS, "TMEM budget");
 };
 
 template <int DQK, int DV>
-__global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kBwdDqThreads, 1) ssa_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   using LY = BwdDqLayout<DQK, DV>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(&g_device_status, kErrLayout);
+    return;
+  }
   const int qb = blockIdx.x, head = blockIdx.y, seq = blockIdx.z;
   const int seq_start = p.cu_seqlens[seq];
   const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
@@ -119,7 +130,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
       mbar_init(bar(LY::BAR_EMPTY + i), 1);
     }
     mbar_init(bar(LY::BAR_DP), 1);
-    mbar_init(bar(LY::BAR_DS), 4);  // one arrival per softmax warp
+    mbar_init(bar(LY::BAR_FREE), 8);  // one arrival per elementwise warp
+    mbar_init(bar(LY::BAR_DS), 8);
     mbar_init(bar(LY::BAR_DQ), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -144,20 +156,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
       int slot = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int b = 0; b < nb && ok; ++b) {
-        const int krow = seq_start + walk.block(b) * kTile;
-        for (int t = 0; t < 2 * LY::NQC + LY::NVC && ok; ++t) {
-          ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
-          if (!ok) break;
-          mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
-          const uint32_t dst = sbase + LY::RING_OFF + slot * kChunkBytes;
-          if (t < LY::NQC)
-            tma_load_3d(dst, &p.tm_k, bar(LY::BAR_FULL + slot), t * 64, head, krow);
-          else if (t < LY::NQC + LY::NVC)
-            tma_load_3d(dst, &p.tm_v, bar(LY::BAR_FULL + slot), (t - LY::NQC) * 64, head, krow);
-          else
-            tma_load_3d(dst, &p.tm_k, bar(LY::BAR_FULL + slot), (t - LY::NQC - LY::NVC) * 64, head, krow);
-          if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+      auto load = [&](const CUtensorMap* map, int col, int row) {
+        ok = mbar_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
+        if (!ok) return;
+        mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), kChunkBytes);
+        tma_load_3d(sbase + LY::RING_OFF + slot * kChunkBytes, map, bar(LY::BAR_FULL + slot), col, head, row);
+        if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+      };
+      for (int b = 0; b <= nb && ok; ++b) {
+        if (b < nb) {
+          const int krow = seq_start + walk.block(b) * kTile;
+          for (int c = 0; c < LY::NQC && ok; ++c) load(&p.tm_k, c * 64, krow);
+          for (int c = 0; c < LY::NVC && ok; ++c) load(&p.tm_v, c * 64, krow);
+        }
+        if (b >= 1) {
+          const int krow = seq_start + walk.block(b - 1) * kTile;
+          for (int c = 0; c < LY::NQC && ok; ++c) load(&p.tm_k, c * 64, krow);
         }
       }
     }
@@ -165,17 +179,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
     // whole warp walks the schedule; one elected lane issues each tcgen05 instruction
     constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);
     constexpr uint32_t idesc_dq = idesc_bf16(128, 64, false, true);
-    const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+    const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256, t_ds = tmem + LY::T_DS;
     int slot = 0;
     uint32_t phase = 0;
     bool ok = warp_wait(bar(LY::BAR_IN), 0, abort_flag);
     tc_fence_after();
-    for (int b = 0; b < nb && ok; ++b) {
-      // S = Q K^T
+    auto next_full = [&]() {
+      ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
+      if (ok) tc_fence_after();
+      return ok;
+    };
+    auto advance = [&]() {
+      if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+    };
+    // S = Q K^T and dP = dO V^T of the next block
+    auto issue_s_dp = [&]() {
       for (int c = 0; c < LY::NQC && ok; ++c) {
-        ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
+        if (!next_full()) break;
         if (elect_one()) {
           const uint32_t a = sbase + LY::Q_OFF + c * kChunkBytes, bb = sbase + LY::RING_OFF + slot * kChunkBytes;
 #pragma unroll
@@ -185,13 +205,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
           mma_commit(bar(LY::BAR_EMPTY + slot));
         }
         __syncwarp();
-        if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+        advance();
       }
-      // dP = dO V^T
       for (int c = 0; c < LY::NVC && ok; ++c) {
-        ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
+        if (!next_full()) break;
         if (elect_one()) {
           const uint32_t a = sbase + LY::DO_OFF + c * kChunkBytes, bb = sbase + LY::RING_OFF + slot * kChunkBytes;
 #pragma unroll
@@ -201,29 +218,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
           mma_commit(bar(LY::BAR_EMPTY + slot));
         }
         __syncwarp();
-        if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+        advance();
       }
-      if (!ok) break;
-      if (elect_one()) mma_commit(bar(LY::BAR_DP));
+      if (ok && elect_one()) mma_commit(bar(LY::BAR_DP));
       __syncwarp();
+    };
+    if (ok) issue_s_dp();
+    for (int b = 0; b < nb && ok; ++b) {
+      if (b + 1 < nb) {
+        // S(b), dP(b) have been read: the next block's products may overwrite them
+        ok = warp_wait(bar(LY::BAR_FREE), b & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s_dp();
+        if (!ok) break;
+      }
       ok = warp_wait(bar(LY::BAR_DS), b & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       // dQ += dS K  (A = dS in TMEM, B = K tiles MN-major)
       for (int c = 0; c < LY::NQC && ok; ++c) {
-        ok = warp_wait(bar(LY::BAR_FULL + slot), phase, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
+        if (!next_full()) break;
         if (elect_one()) {
           const uint32_t bb = sbase + LY::RING_OFF + slot * kChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(t_dq + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_dq,
+            mma_ts(t_dq + 64 * c, t_ds + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_dq,
                    (b > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(LY::BAR_EMPTY + slot));
         }
         __syncwarp();
-        if (++slot == LY::NSTAGE) { slot = 0; phase ^= 1; }
+        advance();
       }
       if (!ok) break;
       if (elect_one()) mma_commit(bar(LY::BAR_DQ));
@@ -231,6 +256,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
     }
   } else {
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // keys [64*half, +64)
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int qpos = qb * kTile + row;
@@ -238,32 +264,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
     const int64_t grow = (int64_t)seq_start + qpos;
     const float lse2 = valid ? p.lse[grow * p.n_heads + head] * 1.4426950408889634f : 0.f;
     const float dd = valid ? p.dvec[grow * p.n_heads + head] : 0.f;
+    const float c2 = p.scale_log2;
     bool ok = true;
     for (int b = 0; b < nb && ok; ++b) {
       ok = warp_wait(bar(LY::BAR_DP), b & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
+      float s[64], dp[64];
+      tmem_ld64x2(lane_addr + 64 * half, lane_addr + 128 + 64 * half, s, dp);
+      // S(b) and dP(b) are in registers: the MMAs of the next block may start
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(LY::BAR_FREE));
       const bool diag = walk.block(b) == qb;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float s[32], dp[32];
-        tmem_ld32(lane_addr + 32 * c, s);
-        tmem_ld32(lane_addr + 128 + 32 * c, dp);
-        uint32_t pk[16];
+      uint32_t pk[2][16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float ds2[2];
+      for (int i = 0; i < 32; ++i) {
+        float ds2[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int key = 32 * c + 2 * i + e;
-            float pr = exp2f(s[2 * i + e] * p.scale_log2 - lse2);
-            if (diag && key > row) pr = 0.f;
-            ds2[e] = pr * (dp[2 * i + e] - dd);
-          }
-          pk[i] = pack_bf16(ds2[0], ds2[1]);
+        for (int e = 0; e < 2; ++e) {
+          const int key = 64 * half + 2 * i + e;
+          float pr = ex2_approx(fmaf(s[2 * i + e], c2, -lse2));
+          if (diag && key > row) pr = 0.f;
+          ds2[e] = pr * (dp[2 * i + e] - dd);
         }
-        tmem_st16(lane_addr + 16 * c, pk);
+        pk[i >> 4][i & 15] = pack_bf16(ds2[0], ds2[1]);
       }
+      // dQ(b-1) has read dS(b-1) (phases waited in order)
+      if (b > 0) {
+        ok = warp_wait(bar(LY::BAR_DQ), (b - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      tmem_st16(lane_addr + LY::T_DS + 32 * half, pk[0]);
+      tmem_st16(lane_addr + LY::T_DS + 32 * half + 16, pk[1]);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -272,18 +306,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dq_kernel(const __grid
     if (ok) ok = warp_wait(bar(LY::BAR_DQ), (nb - 1) & 1, abort_flag);
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* dst = p.dq + (grow * p.n_heads + head) * (int64_t)DQK;
+      const int64_t grow0 = (int64_t)seq_start + qb * kTile;
+      const int n_valid = min(kTile, seq_len - qb * kTile);
+      // dQ in 64-column groups g = half, half + 2, ...: each 8-lane group
+      // transposes its 8 rows x 8 chunks of 16 bytes so that every store of
+      // the warp writes four whole 128-byte row segments
+      const int j8 = lane & 7;
+      const int r8 = quarter * 32 + (lane & ~7);
 #pragma unroll 1
-      for (int c = 0; c < DQK / 32; ++c) {
-        float o[32];
-        tmem_ld32(lane_addr + 256 + 32 * c, o);
-        uint32_t w[16];
+      for (int g = half; g < DQK / 64; g += 2) {
+        float o[32], o2[32];
+        tmem_ld32(lane_addr + 256 + 64 * g, o);
+        tmem_ld32(lane_addr + 256 + 64 * g + 32, o2);
+        uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * p.scale, o[2 * i + 1] * p.scale);
-        if (valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+        for (int i = 0; i < 16; ++i) {
+          w[i] = pack_bf16(o[2 * i] * p.scale, o[2 * i + 1] * p.scale);
+          w[16 + i] = pack_bf16(o2[2 * i] * p.scale, o2[2 * i + 1] * p.scale);
+        }
+        transpose8x8_u4(w, lane);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int k = 0; k < 8; ++k) {
+          if (r8 + k < n_valid) {
+            __nv_bfloat16* dst = p.dq + ((grow0 + r8 + k) * p.n_heads + head) * (int64_t)DQK + 64 * g + 8 * j8;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
         }
       }
     }

@@ -253,7 +253,7 @@ loza_status launch_backward(BwdParams& prm, const void* out, const void* dout, i
                            LK::SMEM_BYTES) != cudaSuccess)
     return LOZA_ERR_CUDA;
   prm.far_mode = 0;
-  ssa_bwd_dq_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdThreads, LQ::SMEM_BYTES, st>>>(prm);
+  ssa_bwd_dq_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdDqThreads, LQ::SMEM_BYTES, st>>>(prm);
   ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdThreads, LK::SMEM_BYTES, st>>>(prm);
   g_launches.fetch_add(2, std::memory_order_relaxed);
   if (prm.n_sink > 0) {
