@@ -354,12 +354,14 @@ struct BwdDkvLayout {
   static constexpr int NQC = DQK / 64, NVC = DV / 64;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = NQC * kChunkBytes;
-  static constexpr int Q_OFF = V_OFF + NVC * kChunkBytes;
-  static constexpr int DO_OFF = Q_OFF + NQC * kChunkBytes;
+  static constexpr int Q_OFF = V_OFF + NVC * kChunkBytes;       // [2 buffers][NQC] tiles
+  static constexpr int DO_OFF = Q_OFF + 2 * NQC * kChunkBytes;
   static constexpr int STAT_OFF = DO_OFF + NVC * kChunkBytes;  // lse2[128], d[128]
   static constexpr int BAR_OFF = STAT_OFF + 2 * 128 * 4;
-  static constexpr int BAR_KV = 0, BAR_QD = 1, BAR_QD_EMPTY = 2, BAR_S = 3, BAR_P = 4, BAR_DP = 5, BAR_DS = 6,
-                       NBAR = 7;
+  // Q of query block j goes to buffer j & 1 and is released after dK(j); dO
+  // is single-buffered and released after dV(j) and dP^T(j) have read it
+  static constexpr int BAR_KV = 0, BAR_Q = 1 /* [2] */, BAR_QE = 3 /* [2] */, BAR_DO = 5, BAR_DOE = 6, BAR_S = 7,
+                       BAR_P = 8, BAR_DP = 9, BAR_DS = 10, NBAR = 11;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr int T_DV = 192, T_DK = 192 + DV;
@@ -417,8 +419,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
 
   if (threadIdx.x == 0) {
     mbar_init(bar(LY::BAR_KV), 1);
-    mbar_init(bar(LY::BAR_QD), 1);
-    mbar_init(bar(LY::BAR_QD_EMPTY), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(LY::BAR_Q + i), 1);
+      mbar_init(bar(LY::BAR_QE + i), 1);
+    }
+    mbar_init(bar(LY::BAR_DO), 1);
+    mbar_init(bar(LY::BAR_DOE), 1);
     mbar_init(bar(LY::BAR_S), 1);
     mbar_init(bar(LY::BAR_P), 4);  // one arrival per softmax warp
     mbar_init(bar(LY::BAR_DP), 1);
@@ -445,14 +451,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
         tma_load_3d(sbase + LY::V_OFF + c * kChunkBytes, &p.tm_v, bar(LY::BAR_KV), c * 64, head, krow);
       bool ok = true;
       for (int jj = 0; jj < nj && ok; ++jj) {
-        ok = mbar_wait(bar(LY::BAR_QD_EMPTY), (jj & 1) ^ 1, abort_flag);
-        if (!ok) break;
         const int qrow = seq_start + (j_lo + jj) * kTile;
-        mbar_arrive_expect_tx(bar(LY::BAR_QD), (LY::NQC + LY::NVC) * kChunkBytes);
+        const int qbuf = jj & 1;
+        ok = mbar_wait(bar(LY::BAR_QE + qbuf), ((jj >> 1) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(LY::BAR_Q + qbuf), LY::NQC * kChunkBytes);
         for (int c = 0; c < LY::NQC; ++c)
-          tma_load_3d(sbase + LY::Q_OFF + c * kChunkBytes, &p.tm_q, bar(LY::BAR_QD), c * 64, head, qrow);
+          tma_load_3d(sbase + LY::Q_OFF + (qbuf * LY::NQC + c) * kChunkBytes, &p.tm_q, bar(LY::BAR_Q + qbuf), c * 64,
+                      head, qrow);
+        ok = mbar_wait(bar(LY::BAR_DOE), (jj & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(LY::BAR_DO), LY::NVC * kChunkBytes);
         for (int c = 0; c < LY::NVC; ++c)
-          tma_load_3d(sbase + LY::DO_OFF + c * kChunkBytes, &p.tm_do, bar(LY::BAR_QD), c * 64, head, qrow);
+          tma_load_3d(sbase + LY::DO_OFF + c * kChunkBytes, &p.tm_do, bar(LY::BAR_DO), c * 64, head, qrow);
       }
     }
   } else if (warp == 1) {
@@ -462,13 +473,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
     const uint32_t t_s = tmem, t_dp = tmem + 64, t_dv = tmem + LY::T_DV, t_dk = tmem + LY::T_DK;
     bool ok = warp_wait(bar(LY::BAR_KV), 0, abort_flag);
     for (int jj = 0; jj < nj && ok; ++jj) {
-      ok = warp_wait(bar(LY::BAR_QD), jj & 1, abort_flag);
+      const int qbuf = jj & 1;
+      const uint32_t q_off = sbase + LY::Q_OFF + qbuf * LY::NQC * kChunkBytes;
+      ok = warp_wait(bar(LY::BAR_Q + qbuf), (jj >> 1) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       // S^T = K Q^T
       if (elect_one()) {
       for (int c = 0; c < LY::NQC; ++c) {
-        const uint32_t a = sbase + LY::K_OFF + c * kChunkBytes, bb = sbase + LY::Q_OFF + c * kChunkBytes;
+        const uint32_t a = sbase + LY::K_OFF + c * kChunkBytes, bb = q_off + c * kChunkBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(t_s, sdesc_sw128(a + 32 * kk, 16, 1024), sdesc_sw128(bb + 32 * kk, 16, 1024), idesc_ss,
@@ -477,7 +490,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       mma_commit(bar(LY::BAR_S));
       }
       __syncwarp();
-      ok = warp_wait(bar(LY::BAR_P), jj & 1, abort_flag);
+      ok = warp_wait(bar(LY::BAR_P), jj & 1, abort_flag) && warp_wait(bar(LY::BAR_DO), jj & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       // dV += P^T dO   (A = P^T in TMEM, B = dO tiles MN-major)
@@ -498,6 +511,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
                  (c | kk) != 0);
       }
       mma_commit(bar(LY::BAR_DP));
+      mma_commit(bar(LY::BAR_DOE));  // dO read by dV and dP^T
       }
       __syncwarp();
       ok = warp_wait(bar(LY::BAR_DS), jj & 1, abort_flag);
@@ -506,13 +520,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       // dK += dS^T Q   (A = dS^T in TMEM, B = Q tiles MN-major)
       if (elect_one()) {
       for (int c = 0; c < LY::NQC; ++c) {
-        const uint32_t bb = sbase + LY::Q_OFF + c * kChunkBytes;
+        const uint32_t bb = q_off + c * kChunkBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(t_dk + 64 * c, t_s + 8 * kk, sdesc_sw128(bb + 2048 * kk, 8192, 1024), idesc_ts,
                  (jj > 0 || kk > 0) ? 1u : 0u);
       }
-      mma_commit(bar(LY::BAR_QD_EMPTY));
+      mma_commit(bar(LY::BAR_QE + qbuf));  // Q(j) no longer read
       }
       __syncwarp();
     }
@@ -545,7 +559,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int col = 32 * c + i;  // query row of block j
-          float v = exp2f(s[i] * p.scale_log2 - s_lse2[col]);
+          float v = ex2_approx(fmaf(s[i], p.scale_log2, -s_lse2[col]));
           if (diag && col < key) v = 0.f;
           pr[col] = v;
         }
@@ -584,7 +598,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       if (lane == 0) mbar_arrive(bar(LY::BAR_DS));  // one arrival per warp
       named_barrier_sync(1, 128);  // statistics of block j no longer read
     }
-    if (ok) ok = warp_wait(bar(LY::BAR_QD_EMPTY), (nj - 1) & 1, abort_flag);
+    if (ok) ok = warp_wait(bar(LY::BAR_QE + ((nj - 1) & 1)), ((nj - 1) >> 1) & 1, abort_flag);  // last dK done
     if (ok) {
       tc_fence_after();
       const int kpos = kblk * kTile + key;
