@@ -25,7 +25,7 @@
 
 namespace loza {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdDkvThreads = 320;  // producer, MMA, 8 elementwise warps
 constexpr int kSinkChunk = 256;  // far query blocks per sink-partial CTA
 
 struct BwdParams {
@@ -361,7 +361,7 @@ struct BwdDkvLayout {
   // Q of query block j goes to buffer j & 1 and is released after dK(j); dO
   // is single-buffered and released after dV(j) and dP^T(j) have read it
   static constexpr int BAR_KV = 0, BAR_Q = 1 /* [2] */, BAR_QE = 3 /* [2] */, BAR_DO = 5, BAR_DOE = 6, BAR_S = 7,
-                       BAR_P = 8, BAR_DP = 9, BAR_DS = 10, NBAR = 11;
+                       BAR_P = 8, BAR_DP = 9, BAR_DS = 10, BAR_ROW = 11 /* [4] */, NBAR = 15;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr int T_DV = 192, T_DK = 192 + DV;
@@ -370,7 +370,7 @@ struct BwdDkvLayout {
 };
 
 template <int DQK, int DV>
-__global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kBwdDkvThreads, 1) ssa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using LY = BwdDkvLayout<DQK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -426,9 +426,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
     mbar_init(bar(LY::BAR_DO), 1);
     mbar_init(bar(LY::BAR_DOE), 1);
     mbar_init(bar(LY::BAR_S), 1);
-    mbar_init(bar(LY::BAR_P), 4);  // one arrival per softmax warp
+    mbar_init(bar(LY::BAR_P), 8);  // one arrival per elementwise warp
     mbar_init(bar(LY::BAR_DP), 1);
-    mbar_init(bar(LY::BAR_DS), 4);
+    mbar_init(bar(LY::BAR_DS), 8);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(LY::BAR_ROW + i), 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -531,14 +532,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       __syncwarp();
     }
   } else {
+    // elementwise: two warps per TMEM lane quarter, warp half h takes the
+    // queries [64h, 64h+64) of every key row
     const int quarter = warp & 3;
-    const int tid = threadIdx.x - 64;
+    const int half = (warp - 2) >> 2;
+    const int tid = threadIdx.x - 64;     // 0..255
     const int key = quarter * 32 + lane;  // TMEM lane == key row of the block
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
     for (int jj = 0; jj < nj && ok; ++jj) {
       const int j = j_lo + jj;
-      {
+      if (tid < 128) {
         // per-query statistics of block j (invalid rows: P = 0, D = 0)
         const int qpos = j * kTile + tid;
         const bool v = qpos < seq_len;
@@ -546,30 +550,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
         s_lse2[tid] = v ? p.lse[g * p.n_heads + head] * 1.4426950408889634f : INFINITY;
         s_d[tid] = v ? p.dvec[g * p.n_heads + head] : 0.f;
       }
-      named_barrier_sync(1, 128);
+      named_barrier_sync(1, 256);
       ok = warp_wait(bar(LY::BAR_S), jj & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const bool diag = (j == kblk);
-      float pr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float s[32];
-        tmem_ld32(lane_addr + 32 * c, s);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = 32 * c + i;  // query row of block j
-          float v = ex2_approx(fmaf(s[i], p.scale_log2, -s_lse2[col]));
-          if (diag && col < key) v = 0.f;
-          pr[col] = v;
-        }
-      }
+      float pr[64];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
+        float sx[32];
+        tmem_ld32(lane_addr + 64 * half + 32 * c, sx);
+        const float4* l4 = reinterpret_cast<const float4*>(s_lse2 + 64 * half + 32 * c);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 l = l4[i4];
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 32 * c + 4 * i4 + e;
+            const int col = 64 * half + i;  // query row of block j
+            float v = ex2_approx(fmaf(sx[4 * i4 + e], p.scale_log2, -lv[e]));
+            if (diag && col < key) v = 0.f;
+            pr[i] = v;
+          }
+        }
+      }
+      // P^T is stored over S^T columns holding queries of both warps of the
+      // row: neither stores before its partner has loaded S^T
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(LY::BAR_ROW + quarter));
+      ok = warp_wait(bar(LY::BAR_ROW + quarter), jj & 1, abort_flag);
+      if (!ok) break;
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(pr[64 * c + 2 * i], pr[64 * c + 2 * i + 1]);
-        tmem_st32(lane_addr + 32 * c, pk);
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(pr[2 * i], pr[2 * i + 1]);
+        tmem_st32(lane_addr + 32 * half, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -579,77 +595,81 @@ __global__ void __launch_bounds__(kBwdThreads, 1) ssa_bwd_dkdv_kernel(const __gr
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float dp[32];
-        tmem_ld32(lane_addr + 64 + 32 * c, dp);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pr[32 * c + i] = pr[32 * c + i] * (dp[i] - s_d[32 * c + i]);
-      }
-#pragma unroll
       for (int c = 0; c < 2; ++c) {
+        float dx[32];
+        tmem_ld32(lane_addr + 64 + 64 * half + 32 * c, dx);
+        const float4* d4 = reinterpret_cast<const float4*>(s_d + 64 * half + 32 * c);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 d = d4[i4];
+          const float dv4[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pr[32 * c + 4 * i4 + e] *= dx[4 * i4 + e] - dv4[e];
+        }
+      }
+      {
+        // dS^T over this warp's own P^T columns (dV and dP^T have read P^T)
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(pr[64 * c + 2 * i], pr[64 * c + 2 * i + 1]);
-        tmem_st32(lane_addr + 32 * c, pk);
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(pr[2 * i], pr[2 * i + 1]);
+        tmem_st32(lane_addr + 32 * half, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(LY::BAR_DS));  // one arrival per warp
-      named_barrier_sync(1, 128);  // statistics of block j no longer read
+      named_barrier_sync(1, 256);  // statistics of block j no longer read
     }
     if (ok) ok = warp_wait(bar(LY::BAR_QE + ((nj - 1) & 1)), ((nj - 1) >> 1) & 1, abort_flag);  // last dK done
     if (ok) {
       tc_fence_after();
-      const int kpos = kblk * kTile + key;
-      const bool valid = kpos < seq_len;
-      const int64_t g = (int64_t)seq_start + kpos;
+      const int64_t g0 = (int64_t)seq_start + kblk * kTile;
+      const int n_valid = min(kTile, seq_len - kblk * kTile);
       if (part) {
+        // fp32 partials, row `key`: dK columns [0, DQK), dV columns [DQK, DQK+DV);
+        // this warp takes the 32-column units u = half, half + 2, ...
         float* prow = part + (int64_t)key * (DQK + DV);
 #pragma unroll 1
-        for (int c = 0; c < DQK / 32; ++c) {
+        for (int u = half; u < (DQK + DV) / 32; u += 2) {
           float o[32];
-          tmem_ld32(lane_addr + LY::T_DK + 32 * c, o);
+          const bool is_k = u < DQK / 32;
+          tmem_ld32(lane_addr + (is_k ? LY::T_DK + 32 * u : LY::T_DV + 32 * u - DQK), o);
+          const float sc = is_k ? p.scale : 1.f;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(prow + 32 * c + i) =
-                make_float4(o[i] * p.scale, o[i + 1] * p.scale, o[i + 2] * p.scale, o[i + 3] * p.scale);
-        }
-#pragma unroll 1
-        for (int c = 0; c < DV / 32; ++c) {
-          float o[32];
-          tmem_ld32(lane_addr + LY::T_DV + 32 * c, o);
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(prow + DQK + 32 * c + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+            *reinterpret_cast<float4*>(prow + 32 * u + i) =
+                make_float4(o[i] * sc, o[i + 1] * sc, o[i + 2] * sc, o[i + 3] * sc);
         }
       } else {
-        __nv_bfloat16* dkr = p.dk + (g * p.n_heads + head) * (int64_t)DQK;
-        __nv_bfloat16* dvr = p.dv + (g * p.n_heads + head) * (int64_t)DV;
+        // bf16 dK, dV in 64-column groups (dK groups, then dV groups; this warp
+        // takes g = half, half + 2, ...): each 8-lane group transposes its 8
+        // rows x 8 chunks of 16 bytes so every store writes whole 128-byte segments
+        const int j8 = lane & 7;
+        const int r8 = quarter * 32 + (lane & ~7);
 #pragma unroll 1
-        for (int c = 0; c < DQK / 32; ++c) {
-          float o[32];
-          tmem_ld32(lane_addr + LY::T_DK + 32 * c, o);
-          uint32_t w[16];
+        for (int gi = half; gi < (DQK + DV) / 64; gi += 2) {
+          const bool is_k = gi < DQK / 64;
+          const int g = is_k ? gi : gi - DQK / 64;
+          const uint32_t col = is_k ? LY::T_DK + 64 * g : LY::T_DV + 64 * g;
+          const float sc = is_k ? p.scale : 1.f;
+          float o[32], o2[32];
+          tmem_ld32(lane_addr + col, o);
+          tmem_ld32(lane_addr + col + 32, o2);
+          uint32_t w[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * p.scale, o[2 * i + 1] * p.scale);
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dkr + 32 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < 16; ++i) {
+            w[i] = pack_bf16(o[2 * i] * sc, o[2 * i + 1] * sc);
+            w[16 + i] = pack_bf16(o2[2 * i] * sc, o2[2 * i + 1] * sc);
           }
-        }
-#pragma unroll 1
-        for (int c = 0; c < DV / 32; ++c) {
-          float o[32];
-          tmem_ld32(lane_addr + LY::T_DV + 32 * c, o);
-          uint32_t w[16];
+          transpose8x8_u4(w, lane);
+          __nv_bfloat16* base = is_k ? p.dk : p.dv;
+          const int width = is_k ? DQK : DV;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i], o[2 * i + 1]);
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dvr + 32 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int k = 0; k < 8; ++k) {
+            if (r8 + k < n_valid) {
+              __nv_bfloat16* dst = base + ((g0 + r8 + k) * p.n_heads + head) * (int64_t)width + 64 * g + 8 * j8;
+              *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            }
           }
         }
       }

@@ -254,12 +254,12 @@ loza_status launch_backward(BwdParams& prm, const void* out, const void* dout, i
     return LOZA_ERR_CUDA;
   prm.far_mode = 0;
   ssa_bwd_dq_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdDqThreads, LQ::SMEM_BYTES, st>>>(prm);
-  ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdThreads, LK::SMEM_BYTES, st>>>(prm);
+  ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdDkvThreads, LK::SMEM_BYTES, st>>>(prm);
   g_launches.fetch_add(2, std::memory_order_relaxed);
   if (prm.n_sink > 0) {
     if (prm.nslots > 1) {
       prm.far_mode = 1;
-      ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(prm.nslots - 1, prm.n_heads * prm.n_sink, batch), kBwdThreads,
+      ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(prm.nslots - 1, prm.n_heads * prm.n_sink, batch), kBwdDkvThreads,
                                      LK::SMEM_BYTES, st>>>(prm);
       g_launches.fetch_add(1, std::memory_order_relaxed);
     }
