@@ -68,10 +68,12 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(files=None):
+    """sha256 (first 16 hex digits) of the given csrc/ files, in sorted order,
+    or of every file in csrc/ when none are given."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_streaming_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files if files else os.listdir(csrc)):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -84,7 +86,7 @@ def profiled_traffic(kernel_key):
         return None
     d = json.load(open(p))
     e = d.get(kernel_key)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("source_files")):
         return None
     return e.get("dram_bytes_per_launch")
 
