@@ -68,6 +68,10 @@ def _load():
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
             _i64p, ctypes.c_int64, _i64p, ctypes.c_int64,
             _f64p, _f64p, _f64p]
+        lib.ssa_oracle_merge.restype = ctypes.c_int
+        lib.ssa_oracle_merge.argtypes = [_u16p, _f64p, _u16p, _f64p, ctypes.c_int64, ctypes.c_int, _f64p, _f64p]
+        lib.ssa_oracle_mix.restype = ctypes.c_int
+        lib.ssa_oracle_mix.argtypes = [_u16p, _u16p, ctypes.c_int64, ctypes.c_double, _f64p]
         lib.ssa_oracle_visible_count.restype = ctypes.c_int64
         lib.ssa_oracle_visible_count.argtypes = [
             ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
@@ -154,3 +158,31 @@ def backward(q, k, v, dout, cu_seqlens, n_heads, n_kv_heads, block_size=128,
 def visible_count(i, block_size=128, n_sink=1, n_local=7) -> int:
     """|A(i)| under the oracle's block-index map."""
     return int(_load().ssa_oracle_visible_count(int(i), block_size, n_sink, n_local))
+
+
+def merge(o_a, lse_a, o_b, lse_b):
+    """Attention over the union of two disjoint key sets from the two branches'
+    (O, LSE): O [rows, d_v] bf16 bits, LSE [rows] (natural log; -inf = no
+    keys). Returns O [rows, d_v] and LSE [rows] as float64."""
+    o_a, o_b = _u16(o_a), _u16(o_b)
+    if o_a.shape != o_b.shape or o_a.ndim != 2:
+        raise ValueError("merge takes two [rows, d_v] outputs of one shape")
+    rows, d_v = o_a.shape
+    la = np.ascontiguousarray(lse_a, dtype=np.float64).reshape(rows)
+    lb = np.ascontiguousarray(lse_b, dtype=np.float64).reshape(rows)
+    o = np.zeros((rows, d_v), np.float64)
+    lse = np.zeros(rows, np.float64)
+    if _load().ssa_oracle_merge(o_a, la, o_b, lb, rows, d_v, o, lse) != 0:
+        raise ValueError("oracle merge rejected its arguments")
+    return o, lse
+
+
+def mix(o_full, o_ssa, alpha):
+    """alpha * O_full + (1 - alpha) * O_ssa, elementwise, float64."""
+    a, b = _u16(o_full), _u16(o_ssa)
+    if a.shape != b.shape:
+        raise ValueError("mix takes two outputs of one shape")
+    o = np.zeros(a.shape, np.float64)
+    if _load().ssa_oracle_mix(a.reshape(-1), b.reshape(-1), a.size, float(alpha), o.reshape(-1)) != 0:
+        raise ValueError("oracle mix rejected its arguments")
+    return o

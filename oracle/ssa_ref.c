@@ -341,3 +341,46 @@ int64_t ssa_oracle_visible_count(int64_t i, int block_size, int n_sink, int n_lo
     free(keys);
     return c;
 }
+
+/*
+ * Combining two attention branches of one query (an adjacent step of the same
+ * operator; page 1 section 01 (1) "calibration": during calibration an MLA
+ * module's output is a weighted mix of its full-attention branch and its
+ * sparse (SSA) branch; the formula is lost in the page text, and this oracle
+ * takes the plain reading alpha * O_full + (1 - alpha) * O_ssa).
+ *
+ * ssa_oracle_merge: branches a and b are softmax attention of the same query
+ * over two disjoint key sets A and B, given as (O, LSE); the result is
+ * attention over A U B:
+ *   LSE = ln(exp(LSE_a) + exp(LSE_b))
+ *   O   = exp(LSE_a - LSE) O_a + exp(LSE_b - LSE) O_b
+ * A branch with LSE = -inf has no keys and weight 0; if both have none the
+ * result is O = 0, LSE = -inf. Rows are (token, head) pairs; O is [rows, d_v]
+ * bf16 bits, LSE [rows] (fp32 values widened to double by the caller).
+ *
+ * ssa_oracle_mix: O = alpha * O_full + (1 - alpha) * O_ssa, elementwise.
+ */
+int ssa_oracle_merge(const uint16_t *o_a, const double *lse_a, const uint16_t *o_b, const double *lse_b,
+                     int64_t rows, int d_v, double *o, double *lse) {
+    if (rows < 0 || d_v < 1) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double la = lse_a[r], lb = lse_b[r];
+        double wa = 0.0, wb = 0.0, l = -INFINITY;
+        if (la != -INFINITY || lb != -INFINITY) {
+            const double m = la > lb ? la : lb;
+            l = m + log(exp(la - m) + exp(lb - m));
+            wa = exp(la - l);
+            wb = exp(lb - l);
+        }
+        lse[r] = l;
+        for (int d = 0; d < d_v; ++d)
+            o[r * d_v + d] = wa * widen(o_a[r * d_v + d]) + wb * widen(o_b[r * d_v + d]);
+    }
+    return 0;
+}
+
+int ssa_oracle_mix(const uint16_t *o_full, const uint16_t *o_ssa, int64_t n, double alpha, double *o) {
+    if (n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) o[i] = alpha * widen(o_full[i]) + (1.0 - alpha) * widen(o_ssa[i]);
+    return 0;
+}
