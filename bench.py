@@ -348,6 +348,40 @@ def prefill_workspace(bss, device, batch, T, L, params, H_=None, Hkv=1, dqk=None
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
+def merge_secondary(bss, device, stream, peaks, peak_kind, steps=20):
+    """LSE merge of two attention branches (O, LSE) at the prefill's output
+    shape: 32,768 tokens x 64 heads x 512 values. Inputs are 4.3 GB (> L2)."""
+    import torch
+    rows, d_v = SEQLEN * H, DV
+    o_a = synth.torch_normal_bf16((rows, d_v), 9001, device)
+    o_b = synth.torch_normal_bf16((rows, d_v), 9002, device)
+    g = torch.Generator(device=device).manual_seed(9003)
+    l_a = torch.rand(rows, device=device, generator=g) * 25 - 5
+    l_b = torch.rand(rows, device=device, generator=g) * 25 - 5
+    out = torch.empty_like(o_a)
+    lse = torch.empty_like(l_a)
+
+    def call():
+        bss.loza_ssa_merge(o_a, l_a, o_b, l_b, out=out, lse_out=lse, stream=stream)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms, _ = time_launches(call, stream, steps)
+    nbytes = rows * (3 * d_v * 2 + 3 * 4)
+    hbm = float(peaks["hbm_gbs"])
+    gbs = nbytes / (ms / 1000.0) / 1e9
+    del o_a, o_b, out
+    torch.cuda.empty_cache()
+    return {"workload": f"merge of two attention branches, {SEQLEN} tokens x {H} heads x {DV}",
+            "metric": "branch merge GB/s", "value": gbs, "unit": "GB/s", "ms_per_call": ms,
+            "bytes_per_call": nbytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "traffic": None, "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
+                         "kernel": "ssa_merge_kernel"},
+            "timing": "mean of per-call CUDA events; inputs larger than L2"}
+
+
 def long_secondary(bss, device, stream, peaks):
     """Workload 4: L = 262144 absorbed prefill, SSA next to full causal attention;
     then SSA and dense decode of 32 sequences of 1,048,576 tokens."""
@@ -510,6 +544,7 @@ def run_ours(args, rank, world, local_rank):
     if args.workload in ("default", "all"):
         secondary["decode"] = decode_secondary(bss, device, stream, peaks, peak_kind, args.decode_batch,
                                                args.decode_ctx)
+        secondary["merge"] = merge_secondary(bss, device, stream, peaks, peak_kind)
     if args.workload in ("long", "all"):
         secondary["long"] = long_secondary(bss, device, stream, peaks)
     if args.workload in ("train", "all"):

@@ -35,6 +35,8 @@ EXPORTED = [
     "loza_ssa_prefill",
     "loza_ssa_decode",
     "loza_ssa_decode_noalloc",
+    "loza_ssa_merge",
+    "loza_ssa_mix",
     "loza_ssa_backward",
     "loza_status_string",
     "loza_device_status",
@@ -83,6 +85,10 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_backward.restype = ctypes.c_int
         L.loza_ssa_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
                                         _i32, _i32, Params, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.loza_ssa_merge.restype = ctypes.c_int
+        L.loza_ssa_merge.argtypes = [_vp, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp]
+        L.loza_ssa_mix.restype = ctypes.c_int
+        L.loza_ssa_mix.argtypes = [_vp, _vp, _i64, ctypes.c_float, _vp, _vp]
         L.loza_status_string.restype = ctypes.c_char_p
         L.loza_status_string.argtypes = [ctypes.c_int]
         L.loza_device_status.restype = ctypes.c_int
@@ -234,3 +240,43 @@ def device_status(stream=None) -> int:
 
 def launch_count() -> int:
     return int(lib().loza_launch_count())
+
+
+def loza_ssa_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None, stream=None):
+    """Attention over the union of two disjoint key sets from two branches:
+    o_* [..., d_v] bf16 contiguous, lse_* of shape o_*.shape[:-1] fp32 (natural
+    log, -inf for a branch without keys). Returns (out, lse_out)."""
+    import torch
+    _require(o_a, "o_a", torch.bfloat16)
+    _require(o_b, "o_b", torch.bfloat16)
+    _require(lse_a, "lse_a", torch.float32)
+    _require(lse_b, "lse_b", torch.float32)
+    if o_a.shape != o_b.shape or lse_a.shape != o_a.shape[:-1] or lse_b.shape != o_a.shape[:-1]:
+        raise ValueError("merge: branch shapes differ")
+    for t, n in ((o_a, "o_a"), (o_b, "o_b"), (lse_a, "lse_a"), (lse_b, "lse_b")):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    d_v = o_a.shape[-1]
+    rows = o_a.numel() // d_v
+    if out is None:
+        out = torch.empty_like(o_a)
+    if lse_out is None:
+        lse_out = torch.empty_like(lse_a)
+    rc = lib().loza_ssa_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), rows, d_v, _ptr(out), _ptr(lse_out),
+                              _stream_ptr(stream))
+    _check(rc, "loza_ssa_merge")
+    return out, lse_out
+
+
+def loza_ssa_mix(o_full, o_ssa, alpha: float, out=None, stream=None):
+    """alpha * o_full + (1 - alpha) * o_ssa (bf16, contiguous, same shape)."""
+    import torch
+    _require(o_full, "o_full", torch.bfloat16)
+    _require(o_ssa, "o_ssa", torch.bfloat16)
+    if o_full.shape != o_ssa.shape or not o_full.is_contiguous() or not o_ssa.is_contiguous():
+        raise ValueError("mix: inputs must be contiguous and of one shape")
+    if out is None:
+        out = torch.empty_like(o_full)
+    rc = lib().loza_ssa_mix(_ptr(o_full), _ptr(o_ssa), o_full.numel(), float(alpha), _ptr(out), _stream_ptr(stream))
+    _check(rc, "loza_ssa_mix")
+    return out

@@ -19,6 +19,7 @@
 #include "decode.cuh"
 #include "decode_mla.cuh"
 #include "decode_mla_hs.cuh"
+#include "merge.cuh"
 #include "backward.cuh"
 
 namespace loza {
@@ -404,12 +405,46 @@ void* decode_scratch_address() {
   return g_scratch_addr[dev];
 }
 
+// Grid for a grid-stride pass over n 16-byte vectors: at most a few waves.
+unsigned stream_grid(int64_t n) {
+  const int64_t per = (int64_t)kMergeThreads;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  return (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + per - 1) / per, cap));
+}
+
 }  // namespace
 }  // namespace loza
 
 using namespace loza;
 
 extern "C" {
+
+loza_status loza_ssa_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, int64_t rows,
+                           int32_t d_v, void* out, float* lse_out, loza_stream_t stream) {
+  if (rows < 0 || d_v < 8 || d_v % 8 != 0) return LOZA_ERR_INVALID_ARG;
+  if (rows == 0) return LOZA_OK;
+  if (!o_a || !o_b || !out || !lse_a || !lse_b || !lse_out) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
+  if (rows > (int64_t(1) << 40) / d_v) return LOZA_ERR_INVALID_ARG;
+  const int vec8 = d_v / 8;
+  ssa_merge_kernel<<<stream_grid(rows * vec8), kMergeThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b, static_cast<uint4*>(out),
+      lse_out, rows, vec8);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
+loza_status loza_ssa_mix(const void* o_full, const void* o_ssa, int64_t n, float alpha, void* out,
+                         loza_stream_t stream) {
+  if (n < 0 || n % 8 != 0) return LOZA_ERR_INVALID_ARG;
+  if (n == 0) return LOZA_OK;
+  if (!o_full || !o_ssa || !out) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(o_full) || !aligned16(o_ssa) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
+  ssa_mix_kernel<<<stream_grid(n / 8), kMergeThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(o_full), static_cast<const uint4*>(o_ssa), static_cast<uint4*>(out), n / 8, alpha);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
 
 const char* loza_status_string(loza_status s) {
   switch (s) {

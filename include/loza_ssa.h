@@ -210,6 +210,35 @@ loza_status loza_ssa_backward(const void *q, const void *k, const void *v, const
                               loza_ssa_params p, void *dq, void *dk, void *dv,
                               void *workspace, size_t workspace_bytes, loza_stream_t stream);
 
+/*
+ * Combine two attention branches of the same (token, head) rows, each given
+ * as O [rows, d_v] bf16 and LSE [rows] fp32 (natural log; -inf = a branch
+ * without keys), where the branches attend to disjoint key sets (for example
+ * SSA's sink + local blocks and a second set of selected blocks). Writes the
+ * attention over the union of the two key sets:
+ *     lse_out = ln(exp(lse_a) + exp(lse_b))
+ *     out     = exp(lse_a - lse_out) o_a + exp(lse_b - lse_out) o_b
+ * (both branches empty: out = 0, lse_out = -inf). This is the LSE combine of
+ * the split-KV decode applied to two whole outputs.
+ *   rows >= 0 (0 launches nothing); d_v a positive multiple of 8.
+ *   o_a, o_b, out: device, 16-byte aligned, contiguous [rows, d_v] bf16;
+ *   lse_a, lse_b, lse_out: device [rows] fp32. out may alias o_a or o_b
+ *   (each element is read before it is written by the same thread).
+ * Returns LOZA_ERR_INVALID_ARG for a bad size, alignment or null pointer.
+ */
+loza_status loza_ssa_merge(const void *o_a, const float *lse_a, const void *o_b, const float *lse_b,
+                           int64_t rows, int32_t d_v, void *out, float *lse_out, loza_stream_t stream);
+
+/*
+ * Calibration mix of a module's full-attention and SSA outputs (page 1
+ * section 01 (1) of the LoZA pages; the formula is lost in the page text, the
+ * plain reading is used): out = alpha * o_full + (1 - alpha) * o_ssa,
+ * elementwise over n bf16 values (n a multiple of 8; device pointers, 16-byte
+ * aligned; out may alias either input).
+ */
+loza_status loza_ssa_mix(const void *o_full, const void *o_ssa, int64_t n, float alpha, void *out,
+                         loza_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *loza_status_string(loza_status s);
 

@@ -71,3 +71,29 @@ def test_prefill_rejects_before_launch(L, over, code):
     count = L.loza_launch_count()
     assert _call_prefill(L, _prefill_args(**over)) == code
     assert L.loza_launch_count() == count
+
+
+@pytest.mark.parametrize("rows,d_v,o_a,code", [
+    (-1, 512, 1 << 20, -1),          # negative row count
+    (4, 12, 1 << 20, -1),            # d_v not a multiple of 8
+    (4, 0, 1 << 20, -1),
+    (4, 512, 0, -1),                 # null branch
+    (4, 512, (1 << 20) + 8, -1),     # misaligned branch
+    (0, 512, 0, 0),                  # nothing to do: no launch, ok
+])
+def test_merge_rejects_before_launch(L, rows, d_v, o_a, code):
+    vp = ctypes.c_void_p
+    count = L.loza_launch_count()
+    rc = L.loza_ssa_merge(vp(o_a), vp(1 << 21), vp(1 << 22), vp(1 << 23), rows, d_v, vp(1 << 24), vp(1 << 25),
+                          vp(0))
+    assert rc == code
+    assert L.loza_launch_count() == count
+
+
+@pytest.mark.parametrize("n,out,code", [(-8, 1 << 22, -1), (12, 1 << 22, -1), (16, 0, -1), (16, (1 << 22) + 4, -1),
+                                        (0, 0, 0)])
+def test_mix_rejects_before_launch(L, n, out, code):
+    vp = ctypes.c_void_p
+    count = L.loza_launch_count()
+    assert L.loza_ssa_mix(vp(1 << 20), vp(1 << 21), n, 0.5, vp(out), vp(0)) == code
+    assert L.loza_launch_count() == count
