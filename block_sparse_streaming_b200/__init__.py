@@ -35,6 +35,7 @@ EXPORTED = [
     "loza_ssa_prefill",
     "loza_ssa_decode",
     "loza_ssa_decode_noalloc",
+    "loza_ssa_decode_paged",
     "loza_ssa_merge",
     "loza_ssa_mix",
     "loza_ssa_backward",
@@ -85,6 +86,9 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_backward.restype = ctypes.c_int
         L.loza_ssa_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
                                         _i32, _i32, Params, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.loza_ssa_decode_paged.restype = ctypes.c_int
+        L.loza_ssa_decode_paged.argtypes = [_vp, _vp, _i32, _i64, _vp, _i32, _vp, _i32, _i32, _i32, Params, _vp, _vp,
+                                            _vp, _sz, _vp]
         L.loza_ssa_merge.restype = ctypes.c_int
         L.loza_ssa_merge.argtypes = [_vp, _vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp]
         L.loza_ssa_mix.restype = ctypes.c_int
@@ -280,3 +284,37 @@ def loza_ssa_mix(o_full, o_ssa, alpha: float, out=None, stream=None):
     rc = lib().loza_ssa_mix(_ptr(o_full), _ptr(o_ssa), o_full.numel(), float(alpha), _ptr(out), _stream_ptr(stream))
     _check(rc, "loza_ssa_mix")
     return out
+
+
+def loza_ssa_decode_paged(q, kv_pool, block_table, seqlens, max_seqlen: int, params: Params, out=None, lse=None,
+                          workspace=None, stream=None):
+    """Absorbed SSA decode from a paged latent cache. q [B,64,576]; kv_pool
+    [num_pages, 128, 576] (or [num_pages * 128, 576]) bf16 with contiguous rows;
+    block_table [B, pages per sequence] int32: the pool page of each logical
+    128-token block. Returns (out [B,64,512], lse [B,64])."""
+    import torch
+    _require(q, "q", torch.bfloat16, 3)
+    _require(kv_pool, "kv_pool", torch.bfloat16)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    if kv_pool.shape[-1] != 576 or kv_pool.stride(-1) != 1:
+        raise ValueError("kv_pool rows must be 576 contiguous latent columns")
+    pool2 = kv_pool.reshape(-1, 576) if kv_pool.dim() == 3 else kv_pool
+    if pool2.dim() != 2 or pool2.shape[0] % 128 != 0:
+        raise ValueError("kv_pool must hold whole pages of 128 rows")
+    if not block_table.is_contiguous():
+        raise ValueError("block_table must be contiguous")
+    B, H, d_qk = q.shape
+    if out is None:
+        out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = workspace_size(LOZA_OP_DECODE, B, 0, int(max_seqlen), H, 1, d_qk, 512, params)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().loza_ssa_decode_paged(_ptr(q), _ptr(pool2), pool2.shape[0] // 128, pool2.stride(0), _ptr(block_table),
+                                     block_table.shape[1], _ptr(seqlens), B, int(max_seqlen), H, params, _ptr(out),
+                                     _ptr(lse), _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check(rc, "loza_ssa_decode_paged")
+    return out, lse

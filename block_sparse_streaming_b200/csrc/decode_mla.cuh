@@ -50,8 +50,10 @@ constexpr int kDecVUnits = 4;            // 512 columns
 
 struct DecodeParams {
   CUtensorMap tm_q;    // q [B, H, 576]       box {64, 64, 1}
-  CUtensorMap tm_kv;   // cache [B, rows, 576] box {64, 128, 1}
+  CUtensorMap tm_kv;   // cache [B, rows, 576] box {64, 128, 1}; paged: the pool [1, pages * 128, 576]
   const int32_t* seqlens;
+  const int32_t* block_table;  // paged cache: [B, bt_stride] pool page of each logical block; nullptr: contiguous
+  int bt_stride;
   float* ws_o;         // workspace mode: [B, nsplit, H, 512] partial O (unnormalised)
   float4* ws_ml;       // workspace mode: [B, nsplit, H] partial (m in log2 units, l exact, l of bf16 P, -)
   int* ws_ticket;      // workspace mode: [B] arrival counters (zero on entry)
@@ -63,6 +65,13 @@ struct DecodeParams {
   int n_local;         // < 0: unbounded
   float scale_log2;
 };
+
+// TMA coordinates (row, batch) of logical block kb of sequence seq: in the
+// sequence's own cache, or on its page of a paged pool (pages of 128 rows).
+__device__ __forceinline__ int2 dec_block_rows(const DecodeParams& p, int seq, int kb) {
+  if (p.block_table) return make_int2(p.block_table[(int64_t)seq * p.bt_stride + kb] * kTile, 0);
+  return make_int2(kb * kTile, seq);
+}
 
 struct DecodeLayout {
   static constexpr int Q_OFF = 0;                                   // 9 Q tiles, 72 KB
@@ -220,7 +229,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       int slot = 0;
       uint32_t phase = 0;
       bool ok = true;
-      auto load_unit = [&](int row, int u) {
+      auto load_unit = [&](int2 rz, int u) {
         ok = warp_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
         if (!ok) return;
         if (elect_one()) {
@@ -228,18 +237,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
           const int ntile = (u < 4) ? 2 : 1;
           mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), ntile * kChunkBytes);
           for (int t = 0; t < ntile; ++t)
-            tma_load_3d(dst + t * kChunkBytes, &p.tm_kv, bar(LY::BAR_FULL + slot), 128 * u + 64 * t, row, seq);
+            tma_load_3d(dst + t * kChunkBytes, &p.tm_kv, bar(LY::BAR_FULL + slot), 128 * u + 64 * t, rz.x, rz.y);
         }
         __syncwarp();
         if (++slot == kDecStages) { slot = 0; phase ^= 1; }
       };
       for (int it = 0; it <= nb && ok; ++it) {
         if (it < nb) {
-          const int krow = walk.block(b_lo + it) * kTile;
+          const int2 krow = dec_block_rows(p, seq, walk.block(b_lo + it));
           for (int u = 0; u < kDecKUnits && ok; ++u) load_unit(krow, u);
         }
         if (it >= 1) {
-          const int vrow = walk.block(b_lo + it - 1) * kTile;
+          const int2 vrow = dec_block_rows(p, seq, walk.block(b_lo + it - 1));
           for (int u = 0; u < kDecVUnits && ok; ++u) load_unit(vrow, u);
         }
       }

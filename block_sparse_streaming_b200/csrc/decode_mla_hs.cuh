@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kHsThreads, 1) ssa_decode_mla_hs_kernel(const 
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
-    auto load_unit = [&](int row, int u) {
+    auto load_unit = [&](int2 rz, int u) {
       ok = warp_wait(bar(LY::BAR_EMPTY + slot), phase ^ 1, abort_flag);
       if (!ok) return;
       if (elect_one()) {
@@ -138,18 +138,18 @@ __global__ void __launch_bounds__(kHsThreads, 1) ssa_decode_mla_hs_kernel(const 
         const int ntile = (u < 4) ? 2 : 1;
         mbar_arrive_expect_tx(bar(LY::BAR_FULL + slot), ntile * kChunkBytes);
         for (int t = 0; t < ntile; ++t)
-          tma_load_3d(dst + t * kChunkBytes, &p.tm_kv, bar(LY::BAR_FULL + slot), 128 * u + 64 * t, row, seq);
+          tma_load_3d(dst + t * kChunkBytes, &p.tm_kv, bar(LY::BAR_FULL + slot), 128 * u + 64 * t, rz.x, rz.y);
       }
       __syncwarp();
       if (++slot == kHsStages) { slot = 0; phase ^= 1; }
     };
     for (int it = 0; it <= nb && ok; ++it) {
       if (it < nb) {
-        const int krow = blk(it) * kTile;
+        const int2 krow = dec_block_rows(p, seq, blk(it));
         for (int u = 0; u < kDecKUnits && ok; ++u) load_unit(krow, u);
       }
       if (it >= 1) {
-        const int vrow = blk(it - 1) * kTile;
+        const int2 vrow = dec_block_rows(p, seq, blk(it - 1));
         for (int u = 0; u < kDecVUnits && ok; ++u) load_unit(vrow, u);
       }
     }

@@ -419,6 +419,43 @@ using namespace loza;
 
 extern "C" {
 
+loza_status loza_ssa_decode_paged(const void* q, const void* kv_pool, int32_t num_pages, int64_t pool_row_stride,
+                                  const int32_t* block_table, int32_t bt_stride, const int32_t* seqlens,
+                                  int32_t batch, int32_t max_seqlen, int32_t n_heads, loza_ssa_params p, void* out,
+                                  float* lse, void* workspace, size_t workspace_bytes, loza_stream_t stream) {
+  if (!block_table || !kv_pool) return LOZA_ERR_INVALID_ARG;
+  if (num_pages < 1 || (int64_t)num_pages * kTile > INT32_MAX) return LOZA_ERR_INVALID_ARG;
+  if (max_seqlen < 1 || bt_stride < (max_seqlen + kTile - 1) / kTile) return LOZA_ERR_INVALID_ARG;
+  if (!stride_ok(pool_row_stride) || pool_row_stride < 576) return LOZA_ERR_INVALID_ARG;
+  DecodeParams prm;
+  DecodePlan plan;
+  // validation and the query map as for a contiguous cache of max_seqlen rows per sequence ...
+  const loza_status rc = setup_decode_mla(q, kv_pool, nullptr, seqlens, batch, max_seqlen,
+                                          (int64_t)max_seqlen * pool_row_stride, pool_row_stride, n_heads, p, out,
+                                          lse, &prm, &plan);
+  if (rc != LOZA_OK) return rc;
+  // ... then the cache map over the whole pool, addressed through the block table
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return LOZA_ERR_CUDA;
+  cuuint64_t dims[3] = {576, (cuuint64_t)num_pages * kTile, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)pool_row_stride * 2, (cuuint64_t)num_pages * kTile * pool_row_stride * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (strides[1] >= (cuuint64_t(1) << 40)) return LOZA_ERR_INVALID_ARG;
+  if (fn(&prm.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv_pool), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return LOZA_ERR_CUDA;
+  prm.block_table = block_table;
+  prm.bt_stride = bt_stride;
+  const DecodeWorkspace wl = decode_workspace(batch, plan);
+  if (wl.total > 0) {
+    if (!workspace || !aligned16(workspace)) return LOZA_ERR_INVALID_ARG;
+    if (workspace_bytes < wl.total) return LOZA_ERR_WORKSPACE;
+  }
+  return launch_decode_mla(prm, plan, batch, static_cast<uint8_t*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
 loza_status loza_ssa_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, int64_t rows,
                            int32_t d_v, void* out, float* lse_out, loza_stream_t stream) {
   if (rows < 0 || d_v < 8 || d_v % 8 != 0) return LOZA_ERR_INVALID_ARG;

@@ -211,6 +211,27 @@ loza_status loza_ssa_backward(const void *q, const void *k, const void *v, const
                               void *workspace, size_t workspace_bytes, loza_stream_t stream);
 
 /*
+ * Absorbed decode (n_kv_heads 1, d_qk 576, d_v 512, n_heads 64) from a paged
+ * latent cache: the pool holds num_pages pages of 128 rows (one SSA block
+ * each), row r of page g at kv_pool + (g * 128 + r) * pool_row_stride
+ * elements; logical block kb of sequence n (rows 128kb .. 128kb+127 of its
+ * context) is page block_table[n * bt_stride + kb]. Every block the window
+ * selects must have a page; other table entries are never read. Same
+ * operation, outputs, workspace (loza_ssa_workspace_size(LOZA_OP_DECODE, ...)
+ * with the same batch and max_seqlen) and errors as loza_ssa_decode; in
+ * addition LOZA_ERR_INVALID_ARG if block_table is NULL, bt_stride <
+ * ceil(max_seqlen / 128), num_pages < 1 or num_pages * 128 > INT32_MAX. A page
+ * number outside [0, num_pages) reads zeros (it is not detected).
+ *   block_table: device int32 [batch, bt_stride]; kv_pool: device bf16,
+ *   16-byte aligned, pool_row_stride >= 576 and a multiple of 8.
+ */
+loza_status loza_ssa_decode_paged(const void *q, const void *kv_pool, int32_t num_pages, int64_t pool_row_stride,
+                                  const int32_t *block_table, int32_t bt_stride, const int32_t *seqlens,
+                                  int32_t batch, int32_t max_seqlen, int32_t n_heads, loza_ssa_params p,
+                                  void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                  loza_stream_t stream);
+
+/*
  * Combine two attention branches of the same (token, head) rows, each given
  * as O [rows, d_v] bf16 and LSE [rows] fp32 (natural log; -inf = a branch
  * without keys), where the branches attend to disjoint key sets (for example

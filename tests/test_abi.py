@@ -97,3 +97,18 @@ def test_mix_rejects_before_launch(L, n, out, code):
     count = L.loza_launch_count()
     assert L.loza_ssa_mix(vp(1 << 20), vp(1 << 21), n, 0.5, vp(out), vp(0)) == code
     assert L.loza_launch_count() == count
+
+
+@pytest.mark.parametrize("table,bt_stride,num_pages,code", [
+    (0, 8, 16, -1),              # no block table
+    (1 << 26, 7, 16, -1),        # fewer table columns than blocks of max_seqlen (1024 -> 8)
+    (1 << 26, 8, 0, -1),         # empty pool
+    (1 << 26, 8, 1 << 24, -1),   # pool rows beyond int32
+])
+def test_decode_paged_rejects_before_launch(L, table, bt_stride, num_pages, code):
+    vp = ctypes.c_void_p
+    count = L.loza_launch_count()
+    rc = L.loza_ssa_decode_paged(vp(1 << 20), vp(1 << 21), num_pages, 576, vp(table), bt_stride, vp(1 << 22), 4,
+                                 1024, 64, bss.Params(1 / 8), vp(1 << 23), vp(1 << 24), vp(0), 0, vp(0))
+    assert rc == code
+    assert L.loza_launch_count() == count

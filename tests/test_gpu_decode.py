@@ -148,3 +148,58 @@ def test_mha_decode_matches_oracle_and_prefill(bss, oracle_mod, dqk, dv):
         torch.cuda.synchronize()
         assert_close_o(from_dev(po[L - 1]), from_dev(out[n]), "decode vs prefill row")
         assert abs(float(pl[L - 1, 0] - lse[n, 0])) <= 1e-3
+
+
+def paged_case(bss, oracle_mod, seed, lens, n_sink=1, n_local=7):
+    """Absorbed decode from a paged pool: each sequence's 128-token blocks sit
+    on shuffled pages of a shared pool (unused pages hold NaN). Compared with
+    the oracle on the logical cache, and bit for bit with loza_ssa_decode on a
+    contiguous cache holding the same rows."""
+    import torch
+    H, D = 64, 576
+    B = len(lens)
+    g = synth.rng(seed)
+    q = synth.normal_bits(g, (B, H, D))
+    nblk = [(L + 127) // 128 for L in lens]
+    n_pages = sum(nblk) + 5
+    perm = g.permutation(n_pages)
+    table = np.full((B, max(nblk) + 2), -1, np.int32)  # entries for absent blocks are never read
+    Lcap = max(nblk) * 128
+    pool = torch.full((n_pages, 128, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    cache = torch.full((B, Lcap, 1, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    host = np.empty((B, Lcap, 1, D), np.uint16)
+    nxt = 0
+    for n, L in enumerate(lens):
+        for kb in range(nblk[n]):
+            table[n, kb] = perm[nxt]
+            nxt += 1
+        rows = selected_rows(L, 128, n_sink, n_local)
+        vals = synth.normal_bits(g, (len(rows), 1, D))
+        host[n, rows] = vals
+        dev_vals = to_dev(vals)
+        cache[n, torch.from_numpy(rows).cuda()] = dev_vals
+        pages = torch.from_numpy(table[n, rows // 128].astype(np.int64)).cuda()
+        pool[pages, torch.from_numpy(rows % 128).cuda()] = dev_vals[:, 0]
+    seqlens = torch.from_numpy(np.array(lens, np.int32)).cuda()
+    scale = 1.0 / math.sqrt(192.0)
+    params = bss.Params(scale, 128, n_sink, n_local)
+    qd = to_dev(q)
+    out_p, lse_p = bss.loza_ssa_decode_paged(qd, pool, torch.from_numpy(table).cuda(), seqlens, Lcap, params)
+    out_c, lse_c = bss.loza_ssa_decode(qd, cache, None, seqlens, Lcap, params)
+    torch.cuda.synchronize()
+    assert bss.device_status() == 0
+    assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
+    o_ref, lse_ref = oracle_mod.decode(q, host, None, np.array(lens, np.int32), H, 1, 128, n_sink, n_local, scale,
+                                       d_v=512)
+    assert_close_o(from_dev(out_p), o_ref, "paged decode O")
+    assert_close_lse(lse_p.cpu().numpy().astype(np.float64), lse_ref, "paged decode LSE")
+
+
+@pytest.mark.parametrize("batch", [6, 40, 80])
+def test_absorbed_decode_paged(bss, oracle_mod, batch):
+    """Paged latent cache under the three plan families (block split over a
+    cluster, head split, one CTA per sequence)."""
+    g = synth.rng(300 + batch)
+    lens = g.integers(1, 3000, size=batch)
+    lens[:3] = [1, 128, 1025]
+    paged_case(bss, oracle_mod, 301 + batch, lens.tolist())
