@@ -377,7 +377,8 @@ def merge_secondary(bss, device, stream, peaks, peak_kind, steps=20):
             "metric": "branch merge GB/s", "value": gbs, "unit": "GB/s", "ms_per_call": ms,
             "bytes_per_call": nbytes,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "traffic": None, "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
+                         "traffic": profiled_traffic("ssa_merge_kernel"),
+                         "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
                          "kernel": "ssa_merge_kernel"},
             "timing": "mean of per-call CUDA events; inputs larger than L2"}
 
