@@ -144,3 +144,93 @@ def prefill_sharded(q_own, k_own, v_own, params, plan: ShardPlan, group=None, la
     cu = torch.tensor([0, q_loc.shape[0]], dtype=torch.int32, device=q_own.device)
     out, lse = loza_ssa_prefill(q_loc, k_loc, v_loc, cu, q_loc.shape[0], params)
     return own_outputs(out, lse, plan)
+
+
+# ---------------------------------------------------------------------------
+# Backward of the sharded prefill.
+#
+# Each rank runs the one-GPU backward on its local sequence [sinks | halo |
+# own]: the prepended rows get zero dO (and zero O), so their queries add
+# nothing to any gradient, and the own rows' dQ is exact. The key gradients of
+# the prepended rows are partial sums that belong to other ranks:
+#   halo rows (local blocks s .. s+l-2): the left neighbour's last l-1 blocks,
+#       sent back to it and added to its own dK, dV;
+#   sink rows (local blocks 0 .. s-1): every rank's share of the sink blocks'
+#       gradients, summed onto rank 0 (which owns the sinks) by a reduce.
+# The additions are done in fp32.
+# ---------------------------------------------------------------------------
+def local_rows(x_own, plan: ShardPlan):
+    """Zero rows for the prepended blocks, then the own rows (q, out, dout, lse)."""
+    return local_queries(x_own, plan)
+
+
+def split_key_grads(dk_loc, dv_loc, plan: ShardPlan, n_sink: int = 1, n_local: int = 7):
+    """The local backward's dK, dV (rows [sinks | halo | own]) as fp32 parts:
+    (own dK, own dV, halo dK, halo dV, sink dK, sink dV); the halo and sink
+    parts are None on rank 0, which has no prepended rows."""
+    off = plan.n_pre * BLOCK
+    own = (dk_loc[off:].float(), dv_loc[off:].float())
+    if plan.n_pre == 0:
+        return own + (None, None, None, None)
+    s_rows, h_rows = n_sink * BLOCK, (n_local - 1) * BLOCK
+    halo = (dk_loc[s_rows:s_rows + h_rows].float(), dv_loc[s_rows:s_rows + h_rows].float())
+    sink = (dk_loc[:s_rows].float(), dv_loc[:s_rows].float())
+    return own + halo + sink
+
+
+def settle_key_grads(dk_loc, dv_loc, plan: ShardPlan, n_sink: int = 1, n_local: int = 7, group=None):
+    """From the local backward's dK, dV (rows [sinks | halo | own]) return this
+    rank's own dK, dV with the other ranks' contributions added (fp32 sums,
+    then the input dtype): its right neighbour's halo part is added to its
+    last l-1 blocks, and on rank 0 every rank's sink part to its first s
+    blocks. Every rank must call it (collective)."""
+    import torch
+    import torch.distributed as dist
+    out_dtype = dk_loc.dtype
+    dk, dv, hk, hv, sk_part, sv_part = split_key_grads(dk_loc, dv_loc, plan, n_sink, n_local)
+    halo_rows = (n_local - 1) * BLOCK
+    sink_rows = n_sink * BLOCK
+    if plan.world > 1:
+        ops = []
+        recv_k = recv_v = None
+        if plan.rank > 0:  # the halo gradients go back to the left neighbour
+            ops.append(dist.P2POp(dist.isend, hk.contiguous(), plan.rank - 1, group=group))
+            ops.append(dist.P2POp(dist.isend, hv.contiguous(), plan.rank - 1, group=group))
+        if plan.rank + 1 < plan.world:
+            recv_k = torch.empty((halo_rows,) + tuple(dk.shape[1:]), dtype=torch.float32, device=dk.device)
+            recv_v = torch.empty((halo_rows,) + tuple(dv.shape[1:]), dtype=torch.float32, device=dv.device)
+            ops.append(dist.P2POp(dist.irecv, recv_k, plan.rank + 1, group=group))
+            ops.append(dist.P2POp(dist.irecv, recv_v, plan.rank + 1, group=group))
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+        if recv_k is not None:
+            dk[dk.shape[0] - halo_rows:] += recv_k
+            dv[dv.shape[0] - halo_rows:] += recv_v
+        # the sink gradients of every other rank, summed onto rank 0
+        sk = sk_part.contiguous() if sk_part is not None else torch.zeros(
+            (sink_rows,) + tuple(dk.shape[1:]), dtype=torch.float32, device=dk.device)
+        sv = sv_part.contiguous() if sv_part is not None else torch.zeros(
+            (sink_rows,) + tuple(dv.shape[1:]), dtype=torch.float32, device=dv.device)
+        dist.reduce(sk, dst=0, op=dist.ReduceOp.SUM, group=group)
+        dist.reduce(sv, dst=0, op=dist.ReduceOp.SUM, group=group)
+        if plan.rank == 0:
+            dk[:sink_rows] += sk
+            dv[:sink_rows] += sv
+    return dk.to(out_dtype), dv.to(out_dtype)
+
+
+def backward_sharded(q_own, k_own, v_own, out_own, dout_own, lse_own, params, plan: ShardPlan, group=None):
+    """SSA backward of this rank's share of one sequence (per-head K, V).
+    Returns (dq, dk, dv) of the own rows."""
+    import torch
+    from . import loza_ssa_backward
+    k_loc = exchange_kv(k_own, plan, params.n_sink, params.n_local, group).contiguous()
+    v_loc = exchange_kv(v_own, plan, params.n_sink, params.n_local, group).contiguous()
+    q_loc = local_rows(q_own, plan).contiguous()
+    o_loc = local_rows(out_own, plan).contiguous()
+    do_loc = local_rows(dout_own, plan).contiguous()
+    lse_loc = local_rows(lse_own, plan).contiguous()
+    cu = torch.tensor([0, q_loc.shape[0]], dtype=torch.int32, device=q_own.device)
+    dq, dk, dv = loza_ssa_backward(q_loc, k_loc, v_loc, o_loc, do_loc, lse_loc, cu, q_loc.shape[0], params)
+    dk_own, dv_own = settle_key_grads(dk, dv, plan, params.n_sink, params.n_local, group)
+    return dq[plan.n_pre * BLOCK:], dk_own, dv_own

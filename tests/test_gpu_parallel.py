@@ -51,3 +51,49 @@ def test_sharded_prefill_equals_whole(bss, shape, world, n_sink):
         torch.cuda.synchronize()
         assert torch.equal(out_own, out_full[lo:hi]), f"rank {r} O"
         assert torch.equal(lse_own, lse_full[lo:hi]), f"rank {r} LSE"
+
+
+@pytest.mark.parametrize("world,n_sink", [(2, 1), (3, 2)])
+def test_sharded_backward_matches_whole(bss, world, n_sink):
+    """The sharded backward on one B200: every rank's local backward through
+    the CUDA kernels, its key gradients split into own / halo / sink parts and
+    summed as the collectives would. dQ is bit-identical to the whole
+    sequence's; dK, dV (extra bf16 roundings of the summed parts) agree within
+    the gradient tolerance."""
+    import torch
+    from block_sparse_streaming_b200 import parallel as par
+    seq_len, H = 5000, 4
+    g = synth.rng(500 + world)
+    q, k = (to_dev(synth.normal_bits(g, (seq_len, H, 192))) for _ in range(2))
+    v, dout = (to_dev(synth.normal_bits(g, (seq_len, H, 128))) for _ in range(2))
+    params = bss.Params(1 / math.sqrt(192), 128, n_sink, 7)
+    cu = torch.tensor([0, seq_len], dtype=torch.int32, device="cuda")
+    out, lse = bss.loza_ssa_prefill(q, k, v, cu, seq_len, params)
+    dq_ref, dk_ref, dv_ref = bss.loza_ssa_backward(q, k, v, out, dout, lse, cu, seq_len, params)
+    plans = [par.shard_plan(seq_len, world, r, n_sink, 7) for r in range(world)]
+    parts = []
+    for plan in plans:
+        lo, hi = plan.own_rows
+        loc = lambda x: par.local_rows(x[lo:hi], plan).contiguous()
+        k_loc = par.local_kv_from_full(k, plan, n_sink, 7).contiguous()
+        v_loc = par.local_kv_from_full(v, plan, n_sink, 7).contiguous()
+        cu_loc = torch.tensor([0, plan.local_len], dtype=torch.int32, device="cuda")
+        dq, dk, dv = bss.loza_ssa_backward(loc(q), k_loc, v_loc, loc(out), loc(dout), loc(lse), cu_loc, plan.local_len,
+                                           params)
+        assert torch.equal(dq[plan.n_pre * 128:], dq_ref[lo:hi]), f"rank {plan.rank} dQ"
+        parts.append(par.split_key_grads(dk, dv, plan, n_sink, 7))
+    # what the exchange does: halo parts to the left neighbour, sink parts onto rank 0
+    dk_sum = [p[0].clone() for p in parts]
+    dv_sum = [p[1].clone() for p in parts]
+    h = 6 * 128
+    for r in range(1, world):
+        dk_sum[r - 1][-h:] += parts[r][2]
+        dv_sum[r - 1][-h:] += parts[r][3]
+        dk_sum[0][: n_sink * 128] += parts[r][4]
+        dv_sum[0][: n_sink * 128] += parts[r][5]
+    dk_got = torch.cat([x.to(torch.bfloat16) for x in dk_sum]).double().cpu().numpy()
+    dv_got = torch.cat([x.to(torch.bfloat16) for x in dv_sum]).double().cpu().numpy()
+    for got, ref, name in ((dk_got, dk_ref.double().cpu().numpy(), "dK"), (dv_got, dv_ref.double().cpu().numpy(), "dV")):
+        err = np.abs(got - ref)
+        assert err.max() <= 1e-2 * max(1.0, np.abs(ref).max()), f"{name} max-abs {err.max()}"
+        assert err.mean() <= 1e-3 * max(1.0, np.abs(ref).mean()), f"{name} mean-abs {err.mean()}"
