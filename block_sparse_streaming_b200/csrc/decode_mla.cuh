@@ -25,13 +25,16 @@
 //
 // Merge of the splits of a sequence (log-sum-exp rule):
 //   CLUSTER  = true : the nsplit (<= 8) CTAs of a sequence form a thread-block
-//                     cluster; after exchanging (m, l), each pushes its
-//                     weighted partial O from TMEM into the shared memory of
-//                     the CTA that owns those output columns (DSMEM stores),
-//                     and each CTA sums its 512/nsplit columns locally.
+//                     cluster; after exchanging (m, l), each stages its
+//                     weighted partial O (from TMEM) for the columns the other
+//                     CTAs own in its shared memory and moves each part with
+//                     one DSMEM bulk copy (nsplit <= 4; with 8 splits, plain
+//                     DSMEM stores), and each CTA sums its 512/nsplit columns.
 //   CLUSTER  = false: partials go to the workspace and the last CTA of the
 //                     sequence (atomic ticket, no waiting) merges them; used
 //                     when a few long sequences need more than 8 splits.
+// Batches that fill the GPU with two CTAs per sequence use the head-split
+// kernel (decode_mla_hs.cuh) instead, which needs no merge.
 #pragma once
 
 #include <cuda.h>
