@@ -203,3 +203,12 @@ def test_absorbed_decode_paged(bss, oracle_mod, batch):
     lens = g.integers(1, 3000, size=batch)
     lens[:3] = [1, 128, 1025]
     paged_case(bss, oracle_mod, 301 + batch, lens.tolist())
+
+
+def test_absorbed_decode_paged_wide_window_workspace_plan(bss, oracle_mod):
+    """A 22-block window on 4 sequences: the plan keeps fp32 partials in the
+    workspace and the last CTA of each sequence merges them; the cache is paged."""
+    g = synth.rng(320)
+    lens = g.integers(2000, 5000, size=4)
+    lens[0] = 129
+    paged_case(bss, oracle_mod, 321, lens.tolist(), n_sink=2, n_local=20)
