@@ -577,29 +577,28 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_e2e(bss, params, device, stream, L, steps):
-    """Same metric through the public API with the inputs in pinned host memory:
-    each step copies Q and the latent host->device, runs the prefill, copies O and
-    LSE device->host; timed with CUDA events on the stream."""
+    """Same metric through the public C-ABI call with HOST buffers
+    (loza_ssa_prefill_host): every step copies Q and the latent from pinned host
+    memory to the device and O and LSE back, inside the call, pipelined over
+    chunks of query blocks; timed with CUDA events on the stream the call
+    completes on."""
     import torch
     q_d, lat_d, cu = make_inputs(device, L, seed_offset=7)
     q_h = torch.empty(q_d.shape, dtype=q_d.dtype, pin_memory=True)
     lat_h = torch.empty(lat_d.shape, dtype=lat_d.dtype, pin_memory=True)
     q_h.copy_(q_d)
     lat_h.copy_(lat_d)
+    del q_d, lat_d
+    torch.cuda.empty_cache()
     out_h = torch.empty((L, H, DV), dtype=torch.bfloat16, pin_memory=True)
     lse_h = torch.empty((L, H), dtype=torch.float32, pin_memory=True)
-    out_d = torch.empty((L, H, DV), dtype=torch.bfloat16, device=device)
-    lse_d = torch.empty((L, H), dtype=torch.float32, device=device)
-    ws = prefill_workspace(bss, device, 1, L, L, params)
+    ws = torch.empty(bss.workspace_size(bss.LOZA_OP_PREFILL_HOST, 1, L, L, H, 1, DQK, DV, params), dtype=torch.uint8,
+                     device=device)
     torch.cuda.synchronize()
 
     def one():
-        q_d.copy_(q_h, non_blocking=True)
-        lat_d.copy_(lat_h, non_blocking=True)
-        bss.loza_ssa_prefill(q_d, lat_d, lat_d[:, :, :DV], cu, L, params, out=out_d, lse=lse_d, workspace=ws,
-                             stream=stream)
-        out_h.copy_(out_d, non_blocking=True)
-        lse_h.copy_(lse_d, non_blocking=True)
+        bss.loza_ssa_prefill_host(q_h, lat_h, lat_h[:, :, :DV], params, out=out_h, lse=lse_h, workspace=ws,
+                                  stream=stream)
 
     one()
     torch.cuda.synchronize()
@@ -613,10 +612,51 @@ def run_e2e(bss, params, device, stream, L, steps):
     ms = e0.elapsed_time(e1) / steps
     h2d = q_h.numel() * 2 + lat_h.numel() * 2
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
-    del q_h, lat_h, out_h, lse_h, q_d, lat_d, out_d, lse_d
+    del ws
+    torch.cuda.empty_cache()
+    floor = copy_floor_ms(stream, [q_h, lat_h], [out_h, lse_h], steps)
+    del q_h, lat_h, out_h, lse_h
     torch.cuda.empty_cache()
     return {"value": prefill_flops(L) / (ms / 1000.0) / 1e12, "unit": UNIT, "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "api": "loza_ssa_prefill_host",
+            "copy_floor_ms": floor, "frac_of_copy_floor": floor / ms,
+            "copy_floor": "the same host<->device bytes alone, both directions at once on two streams, no kernels"}
+
+
+def copy_floor_ms(stream, host_in, host_out, steps):
+    """Time of the step's PCIe traffic alone: the pinned inputs copied to the
+    device while same-sized device buffers are copied to the pinned outputs,
+    on two streams; the e2e step cannot be faster than this."""
+    import torch
+    dev_in = [torch.empty_like(t, device="cuda") for t in host_in]
+    dev_out = [torch.empty_like(t, device="cuda") for t in host_out]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def one():
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        with torch.cuda.stream(s_in):
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            for h, d in zip(host_out, dev_out):
+                h.copy_(d, non_blocking=True)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+
+    one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del dev_in, dev_out
+    return ms
 
 
 def main():

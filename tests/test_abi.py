@@ -112,3 +112,49 @@ def test_decode_paged_rejects_before_launch(L, table, bt_stride, num_pages, code
                                  1024, 64, bss.Params(1 / 8), vp(1 << 23), vp(1 << 24), vp(0), 0, vp(0))
     assert rc == code
     assert L.loza_launch_count() == count
+
+
+def _call_prefill_host(L, q=1 << 20, k=1 << 21, v=1 << 22, seq_len=4096, H=4, Hkv=4, dqk=64, dv=64,
+                       params=None, ws=1 << 28, ws_bytes=1 << 40):
+    vp = ctypes.c_void_p
+    params = params if params is not None else bss.Params(0.125)
+    return L.loza_ssa_prefill_host(vp(q), vp(k), vp(v), seq_len, H, Hkv, dqk, dv, params, vp(1 << 24),
+                                   vp(1 << 25), vp(ws), ws_bytes, vp(0))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=0), -1),                                  # null pointer
+    (dict(seq_len=0), -1),                            # empty sequence
+    (dict(seq_len=1 << 31), -1),                      # beyond int32 rows
+    (dict(H=6, Hkv=4), -1),                           # heads not a multiple of kv heads
+    (dict(H=4, Hkv=2), -2),                           # grouped heads not compiled
+    (dict(dqk=96, dv=96), -2),                        # head dims not compiled
+    (dict(dqk=576, dv=512, H=3, Hkv=1), -2),          # absorbed needs an even head count
+    (dict(params=bss.Params(0.1, n_local=0)), -2),    # empty local window
+    (dict(ws=0), -1),                                 # no workspace
+    (dict(ws=(1 << 28) + 16), -1),                    # workspace not 256-byte aligned
+    (dict(ws_bytes=1024), -3),                        # workspace too small
+])
+def test_prefill_host_rejects_before_launch(L, over, code):
+    count = L.loza_launch_count()
+    assert _call_prefill_host(L, **over) == code
+    assert L.loza_launch_count() == count
+
+
+def test_prefill_host_workspace_size():
+    p = bss.Params(1 / math.sqrt(576))
+    size = lambda *a: bss.workspace_size(bss.LOZA_OP_PREFILL_HOST, *a)
+    assert size(2, 4096, 4096, 64, 1, 576, 512, p) == 0          # one sequence per call
+    assert size(1, 4096, 2048, 64, 1, 576, 512, p) == 0          # total_tokens == max_seqlen == seq_len
+    assert size(1, 4096, 4096, 64, 4, 576, 512, p) == 0          # absorbed is one kv head
+    small = size(1, 300, 300, 64, 1, 576, 512, p)
+    big = size(1, 32768, 32768, 64, 1, 576, 512, p)
+    huge = size(1, 1 << 20, 1 << 20, 64, 1, 576, 512, p)
+    # one chunk slot at least holds the short sequence's q, latent, out and lse
+    assert small >= 300 * (64 * 576 * 2 + 2 * 576 * 2 + 64 * 512 * 2 + 64 * 4)
+    # chunks are bounded (at most 64 own + s + l - 1 prepended blocks, three slots)
+    assert small < big <= huge
+    assert huge < 3 * (71 * 128) * (64 * 576 * 2 + 64 * 512 * 2 + 2 * 576 * 2 + 64 * 4) + (256 << 20)
+    # the unbounded window runs as one chunk: one slot of the whole sequence
+    dense = size(1, 8192, 8192, 4, 4, 64, 64, bss.Params(0.125, n_local=bss.LOZA_UNBOUNDED))
+    assert dense >= 8192 * 4 * (64 * 2 * 4 + 4)
