@@ -329,9 +329,9 @@ def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None, ctx=None
            "metric": "SSA decode GB/s (bytes touched)", "value": ssa["GB/s"], "unit": "GB/s",
            "ms_per_call": ssa["ms"], "bytes_per_call": ssa["bytes"],
            "roofline": {"bound": "hbm", "achieved": ssa["GB/s"], "peak": hbm, "unit": "GB/s",
-                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic("ssa_decode_mla_hs_kernel"),
+                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic("ssa_decode_mla_hb_kernel"),
                         "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
-                        "kernel": "ssa_decode_mla_hs_kernel"},
+                        "kernel": "ssa_decode_mla_hb_kernel"},
            "timing": "mean of per-call CUDA events, L2 flushed (256 MB write) before each call"}
     if "dense" in r:
         d = r["dense"]

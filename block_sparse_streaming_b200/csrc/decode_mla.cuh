@@ -24,17 +24,20 @@
 // by more than 2^8).
 //
 // Merge of the splits of a sequence (log-sum-exp rule):
-//   CLUSTER  = true : the nsplit (<= 8) CTAs of a sequence form a thread-block
+//   CLUSTER  = true : the nsplit (<= 4) CTAs of a sequence form a thread-block
 //                     cluster; after exchanging (m, l), each stages its
 //                     weighted partial O (from TMEM) for the columns the other
 //                     CTAs own in its shared memory and moves each part with
-//                     one DSMEM bulk copy (nsplit <= 4; with 8 splits, plain
-//                     DSMEM stores), and each CTA sums its 512/nsplit columns.
+//                     one DSMEM bulk copy, and each CTA sums its 512/nsplit
+//                     columns. The decode plan uses it with one CTA per
+//                     sequence (large batches), which writes all columns.
 //   CLUSTER  = false: partials go to the workspace and the last CTA of the
 //                     sequence (atomic ticket, no waiting) merges them; used
 //                     when a few long sequences need more than 8 splits.
-// Batches that fill the GPU with two CTAs per sequence use the head-split
-// kernel (decode_mla_hs.cuh) instead, which needs no merge.
+// Batches of at most half as many sequences as SMs use the half-block kernel
+// (decode_mla_hb.cuh) instead, which reads every selected row once; this
+// kernel then runs either as one CTA per sequence (no merge) or with many
+// splits merged through the workspace.
 #pragma once
 
 #include <cuda.h>
@@ -54,6 +57,7 @@ constexpr int kDecVUnits = 4;            // 512 columns
 struct DecodeParams {
   CUtensorMap tm_q;    // q [B, H, 576]       box {64, 64, 1}
   CUtensorMap tm_kv;   // cache [B, rows, 576] box {64, 128, 1}; paged: the pool [1, pages * 128, 576]
+  CUtensorMap tm_kv64; // the same tensor with box {64, 64, 1} (half blocks)
   const int32_t* seqlens;
   const int32_t* block_table;  // paged cache: [B, bt_stride] pool page of each logical block; nullptr: contiguous
   int bt_stride;
@@ -478,7 +482,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
     p.ws_ml[part * kDecHeads + threadIdx.x] = make_float4(-INFINITY, 0.f, 0.f, 0.f);  // a split without blocks
   }
 
-  if (CLUSTER && p.nsplit <= 4) {
+  if (CLUSTER) {
     // ---------------------------------------------------------- on-chip merge
     // Split r owns output columns [r*W, (r+1)*W), W = 512 / nsplit.
     // 1. every CTA reads all splits' (m, l) over DSMEM and computes the same
@@ -589,86 +593,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
     tc_fence_before();
     __syncthreads();
     cluster_sync_all();  // every bulk copy has finished reading its source before any CTA exits
-  } else if (CLUSTER) {
-    // ---------------------------------------------------------- on-chip merge, 8 splits
-    // 1. every CTA reads all splits' (m, l) over DSMEM and computes the same
-    //    merge weights; 2. each thread scales its O^T values (read from TMEM)
-    //    by its split's weight and pushes them, with plain DSMEM stores, into
-    //    the receive buffer of the CTA that owns those output columns
-    //    (split r owns columns [r*W, (r+1)*W), W = 512 / nsplit);
-    // 3. after one cluster barrier every CTA sums its buffer locally.
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();  // (m, l) of every split visible
-    const int r = (int)cluster_rank();
-    const int ns = p.nsplit;
-    const int W = 512 / ns;
-    float* wgt = reinterpret_cast<float*>(smem + LY::Q_OFF);  // [8][64]; Q tiles are idle now
-    float* mls = wgt + 8 * 64;                                 // [3][8][64] all splits' m, l, r
-    float* recv = reinterpret_cast<float*>(smem + LY::RING_OFF);  // [ns][64][W]; the ring is idle now
-    for (int idx = threadIdx.x; idx < ns * 64; idx += blockDim.x) {
-      const int s2 = idx >> 6, h = idx & 63;
-      mls[idx] = *static_cast<const float*>(__cluster_map_shared_rank(m_run + h, s2));
-      mls[8 * 64 + idx] = *static_cast<const float*>(__cluster_map_shared_rank(l_run + h, s2));
-      mls[16 * 64 + idx] = *static_cast<const float*>(__cluster_map_shared_rank(r_run + h, s2));
-    }
-    __syncthreads();
-    if (threadIdx.x < 64) {
-      const int h = threadIdx.x;
-      float M = -INFINITY;
-      for (int s2 = 0; s2 < ns; ++s2)
-        if (mls[8 * 64 + s2 * 64 + h] > 0.f) M = fmaxf(M, mls[s2 * 64 + h]);
-      // O is normalised by the merged sum of the bf16 P that multiplied V,
-      // the LSE by the merged exact sum
-      float Ls = 0.f, Rs = 0.f;
-      for (int s2 = 0; s2 < ns; ++s2) {
-        const float l = mls[8 * 64 + s2 * 64 + h];
-        const float w = l > 0.f ? ex2_approx(mls[s2 * 64 + h] - M) : 0.f;
-        wgt[s2 * 64 + h] = w;
-        Ls += l * w;
-        Rs += mls[16 * 64 + s2 * 64 + h] * w;
-      }
-      const float inv = 1.f / Rs;
-      for (int s2 = 0; s2 < ns; ++s2) wgt[s2 * 64 + h] *= inv;
-      if (r == 0) p.lse[(int64_t)seq * kDecHeads + h] = (M + log2f(Ls)) * 0.69314718055994530942f;
-    }
-    __syncthreads();
-    if (nb > 0 && warp >= 2) {
-      const int quarter = warp & 3, grp = (warp - 2) >> 2, key = quarter * 32 + lane;
-      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll 1
-      for (int u = 0; u < 4; ++u) {
-        const int d = 128 * u + key;  // latent column of this lane
-        const int owner = d / W;
-        float* dst = static_cast<float*>(__cluster_map_shared_rank(recv, owner)) + (size_t)r * 64 * W + (d - owner * W);
-        float o[32];
-        tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int h = 32 * grp + i;
-          dst[(size_t)h * W] = o[i] * wgt[r * 64 + h];
-        }
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();  // every push landed; no CTA touches another's memory after this
-    const int W4 = W / 4;
-    for (int idx = threadIdx.x; idx < kDecHeads * W4; idx += blockDim.x) {
-      const int h = idx / W4;
-      const int j = (idx % W4) * 4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s2 = 0; s2 < ns; ++s2) {
-        if (wgt[s2 * 64 + h] == 0.f) continue;  // a split without blocks pushed nothing
-        const float4 o = *reinterpret_cast<const float4*>(recv + ((size_t)s2 * 64 + h) * W + j);
-        acc.x += o.x;
-        acc.y += o.y;
-        acc.z += o.z;
-        acc.w += o.w;
-      }
-      __nv_bfloat16* dst = p.out + ((int64_t)seq * kDecHeads + h) * 512 + r * W + j;
-      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
-    }
   } else {
     // ---------------------------------------------------------- last CTA merges
     __threadfence();

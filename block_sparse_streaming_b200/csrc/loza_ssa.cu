@@ -18,7 +18,7 @@
 #include "prefill_mla.cuh"
 #include "decode.cuh"
 #include "decode_mla.cuh"
-#include "decode_mla_hs.cuh"
+#include "decode_mla_hb.cuh"
 #include "merge.cuh"
 #include "backward.cuh"
 
@@ -80,14 +80,25 @@ int sm_count() {
 }
 
 // Split-KV plan of the absorbed decode: CTAs per sequence (nsplit) and selected
-// blocks per CTA (bps), sized so that batch * nsplit CTAs fill the GPU in one
-// wave. Up to 8 splits form one thread-block cluster per sequence and merge
-// on chip (no workspace). Only when a few sequences have long windows (more
-// than 8 splits pay off) do the splits merge through the workspace.
+// blocks (or half blocks) per CTA (bps), sized so that batch * nsplit CTAs fill
+// the GPU in one wave.
+//   - a few sequences with long windows (more than 8 blocks, batch * 16 <= SMs):
+//     the block kernel, many splits, merged through the workspace;
+//   - windows of at most 16 blocks while two CTAs per sequence fit (batch * 2
+//     <= SMs): the half-block kernel, up to 4 splits per sequence in a
+//     cluster, merged on chip;
+//   - otherwise the block kernel with up to 4 splits per sequence in a
+//     cluster (one CTA per sequence for large batches), merged on chip.
+// Measured kernel times (64 heads, 8-block window, contexts of 64K-128K;
+// half-block vs the block kernel's best plan): 1 sequence 21.8 vs 25.4 us,
+// 8: 22.2 vs 24.5, 64: 32.5 vs 34.3 (a head-split kernel), 96: 47.2 vs 43.6,
+// 128: 49.0 vs 47.6. With the whole context selected (the dense decode of
+// 64 sequences of 64K-128K) the block kernel took 1.74 ms, the half-block one
+// 2.22 ms.
 struct DecodePlan {
-  int bps, nsplit;
-  bool cluster;
-  bool head_split;  // kHsHeads heads per CTA, every CTA walks all of its sequence's blocks
+  int bps, nsplit;  // half_block: half blocks per split
+  bool cluster;     // the splits of a sequence form a cluster and merge on chip
+  bool half_block;  // 64-row units resident for both MMAs (decode_mla_hb.cuh)
 };
 DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t batch) {
   const int max_blocks = (max_seqlen + kTile - 1) / kTile;
@@ -101,17 +112,17 @@ DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t bat
     const int bps = (count + ns - 1) / ns;
     return {bps, (count + bps - 1) / bps, false, false};
   }
-  // a window of at most 16 blocks and a batch that fills half the GPU or
-  // more with two CTAs per sequence: split the heads, not the blocks, so no
-  // partial results need merging
-  const int per_seq = kDecHeads / kHsHeads;
-  if (count <= 16 && (int64_t)batch * per_seq <= sms && (int64_t)batch * per_seq * 2 > sms)
-    return {count, 1, false, true};
-  // Clusters of 8 CTAs that each hold a full SM's shared memory fit about one
-  // per GPC at a time: more than 8 of them (batch > 8) run in two waves
-  // (measured: 16 sequences took 45 us with 8 CTAs per sequence, 31 us with 4).
+  if (count <= 16 && (int64_t)batch * 2 <= sms) {
+    // half blocks: up to 4 CTAs per sequence in one cluster, each pulling
+    // its share of the rows once
+    const int nh = 2 * count;
+    int ns = 1;
+    while (ns < kHbMaxSplit && ns * 2 <= nh && (int64_t)batch * ns * 2 <= sms) ns *= 2;
+    const int hps = (nh + ns - 1) / ns;
+    return {hps, (nh + hps - 1) / hps, true, true};
+  }
   int ns = 1;
-  while (ns < 8 && ns * 2 <= count && (int64_t)batch * ns * 2 <= sms && !(ns == 4 && batch > 8)) ns *= 2;
+  while (ns < 4 && ns * 2 <= count && (int64_t)batch * ns * 2 <= sms) ns *= 2;
   return {(count + ns - 1) / ns, ns, true, false};
 }
 
@@ -120,7 +131,7 @@ struct DecodeWorkspace {
 };
 DecodeWorkspace decode_workspace(int32_t batch, const DecodePlan& plan) {
   DecodeWorkspace w{0, 0, 0, 0};
-  if (plan.cluster || plan.head_split) return w;
+  if (plan.cluster) return w;
   const size_t parts = (size_t)batch * plan.nsplit * kDecHeads;
   w.o_off = 0;
   w.ml_off = parts * 512 * sizeof(float);
@@ -151,7 +162,7 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
   {
     cuuint64_t dims[3] = {576, (cuuint64_t)n_heads, (cuuint64_t)batch};
     cuuint64_t strides[2] = {576 * 2, (cuuint64_t)n_heads * 576 * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)(plan->head_split ? kHsHeads : kDecHeads), 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)kDecHeads, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     if (fn(&prm->tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -162,9 +173,13 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
     cuuint64_t dims[3] = {576, (cuuint64_t)max_seqlen, (cuuint64_t)batch};
     cuuint64_t strides[2] = {(cuuint64_t)cache_row_stride * 2, (cuuint64_t)cache_batch_stride * 2};
     cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box64[3] = {64, 64, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     if (fn(&prm->tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        fn(&prm->tm_kv64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box64,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return LOZA_ERR_CUDA;
   }
@@ -182,11 +197,23 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
 // Point the kernel at its workspace (unless the plan merges on chip) and launch.
 loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t batch, uint8_t* ws,
                               cudaStream_t st) {
-  if (plan.head_split) {
-    if (cudaFuncSetAttribute(ssa_decode_mla_hs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DecodeHsLayout::SMEM_BYTES) != cudaSuccess)
+  if (plan.half_block) {
+    if (cudaFuncSetAttribute(ssa_decode_mla_hb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeHbLayout::SMEM_BYTES) != cudaSuccess)
       return LOZA_ERR_CUDA;
-    ssa_decode_mla_hs_kernel<<<dim3(kDecHeads / kHsHeads, batch), kHsThreads, DecodeHsLayout::SMEM_BYTES, st>>>(prm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.nsplit, batch, 1);
+    cfg.blockDim = dim3(kHbThreads, 1, 1);
+    cfg.dynamicSmemBytes = DecodeHbLayout::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = plan.nsplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, ssa_decode_mla_hb_kernel, prm) != cudaSuccess) return LOZA_ERR_CUDA;
   } else if (!plan.cluster) {
     const DecodeWorkspace wl = decode_workspace(batch, plan);
     prm.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
@@ -447,7 +474,11 @@ loza_status loza_ssa_decode_paged(const void* q, const void* kv_pool, int32_t nu
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   if (strides[1] >= (cuuint64_t(1) << 40)) return LOZA_ERR_INVALID_ARG;
+  cuuint32_t box64[3] = {64, 64, 1};
   if (fn(&prm.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv_pool), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+      fn(&prm.tm_kv64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv_pool), dims, strides, box64, estr,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return LOZA_ERR_CUDA;

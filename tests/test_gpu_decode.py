@@ -92,6 +92,14 @@ def test_absorbed_decode_split_plans(bss, oracle_mod, batch):
     absorbed_case(bss, oracle_mod, 71 + batch, lens.tolist(), 6144)
 
 
+def test_absorbed_decode_half_block_boundaries(bss, oracle_mod):
+    """Positions at and around the half-block boundaries of the own block (its
+    second half present or not, full or partial), the sink block as the own
+    block, and more splits (4 per sequence) than some sequences have half blocks."""
+    lens = [1, 63, 64, 65, 100, 128, 129, 192, 193, 256, 1025, 1088, 1089]
+    absorbed_case(bss, oracle_mod, 93, lens, 1152)
+
+
 def test_absorbed_decode_wide_window_two_splits(bss, oracle_mod):
     """A 22-block window (s=2, l=20) on 40 sequences: two CTAs of a cluster
     split each sequence's blocks and merge on chip."""
