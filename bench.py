@@ -262,6 +262,52 @@ def time_launches(fn, stream, n, flush=None):
     return statistics.mean(ts), ts
 
 
+def time_rotating(bss, q, cache, seqlens, cap, params, ws, copies, reps=10):
+    """Mean device time (ms) of one decode call when calls run back to back
+    over `copies` independent copies of q, the cache and the outputs: each
+    call's data was last touched copies - 1 calls earlier, with more bytes
+    than L2 holds touched in between, so no flush (and none of the write-back
+    a flush write leaves in L2) is needed. One pass over the copies is
+    captured in a CUDA graph, so no host time separates the calls."""
+    import torch
+    qs = [q] + [q.clone() for _ in range(copies - 1)]
+    caches = [cache] + [cache.clone() for _ in range(copies - 1)]
+    outs = [torch.empty((q.shape[0], H, DV), dtype=torch.bfloat16, device=q.device) for _ in range(copies)]
+    lses = [torch.empty((q.shape[0], H), dtype=torch.float32, device=q.device) for _ in range(copies)]
+
+    def one_pass():
+        for i in range(copies):
+            bss.loza_ssa_decode(qs[i], caches[i], None, seqlens, cap, params, out=outs[i], lse=lses[i],
+                                workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            one_pass()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    # relaxed: the library sets kernel attributes (not stream work) on every call
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        one_pass()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for _ in range(reps):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * copies)
+    del g, qs, caches, outs, lses
+    torch.cuda.empty_cache()
+    return ms
+
+
 def decode_bytes(lens, n_local=LW):
     """Algorithmic bytes of one absorbed decode call: every selected latent row once
     (576 bf16; K and V share it), q, out and lse."""
@@ -277,9 +323,11 @@ def decode_bytes(lens, n_local=LW):
     return rows * DQK * 2 + n * H * (DQK * 2 + DV * 2 + 4)
 
 
-def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20):
+def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20, rotating=0):
     """SSA decode (and the dense full-context decode) on a latent cache
-    [len(lens), cap, 576]; L2 flushed (256 MB write) before every timed call."""
+    [len(lens), cap, 576]; L2 flushed (256 MB write) before every timed call.
+    rotating > 1: also time the SSA decode over that many copies of the inputs
+    and outputs, back to back in a CUDA graph (time_rotating)."""
     import torch
     Bn = len(lens)
     q = synth.torch_normal_bf16((Bn, H, DQK), synth.workload_seed(3) * 1000 + 1, device)
@@ -307,6 +355,14 @@ def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20):
         res[name] = {"ms": ms, "bytes": nbytes, "GB/s": nbytes / (ms / 1000.0) / 1e9, "launches_timed": n}
         if bss.device_status() != 0:
             raise RuntimeError("device status reports a timed-out wait in decode")
+        if name == "ssa" and rotating > 1:
+            try:
+                ms_r = time_rotating(bss, q, cache, seqlens, cap, params, ws, rotating)
+                res["ssa_rotating"] = {"ms": ms_r, "bytes": nbytes, "GB/s": nbytes / (ms_r / 1000.0) / 1e9,
+                                       "copies": rotating}
+            except RuntimeError as e:  # a secondary timing; the flushed one above stands
+                torch.cuda.synchronize()
+                print(f"rotating decode timing skipped: {e}", file=sys.stderr)
     del cache
     torch.cuda.empty_cache()
     return res
@@ -319,7 +375,7 @@ def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None, ctx=None
     lens = synth.uniform_lengths(g, w["batch"], lo, hi).tolist()
     if batch is not None:
         lens = lens[:batch]
-    r = run_decode(bss, device, stream, lens, hi)
+    r = run_decode(bss, device, stream, lens, hi, rotating=4)
     hbm = float(peaks["hbm_gbs"])
     ssa = r["ssa"]
     name = w["name"] if len(lens) == w["batch"] else f"{w['name']} (first {len(lens)} sequences)"
@@ -333,6 +389,12 @@ def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None, ctx=None
                         "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
                         "kernel": "ssa_decode_mla_hb_kernel"},
            "timing": "mean of per-call CUDA events, L2 flushed (256 MB write) before each call"}
+    if "ssa_rotating" in r:
+        rr = r["ssa_rotating"]
+        out["rotating"] = {"ms_per_call": rr["ms"], "GB/s": rr["GB/s"], "frac_of_hbm": rr["GB/s"] / hbm,
+                           "timing": f"calls back to back over {rr['copies']} copies of q, cache and outputs "
+                                     "(more than L2 touched between two uses of a copy; no flush), one pass "
+                                     "over the copies captured in a CUDA graph, mean over 10 replays"}
     if "dense" in r:
         d = r["dense"]
         out["dense"] = {"ms_per_call": d["ms"], "bytes_per_call": d["bytes"], "GB/s": d["GB/s"],
