@@ -137,16 +137,33 @@ struct HostPipe {
 };
 HostPipe g_host_pipes[kMaxDevices];
 
+void host_pipe_release(HostPipe& hp) {
+  if (hp.h2d) cudaStreamDestroy(hp.h2d);
+  if (hp.d2h) cudaStreamDestroy(hp.d2h);
+  if (hp.start) cudaEventDestroy(hp.start);
+  for (int i = 0; i < kHostSlots; ++i) {
+    if (hp.in_done[i]) cudaEventDestroy(hp.in_done[i]);
+    if (hp.run_done[i]) cudaEventDestroy(hp.run_done[i]);
+    if (hp.out_done[i]) cudaEventDestroy(hp.out_done[i]);
+    hp.in_done[i] = hp.run_done[i] = hp.out_done[i] = nullptr;
+  }
+  hp.h2d = hp.d2h = nullptr;
+  hp.start = nullptr;
+}
+
+// All or nothing: a failed creation releases what was created before it.
 bool host_pipe_init(HostPipe& hp) {
   if (hp.ready) return true;
-  if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
-  if (cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess) return false;
-  if (cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) != cudaSuccess) return false;
-  for (int i = 0; i < kHostSlots; ++i) {
-    if (cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&hp.run_done[i], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) != cudaSuccess)
-      return false;
+  bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; ok && i < kHostSlots; ++i)
+    ok = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&hp.run_done[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    host_pipe_release(hp);
+    return false;
   }
   hp.ready = true;
   return true;
