@@ -158,3 +158,25 @@ def test_prefill_host_workspace_size():
     # the unbounded window runs as one chunk: one slot of the whole sequence
     dense = size(1, 8192, 8192, 4, 4, 64, 64, bss.Params(0.125, n_local=bss.LOZA_UNBOUNDED))
     assert dense >= 8192 * 4 * (64 * 2 * 4 + 4)
+
+
+def test_prefill_host_binding_rejects_before_any_device_work(L):
+    """The binding checks dtypes, ranks and contiguity, and the shape through the
+    workspace query, before it allocates or launches anything (runs without a GPU)."""
+    import torch
+    p = bss.Params(1 / math.sqrt(192))
+    q = torch.zeros((256, 4, 576), dtype=torch.bfloat16)
+    lat = torch.zeros((256, 1, 576), dtype=torch.bfloat16)
+    count = L.loza_launch_count()
+    with pytest.raises(TypeError):
+        bss.loza_ssa_prefill_host(q.float(), lat, lat[:, :, :512], p)
+    with pytest.raises(TypeError):
+        bss.loza_ssa_prefill_host(q[0], lat, lat[:, :, :512], p)
+    with pytest.raises(ValueError):
+        bss.loza_ssa_prefill_host(q.transpose(1, 2).contiguous().transpose(1, 2), lat, lat[:, :, :512], p)
+    with pytest.raises(ValueError):  # a latent V must share K's rows
+        bss.loza_ssa_prefill_host(q, lat, lat.reshape(128, 2, 576)[:, :1, :512], p)
+    with pytest.raises(bss.LozaError) as e:  # the whole 576-wide latent as V: no such head dims
+        bss.loza_ssa_prefill_host(q, lat, lat, p)
+    assert e.value.status == -2
+    assert L.loza_launch_count() == count
