@@ -9,7 +9,8 @@ The arithmetic lives in ``ssa_ref.c`` (plain C, double precision, OpenMP over
 rows); this module only compiles it with gcc and marshals numpy arrays. What it
 computes is stated in the header of ``ssa_ref.c`` with the passages it follows
 (Efficient Context Scaling with LongCat ZigZag Attention: page 1 section 01,
-page 2 section 2.2, page 5).
+page 2 section 2.2, page 5), and for the token-granular variant, page 4's
+streaming-aware index (a fixed set of sink tokens plus a sliding window).
 
 Every array argument holding model values is a numpy ``uint16`` array of bf16
 bit patterns; the C side widens each exactly to double.
@@ -54,6 +55,12 @@ def _load():
             _u16p, _u16p, _u16p, _i32p, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            _i64p, ctypes.c_int64, _f64p, _f64p]
+        lib.ssa_oracle_forward_tokens_rows.restype = ctypes.c_int
+        lib.ssa_oracle_forward_tokens_rows.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
             _i64p, ctypes.c_int64, _f64p, _f64p]
         lib.ssa_oracle_decode.restype = ctypes.c_int
         lib.ssa_oracle_decode.argtypes = [
@@ -103,6 +110,26 @@ def forward(q, k, v, cu_seqlens, n_heads, n_kv_heads, block_size=128, n_sink=1,
                                          float(scale), rows, len(rows), o, lse)
     if rc != 0:
         raise ValueError("oracle forward rejected its arguments")
+    return o, lse
+
+
+def forward_tokens(q, k, v, cu_seqlens, n_heads, n_kv_heads, sink_tokens=16, window_tokens=1024,
+                   scale=1.0, rows=None):
+    """Token-granular variant: query i sees the keys t <= i with t < sink_tokens
+    or i - t < window_tokens (page 4: 16 sink tokens and a 1,024-token sliding
+    window). Same arguments and results as forward() otherwise."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    T = int(cu[-1])
+    d_qk, d_v = q.shape[-1], v.shape[-1]
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    o = np.zeros((len(rows), n_heads, d_v), np.float64)
+    lse = np.zeros((len(rows), n_heads), np.float64)
+    rc = _load().ssa_oracle_forward_tokens_rows(q, k, v, cu, len(cu) - 1, n_heads, n_kv_heads, d_qk, d_v,
+                                                int(sink_tokens), int(window_tokens), float(scale), rows,
+                                                len(rows), o, lse)
+    if rc != 0:
+        raise ValueError("oracle forward (token window) rejected its arguments")
     return o, lse
 
 

@@ -78,12 +78,25 @@ static int64_t visible_keys(int64_t i, int b, int n_sink, int n_local, int64_t *
     return c;
 }
 
+/* The token-granular variant (page 4, the LSA article's streaming-aware
+ * index: a fixed part of every query's key set made of the first sink tokens
+ * and a sliding window of the most recent tokens, 16 + 1,024 there):
+ *   A(i) = { t <= i : t < sink_tokens  or  i - t < window_tokens }.
+ * Written into keys[] in increasing order of t; returns |A(i)|. */
+static int64_t visible_tokens(int64_t i, int64_t sink_tokens, int64_t window_tokens, int64_t *keys) {
+    int64_t c = 0;
+    for (int64_t t = 0; t <= i; ++t)
+        if (t < sink_tokens || i - t < window_tokens) keys[c++] = t;
+    return c;
+}
+
 typedef struct {
     const uint16_t *q, *k, *v;   /* [T,H,dqk], [T,Hkv,dqk], [T,Hkv,dv] */
     int64_t total;
     int n_heads, n_kv_heads, d_qk, d_v;
     int b, n_sink, n_local;
     double scale;
+    int64_t sink_tokens, window_tokens;  /* token-granular variant when window_tokens > 0 */
 } problem;
 
 /* Steps 3-5 for query position i of the sequence starting at global row base,
@@ -93,7 +106,8 @@ static double row_forward(const problem *p, int64_t base, int64_t i, int h,
                           int64_t *keys, double *z, int64_t *count, double *o) {
     const int hk = h / (p->n_heads / p->n_kv_heads);
     const uint16_t *qi = p->q + ((base + i) * p->n_heads + h) * (int64_t)p->d_qk;
-    const int64_t c = visible_keys(i, p->b, p->n_sink, p->n_local, keys);
+    const int64_t c = p->window_tokens > 0 ? visible_tokens(i, p->sink_tokens, p->window_tokens, keys)
+                                           : visible_keys(i, p->b, p->n_sink, p->n_local, keys);
     double m = -INFINITY;
     for (int64_t a = 0; a < c; ++a) {
         const uint16_t *kt = p->k + ((base + keys[a]) * p->n_kv_heads + hk) * (int64_t)p->d_qk;
@@ -136,21 +150,11 @@ static int check_shape(const int32_t *cu, int batch, int n_heads, int n_kv_heads
     return 0;
 }
 
-/*
- * Forward for a list of global query rows (all heads of each row).
- * rows: n_rows global row indices in [0, cu[batch]).
- * o_out [n_rows, H, d_v], lse_out [n_rows, H].
- */
-int ssa_oracle_forward_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                            const int32_t *cu_seqlens, int batch,
-                            int n_heads, int n_kv_heads, int d_qk, int d_v,
-                            int block_size, int n_sink, int n_local, double scale,
-                            const int64_t *rows, int64_t n_rows,
-                            double *o_out, double *lse_out) {
-    if (!q || !k || !v || !cu_seqlens || !rows || !o_out || !lse_out) return -1;
-    if (check_shape(cu_seqlens, batch, n_heads, n_kv_heads, d_qk, d_v, block_size)) return -1;
-    problem p = {q, k, v, cu_seqlens[batch], n_heads, n_kv_heads, d_qk, d_v,
-                 block_size, n_sink, n_local, scale};
+/* Steps 3-5 for a list of global query rows, all heads of each row. */
+static int forward_rows(const problem *pp, const int32_t *cu_seqlens, int batch, const int64_t *rows,
+                        int64_t n_rows, double *o_out, double *lse_out) {
+    const problem p = *pp;
+    const int n_heads = p.n_heads, d_v = p.d_v;
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int64_t r = 0; r < n_rows * n_heads; ++r) {
@@ -169,6 +173,42 @@ int ssa_oracle_forward_rows(const uint16_t *q, const uint16_t *k, const uint16_t
         free(z);
     }
     return bad ? -1 : 0;
+}
+
+/*
+ * Forward for a list of global query rows (all heads of each row).
+ * rows: n_rows global row indices in [0, cu[batch]).
+ * o_out [n_rows, H, d_v], lse_out [n_rows, H].
+ */
+int ssa_oracle_forward_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *cu_seqlens, int batch,
+                            int n_heads, int n_kv_heads, int d_qk, int d_v,
+                            int block_size, int n_sink, int n_local, double scale,
+                            const int64_t *rows, int64_t n_rows,
+                            double *o_out, double *lse_out) {
+    if (!q || !k || !v || !cu_seqlens || !rows || !o_out || !lse_out) return -1;
+    if (check_shape(cu_seqlens, batch, n_heads, n_kv_heads, d_qk, d_v, block_size)) return -1;
+    problem p = {q, k, v, cu_seqlens[batch], n_heads, n_kv_heads, d_qk, d_v,
+                 block_size, n_sink, n_local, scale, 0, 0};
+    return forward_rows(&p, cu_seqlens, batch, rows, n_rows, o_out, lse_out);
+}
+
+/*
+ * The same for the token-granular window (visible_tokens): sink_tokens >= 0,
+ * window_tokens >= 1.
+ */
+int ssa_oracle_forward_tokens_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                   const int32_t *cu_seqlens, int batch,
+                                   int n_heads, int n_kv_heads, int d_qk, int d_v,
+                                   int64_t sink_tokens, int64_t window_tokens, double scale,
+                                   const int64_t *rows, int64_t n_rows,
+                                   double *o_out, double *lse_out) {
+    if (!q || !k || !v || !cu_seqlens || !rows || !o_out || !lse_out) return -1;
+    if (check_shape(cu_seqlens, batch, n_heads, n_kv_heads, d_qk, d_v, 1)) return -1;
+    if (sink_tokens < 0 || window_tokens < 1) return -1;
+    problem p = {q, k, v, cu_seqlens[batch], n_heads, n_kv_heads, d_qk, d_v,
+                 1, 0, 0, scale, sink_tokens, window_tokens};
+    return forward_rows(&p, cu_seqlens, batch, rows, n_rows, o_out, lse_out);
 }
 
 /*
@@ -248,7 +288,7 @@ int ssa_oracle_backward_rows(const uint16_t *q, const uint16_t *k, const uint16_
     if (n_k_rows > 0 && (!k_rows || !dk_out || !dv_out)) return -1;
     if (check_shape(cu_seqlens, batch, n_heads, n_kv_heads, d_qk, d_v, block_size)) return -1;
     problem p = {q, k, v, cu_seqlens[batch], n_heads, n_kv_heads, d_qk, d_v,
-                 block_size, n_sink, n_local, scale};
+                 block_size, n_sink, n_local, scale, 0, 0};
     const int group = n_heads / n_kv_heads;
     int bad = 0;
 
