@@ -198,6 +198,8 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
 loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t batch, uint8_t* ws,
                               cudaStream_t st) {
   if (plan.half_block) {
+    // the kernel's merge buffers hold at most kHbMaxSplit splits
+    if (plan.nsplit < 1 || plan.nsplit > kHbMaxSplit) return LOZA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(ssa_decode_mla_hb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DecodeHbLayout::SMEM_BYTES) != cudaSuccess)
       return LOZA_ERR_CUDA;
@@ -226,6 +228,8 @@ loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t
       return LOZA_ERR_CUDA;
     ssa_decode_mla_kernel<false><<<dim3(plan.nsplit, batch), kDecThreads, DecodeLayout::SMEM_BYTES, st>>>(prm);
   } else {
+    // the cluster merge handles at most 4 splits
+    if (plan.nsplit < 1 || plan.nsplit > 4) return LOZA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(ssa_decode_mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DecodeLayout::SMEM_BYTES) != cudaSuccess)
       return LOZA_ERR_CUDA;
