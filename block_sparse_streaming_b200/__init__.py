@@ -79,8 +79,8 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_prefill.argtypes = [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
                                        _i64, _i64, _i64, Params, _vp, _vp, _vp, _sz, _vp]
         L.loza_ssa_prefill_host.restype = ctypes.c_int
-        L.loza_ssa_prefill_host.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, Params, _vp, _vp, _vp, _sz,
-                                            _vp]
+        L.loza_ssa_prefill_host.argtypes = [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, Params,
+                                            _vp, _vp, _vp, _sz, _vp]
         L.loza_ssa_decode.restype = ctypes.c_int
         L.loza_ssa_decode.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i64, _i64, _i32, _i32, _i32, _i32,
                                       Params, _vp, _vp, _vp, _sz, _vp]
@@ -170,19 +170,23 @@ def loza_ssa_prefill(q, k, v, cu_seqlens, max_seqlen: int, params: Params, out=N
     return out, lse
 
 
-def loza_ssa_prefill_host(q, k, v, params: Params, out=None, lse=None, workspace=None, stream=None):
-    """Prefill of one sequence from and to host memory (copies inside the call,
-    overlapped with the kernels). q [L, H, d_qk], k [L, Hkv, d_qk], v [L, Hkv, d_v]:
+def loza_ssa_prefill_host(q, k, v, params: Params, cu_seqlens=None, max_seqlen=None, out=None, lse=None,
+                          workspace=None, stream=None):
+    """Prefill of a packed batch from and to host memory (copies inside the call,
+    overlapped with the kernels). q [T, H, d_qk], k [T, Hkv, d_qk], v [T, Hkv, d_v]:
     contiguous bf16 CPU tensors (pinned for overlap); absorbed MLA: pass the
-    latent [L, 1, 576] as k and v (the same tensor, or its first 512 columns).
-    Returns (out [L, H, d_v] bf16, lse [L, H] fp32) as CPU tensors; they hold
-    the results once `stream` (default: the current CUDA stream) has passed
-    the call. The workspace is a CUDA uint8 tensor (allocated if None)."""
+    latent [T, 1, 576] as k and v (the same tensor, or its first 512 columns).
+    cu_seqlens: host sequence offsets [0, ..., T] (a list, numpy array or CPU
+    tensor; None = one sequence of T tokens). Returns (out [T, H, d_v] bf16,
+    lse [T, H] fp32) as CPU tensors; they hold the results once `stream`
+    (default: the current CUDA stream) has passed the call. The workspace is a
+    CUDA uint8 tensor (allocated if None)."""
+    import numpy as np
     import torch
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.dim() != 3:
             raise TypeError(f"{n} must be a 3-D bf16 tensor")
-    L, H, d_qk = q.shape
+    T, H, d_qk = q.shape
     Hkv, d_v = k.shape[1], v.shape[2]
     latent = v.data_ptr() == k.data_ptr()
     for t, n in ((q, "q"), (k, "k")) + (() if latent else ((v, "v"),)):
@@ -190,21 +194,33 @@ def loza_ssa_prefill_host(q, k, v, params: Params, out=None, lse=None, workspace
             raise ValueError(f"{n} must be contiguous")
     if latent and v.stride(0) != k.stride(0):
         raise ValueError("a latent v must be a column slice of k")
+    if cu_seqlens is None:
+        cu_seqlens = [0, T]
+    if isinstance(cu_seqlens, torch.Tensor):
+        cu_seqlens = cu_seqlens.cpu().numpy()
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    if cu.ndim != 1 or cu.size < 2:
+        raise ValueError("cu_seqlens needs at least two offsets")
+    batch = cu.size - 1
+    if max_seqlen is None:
+        max_seqlen = max(1, int(np.max(np.diff(cu))))
     pin = q.device.type == "cpu" and q.is_pinned()
     if out is None:
-        out = torch.empty((L, H, d_v), dtype=torch.bfloat16, device=q.device, pin_memory=pin)
+        out = torch.empty((T, H, d_v), dtype=torch.bfloat16, device=q.device, pin_memory=pin)
     if lse is None:
-        lse = torch.empty((L, H), dtype=torch.float32, device=q.device, pin_memory=pin)
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device, pin_memory=pin)
     if not out.is_contiguous() or not lse.is_contiguous():
         raise ValueError("out and lse must be contiguous")
     if workspace is None:
-        n = workspace_size(LOZA_OP_PREFILL_HOST, 1, L, L, H, Hkv, d_qk, d_v, params)
+        n = workspace_size(LOZA_OP_PREFILL_HOST, batch, T, int(max_seqlen), H, Hkv, d_qk, d_v, params)
         if n == 0:
             raise LozaError(-2, "loza_ssa_prefill_host")
         workspace = torch.empty(n, dtype=torch.uint8, device="cuda")
     _require(workspace, "workspace", torch.uint8)
-    rc = lib().loza_ssa_prefill_host(_ptr(q), _ptr(k), _ptr(k if latent else v), L, H, Hkv, d_qk, d_v, params,
-                                     _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    rc = lib().loza_ssa_prefill_host(_ptr(q), _ptr(k), _ptr(k if latent else v),
+                                     cu.ctypes.data_as(ctypes.c_void_p), batch, T, int(max_seqlen), H, Hkv, d_qk,
+                                     d_v, params, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                     _stream_ptr(stream))
     _check(rc, "loza_ssa_prefill_host")
     return out, lse
 

@@ -565,11 +565,12 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
     return 0;
   }
   if (op == LOZA_OP_PREFILL_HOST) {
-    if (batch != 1 || total_tokens != max_seqlen || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v)) return 0;
-    const HostChunkPlan h = host_chunk_plan(total_tokens, p);
+    if (total_tokens < max_seqlen || total_tokens > INT32_MAX || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v))
+      return 0;
+    const HostChunkPlan h = host_chunk_plan(max_seqlen, p);
     const size_t pf = loza_ssa_workspace_size(LOZA_OP_PREFILL, 1, h.rows_max, (int32_t)h.rows_max, n_heads,
                                               n_kv_heads, d_qk, d_v, p);
-    return host_layout(h, pf, n_heads, n_kv_heads, d_qk, d_v).total;
+    return host_layout(h, host_chunk_cap(batch, total_tokens), pf, n_heads, n_kv_heads, d_qk, d_v).total;
   }
   if (op == LOZA_OP_BACKWARD) {
     if (n_kv_heads != n_heads || p.n_local == LOZA_UNBOUNDED || total_tokens < 1) return 0;
@@ -677,20 +678,43 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
   }
 }
 
-loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, int64_t seq_len, int32_t n_heads,
+loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                  int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t n_heads,
                                   int32_t n_kv_heads, int32_t d_qk, int32_t d_v, loza_ssa_params p, void* out,
                                   float* lse, void* workspace, size_t workspace_bytes, loza_stream_t stream) {
-  if (!q || !k || !v || !out || !lse) return LOZA_ERR_INVALID_ARG;
-  if (seq_len < 1 || seq_len > INT32_MAX) return LOZA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !cu_seqlens || !out || !lse) return LOZA_ERR_INVALID_ARG;
+  if (batch < 1 || total_tokens < 1 || total_tokens > INT32_MAX || max_seqlen < 1 || max_seqlen > total_tokens)
+    return LOZA_ERR_INVALID_ARG;
+  // cu_seqlens is host memory: {0, ..., total_tokens}, non-decreasing, no sequence longer than max_seqlen
+  if (cu_seqlens[0] != 0 || cu_seqlens[batch] != total_tokens) return LOZA_ERR_INVALID_ARG;
+  for (int32_t n = 0; n < batch; ++n)
+    if (cu_seqlens[n + 1] < cu_seqlens[n] || cu_seqlens[n + 1] - cu_seqlens[n] > max_seqlen)
+      return LOZA_ERR_INVALID_ARG;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
   if (!window_ok(p) || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v)) return LOZA_ERR_UNSUPPORTED;
   const bool latent_v = (v == k);
   if (latent_v && d_v > d_qk) return LOZA_ERR_INVALID_ARG;
-  const size_t need = loza_ssa_workspace_size(LOZA_OP_PREFILL_HOST, 1, seq_len, (int32_t)seq_len, n_heads,
+  const size_t need = loza_ssa_workspace_size(LOZA_OP_PREFILL_HOST, batch, total_tokens, max_seqlen, n_heads,
                                               n_kv_heads, d_qk, d_v, p);
   if (need == 0) return LOZA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LOZA_ERR_INVALID_ARG;
   if (workspace_bytes < need) return LOZA_ERR_WORKSPACE;
+
+  // every chunk of every sequence, in order
+  struct Work {
+    int64_t row0;  // the sequence's first packed row
+    HostChunk ck;
+  };
+  std::vector<Work> work;
+  for (int32_t n = 0; n < batch; ++n) {
+    const int64_t L = cu_seqlens[n + 1] - cu_seqlens[n];
+    if (L == 0) continue;
+    const HostChunkPlan hn = host_chunk_plan(L, p);
+    for (int64_t c = 0; c < hn.n_chunks; ++c) work.push_back({(int64_t)cu_seqlens[n], host_chunk(hn, c, L, p)});
+  }
+  const HostChunkPlan h = host_chunk_plan(max_seqlen, p);
+  const int64_t cap = host_chunk_cap(batch, total_tokens);
+  if ((int64_t)work.size() > cap) return LOZA_ERR_UNSUPPORTED;  // cannot happen: the cap bounds every plan
 
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LOZA_ERR_CUDA;
@@ -698,10 +722,10 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, i
   std::lock_guard<std::mutex> lock(hp.mu);
   if (!host_pipe_init(hp)) return LOZA_ERR_CUDA;
 
-  const HostChunkPlan h = host_chunk_plan(seq_len, p);
   const size_t pf = loza_ssa_workspace_size(LOZA_OP_PREFILL, 1, h.rows_max, (int32_t)h.rows_max, n_heads,
                                             n_kv_heads, d_qk, d_v, p);
-  const HostLayout w = host_layout(h, pf, n_heads, n_kv_heads, d_qk, d_v);
+  const HostLayout w = host_layout(h, cap, pf, n_heads, n_kv_heads, d_qk, d_v);
+  const int slots = (int)std::min<int64_t>(w.slots, (int64_t)work.size());
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t q_row = (size_t)n_heads * d_qk * 2, k_row = (size_t)n_kv_heads * d_qk * 2;
   const size_t v_row = (size_t)n_kv_heads * d_v * 2, o_row = (size_t)n_heads * d_v * 2;
@@ -712,16 +736,17 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, i
   uint8_t* oh = static_cast<uint8_t*>(out);
   uint8_t* lh = reinterpret_cast<uint8_t*>(lse);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (work.empty()) return LOZA_OK;  // only empty sequences
 #define LOZA_CU(x) \
   do {                                  \
     if ((x) != cudaSuccess) return LOZA_ERR_CUDA; \
   } while (0)
 
   // the local cu_seqlens {0, local length} of every chunk, staged from pageable memory
-  std::vector<int32_t> cu((size_t)h.n_chunks * 2);
-  for (int64_t c = 0; c < h.n_chunks; ++c) {
-    cu[2 * c] = 0;
-    cu[2 * c + 1] = (int32_t)host_chunk(h, c, seq_len, p).local_len();
+  std::vector<int32_t> cu(work.size() * 2);
+  for (size_t g = 0; g < work.size(); ++g) {
+    cu[2 * g] = 0;
+    cu[2 * g + 1] = (int32_t)work[g].ck.local_len();
   }
   // the copy streams start after the caller's earlier work on `stream`
   LOZA_CU(cudaEventRecord(hp.start, st));
@@ -730,9 +755,10 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, i
   int32_t* cu_dev = reinterpret_cast<int32_t*>(ws + w.cu_off);
   LOZA_CU(cudaMemcpyAsync(cu_dev, cu.data(), cu.size() * sizeof(int32_t), cudaMemcpyHostToDevice, hp.h2d));
 
-  for (int64_t c = 0; c < h.n_chunks; ++c) {
-    const int sl = (int)(c % h.slots);
-    const HostChunk ck = host_chunk(h, c, seq_len, p);
+  for (size_t g = 0; g < work.size(); ++g) {
+    const int sl = (int)(g % slots);
+    const HostChunk& ck = work[g].ck;
+    const int64_t r0 = work[g].row0;  // sequence-relative rows + r0 = packed rows
     uint8_t* slot = ws + w.slot_off + (size_t)sl * w.slot_bytes;
     uint8_t* qd = slot + w.q_off;
     uint8_t* kd = slot + w.k_off;
@@ -742,28 +768,30 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, i
     const int64_t pre_rows = ck.pre * kTile, own = ck.q1 - ck.q0;
 
     // copy in: the slot's inputs are free once the chunk that used them ran
-    if (c >= h.slots) LOZA_CU(cudaStreamWaitEvent(hp.h2d, hp.run_done[sl], 0));
+    if (g >= (size_t)slots) LOZA_CU(cudaStreamWaitEvent(hp.h2d, hp.run_done[sl], 0));
     if (pre_rows > 0) LOZA_CU(cudaMemsetAsync(qd, 0, (size_t)pre_rows * q_row, hp.h2d));
-    LOZA_CU(cudaMemcpyAsync(qd + (size_t)pre_rows * q_row, qh + (size_t)ck.q0 * q_row, (size_t)own * q_row,
+    LOZA_CU(cudaMemcpyAsync(qd + (size_t)pre_rows * q_row, qh + (size_t)(r0 + ck.q0) * q_row, (size_t)own * q_row,
                             cudaMemcpyDefault, hp.h2d));
-    LOZA_CU(cudaMemcpyAsync(kd, kh + (size_t)ck.src0 * k_row, (size_t)ck.n0 * k_row, cudaMemcpyDefault, hp.h2d));
+    LOZA_CU(cudaMemcpyAsync(kd, kh + (size_t)(r0 + ck.src0) * k_row, (size_t)ck.n0 * k_row, cudaMemcpyDefault,
+                            hp.h2d));
     if (ck.n1 > 0)
-      LOZA_CU(cudaMemcpyAsync(kd + (size_t)ck.n0 * k_row, kh + (size_t)ck.src1 * k_row, (size_t)ck.n1 * k_row,
+      LOZA_CU(cudaMemcpyAsync(kd + (size_t)ck.n0 * k_row, kh + (size_t)(r0 + ck.src1) * k_row, (size_t)ck.n1 * k_row,
                               cudaMemcpyDefault, hp.h2d));
     if (!latent_v) {
-      LOZA_CU(cudaMemcpyAsync(vd, vh + (size_t)ck.src0 * v_row, (size_t)ck.n0 * v_row, cudaMemcpyDefault, hp.h2d));
+      LOZA_CU(cudaMemcpyAsync(vd, vh + (size_t)(r0 + ck.src0) * v_row, (size_t)ck.n0 * v_row, cudaMemcpyDefault,
+                              hp.h2d));
       if (ck.n1 > 0)
-        LOZA_CU(cudaMemcpyAsync(vd + (size_t)ck.n0 * v_row, vh + (size_t)ck.src1 * v_row, (size_t)ck.n1 * v_row,
-                                cudaMemcpyDefault, hp.h2d));
+        LOZA_CU(cudaMemcpyAsync(vd + (size_t)ck.n0 * v_row, vh + (size_t)(r0 + ck.src1) * v_row,
+                                (size_t)ck.n1 * v_row, cudaMemcpyDefault, hp.h2d));
     }
     LOZA_CU(cudaEventRecord(hp.in_done[sl], hp.h2d));
 
     // compute on the caller's stream: the slot's outputs are free once copied out
     LOZA_CU(cudaStreamWaitEvent(st, hp.in_done[sl], 0));
-    if (c >= h.slots) LOZA_CU(cudaStreamWaitEvent(st, hp.out_done[sl], 0));
+    if (g >= (size_t)slots) LOZA_CU(cudaStreamWaitEvent(st, hp.out_done[sl], 0));
     const int32_t len = (int32_t)ck.local_len();
     const loza_status rc = loza_ssa_prefill(
-        qd, kd, vd, cu_dev + 2 * c, 1, len, len, n_heads, n_kv_heads, d_qk, d_v, (int64_t)n_heads * d_qk,
+        qd, kd, vd, cu_dev + 2 * g, 1, len, len, n_heads, n_kv_heads, d_qk, d_v, (int64_t)n_heads * d_qk,
         (int64_t)n_kv_heads * d_qk, latent_v ? (int64_t)n_kv_heads * d_qk : (int64_t)n_kv_heads * d_v, p, od, ld,
         pf > 0 ? ws + w.pf_off : nullptr, pf, stream);
     if (rc != LOZA_OK) return rc;
@@ -771,14 +799,15 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, i
 
     // copy out the own rows
     LOZA_CU(cudaStreamWaitEvent(hp.d2h, hp.run_done[sl], 0));
-    LOZA_CU(cudaMemcpyAsync(oh + (size_t)ck.q0 * o_row, od + (size_t)pre_rows * o_row, (size_t)own * o_row,
+    LOZA_CU(cudaMemcpyAsync(oh + (size_t)(r0 + ck.q0) * o_row, od + (size_t)pre_rows * o_row, (size_t)own * o_row,
                             cudaMemcpyDefault, hp.d2h));
-    LOZA_CU(cudaMemcpyAsync(lh + (size_t)ck.q0 * l_row, reinterpret_cast<uint8_t*>(ld) + (size_t)pre_rows * l_row,
-                            (size_t)own * l_row, cudaMemcpyDefault, hp.d2h));
+    LOZA_CU(cudaMemcpyAsync(lh + (size_t)(r0 + ck.q0) * l_row,
+                            reinterpret_cast<uint8_t*>(ld) + (size_t)pre_rows * l_row, (size_t)own * l_row,
+                            cudaMemcpyDefault, hp.d2h));
     LOZA_CU(cudaEventRecord(hp.out_done[sl], hp.d2h));
   }
   // the caller's stream completes when the last rows have reached the host
-  LOZA_CU(cudaStreamWaitEvent(st, hp.out_done[(h.n_chunks - 1) % h.slots], 0));
+  LOZA_CU(cudaStreamWaitEvent(st, hp.out_done[(work.size() - 1) % slots], 0));
 #undef LOZA_CU
   return LOZA_OK;
 }

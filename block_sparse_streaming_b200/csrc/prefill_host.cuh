@@ -1,7 +1,8 @@
 // prefill_host.cuh - host-side pipeline of loza_ssa_prefill_host: the prefill of
-// one sequence whose tensors live in host memory, streamed through the GPU in
-// chunks of query blocks so that the PCIe copies in both directions overlap
-// each other and the kernels.
+// a packed batch of sequences whose tensors live in host memory, streamed
+// through the GPU in chunks of query blocks (each chunk inside one sequence)
+// so that the PCIe copies in both directions overlap each other and the
+// kernels.
 //
 // A query in block j reads the sink blocks 0 .. s-1 and the local blocks
 // j-l+1 .. j (LongCat ZigZag Attention, page 1 section 01 (1)-(2)). A chunk of
@@ -37,7 +38,6 @@ struct HostChunkPlan {
   int64_t cb;        // own blocks per chunk
   int64_t n_chunks;
   int64_t pre_max;   // prepended blocks at most
-  int slots;
   int64_t rows_max;  // local rows of the largest chunk
 };
 
@@ -57,7 +57,6 @@ HostChunkPlan host_chunk_plan(int64_t seq_len, const loza_ssa_params& p) {
     h.cb = std::min(cb, h.nb);
   }
   h.n_chunks = (h.nb + h.cb - 1) / h.cb;
-  h.slots = (int)std::min<int64_t>(kHostSlots, h.n_chunks);
   // a local sequence never holds more rows than the prefix up to its chunk's end
   h.rows_max = std::min((h.pre_max + h.cb) * kTile, seq_len);
   return h;
@@ -93,20 +92,31 @@ HostChunk host_chunk(const HostChunkPlan& h, int64_t c, int64_t seq_len, const l
   return k;
 }
 
+// Upper bound of the chunks of a packed batch: a sequence of nb blocks is one
+// chunk if nb < kHostMinBlocks, otherwise chunks of at least kHostMinBlocks
+// blocks, at most nb / kHostMinBlocks + 1 of them.
+int64_t host_chunk_cap(int32_t batch, int64_t total_tokens) {
+  return 2 * (int64_t)batch + total_tokens / (kTile * kHostMinBlocks) + 1;
+}
+
 struct HostLayout {
   size_t cu_off, pf_off, pf_bytes, slot_off, slot_bytes;
   size_t q_off, k_off, v_off, o_off, l_off;  // within a slot
+  int slots;
   size_t total;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-HostLayout host_layout(const HostChunkPlan& h, size_t pf_bytes, int32_t n_heads, int32_t n_kv_heads, int32_t d_qk,
-                       int32_t d_v) {
+// Workspace of a packed batch: slots sized for the longest sequence's largest
+// chunk (chunks grow with the sequence), the local cu_seqlens of every chunk.
+HostLayout host_layout(const HostChunkPlan& h, int64_t chunk_cap, size_t pf_bytes, int32_t n_heads,
+                       int32_t n_kv_heads, int32_t d_qk, int32_t d_v) {
   HostLayout w;
   const size_t rows = (size_t)h.rows_max;
+  w.slots = (int)std::min<int64_t>(kHostSlots, chunk_cap);
   w.cu_off = 0;
-  w.pf_off = align256((size_t)h.n_chunks * 2 * sizeof(int32_t));
+  w.pf_off = align256((size_t)chunk_cap * 2 * sizeof(int32_t));
   w.pf_bytes = pf_bytes;
   w.slot_off = align256(w.pf_off + pf_bytes);
   w.q_off = 0;
@@ -115,7 +125,7 @@ HostLayout host_layout(const HostChunkPlan& h, size_t pf_bytes, int32_t n_heads,
   w.o_off = align256(w.v_off + rows * n_kv_heads * d_v * 2);
   w.l_off = align256(w.o_off + rows * n_heads * d_v * 2);
   w.slot_bytes = align256(w.l_off + rows * n_heads * sizeof(float));
-  w.total = w.slot_off + (size_t)h.slots * w.slot_bytes;
+  w.total = w.slot_off + (size_t)w.slots * w.slot_bytes;
   return w;
 }
 

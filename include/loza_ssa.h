@@ -124,43 +124,49 @@ loza_status loza_ssa_prefill(const void *q, const void *k, const void *v,
                              void *workspace, size_t workspace_bytes, loza_stream_t stream);
 
 /*
- * Prefill of ONE sequence whose tensors live in host memory: the operation
+ * Prefill of a packed batch whose tensors live in host memory: the operation
  * and results of loza_ssa_prefill (same kernels; every output row is computed
- * exactly as in a device-resident call with cu_seqlens {0, seq_len}), with the
+ * exactly as in a device-resident call with the same cu_seqlens), with the
  * host-to-device copies of the inputs and the device-to-host copies of the
  * outputs inside the call. (The LoZA pages have no counterpart to this entry
  * point; it exists for callers whose activations are on the host.)
- *   q   [seq_len, n_heads, d_qk]     bf16, contiguous rows
- *   k   [seq_len, n_kv_heads, d_qk]  bf16, contiguous rows
- *   v   [seq_len, n_kv_heads, d_v]   bf16, contiguous rows; absorbed MLA: v == k
- *                                    (V = the first d_v columns of the latent row)
- *   out [seq_len, n_heads, d_v] bf16 and lse [seq_len, n_heads] fp32 (written)
- * These five pointers may be host memory (page-locked memory lets the copies
+ *   q   [T, n_heads, d_qk]     bf16, contiguous rows
+ *   k   [T, n_kv_heads, d_qk]  bf16, contiguous rows
+ *   v   [T, n_kv_heads, d_v]   bf16, contiguous rows; absorbed MLA: v == k
+ *                              (V = the first d_v columns of the latent row)
+ *   out [T, n_heads, d_v] bf16 and lse [T, n_heads] fp32 (written)
+ *   cu_seqlens: HOST int32 [batch+1], 0 = cu_seqlens[0] <= ... <=
+ *               cu_seqlens[batch] = total_tokens (T); no sequence longer than
+ *               max_seqlen; empty sequences are allowed
+ * These five tensors may be host memory (page-locked memory lets the copies
  * run asynchronously and overlap; pageable memory gives the same results but
  * the copies serialise) or device memory; they are addressed through the
  * unified address space.
- * How it runs: the query blocks are cut into chunks (about 16 per sequence,
- * 8 to 64 blocks of 128 rows each, at least s + l - 1 blocks; the unbounded
- * window is one chunk). A chunk's own blocks [j0, j1) run as the local
- * sequence [sink blocks | blocks j0-l+1 .. j0-1 | own blocks] with zero query
- * rows for the prepended blocks: by the window rule (page 1 section 01 (1) of
- * the LoZA pages) every own query sees exactly its keys of the whole
- * sequence. Up to three chunks are in flight: the copy-in of one, the kernels
- * of the next and the copy-out of a third overlap, on two copy streams that
- * the library creates on the first call per device and keeps until exit.
- * The call is asynchronous on `stream`: when `stream` reaches this point of
- * its work, out and lse hold the results. Supported shapes are those of
- * loza_ssa_prefill with n_kv_heads in {1, n_heads}: (d_qk, d_v) in {(64, 64),
- * (192, 128)} and the absorbed (576, 512) with an even n_heads.
+ * How it runs: each sequence's query blocks are cut into chunks (about 16 per
+ * sequence, 8 to 64 blocks of 128 rows each, at least s + l - 1 blocks; the
+ * unbounded window is one chunk per sequence). A chunk's own blocks
+ * [j0, j1) run as the local sequence [sink blocks | blocks j0-l+1 .. j0-1 |
+ * own blocks] with zero query rows for the prepended blocks: by the window
+ * rule (page 1 section 01 (1) of the LoZA pages) every own query sees exactly
+ * its keys of the whole sequence. Up to three chunks are in flight: the
+ * copy-in of one, the kernels of the next and the copy-out of a third
+ * overlap, on two copy streams that the library creates on the first call per
+ * device and keeps until exit. The call is asynchronous on `stream`: when
+ * `stream` reaches this point of its work, out and lse hold the results.
+ * Supported shapes are those of loza_ssa_prefill with n_kv_heads in
+ * {1, n_heads}: (d_qk, d_v) in {(64, 64), (192, 128)} and the absorbed
+ * (576, 512) with an even n_heads.
  *   workspace: device memory, 256-byte aligned, of at least
- *   loza_ssa_workspace_size(LOZA_OP_PREFILL_HOST, 1, seq_len, seq_len, ...)
- *   bytes (per chunk slot: its local q, k, v, out and lse), owned by the
- *   caller and used by nothing else until `stream` has passed this call.
+ *   loza_ssa_workspace_size(LOZA_OP_PREFILL_HOST, batch, T, max_seqlen, ...)
+ *   bytes (chunk slots sized for the longest sequence, and the chunks' local
+ *   cu_seqlens), owned by the caller and used by nothing else until `stream`
+ *   has passed this call.
  *   Errors: LOZA_ERR_INVALID_ARG / LOZA_ERR_UNSUPPORTED / LOZA_ERR_WORKSPACE
  *   before anything is enqueued; LOZA_ERR_CUDA if enqueueing fails part way
  *   (synchronise `stream` before reusing any buffer in that case).
  */
-loza_status loza_ssa_prefill_host(const void *q, const void *k, const void *v, int64_t seq_len,
+loza_status loza_ssa_prefill_host(const void *q, const void *k, const void *v, const int32_t *cu_seqlens,
+                                  int32_t batch, int64_t total_tokens, int32_t max_seqlen,
                                   int32_t n_heads, int32_t n_kv_heads, int32_t d_qk, int32_t d_v,
                                   loza_ssa_params p, void *out, float *lse,
                                   void *workspace, size_t workspace_bytes, loza_stream_t stream);

@@ -114,18 +114,28 @@ def test_decode_paged_rejects_before_launch(L, table, bt_stride, num_pages, code
     assert L.loza_launch_count() == count
 
 
-def _call_prefill_host(L, q=1 << 20, k=1 << 21, v=1 << 22, seq_len=4096, H=4, Hkv=4, dqk=64, dv=64,
-                       params=None, ws=1 << 28, ws_bytes=1 << 40):
+def _call_prefill_host(L, q=1 << 20, k=1 << 21, v=1 << 22, cu=(0, 4096), batch=None, total=None, max_seqlen=None,
+                       H=4, Hkv=4, dqk=64, dv=64, params=None, ws=1 << 28, ws_bytes=1 << 40, null_cu=False):
+    import numpy as np
     vp = ctypes.c_void_p
     params = params if params is not None else bss.Params(0.125)
-    return L.loza_ssa_prefill_host(vp(q), vp(k), vp(v), seq_len, H, Hkv, dqk, dv, params, vp(1 << 24),
-                                   vp(1 << 25), vp(ws), ws_bytes, vp(0))
+    cu_arr = np.ascontiguousarray(cu, dtype=np.int32)  # host memory, as the entry point requires
+    batch = len(cu) - 1 if batch is None else batch
+    total = int(cu[-1]) if total is None else total
+    max_seqlen = int(max(np.diff(cu))) if max_seqlen is None else max_seqlen
+    cu_ptr = vp(0) if null_cu else cu_arr.ctypes.data_as(vp)
+    return L.loza_ssa_prefill_host(vp(q), vp(k), vp(v), cu_ptr, batch, total, max_seqlen, H, Hkv, dqk, dv, params,
+                                   vp(1 << 24), vp(1 << 25), vp(ws), ws_bytes, vp(0))
 
 
 @pytest.mark.parametrize("over,code", [
     (dict(q=0), -1),                                  # null pointer
-    (dict(seq_len=0), -1),                            # empty sequence
-    (dict(seq_len=1 << 31), -1),                      # beyond int32 rows
+    (dict(null_cu=True), -1),                         # no sequence offsets
+    (dict(cu=(0, 0), max_seqlen=1), -1),              # no tokens at all
+    (dict(cu=(0, 100, 50, 200)), -1),                 # offsets going backwards
+    (dict(cu=(1, 100)), -1),                          # offsets not starting at 0
+    (dict(cu=(0, 100, 300), max_seqlen=150), -1),     # a sequence longer than max_seqlen
+    (dict(cu=(0, 100, 300), total=299), -1),          # last offset is not the token count
     (dict(H=6, Hkv=4), -1),                           # heads not a multiple of kv heads
     (dict(H=4, Hkv=2), -2),                           # grouped heads not compiled
     (dict(dqk=96, dv=96), -2),                        # head dims not compiled
@@ -144,8 +154,7 @@ def test_prefill_host_rejects_before_launch(L, over, code):
 def test_prefill_host_workspace_size():
     p = bss.Params(1 / math.sqrt(576))
     size = lambda *a: bss.workspace_size(bss.LOZA_OP_PREFILL_HOST, *a)
-    assert size(2, 4096, 4096, 64, 1, 576, 512, p) == 0          # one sequence per call
-    assert size(1, 4096, 2048, 64, 1, 576, 512, p) == 0          # total_tokens == max_seqlen == seq_len
+    assert size(1, 2048, 4096, 64, 1, 576, 512, p) == 0          # max_seqlen beyond the token count
     assert size(1, 4096, 4096, 64, 4, 576, 512, p) == 0          # absorbed is one kv head
     small = size(1, 300, 300, 64, 1, 576, 512, p)
     big = size(1, 32768, 32768, 64, 1, 576, 512, p)
@@ -155,7 +164,10 @@ def test_prefill_host_workspace_size():
     # chunks are bounded (at most 64 own + s + l - 1 prepended blocks, three slots)
     assert small < big <= huge
     assert huge < 3 * (71 * 128) * (64 * 576 * 2 + 64 * 512 * 2 + 2 * 576 * 2 + 64 * 4) + (256 << 20)
-    # the unbounded window runs as one chunk: one slot of the whole sequence
+    # a packed batch needs slots for its longest sequence only, plus a longer chunk table
+    packed = size(8, 8 * 32768, 32768, 64, 1, 576, 512, p)
+    assert big <= packed < big + (1 << 20)
+    # the unbounded window runs as one chunk per sequence: a slot of the longest sequence
     dense = size(1, 8192, 8192, 4, 4, 64, 64, bss.Params(0.125, n_local=bss.LOZA_UNBOUNDED))
     assert dense >= 8192 * 4 * (64 * 2 * 4 + 4)
 

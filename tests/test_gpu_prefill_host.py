@@ -30,21 +30,25 @@ def host_bf16(bits, pinned):
     return t.pin_memory() if pinned else t.clone()
 
 
-def check_host_call(bss, oracle_mod, params, qh, kh, vh, qd, kd, vd, q_bits, k_bits, v_bits, Hkv, rows=None):
+def check_host_call(bss, oracle_mod, params, qh, kh, vh, qd, kd, vd, q_bits, k_bits, v_bits, Hkv, rows=None,
+                    lens=None):
     """Run the host entry point, then compare it bit for bit with the device call
-    and element by element with the oracle (on ``rows``, all rows if None)."""
+    and element by element with the oracle (on ``rows``, all rows if None).
+    lens: the packed sequence lengths (one sequence of all rows if None)."""
     import torch
     L, H = qh.shape[0], qh.shape[1]
-    out_h, lse_h = bss.loza_ssa_prefill_host(qh, kh, vh, params)
+    lens = [L] if lens is None else lens
+    cu_np = synth.cu_seqlens(lens)
+    out_h, lse_h = bss.loza_ssa_prefill_host(qh, kh, vh, params, cu_seqlens=None if len(lens) == 1 else cu_np)
     torch.cuda.synchronize()
     assert bss.device_status() == 0
     assert out_h.device.type == "cpu" and lse_h.device.type == "cpu"
-    cu = torch.tensor([0, L], dtype=torch.int32, device="cuda")
-    out_d, lse_d = bss.loza_ssa_prefill(qd, kd, vd, cu, L, params)
+    cu = torch.from_numpy(cu_np).cuda()
+    out_d, lse_d = bss.loza_ssa_prefill(qd, kd, vd, cu, max(lens), params)
     torch.cuda.synchronize()
     assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16)), "O differs from the device call"
     assert torch.equal(lse_h.view(torch.int32), lse_d.cpu().view(torch.int32)), "LSE differs from the device call"
-    o_ref, lse_ref = oracle_mod.forward(q_bits, k_bits, v_bits, synth.cu_seqlens([L]), H, Hkv, 128, params.n_sink,
+    o_ref, lse_ref = oracle_mod.forward(q_bits, k_bits, v_bits, cu_np, H, Hkv, 128, params.n_sink,
                                         params.n_local, params.scale, rows=rows)
     o_got = out_h.to(torch.float32).numpy().astype(np.float64)
     lse_got = lse_h.numpy().astype(np.float64)
@@ -56,7 +60,8 @@ def check_host_call(bss, oracle_mod, params, qh, kh, vh, qd, kd, vd, q_bits, k_b
 
 
 def host_case(bss, oracle_mod, seed, L, H, Hkv, dqk, dv, scale, n_sink=1, n_local=7, latent=False,
-              pinned=True):
+              pinned=True, lens=None):
+    """L tokens, one sequence or packed as `lens` (summing to L)."""
     g = synth.rng(seed)
     q = synth.normal_bits(g, (L, H, dqk))
     if latent:
@@ -73,7 +78,7 @@ def host_case(bss, oracle_mod, seed, L, H, Hkv, dqk, dv, scale, n_sink=1, n_loca
         kd, vd = to_dev(k_bits), to_dev(v_bits)
     params = bss.Params(scale, 128, n_sink, n_local)
     check_host_call(bss, oracle_mod, params, host_bf16(q, pinned), kh, vh, to_dev(q), kd, vd, q, k_bits, v_bits,
-                    Hkv)
+                    Hkv, lens=lens)
 
 
 @pytest.mark.parametrize("L", [1, 200, 3000, 5000])
@@ -92,6 +97,20 @@ def test_host_windows_d64(bss, oracle_mod, n_sink, n_local):
 
 def test_host_192_128(bss, oracle_mod):
     host_case(bss, oracle_mod, 420, 4200, 4, 4, 192, 128, 1 / math.sqrt(192))
+
+
+@pytest.mark.parametrize("lens", [[3000, 1, 700, 5000], [129, 1024, 1025, 2049, 64]])
+def test_host_absorbed_packed(bss, oracle_mod, lens):
+    """A packed batch: each sequence chunked on its own (1 to 5 chunks), the
+    chunks of all sequences streamed through the same three slots."""
+    host_case(bss, oracle_mod, 450 + len(lens), sum(lens), 4, 1, 576, 512, 1 / math.sqrt(192), latent=True,
+              lens=lens)
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(1, 7), (2, 3), (0, -1)])
+def test_host_packed_d64_and_192(bss, oracle_mod, n_sink, n_local):
+    host_case(bss, oracle_mod, 460, 4300, 2, 2, 64, 64, 0.125, n_sink, n_local, lens=[2500, 300, 1500])
+    host_case(bss, oracle_mod, 461, 3100, 2, 2, 192, 128, 1 / math.sqrt(192), n_sink, n_local, lens=[1100, 2000])
 
 
 def test_host_pageable(bss, oracle_mod):
