@@ -90,9 +90,10 @@ int sm_count() {
 //   - otherwise the block kernel with up to 4 splits per sequence in a
 //     cluster (one CTA per sequence for large batches), merged on chip.
 // Measured kernel times (64 heads, 8-block window, contexts of 64K-128K;
-// half-block vs the block kernel's best plan): 1 sequence 21.8 vs 25.4 us,
-// 8: 22.2 vs 24.5, 64: 32.5 vs 34.3 (a head-split kernel), 96: 47.2 vs 43.6,
-// 128: 49.0 vs 47.6. With the whole context selected (the dense decode of
+// half-block vs the best alternative measured: the block kernel, or at 64
+// sequences a kernel splitting the heads over two CTAs per sequence):
+// 1 sequence 21.8 vs 25.4 us, 8: 22.2 vs 24.5, 64: 32.5 vs 34.3,
+// 96: 47.2 vs 43.6, 128: 49.0 vs 47.6. With the whole context selected (the dense decode of
 // 64 sequences of 64K-128K) the block kernel took 1.74 ms, the half-block one
 // 2.22 ms.
 struct DecodePlan {

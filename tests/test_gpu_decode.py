@@ -205,8 +205,9 @@ def paged_case(bss, oracle_mod, seed, lens, n_sink=1, n_local=7):
 
 @pytest.mark.parametrize("batch", [6, 40, 80])
 def test_absorbed_decode_paged(bss, oracle_mod, batch):
-    """Paged latent cache under the three plan families (block split over a
-    cluster, head split, one CTA per sequence)."""
+    """Paged latent cache under the decode plans: half blocks split over a
+    cluster of 4 CTAs (6 sequences) or 2 (40), and the block kernel with one CTA
+    per sequence (80)."""
     g = synth.rng(300 + batch)
     lens = g.integers(1, 3000, size=batch)
     lens[:3] = [1, 128, 1025]
