@@ -45,6 +45,12 @@
  * All inputs are bf16 bit patterns (uint16) widened exactly to double. n_local
  * < 0 means an unbounded local window (plain causal attention when n_sink = 0).
  * kv head hk = h / (n_heads / n_kv_heads).
+ *
+ * A second window, token-granular (ssa_oracle_forward_tokens_rows; page 4, the
+ * LSA article's streaming-aware index of 16 sink tokens and a 1,024-token
+ * sliding window), replaces steps 1-2 by
+ *   A(i) = { t <= i : t < sink_tokens  or  i - t < window_tokens }
+ * and keeps steps 3-5.
  */
 #include <math.h>
 #include <stdint.h>
