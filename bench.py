@@ -325,7 +325,8 @@ def decode_bytes(lens, n_local=LW):
 
 def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20, rotating=0):
     """SSA decode (and the dense full-context decode) on a latent cache
-    [len(lens), cap, 576]; L2 flushed (256 MB write) before every timed call.
+    [len(lens), cap, 576]; L2 flushed (256 MB write, then a 256 MB read) before
+    every timed call.
     rotating > 1: also time the SSA decode over that many copies of the inputs
     and outputs, back to back in a CUDA graph (time_rotating)."""
     import torch
@@ -333,7 +334,14 @@ def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20, rotati
     q = synth.torch_normal_bf16((Bn, H, DQK), synth.workload_seed(3) * 1000 + 1, device)
     cache = synth.torch_normal_bf16((Bn, cap, 1, DQK), synth.workload_seed(3) * 1000 + 2, device)
     seqlens = torch.tensor(lens, dtype=torch.int32, device=device)
-    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=device)
+
+    def flush():
+        # evict the inputs: write 256 MB, then read 256 MB more, so that the
+        # write's dirty lines are written back here and not inside the timed call
+        flush_w.zero_()
+        flush_r.sum()
     out = torch.empty((Bn, H, DV), dtype=torch.bfloat16, device=device)
     lse = torch.empty((Bn, H), dtype=torch.float32, device=device)
     res = {}
@@ -350,7 +358,7 @@ def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20, rotati
         for _ in range(3):
             call()
         torch.cuda.synchronize()
-        ms, _ = time_launches(call, stream, n, flush=lambda: flush_buf.zero_())
+        ms, _ = time_launches(call, stream, n, flush=flush)
         nbytes = decode_bytes(lens, nl)
         res[name] = {"ms": ms, "bytes": nbytes, "GB/s": nbytes / (ms / 1000.0) / 1e9, "launches_timed": n}
         if bss.device_status() != 0:
@@ -366,6 +374,10 @@ def run_decode(bss, device, stream, lens, cap, with_dense=True, steps=20, rotati
     del cache
     torch.cuda.empty_cache()
     return res
+
+
+# the kernel the library's decode plan picks for the 1 + 7 window at these batches
+DECODE_KERNEL = "ssa_decode_mla_hb_kernel"
 
 
 def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None, ctx=None):
@@ -385,10 +397,11 @@ def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None, ctx=None
            "metric": "SSA decode GB/s (bytes touched)", "value": ssa["GB/s"], "unit": "GB/s",
            "ms_per_call": ssa["ms"], "bytes_per_call": ssa["bytes"],
            "roofline": {"bound": "hbm", "achieved": ssa["GB/s"], "peak": hbm, "unit": "GB/s",
-                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic("ssa_decode_mla_hb_kernel"),
+                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic(DECODE_KERNEL),
                         "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
-                        "kernel": "ssa_decode_mla_hb_kernel"},
-           "timing": "mean of per-call CUDA events, L2 flushed (256 MB write) before each call"}
+                        "kernel": DECODE_KERNEL},
+           "timing": "mean of per-call CUDA events; before each call (outside the events) the L2 is flushed "
+                     "by a 256 MB write and then a 256 MB read, so the call starts with no dirty lines to write back"}
     if "ssa_rotating" in r:
         rr = r["ssa_rotating"]
         out["rotating"] = {"ms_per_call": rr["ms"], "GB/s": rr["GB/s"], "frac_of_hbm": rr["GB/s"] / hbm,
@@ -445,41 +458,77 @@ def merge_secondary(bss, device, stream, peaks, peak_kind, steps=20):
             "timing": "mean of per-call CUDA events; inputs larger than L2"}
 
 
-def long_secondary(bss, device, stream, peaks):
-    """Workload 4: L = 262144 absorbed prefill, SSA next to full causal attention;
-    then SSA and dense decode of 32 sequences of 1,048,576 tokens."""
+def tensor_roofline(flop, ms, peaks, peak_kind, kernel):
+    pk = float(peaks["bf16_tflops"])
+    a = flop / (ms / 1000.0) / 1e12
+    return {"bound": "tensor", "achieved": a, "peak": pk, "unit": "TFLOP/s", "frac": a / pk,
+            "traffic": profiled_traffic(kernel),
+            "peak_kind": f"{peak_kind} bf16 dense burst (MEASURED_PEAKS.json bf16_tflops)", "kernel": kernel}
+
+
+def hbm_roofline(nbytes, ms, peaks, peak_kind, kernel):
+    hbm = float(peaks["hbm_gbs"])
+    a = nbytes / (ms / 1000.0) / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
+            "traffic": profiled_traffic(kernel),
+            "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)", "kernel": kernel}
+
+
+def long_secondary(bss, device, stream, peaks, peak_kind):
+    """Workload 4: L = 262144 absorbed prefill, SSA next to full causal attention
+    (the same library, unbounded window); then SSA and dense decode of 32
+    sequences of 1,048,576 tokens."""
     import torch
     w = synth.WORKLOADS[4]
     L = w["seqlen"]
     q, lat, cu = make_inputs(device, L, seed_offset=40)
     out = torch.empty((L, H, DV), dtype=torch.bfloat16, device=device)
     lse = torch.empty((L, H), dtype=torch.float32, device=device)
-    res = {"workload": w["name"]}
-    for name, nl, n in (("ssa", LW, 5), ("dense", -1, 1)):
+    lines = {}
+    for name, nl, warm, n in (("ssa", LW, 2, 5), ("dense", -1, 0, 1)):
         params = bss.Params(SCALE, B, S if nl > 0 else 0, nl)
         ws = prefill_workspace(bss, device, 1, L, L, params)
 
         def call():
             bss.loza_ssa_prefill(q, lat, lat[:, :, :DV], cu, L, params, out=out, lse=lse, workspace=ws, stream=stream)
 
-        call()
+        for _ in range(warm):
+            call()
         torch.cuda.synchronize()
         ms, _ = time_launches(call, stream, n)
+        if bss.device_status() != 0:
+            raise RuntimeError("device status reports a timed-out wait in the long prefill")
         fl = prefill_flops(L) if nl > 0 else 2.0 * (DQK + DV) * H * L * (L + 1) / 2
-        res[f"prefill_{name}"] = {"ms": ms, "algorithmic_tflop": fl / 1e12, "TFLOP/s": fl / (ms / 1000) / 1e12,
-                                  "frac_of_peak": fl / (ms / 1000) / 1e12 / float(peaks["bf16_tflops"])}
-    res["prefill_dense_over_ssa_time"] = res["prefill_dense"]["ms"] / res["prefill_ssa"]["ms"]
+        # the library's choice for these shapes: the two-pass kernel needs a
+        # workspace and a bounded window, the unbounded window runs on the pair kernel
+        kern = "ssa_prefill_mla_kernel" if (nl > 0 and ws is not None) else "ssa_prefill_pair_kernel"
+        lines[name] = {"ms_per_call": ms, "launches_timed": n, "algorithmic_tflop": fl / 1e12,
+                       "TFLOP/s": fl / (ms / 1000) / 1e12,
+                       "roofline": tensor_roofline(fl, ms, peaks, peak_kind, kern)}
+        del ws
     del q, lat, out, lse
     torch.cuda.empty_cache()
+    res = {"workload": "MLA-absorbed SSA prefill L=262144 (64 heads, latent 576, V = first 512)",
+           "metric": "SSA prefill TFLOP/s", "value": lines["ssa"]["TFLOP/s"], "unit": "TFLOP/s",
+           "ms_per_call": lines["ssa"]["ms_per_call"], "roofline": lines["ssa"]["roofline"],
+           "dense": dict(lines["dense"], dense_over_ssa_time=lines["dense"]["ms_per_call"] / lines["ssa"]["ms_per_call"],
+                         algorithmic_ratio=lines["dense"]["algorithmic_tflop"] / lines["ssa"]["algorithmic_tflop"]),
+           "timing": "mean of per-call CUDA events (SSA: 2 warm-up, 5 timed; dense: 1 timed launch of ~5 s); "
+                     "inputs larger than L2"}
     r = run_decode(bss, device, stream, [w["decode_ctx"]] * w["decode_batch"], w["decode_ctx"])
-    hbm = float(peaks["hbm_gbs"])
-    res["decode_1m"] = {"ssa": dict(r["ssa"], frac_of_hbm=r["ssa"]["GB/s"] / hbm),
-                        "dense": dict(r["dense"], frac_of_hbm=r["dense"]["GB/s"] / hbm),
-                        "dense_over_ssa_time": r["dense"]["ms"] / r["ssa"]["ms"]}
-    return res
+    ssa, dense = r["ssa"], r["dense"]
+    dec = {"workload": f"MLA-absorbed SSA decode, {w['decode_batch']} seqs x {w['decode_ctx']} tokens",
+           "metric": "SSA decode GB/s (bytes touched)", "value": ssa["GB/s"], "unit": "GB/s",
+           "ms_per_call": ssa["ms"], "bytes_per_call": ssa["bytes"],
+           "roofline": hbm_roofline(ssa["bytes"], ssa["ms"], peaks, peak_kind, DECODE_KERNEL),
+           "dense": {"ms_per_call": dense["ms"], "bytes_per_call": dense["bytes"], "GB/s": dense["GB/s"],
+                     "frac_of_hbm": dense["GB/s"] / float(peaks["hbm_gbs"]),
+                     "dense_over_ssa_time": dense["ms"] / ssa["ms"]},
+           "timing": "mean of per-call CUDA events; L2 flushed (256 MB write, then 256 MB read) before each call"}
+    return res, dec
 
 
-def train_secondary(bss, device, stream, peaks, train_len=None):
+def train_secondary(bss, device, stream, peaks, peak_kind, train_len=None):
     """Workload 5: varlen forward + backward, per-head 192/128 dims, 64 heads
     (train_len: one sequence of that many tokens instead, for profiling)."""
     import torch
@@ -515,19 +564,24 @@ def train_secondary(bss, device, stream, peaks, train_len=None):
         bss.loza_ssa_backward(q, k, v, out, do, lse, cu, int(lens.max()), params, dq=dq, dk=dk, dv=dvv,
                               workspace=ws, stream=stream)
 
-    fwd(); bwd()
+    for _ in range(3):
+        fwd()
+        bwd()
     torch.cuda.synchronize()
-    mf, _ = time_launches(fwd, stream, 3)
-    mb, _ = time_launches(bwd, stream, 3)
+    mf, _ = time_launches(fwd, stream, 5)
+    mb, _ = time_launches(bwd, stream, 5)
     if bss.device_status() != 0:
         raise RuntimeError("device status reports a timed-out wait in training")
-    pk = float(peaks["bf16_tflops"])
-    res = {"workload": w["name"] if not train_len else f"training fwd+bwd, one sequence of {train_len} tokens",
-           "lengths": lens.tolist(), "total_tokens": T,
-           "forward": {"ms": mf, "TFLOP/s": f_fwd / (mf / 1000) / 1e12, "frac_of_peak": f_fwd / (mf / 1000) / 1e12 / pk,
-                       "algorithmic_tflop": f_fwd / 1e12},
-           "backward": {"ms": mb, "TFLOP/s": f_bwd / (mb / 1000) / 1e12, "frac_of_peak": f_bwd / (mb / 1000) / 1e12 / pk,
-                        "algorithmic_tflop": f_bwd / 1e12}}
+    name = w["name"] if not train_len else f"training fwd+bwd, one sequence of {train_len} tokens"
+    res = {"workload": f"{name}, {Hh} heads, q/k {dqk}, v {dv}", "lengths": lens.tolist(), "total_tokens": T,
+           "metric": "SSA training TFLOP/s (forward, backward)", "unit": "TFLOP/s",
+           "value": (f_fwd + f_bwd) / ((mf + mb) / 1000) / 1e12,
+           "forward": {"ms_per_call": mf, "TFLOP/s": f_fwd / (mf / 1000) / 1e12, "algorithmic_tflop": f_fwd / 1e12,
+                       "roofline": tensor_roofline(f_fwd, mf, peaks, peak_kind, "ssa_prefill_mha2_kernel")},
+           "backward": {"ms_per_call": mb, "TFLOP/s": f_bwd / (mb / 1000) / 1e12, "algorithmic_tflop": f_bwd / 1e12,
+                        "roofline": tensor_roofline(f_bwd, mb, peaks, peak_kind, "ssa_bwd"),
+                        "flop_per_pair_head": 2 * (3 * dqk + 2 * dv)},
+           "timing": "mean of per-call CUDA events, 3 warm-up and 5 timed calls each; inputs larger than L2"}
     del q, k, v, do, out, lse, dq, dk, dvv, ws
     torch.cuda.empty_cache()
     return res
@@ -610,14 +664,15 @@ def run_ours(args, rank, world, local_rank):
                 "avg_launch_ms": avg_launch_ms}
 
     secondary = {}
-    if args.workload in ("default", "all"):
+    if args.workload in ("default", "decode"):
         secondary["decode"] = decode_secondary(bss, device, stream, peaks, peak_kind, args.decode_batch,
                                                args.decode_ctx)
+    if args.workload == "default":
         secondary["merge"] = merge_secondary(bss, device, stream, peaks, peak_kind)
-    if args.workload in ("long", "all"):
-        secondary["long"] = long_secondary(bss, device, stream, peaks)
-    if args.workload in ("train", "all"):
-        secondary["train"] = train_secondary(bss, device, stream, peaks, args.train_len)
+    if args.workload in ("default", "long"):
+        secondary["long"], secondary["decode_1m"] = long_secondary(bss, device, stream, peaks, peak_kind)
+    if args.workload in ("default", "train"):
+        secondary["train"] = train_secondary(bss, device, stream, peaks, peak_kind, args.train_len)
 
     line = None
     if rank == 0:
@@ -744,8 +799,10 @@ def main():
                          "sequence, a smaller cache)")
     ap.add_argument("--train-len", type=int, default=None,
                     help="training workload as one sequence of this length (profiling)")
-    ap.add_argument("--workload", choices=["default", "prefill", "long", "train", "all"], default="default",
-                    help="default: prefill line plus the 64-sequence decode; long/train/all add workloads 4/5")
+    ap.add_argument("--workload", choices=["default", "prefill", "decode", "long", "train"], default="default",
+                    help="default: the prefill line with every other workload as secondary lines (the "
+                         "64-sequence decode, the branch merge, workload 4's long prefill and 1M decode, "
+                         "workload 5's training); the others: the prefill line plus only that one")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -417,27 +417,22 @@ loza_status launch_prefill_mla(PrefillMlaParams& prm, void* workspace, cudaStrea
 // workspace. It is ordinary device memory of this module: every GPU that loads
 // the library reserves kNoAllocScratchBytes for it until the process exits.
 // Host code must not use the name g_decode_scratch as a pointer; the device
-// address comes from cudaGetSymbolAddress, once per device.
+// address comes from cudaGetSymbolAddress.
 // ---------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) uint8_t g_decode_scratch[kNoAllocScratchBytes];
 
+// Devices of one process for which per-device host state is kept.
 constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device (looked up on the
-// first call per device). Returns nullptr if the lookup fails.
+// Device address of g_decode_scratch on the current device, looked up on
+// every call: the lookup is cheap once the module is loaded, and a module
+// loaded again after cudaDeviceReset may place the array elsewhere. Returns
+// nullptr if the lookup fails.
 void* decode_scratch_address() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
-    g_scratch_addr[dev] = p;
-  }
-  return g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 // Grid for a grid-stride pass over n 16-byte vectors: at most a few waves.

@@ -215,7 +215,11 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  * fixed 16 MiB array that is part of the library itself. Every other call
  * merges its partials on chip and needs none.
  *   - The library never allocates: every GPU that loads the library holds the
- *     16 MiB array until the process exits.
+ *     16 MiB array until the process exits. With CUDA's lazy module loading
+ *     (the default since CUDA 12.2) the array is placed on a device at the
+ *     first call into this library on that device, whichever entry point it
+ *     is; a runtime that reserves nearly all device memory for its own pool
+ *     should make one call into the library on each device before it does so.
  *   - Limit: a call that needs scratch needs batch * nsplit * 132,096 bytes
  *     plus 256 for the counters, with nsplit = min(selected blocks,
  *     ceil(SMs / batch)), so it fits when batch * nsplit <= 127; e.g. with
@@ -223,9 +227,11 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  *     tokens or four of up to 3,968 tokens. A larger call returns
  *     LOZA_ERR_WORKSPACE before anything is launched; use loza_ssa_decode with
  *     a workspace instead, or split the batch.
- *   - The first call on each device that needs scratch looks up the array's
- *     device address (with that device current); make that first call before
- *     any stream capture on that device.
+ *   - Every call that needs scratch looks up the array's device address on
+ *     the current device (the first such call on a device also loads the
+ *     library's device code there, if no earlier call did); make that first
+ *     call before any stream capture on that device. After cudaDeviceReset
+ *     the next call finds the array at its new address.
  *   - Every call uses the same array and leaves its last contents there; the
  *     arrival counters are cleared on the caller's stream at the start of each
  *     call. Two calls whose kernels can overlap on the GPU (different streams

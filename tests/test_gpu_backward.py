@@ -11,18 +11,9 @@ import numpy as np
 import pytest
 
 import synth
-from helpers import from_dev, to_dev
+from helpers import assert_close_grad, from_dev, to_dev
 
 pytestmark = pytest.mark.gpu
-
-
-def assert_close_grad(got, ref, what):
-    err = np.abs(got - ref)
-    assert np.isfinite(got).all(), f"{what}: non-finite"
-    tol_max = 1e-2 * max(1.0, float(np.abs(ref).max()))
-    tol_mean = 1e-3 * max(1.0, float(np.abs(ref).mean()))
-    assert err.max() <= tol_max, f"{what}: max-abs {err.max():.3e} > {tol_max:.3e}"
-    assert err.mean() <= tol_mean, f"{what}: mean-abs {err.mean():.3e} > {tol_mean:.3e}"
 
 
 @pytest.fixture(scope="module")

@@ -122,8 +122,42 @@ def test_absorbed_decode_workload3_full_size(bss, oracle_mod):
 
 
 def test_absorbed_decode_1m_context(bss, oracle_mod):
-    """Contexts of 1,048,576 tokens (4 sequences here; the workload has 32)."""
-    absorbed_case(bss, oracle_mod, synth.workload_seed(4) + 2, [1 << 20] * 4, 1 << 20)
+    """Workload 4's decode at its stated size: 32 sequences of 1,048,576 tokens,
+    cache [32, 1048576, 576] (38.7 GB; every row outside the windows is NaN)."""
+    w = synth.WORKLOADS[4]
+    absorbed_case(bss, oracle_mod, synth.workload_seed(4) + 2, [w["decode_ctx"]] * w["decode_batch"],
+                  w["decode_ctx"])
+
+
+@pytest.mark.parametrize("lens", [[1, 64, 129, 1000], [5000, 70001, 65536]])
+def test_absorbed_decode_equals_last_prefill_row(bss, lens):
+    """Decode of the last token equals the last row of the prefill over the same
+    latent rows (the streaming pattern serves both phases: page 1 section 01),
+    for the absorbed 576/512 shapes, on the GPU: each sequence's prefill, with
+    the decode query as its last query row, against one batched decode call."""
+    import torch
+    H, D, DV = 64, 576, 512
+    g = synth.rng(400 + len(lens))
+    B, Lcap = len(lens), max(lens)
+    qd = synth.normal_bits(g, (B, H, D))
+    cache = torch.zeros((B, Lcap, 1, D), dtype=torch.bfloat16, device="cuda")
+    for n, L in enumerate(lens):
+        cache[n, :L] = to_dev(synth.normal_bits(g, (L, 1, D)))
+    params = bss.Params(1.0 / math.sqrt(192.0))
+    seqlens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    out, lse = bss.loza_ssa_decode(to_dev(qd), cache, None, seqlens, Lcap, params)
+    torch.cuda.synchronize()
+    assert bss.device_status() == 0
+    for n, L in enumerate(lens):
+        q = torch.zeros((L, H, D), dtype=torch.bfloat16, device="cuda")
+        q[L - 1] = to_dev(qd[n])
+        lat = cache[n, :L].contiguous()
+        cu = torch.tensor([0, L], dtype=torch.int32, device="cuda")
+        po, pl = bss.loza_ssa_prefill(q, lat, lat[:, :, :DV], cu, L, params)
+        torch.cuda.synchronize()
+        assert_close_o(from_dev(po[L - 1]), from_dev(out[n]), f"absorbed decode vs prefill row, L={L}")
+        assert_close_lse(pl[L - 1].cpu().numpy().astype(np.float64), lse[n].cpu().numpy().astype(np.float64),
+                         f"absorbed decode vs prefill row LSE, L={L}")
 
 
 @pytest.mark.parametrize("dqk,dv", [(64, 64), (192, 128)])

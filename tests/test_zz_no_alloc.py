@@ -43,26 +43,32 @@ def test_noalloc_decode_matches_workspace_decode_twice():
         ref_o, ref_l = bss.loza_ssa_decode(q, cache, None, seqlens, Lcap, params)
         out = torch.empty_like(ref_o)
         lse = torch.empty_like(ref_l)
+        torch.cuda.synchronize()
         before = torch.cuda.memory_allocated()
+        free_before, _ = torch.cuda.mem_get_info()    # device-wide: any allocation by anyone
         bss.loza_ssa_decode_noalloc(q, cache, None, seqlens, Lcap, params, out, lse)
         torch.cuda.synchronize()
         assert torch.cuda.memory_allocated() == before
+        assert torch.cuda.mem_get_info()[0] == free_before
         assert bss.device_status() == 0
         assert_close_o(from_dev(out), from_dev(ref_o), "noalloc vs workspace decode O")
         assert_close_lse(lse.cpu().numpy().astype(np.float64), ref_l.cpu().numpy().astype(np.float64),
                          "noalloc vs workspace decode LSE")
+        # the same plan on the same data: the results agree bit for bit
+        assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
 
 
 def test_noalloc_decode_rejects_batch_beyond_builtin_scratch():
     """4 sequences of up to 4,096 tokens with the unbounded window need more than
     the 16 MiB built in: rejected with LOZA_ERR_WORKSPACE before anything runs
-    (no GPU needed)."""
+    (no GPU needed). q is NULL: had the size check been skipped, the argument
+    check would refuse the call (LOZA_ERR_INVALID_ARG) before any launch."""
     import block_sparse_streaming_b200 as bss
     bss.build()
     L = bss.lib()
     vp = ctypes.c_void_p
     count = L.loza_launch_count()
-    rc = L.loza_ssa_decode_noalloc(vp(1 << 20), vp(1 << 21), vp(0), vp(1 << 22), 4, 4096, 4096 * 576, 576,
+    rc = L.loza_ssa_decode_noalloc(vp(0), vp(1 << 21), vp(0), vp(1 << 22), 4, 4096, 4096 * 576, 576,
                                    64, 1, 576, 512, bss.Params(0.07, 128, 0, bss.LOZA_UNBOUNDED), vp(1 << 23),
                                    vp(1 << 24), vp(0))
     assert rc == -3
