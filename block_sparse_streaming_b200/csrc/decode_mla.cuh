@@ -58,6 +58,9 @@ struct DecodeParams {
   CUtensorMap tm_q;    // q [B, H, 576]       box {64, 64, 1}
   CUtensorMap tm_kv;   // cache [B, rows, 576] box {64, 128, 1}; paged: the pool [1, pages * 128, 576]
   CUtensorMap tm_kv64; // the same tensor with box {64, 64, 1} (half blocks)
+  // 4-D views {64 columns, rows, 9 column tiles, batch} (tile stride 128 B):
+  CUtensorMap tm_q3;   // q, box {64, 64 heads, 3, 1}: three Q tiles per request
+  CUtensorMap tm_kv3;  // cache, box {64, 64 rows, 3, 1}: three half-block tiles per request
   const int32_t* seqlens;
   const int32_t* block_table;  // paged cache: [B, bt_stride] pool page of each logical block; nullptr: contiguous
   int bt_stride;

@@ -19,10 +19,10 @@
 // [64 heads x 64 keys], K-major) replaces the half block's rope tile (columns
 // 512..575), which no MMA reads after S.
 //
-// Roles: a TMA producer warp, an S issuer (one MMA group per tile as the tile
-// lands), a P.V issuer (separate, so that P.V of one half block never waits
-// for the load of the next; each 128-column chunk of P.V frees its two tiles
-// for the load after next) and 8 softmax warps. O^T is rescaled only when a
+// Roles: a TMA producer warp (three 24 KB boxes per half block), an S issuer
+// (one MMA group per box as it lands), a P.V issuer (separate, so that P.V of
+// one half block never waits for the load of the next; its 128-column chunks
+// free the tiles for the load after next box by box) and 8 softmax warps. O^T is rescaled only when a
 // head's maximum grows by more than 2^8; the softmax warps agree on that once
 // per half block at one named barrier.
 //
@@ -31,10 +31,13 @@
 // among nsplit <= 4 CTAs of a thread-block cluster. They merge on chip by the
 // log-sum-exp rule: split r owns output columns [r W, (r+1) W), W = 512 /
 // nsplit. When its own MMAs are done, each split tells the others that its
-// shared memory is free; each then pushes its (m, l, r) and its unscaled
-// partial O^T for the columns the others own straight into their shared
-// memory (16-byte DSMEM stores, no multicast) and arrives on their mbarrier;
-// each owner weights, sums and writes its columns.
+// shared memory is free, stages its (m, l, r) and its unscaled partial O^T
+// for the columns each other split owns in its own shared memory, and moves
+// each part with one bulk copy (no multicast) into the owner's receive area,
+// where it completes as transaction bytes on the owner's mbarrier; each owner
+// weights, sums and writes its columns. The L2 is asked for the half blocks
+// after the first two of each split at the start, so HBM keeps streaming
+// while the two slots turn over.
 #pragma once
 
 #include <cuda.h>
@@ -54,28 +57,39 @@ constexpr int kHbRecvPitch = 64 * 4 + 16;   // one received latent column: 64 he
 struct DecodeHbLayout {
   static constexpr int Q_OFF = 0;                                   // 9 Q tiles [64 heads x 64], 72 KB
   static constexpr int SLOT_OFF = 9 * kDecQTile;                    // 2 half-block slots, 144 KB
-  static constexpr int STAT_OFF = SLOT_OFF + 2 * kHbSlot;           // (m, l, r) [kHbMaxSplit][3][64]
-  static constexpr int WGT_OFF = STAT_OFF + kHbMaxSplit * 3 * 64 * 4;  // merge weights [kHbMaxSplit][64]
+  static constexpr int STAT_OFF = SLOT_OFF + 2 * kHbSlot;           // (m, l0, l1, r0, r1) [5][64]
+  static constexpr int WGT_OFF = STAT_OFF + 5 * 64 * 4;             // merge weights [kHbMaxSplit][64]
   static constexpr int ALPHA_OFF = WGT_OFF + kHbMaxSplit * 64 * 4;  // O^T rescale factors [2][64]
-  static constexpr int LPART_OFF = ALPHA_OFF + 2 * 64 * 4;          // second key group's (l, r) [2][64]
-  static constexpr int FLAG_OFF = LPART_OFF + 2 * 64 * 4;           // rescale flags [2]
+  static constexpr int FLAG_OFF = ALPHA_OFF + 2 * 64 * 4;           // rescale flags [2]
   static constexpr int BAR_OFF = FLAG_OFF + 16;
-  // barriers: q[9] (Q tile t), full[2][9] (slot, tile), empty[2][4] (slot, 128-column
-  // chunk of P.V: tiles 2c, 2c+1, and the P tile with the last chunk), s_full[2],
-  // s_free[2] (the softmax warps have read an S buffer), p_ready, pv_done[2]
-  // (P.V of even / odd half blocks), ready (the other splits' shared memory is
-  // free for the merge), data (the other splits' parts have landed)
-  static constexpr int BAR_Q = 0, BAR_FULL = 9, BAR_EMPTY = 27, BAR_S = 35, BAR_SFREE = 37, BAR_P = 39,
-                       BAR_PV = 40, BAR_READY = 42, BAR_DATA = 43, NBAR = 44;
+  // barriers: q[3] (Q tiles 3g .. 3g+2), full[2][3] (slot, tiles 3g .. 3g+2),
+  // empty[2][3] (slot, tiles 3g .. 3g+2 free: after 128-column chunk g+1 of
+  // P.V; the P tile, 8, with the last chunk), s_full[2], s_free[2] (the
+  // softmax warps have read an S buffer), p_ready, pv_done[2] (P.V of even /
+  // odd half blocks), ready (the other splits' shared memory is free for the
+  // merge), data (the other splits' parts have landed), sent (the other
+  // splits have received this split's parts: its shared memory may go)
+  static constexpr int BAR_Q = 0, BAR_FULL = 3, BAR_EMPTY = 9, BAR_S = 15, BAR_SFREE = 17, BAR_P = 19,
+                       BAR_PV = 20, BAR_READY = 22, BAR_DATA = 23, BAR_SENT = 24, NBAR = 25;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;               // tmem base, abort
   static constexpr int SMEM_BYTES = MISC_OFF + 16;
-  // merge receive buffer over Q and the slots: [nsplit - 1][W][kHbRecvPitch]
-  static constexpr int RECV_OFF = 0;
+  // merge, over Q and the slots once the MMAs are done: the parts this split
+  // sends (stage) and receives, [nsplit - 1] parts each of
+  // [(m, l0, l1, r0, r1) x 64][W = 512 / nsplit latent columns x kHbRecvPitch]
+  static constexpr int kPartHead = 5 * 64 * 4;
+  static constexpr __host__ __device__ int part_bytes(int ns) { return kPartHead + (512 / ns) * kHbRecvPitch; }
+  static constexpr int STAGE_OFF = 0;
+  static constexpr int RECV_OFF = 110592;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(BAR_OFF % 8 == 0, "mbarrier alignment");
-  static_assert((kHbMaxSplit - 1) * (512 / kHbMaxSplit) * kHbRecvPitch <= STAT_OFF, "merge receive buffer");
-  static_assert(1 * 256 * kHbRecvPitch <= STAT_OFF, "merge receive buffer");
 };
+static_assert(DecodeHbLayout::part_bytes(2) % 16 == 0 && DecodeHbLayout::part_bytes(4) % 16 == 0, "bulk copy sizes");
+static_assert(DecodeHbLayout::STAGE_OFF + 3 * DecodeHbLayout::part_bytes(4) <= DecodeHbLayout::RECV_OFF &&
+                  DecodeHbLayout::STAGE_OFF + DecodeHbLayout::part_bytes(2) <= DecodeHbLayout::RECV_OFF,
+              "merge stage");
+static_assert(DecodeHbLayout::RECV_OFF + 3 * DecodeHbLayout::part_bytes(4) <= DecodeHbLayout::STAT_OFF &&
+                  DecodeHbLayout::RECV_OFF + DecodeHbLayout::part_bytes(2) <= DecodeHbLayout::STAT_OFF,
+              "merge receive");
 
 __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const __grid_constant__ DecodeParams p) {
   using LY = DecodeHbLayout;
@@ -104,19 +118,17 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
   auto bar = [&](int i) { return bar0 + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::MISC_OFF + 4);
-  float* stats = reinterpret_cast<float*>(smem + LY::STAT_OFF);   // [split][m, l, r][64]
+  float* stats = reinterpret_cast<float*>(smem + LY::STAT_OFF);   // [m, l0, l1, r0, r1][64]
   float* wgt = reinterpret_cast<float*>(smem + LY::WGT_OFF);      // [split][64]
   float* alpha = reinterpret_cast<float*>(smem + LY::ALPHA_OFF);  // [b & 1][64]
-  float* lpart = reinterpret_cast<float*>(smem + LY::LPART_OFF);  // [l, r][64]
   volatile int* rflag = reinterpret_cast<volatile int*>(smem + LY::FLAG_OFF);
 
   if (threadIdx.x == 0) {
-    for (int t = 0; t < 9; ++t) {
-      mbar_init(bar(LY::BAR_Q + t), 1);
-      mbar_init(bar(LY::BAR_FULL + t), 1);
-      mbar_init(bar(LY::BAR_FULL + 9 + t), 1);
+    for (int g = 0; g < 3; ++g) mbar_init(bar(LY::BAR_Q + g), 1);
+    for (int g = 0; g < 6; ++g) {
+      mbar_init(bar(LY::BAR_FULL + g), 1);
+      mbar_init(bar(LY::BAR_EMPTY + g), 1);
     }
-    for (int c = 0; c < 8; ++c) mbar_init(bar(LY::BAR_EMPTY + c), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(LY::BAR_S + i), 1);
       mbar_init(bar(LY::BAR_SFREE + i), 8);  // one arrival per softmax warp
@@ -124,7 +136,10 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
     }
     mbar_init(bar(LY::BAR_P), 8);  // one arrival per softmax warp
     mbar_init(bar(LY::BAR_READY), ns > 1 ? ns - 1 : 1);          // one arrival per other split
-    mbar_init(bar(LY::BAR_DATA), ns > 1 ? 8 * (ns - 1) : 1);     // one per softmax warp of each other split
+    mbar_init(bar(LY::BAR_DATA), 1);
+    mbar_init(bar(LY::BAR_SENT), ns > 1 ? ns - 1 : 1);
+    // every other split's part arrives by a bulk copy as transaction bytes
+    if (ns > 1) mbar_arrive_expect_tx(bar(LY::BAR_DATA), (uint32_t)((ns - 1) * LY::part_bytes(ns)));
     *abort_flag = 0;
     rflag[0] = -1;
     rflag[1] = -1;
@@ -139,16 +154,19 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // the other splits may signal this CTA's barriers only after they were
-  // initialised: the matching wait comes before the first remote access
+  // initialised: the softmax warps, which make every remote access, wait for
+  // that before their main loop; the other warps before they leave
   if (ns > 1) cluster_arrive();
 
   if (nh > 0 && warp == 0) {
     // ---------------------------------------------------------- producer
-    // Q tile t just before the first half block's tile t, so that S starts on
-    // the first tiles while the rest land
+    // three requests per half block (tiles 3g .. 3g+2 each, 24 KB: a TMA
+    // request has a fixed cost, so few large boxes keep more bytes in flight
+    // than nine 8 KB tiles); Q's three groups just before the first half
+    // block's, so that S starts on the first tiles while the rest land
     if (elect_one()) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_kv64);
+      tma_prefetch_desc(&p.tm_q3);
+      tma_prefetch_desc(&p.tm_kv3);
     }
     __syncwarp();
     bool ok = true;
@@ -157,24 +175,33 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
       const int h = h_lo + it;
       const int2 rz = dec_block_rows(p, seq, walk.block(h >> 1));
       const uint32_t dst = sbase + LY::SLOT_OFF + slot * kHbSlot;
-      for (int t = 0; t < 9 && ok; ++t) {
-        // tiles 2c, 2c+1 are free once chunk c of the P.V two half blocks back
-        // completed; the P tile (8) with the last chunk
-        if (it >= 2 && (t & 1) == 0 && t < 8) {
-          ok = warp_wait(bar(LY::BAR_EMPTY + 4 * slot + t / 2), ((it >> 1) & 1) ^ 1, abort_flag);
+      for (int g = 0; g < 3 && ok; ++g) {
+        // tiles 3g .. 3g+2 are free once P.V of the half block two back has
+        // completed the chunks that read them
+        if (it >= 2) {
+          ok = warp_wait(bar(LY::BAR_EMPTY + 3 * slot + g), ((it >> 1) & 1) ^ 1, abort_flag);
           if (!ok) break;
         }
         if (elect_one()) {
           if (it == 0) {
-            mbar_arrive_expect_tx(bar(LY::BAR_Q + t), kDecQTile);
-            tma_load_3d(sbase + LY::Q_OFF + t * kDecQTile, &p.tm_q, bar(LY::BAR_Q + t), t * 64, 0, seq);
+            mbar_arrive_expect_tx(bar(LY::BAR_Q + g), 3 * kDecQTile);
+            tma_load_4d(sbase + LY::Q_OFF + 3 * g * kDecQTile, &p.tm_q3, bar(LY::BAR_Q + g), 0, 0, 3 * g, seq);
           }
-          mbar_arrive_expect_tx(bar(LY::BAR_FULL + 9 * slot + t), kHbTile);
-          tma_load_3d(dst + t * kHbTile, &p.tm_kv64, bar(LY::BAR_FULL + 9 * slot + t), 64 * t,
-                      rz.x + kHbRows * (h & 1), rz.y);
+          mbar_arrive_expect_tx(bar(LY::BAR_FULL + 3 * slot + g), 3 * kHbTile);
+          tma_load_4d(dst + 3 * g * kHbTile, &p.tm_kv3, bar(LY::BAR_FULL + 3 * slot + g), 0,
+                      rz.x + kHbRows * (h & 1), 3 * g, rz.y);
         }
         __syncwarp();
       }
+      if (it == 1 && elect_one()) {
+        // the half blocks after the first two into L2 now, so that HBM streams
+        // while the slots turn over; their loads into the slots then hit L2
+        for (int h2 = h_lo + 2; h2 < h_lo + nh; ++h2) {
+          const int2 r2 = dec_block_rows(p, seq, walk.block(h2 >> 1));
+          for (int g = 0; g < 3; ++g) tma_prefetch_l2_4d(&p.tm_kv3, 0, r2.x + kHbRows * (h2 & 1), 3 * g, r2.y);
+        }
+      }
+      __syncwarp();
     }
   } else if (nh > 0 && warp == 1) {
     // ---------------------------------------------------------- S issuer
@@ -191,18 +218,20 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
         if (!ok) break;
       }
       const uint32_t tmem_s = tmem + 64 * slot;
-      for (int t = 0; t < 9 && ok; ++t) {
-        if (it == 0) ok = warp_wait(bar(LY::BAR_Q + t), 0, abort_flag);
-        if (ok) ok = warp_wait(bar(LY::BAR_FULL + 9 * slot + t), (it >> 1) & 1, abort_flag);
+      for (int g = 0; g < 3 && ok; ++g) {
+        if (it == 0) ok = warp_wait(bar(LY::BAR_Q + g), 0, abort_flag);
+        if (ok) ok = warp_wait(bar(LY::BAR_FULL + 3 * slot + g), (it >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
-          const uint64_t da = desc_add(dq0, t * kDecQTile);
-          const uint64_t db = desc_add(dk0, slot * kHbSlot + t * kHbTile);
+          for (int t = 3 * g; t < 3 * g + 3; ++t) {
+            const uint64_t da = desc_add(dq0, t * kDecQTile);
+            const uint64_t db = desc_add(dk0, slot * kHbSlot + t * kHbTile);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem_s, desc_add(da, 32 * kk), desc_add(db, 32 * kk), idesc_s, (t | kk) != 0);
-          if (t == 8) mma_commit(bar(LY::BAR_S + slot));
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem_s, desc_add(da, 32 * kk), desc_add(db, 32 * kk), idesc_s, (t | kk) != 0);
+          }
+          if (g == 2) mma_commit(bar(LY::BAR_S + slot));
         }
         __syncwarp();
       }
@@ -229,9 +258,10 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
             mma_ss(tmem_o + 64 * u, desc_add(da, 2048 * kk), desc_add(dp, 32 * kk), idesc_o,
                    (b > 0 || kk > 0) ? 1u : 0u);
           // pv_done before the last chunk's empty: a reload of the P tile
-          // implies P.V(b) is signalled
+          // implies P.V(b) is signalled. Chunk u >= 1 frees tiles 3(u-1) ..
+          // 3(u-1)+2 (chunks complete in order; the last also frees the P tile)
           if (u == 3) mma_commit(bar(LY::BAR_PV + (b & 1)));
-          mma_commit(bar(LY::BAR_EMPTY + 4 * slot + u));
+          if (u >= 1) mma_commit(bar(LY::BAR_EMPTY + 3 * slot + (u - 1)));
         }
       }
       __syncwarp();
@@ -254,6 +284,7 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
   float l_a = 0.f, l_b = 0.f;              // sums of exact P
   float r_a = 0.f, r_b = 0.f;              // sums of bf16-rounded P (normalise O)
   bool ok = true;
+  if (smx && ns > 1) cluster_wait();
   if (smx && nh > 0) {
     const float cs = p.scale_log2;
     for (int b = 0; b < nh; ++b) {
@@ -383,6 +414,9 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
   }
 
   // ---------------------------------------------------------- this split's (m, l, r)
+  // m, and the sums of each key group kept apart (the owner adds them):
+  // [m, l of group 0, l of group 1, r of group 0, r of group 1][64 heads],
+  // here and at the head of every part staged for another split
   if (smx) {
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
@@ -392,99 +426,112 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
     r_a += __shfl_xor_sync(0xffffffffu, r_a, 2);
     r_b += __shfl_xor_sync(0xffffffffu, r_b, 2);
-    if (grp == 1 && t4 == 0) {
-      lpart[ha] = l_a;
-      lpart[hb2] = l_b;
-      lpart[64 + ha] = r_a;
-      lpart[64 + hb2] = r_b;
+    if (t4 == 0) {
+      for (int j = -1; j < ns - 1; ++j) {
+        float* st = j < 0 ? stats : reinterpret_cast<float*>(smem + LY::STAGE_OFF + j * LY::part_bytes(ns));
+        if (grp == 0) {
+          st[ha] = m_a;
+          st[hb2] = m_b;
+        }
+        st[64 * (1 + grp) + ha] = l_a;
+        st[64 * (1 + grp) + hb2] = l_b;
+        st[64 * (3 + grp) + ha] = r_a;
+        st[64 * (3 + grp) + hb2] = r_b;
+      }
     }
-    named_barrier_sync(1, 256);
-    if (grp == 0 && t4 == 0) {
-      float* st = stats + split * 192;
-      st[ha] = m_a;
-      st[hb2] = m_b;
-      st[64 + ha] = nh > 0 ? l_a + lpart[ha] : 0.f;
-      st[64 + hb2] = nh > 0 ? l_b + lpart[hb2] : 0.f;
-      st[128 + ha] = nh > 0 ? r_a + lpart[64 + ha] : 0.f;
-      st[128 + hb2] = nh > 0 ? r_b + lpart[64 + hb2] : 0.f;
-    }
-    named_barrier_sync(1, 256);
   }
 
   // ---------------------------------------------------------- on-chip merge of the splits
+  // Each split stages, for every other split, its (m, l, r) and its unscaled
+  // partial O^T of that split's columns in its own shared memory (free once
+  // its MMAs are done), and moves each part with one bulk copy into the
+  // owner's receive area once the owner has said that area is free. The
+  // copies complete as transaction bytes on the owner's data barrier.
   const int W = 512 / ns;
-  float* recv = reinterpret_cast<float*>(smem + LY::RECV_OFF);
+  const int DB = LY::part_bytes(ns);
   if (ns > 1) {
-    cluster_wait();  // every split's barriers are initialised
     if (smx) {
-      // this CTA's MMAs are done (or it had none): its shared memory may
-      // receive; then wait until every other split's may
+      if (tid == 32) {
+        // this CTA's MMAs are done (or it had none): its receive area is free
+        // (a plain arrive: the MMAs that read the area have completed)
+        for (int s2 = 0; s2 < ns; ++s2)
+          if (s2 != split) mbar_arrive_cluster(peer_addr(bar(LY::BAR_READY), (uint32_t)s2));
+      }
+      {
+        // lane = latent column, 32 heads per thread as eight 16-byte stores
+        // (zeros from a split without keys, so the owner needs no test)
+#pragma unroll 1
+        for (int u = 0; u < 4; ++u) {
+          const int d = 128 * u + 32 * quarter + lane;
+          const int owner = d / W;
+          if (owner == split) continue;
+          float o[32];
+          if (nh > 0 && ok) {
+            tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          }
+          const int j = owner < split ? owner : owner - 1;
+          uint4* dst = reinterpret_cast<uint4*>(smem + LY::STAGE_OFF + j * DB + LY::kPartHead +
+                                                (d - owner * W) * kHbRecvPitch + grp * 128);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            dst[q4] = make_uint4(__float_as_uint(o[4 * q4]), __float_as_uint(o[4 * q4 + 1]),
+                                 __float_as_uint(o[4 * q4 + 2]), __float_as_uint(o[4 * q4 + 3]));
+        }
+      }
+      fence_proxy_async_smem();  // the staged parts are read by the bulk copies
+      named_barrier_sync(1, 256);
+      // every other split's receive area is free: one bulk copy per owner
+      if (warp_wait_cluster(bar(LY::BAR_READY), 0, abort_flag) && tid == 0) {
+        for (int o2 = 0; o2 < ns; ++o2) {
+          if (o2 == split) continue;
+          const int j = o2 < split ? o2 : o2 - 1;       // the part for o2 in this split's stage
+          const int jr = split < o2 ? split : split - 1; // this split's part in o2's receive area
+          bulk_copy_to_peer(peer_addr(sbase + LY::RECV_OFF + jr * DB, (uint32_t)o2), sbase + LY::STAGE_OFF + j * DB,
+                            DB, peer_addr(bar(LY::BAR_DATA), (uint32_t)o2));
+        }
+      }
+      ok = warp_wait(bar(LY::BAR_DATA), 0, abort_flag) && ok;
+      // every part copied into this CTA has landed: tell each sender that it
+      // may leave (its copies have read their source)
       if (tid == 0) {
         for (int s2 = 0; s2 < ns; ++s2)
-          if (s2 != split) mbar_arrive_cluster_release(peer_addr(bar(LY::BAR_READY), (uint32_t)s2));
+          if (s2 != split) mbar_arrive_cluster(peer_addr(bar(LY::BAR_SENT), (uint32_t)s2));
       }
-      const bool rdy = warp_wait_cluster(bar(LY::BAR_READY), 0, abort_flag);
-      if (rdy) {
-        if (tid < 64) {
-          const float* st = stats + split * 192;
-          for (int s2 = 0; s2 < ns; ++s2) {
-            if (s2 == split) continue;
-            const uint32_t dst = peer_addr(smem_u32(stats + split * 192 + tid), (uint32_t)s2);
-            st_cluster_u32(dst, __float_as_uint(st[tid]));
-            st_cluster_u32(dst + 256, __float_as_uint(st[64 + tid]));
-            st_cluster_u32(dst + 512, __float_as_uint(st[128 + tid]));
-          }
-        }
-        if (nh > 0 && ok) {
-          // the unscaled partial O^T of the columns other splits own: lane =
-          // latent column, 32 heads per thread as eight 16-byte stores
-#pragma unroll 1
-          for (int u = 0; u < 4; ++u) {
-            const int d = 128 * u + 32 * quarter + lane;
-            const int owner = d / W;
-            if (owner == split) continue;
-            float o[32];
-            tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, o);
-            const int slot_in = split < owner ? split : split - 1;
-            const uint32_t dst = peer_addr(
-                smem_u32(reinterpret_cast<uint8_t*>(recv) + (size_t)(slot_in * W + (d - owner * W)) * kHbRecvPitch +
-                         grp * 128),
-                (uint32_t)owner);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              st_cluster_v4(dst + 16 * j, __float_as_uint(o[4 * j]), __float_as_uint(o[4 * j + 1]),
-                            __float_as_uint(o[4 * j + 2]), __float_as_uint(o[4 * j + 3]));
-          }
-        }
-      }
-      fence_acq_rel_cluster();
-      __syncwarp();
-      if (lane == 0) {
-        for (int s2 = 0; s2 < ns; ++s2)
-          if (s2 != split) mbar_arrive_cluster_release(peer_addr(bar(LY::BAR_DATA), (uint32_t)s2));
-      }
-      ok = warp_wait_cluster(bar(LY::BAR_DATA), 0, abort_flag) && ok && rdy;
     }
   }
   if (smx) {
+    // weights of the splits' partial O by the log-sum-exp rule
+    if (ns == 1) named_barrier_sync(1, 256);  // the statistics above are complete
+    // [m, l0, l1, r0, r1] of split s2: this split's own, or the head of its received part
+    auto part = [&](int s2) -> const float* {
+      if (s2 == split) return stats;
+      return reinterpret_cast<const float*>(smem + LY::RECV_OFF + (s2 < split ? s2 : s2 - 1) * DB);
+    };
     if (tid < 64) {
       const int h = tid;
       float M = -INFINITY;
-      for (int s2 = 0; s2 < ns; ++s2)
-        if (stats[s2 * 192 + 64 + h] > 0.f) M = fmaxf(M, stats[s2 * 192 + h]);
+      for (int s2 = 0; s2 < ns; ++s2) {
+        const float* st = part(s2);
+        if (st[64 + h] + st[128 + h] > 0.f) M = fmaxf(M, st[h]);
+      }
       // O is normalised by the merged sum of the bf16 P that multiplied V,
       // the LSE by the merged exact sum
       float Ls = 0.f, Rs = 0.f;
       for (int s2 = 0; s2 < ns; ++s2) {
-        const float l = stats[s2 * 192 + 64 + h];
-        const float w = l > 0.f ? ex2_approx(stats[s2 * 192 + h] - M) : 0.f;
+        const float* st = part(s2);
+        const float l = st[64 + h] + st[128 + h];
+        const float w = l > 0.f ? ex2_approx(st[h] - M) : 0.f;
         wgt[s2 * 64 + h] = w;
         Ls += l * w;
-        Rs += stats[s2 * 192 + 128 + h] * w;
+        Rs += (st[192 + h] + st[256 + h]) * w;
       }
-      const float inv = Rs > 0.f ? 1.f / Rs : 0.f;
+      const float inv = Rs > 0.f ? rcp_approx(Rs) : 0.f;
       for (int s2 = 0; s2 < ns; ++s2) wgt[s2 * 64 + h] *= inv;
-      if (split == 0) p.lse[(int64_t)seq * kDecHeads + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994530942f : -INFINITY;
+      if (split == 0)
+        p.lse[(int64_t)seq * kDecHeads + h] = Ls > 0.f ? (M + lg2_approx(Ls)) * 0.69314718055994530942f : -INFINITY;
     }
     named_barrier_sync(1, 256);
 #pragma unroll 1
@@ -494,27 +541,32 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
       float acc[32];
       if (nh > 0 && ok) {
         tmem_ld32(lane_addr + 128 + 64 * u + 32 * grp, acc);
+        const float4* w4 = reinterpret_cast<const float4*>(wgt + split * 64 + 32 * grp);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] *= wgt[split * 64 + 32 * grp + i];
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 w = w4[q4];
+          acc[4 * q4] *= w.x;
+          acc[4 * q4 + 1] *= w.y;
+          acc[4 * q4 + 2] *= w.z;
+          acc[4 * q4 + 3] *= w.w;
+        }
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = 0.f;
       }
       for (int s2 = 0; s2 < ns; ++s2) {
         if (s2 == split) continue;
-        const int slot_in = s2 < split ? s2 : s2 - 1;
-        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const uint8_t*>(recv) +
-                                                            (size_t)(slot_in * W + (d - split * W)) * kHbRecvPitch +
-                                                            grp * 128);
+        const int j = s2 < split ? s2 : s2 - 1;
+        const float4* src = reinterpret_cast<const float4*>(smem + LY::RECV_OFF + j * DB + LY::kPartHead +
+                                                            (d - split * W) * kHbRecvPitch + grp * 128);
+        const float4* w4 = reinterpret_cast<const float4*>(wgt + s2 * 64 + 32 * grp);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 v = src[j];
-          const float* w = wgt + s2 * 64 + 32 * grp + 4 * j;
-          // a split without keys pushed no O (its weight is 0)
-          if (w[0] != 0.f) acc[4 * j] += v.x * w[0];
-          if (w[1] != 0.f) acc[4 * j + 1] += v.y * w[1];
-          if (w[2] != 0.f) acc[4 * j + 2] += v.z * w[2];
-          if (w[3] != 0.f) acc[4 * j + 3] += v.w * w[3];
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 v = src[q4], w = w4[q4];
+          acc[4 * q4] = fmaf(v.x, w.x, acc[4 * q4]);
+          acc[4 * q4 + 1] = fmaf(v.y, w.y, acc[4 * q4 + 1]);
+          acc[4 * q4 + 2] = fmaf(v.z, w.z, acc[4 * q4 + 2]);
+          acc[4 * q4 + 3] = fmaf(v.w, w.w, acc[4 * q4 + 3]);
         }
       }
       __nv_bfloat16* dst = p.out + (int64_t)seq * kDecHeads * 512 + d;
@@ -522,6 +574,9 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
       for (int i = 0; i < 32; ++i) dst[(int64_t)(32 * grp + i) * 512] = __float2bfloat16_rn(acc[i]);
     }
   }
+  // no split leaves while a bulk copy out of its shared memory may still run
+  if (ns > 1 && smx) ok = warp_wait_cluster(bar(LY::BAR_SENT), 0, abort_flag) && ok;
+  if (ns > 1 && !smx) cluster_wait();  // the other warps' half of the barrier at the start
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

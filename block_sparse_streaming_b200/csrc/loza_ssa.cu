@@ -141,6 +141,23 @@ DecodeWorkspace decode_workspace(int32_t batch, const DecodePlan& plan) {
   return w;
 }
 
+// 4-D bf16 map {64 columns, rows, 9 column tiles, batch} over a latent tensor
+// [batch][rows][576] with the given row and batch strides (elements): the
+// tile dimension's stride is 128 bytes, so a box {64, box_rows, 3, 1} lands as
+// three consecutive [box_rows x 64] 128-byte-swizzled tiles.
+bool make_map_latent3(CUtensorMap* m, const void* base, int64_t rows, int64_t batch, int64_t row_stride,
+                      int64_t batch_stride, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, (cuuint64_t)rows, 9, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)row_stride * 2, 128, (cuuint64_t)batch_stride * 2};
+  cuuint32_t box[4] = {64, box_rows, 3, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Validate an absorbed-MLA decode call and build its kernel parameters
 // (everything except the workspace pointers).
 loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
@@ -184,6 +201,9 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return LOZA_ERR_CUDA;
   }
+  if (!make_map_latent3(&prm->tm_q3, q, n_heads, batch, 576, (int64_t)n_heads * 576, (uint32_t)kDecHeads) ||
+      !make_map_latent3(&prm->tm_kv3, k_cache, max_seqlen, batch, cache_row_stride, cache_batch_stride, 64))
+    return LOZA_ERR_CUDA;
   prm->seqlens = seqlens;
   prm->out = reinterpret_cast<__nv_bfloat16*>(out);
   prm->lse = lse;
@@ -481,6 +501,9 @@ loza_status loza_ssa_decode_paged(const void* q, const void* kv_pool, int32_t nu
       fn(&prm.tm_kv64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv_pool), dims, strides, box64, estr,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return LOZA_ERR_CUDA;
+  if (!make_map_latent3(&prm.tm_kv3, kv_pool, (int64_t)num_pages * kTile, 1, pool_row_stride,
+                        (int64_t)num_pages * kTile * pool_row_stride, 64))
     return LOZA_ERR_CUDA;
   prm.block_table = block_table;
   prm.bt_stride = bt_stride;

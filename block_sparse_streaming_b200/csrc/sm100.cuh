@@ -165,6 +165,26 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(desc)) : "memory");
 }
 
+// Ask for a box to be brought into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const void* desc, int32_t c0, int32_t c1, int32_t c2,
+                                                   int32_t c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+               ::"l"(reinterpret_cast<uint64_t>(desc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
+
+// 4-D box load. With dims {64 columns, rows, column tile, batch} over a
+// row-major [batch][rows][tiles * 64] bf16 tensor (the tile dimension's
+// stride is 128 bytes), one box of {64, R, T, 1} lands as T consecutive
+// [R x 64] 128-byte-swizzled tiles: one request instead of T.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* desc, uint32_t bar, int32_t c0, int32_t c1,
+                                            int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* desc, uint32_t bar,
                                             int32_t c0, int32_t c1) {
   asm volatile(
@@ -550,6 +570,19 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 1/x and log2(x) on the special-function unit (rcp.approx / lg2.approx,
+// flush to zero; relative errors ~2^-23 and ~2^-22).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
