@@ -29,6 +29,7 @@ struct DecodeMhaParams {
   float* lse;                  // [B, H]
   int n_heads, n_kv_heads;
   int n_sink, n_local;
+  int block;  // b, tokens per block of the window
   float scale_log2;
 };
 
@@ -41,7 +42,10 @@ __global__ void __launch_bounds__(128) ssa_decode_mha_kernel(const DecodeMhaPara
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = p.seqlens[seq];
   const int i_q = L - 1;
-  const BlockWalk walk(i_q / kTile, p.n_sink, p.n_local);
+  // the window of the query: keys [0, sink_end) and [lo, i_q], each once
+  const SsaWindow win{p.block, p.n_sink * p.block, p.n_local};
+  const int r0_end = min(win.sink_end, i_q + 1);
+  const int r1_lo = max(win.lo(i_q), r0_end);
   float qv[QPL];
   const __nv_bfloat16* qp = p.q + ((int64_t)seq * p.n_heads + h) * DQK;
 #pragma unroll
@@ -49,11 +53,11 @@ __global__ void __launch_bounds__(128) ssa_decode_mha_kernel(const DecodeMhaPara
   float m = -INFINITY, l = 0.f, acc[VPL];
 #pragma unroll
   for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
-  // keys of the window, warp w takes every 4th key
-  for (int b = 0; b < walk.count; ++b) {
-    const int kb = walk.block(b);
-    const int t_end = min(kb * kTile + kTile, i_q + 1);
-    for (int t = kb * kTile + warp; t < t_end; t += 4) {
+  // keys of the window (the sink range, then the local range), warp w takes every 4th key
+  for (int range = 0; range < 2; ++range) {
+    const int t_lo = range == 0 ? 0 : r1_lo;
+    const int t_end = range == 0 ? r0_end : i_q + 1;
+    for (int t = t_lo + warp; t < t_end; t += 4) {
       const __nv_bfloat16* kp = p.k + seq * p.k_batch_stride + (int64_t)t * p.k_row_stride + (int64_t)hk * DQK;
       float s = 0.f;
 #pragma unroll

@@ -73,6 +73,7 @@ struct DecodeParams {
   int bps;             // selected blocks per split
   int n_sink;
   int n_local;         // < 0: unbounded
+  int block;           // b, tokens per block of the window
   float scale_log2;
 };
 
@@ -174,7 +175,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
   const int L = p.seqlens[seq];
   const int i_q = L - 1;                 // decode query position
   const int jq = i_q / kTile;            // its block
-  const BlockWalk walk(jq, p.n_sink, p.n_local);
+  // the 128-row units of the window of position i_q (the own block last)
+  const SsaWindow win{p.block, p.n_sink * p.block, p.n_local};
+  const RowWalk walk(win, i_q, kTile);
+  const int lo_q = win.lo(i_q);
   const int b_lo = split * p.bps;
   const int nb = max(0, min(walk.count, b_lo + p.bps) - b_lo);
 
@@ -254,11 +258,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
       };
       for (int it = 0; it <= nb && ok; ++it) {
         if (it < nb) {
-          const int2 krow = dec_block_rows(p, seq, walk.block(b_lo + it));
+          const int2 krow = dec_block_rows(p, seq, walk.unit_at(b_lo + it));
           for (int u = 0; u < kDecKUnits && ok; ++u) load_unit(krow, u);
         }
         if (it >= 1) {
-          const int2 vrow = dec_block_rows(p, seq, walk.block(b_lo + it - 1));
+          const int2 vrow = dec_block_rows(p, seq, walk.unit_at(b_lo + it - 1));
           for (int u = 0; u < kDecVUnits && ok; ++u) load_unit(vrow, u);
         }
       }
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
         if (it >= 1) {
           // O^T += V^T . P^T(b), V unit u = latent columns 128u .. 128u+127
           const int b = it - 1;
-          if (walk.block(b_lo + b) == jq) {
+          if (walk.unit_at(b_lo + b) == jq) {
             // the query's own block may end inside the block: once its V units
             // are resident, let the softmax warps zero the rows past the end
             for (int u = 0; u < kDecVUnits && ok; ++u) {
@@ -356,8 +360,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
         if (tid == 0) *rescale_flag = 0;  // read by all only after the next two barriers
         float x[32];
         tmem_ld32(lane_addr + 64 * (b & 1) + 32 * grp, x);
-        const int kb = walk.block(b_lo + b);
-        const bool valid = kb * kTile + key <= i_q;
+        const int kb = walk.unit_at(b_lo + b);
+        const int tpos = kb * kTile + key;
+        const bool valid = tpos <= i_q && (tpos < win.sink_end || tpos >= lo_q);
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] = valid ? x[i] : -INFINITY;
         redmax[quarter * 64 + grp * 32 + lane] = warp_reduce_scatter32<true>(x);
@@ -443,7 +448,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
           // hold anything there) so that 0 * garbage cannot reach O
           ok = warp_wait(bar(LY::BAR_VT), 0, abort_flag);
           if (!ok) break;
-          if (!valid) {
+          if (tpos > i_q) {
             const uint4 z = make_uint4(0, 0, 0, 0);
             for (int u = 2 * grp; u < 2 * grp + 2; ++u) {
               const int slot_u = dec_v_pos(b, u, nb) % kDecStages;

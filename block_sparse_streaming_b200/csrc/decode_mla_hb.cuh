@@ -103,11 +103,12 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
   const int ns = p.nsplit;
   const int L = p.seqlens[seq];
   const int i_q = L - 1;                                 // decode query position
-  const int jq = i_q >= 0 ? i_q / kTile : 0;             // its block
-  const int hq = i_q >= 0 ? (i_q % kTile) / kHbRows : 0; // the half of its block that holds it
-  const BlockWalk walk(jq, p.n_sink, p.n_local);
-  // half blocks in walk order (the own block is last; its second half only if hq == 1)
-  const int nh_total = i_q >= 0 ? 2 * walk.count - (hq == 0 ? 1 : 0) : 0;
+  // the half blocks (64-row units) of the window of position i_q, sinks
+  // first, the unit holding i_q last; each holds at least one visible key
+  const SsaWindow win{p.block, p.n_sink * p.block, p.n_local};
+  const RowWalk walk(win, max(i_q, 0), kHbRows);
+  const int lo_q = win.lo(max(i_q, 0));
+  const int nh_total = i_q >= 0 ? walk.count : 0;
   const int h_lo = split * p.bps;
   const int nh = max(0, min(nh_total, h_lo + p.bps) - h_lo);
 
@@ -172,8 +173,8 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
     bool ok = true;
     for (int it = 0; it < nh && ok; ++it) {
       const int slot = it & 1;
-      const int h = h_lo + it;
-      const int2 rz = dec_block_rows(p, seq, walk.block(h >> 1));
+      const int h = walk.unit_at(h_lo + it);  // rows 64h .. 64h+63 of the context
+      const int2 rz = dec_block_rows(p, seq, h >> 1);
       const uint32_t dst = sbase + LY::SLOT_OFF + slot * kHbSlot;
       for (int g = 0; g < 3 && ok; ++g) {
         // tiles 3g .. 3g+2 are free once P.V of the half block two back has
@@ -196,8 +197,9 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
       if (it == 1 && elect_one()) {
         // the half blocks after the first two into L2 now, so that HBM streams
         // while the slots turn over; their loads into the slots then hit L2
-        for (int h2 = h_lo + 2; h2 < h_lo + nh; ++h2) {
-          const int2 r2 = dec_block_rows(p, seq, walk.block(h2 >> 1));
+        for (int i2 = h_lo + 2; i2 < h_lo + nh; ++i2) {
+          const int h2 = walk.unit_at(i2);
+          const int2 r2 = dec_block_rows(p, seq, h2 >> 1);
           for (int g = 0; g < 3; ++g) tma_prefetch_l2_4d(&p.tm_kv3, 0, r2.x + kHbRows * (h2 & 1), 3 * g, r2.y);
         }
       }
@@ -299,16 +301,16 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(LY::BAR_SFREE + slot));
-      const int h = h_lo + b;
-      const int kb = walk.block(h >> 1);
-      const int base_pos = kb * kTile + kHbRows * (h & 1);
-      const int cut = i_q - base_pos;  // keys c <= cut are visible (>= 63: all)
-      if (cut < 63) {
+      const int base_pos = kHbRows * walk.unit_at(h_lo + b);
+      const int cut = i_q - base_pos;         // keys c <= cut exist (>= 63: all)
+      const int e = win.sink_end - base_pos;  // c < e: sink keys
+      const int f = lo_q - base_pos;          // c >= f: the local range
+      if (cut < 63 || (e < 64 && f > 0)) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int c = 8 * k + 2 * t4;
-          if (c > cut) { x[4 * k] = -INFINITY; x[4 * k + 2] = -INFINITY; }
-          if (c + 1 > cut) { x[4 * k + 1] = -INFINITY; x[4 * k + 3] = -INFINITY; }
+          if (!(c <= cut && (c < e || c >= f))) { x[4 * k] = -INFINITY; x[4 * k + 2] = -INFINITY; }
+          if (!(c + 1 <= cut && (c + 1 < e || c + 1 >= f))) { x[4 * k + 1] = -INFINITY; x[4 * k + 3] = -INFINITY; }
         }
       }
       // row maxima over all 64 keys (both key groups compute the same)

@@ -62,10 +62,55 @@ bool make_map_3d(CUtensorMap* m, const void* base, int64_t dim, int64_t heads, i
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool stride_ok(int64_t s) { return s > 0 && (s * 2) % 16 == 0 && s * 2 < (int64_t(1) << 40); }
 
+// A window the prefill and decode kernels take: b a power of two from 1 to
+// 65,536 tokens per block; s >= 0 sink blocks and l >= 1 local blocks, or the
+// unbounded window (l = LOZA_UNBOUNDED: every earlier key; s is then unused).
 bool window_ok(const loza_ssa_params& p) {
-  if (p.block_size != kTile) return false;
-  if (p.n_local != LOZA_UNBOUNDED && (p.n_local < 1 || p.n_sink < 0)) return false;
+  const int b = p.block_size;
+  if (b < 1 || b > 65536 || (b & (b - 1)) != 0) return false;
+  if (p.n_local == LOZA_UNBOUNDED) return true;
+  if (p.n_local < 1 || p.n_sink < 0) return false;
+  if ((int64_t)p.n_sink * b > (int64_t(1) << 30) || (int64_t)p.n_local * b > (int64_t(1) << 30)) return false;
   return true;
+}
+// The backward, the host-buffer prefill and the sharded prefill work in
+// whole blocks of 128 tokens.
+bool window_block128(const loza_ssa_params& p) { return window_ok(p) && p.block_size == kTile; }
+
+SsaWindow host_window(const loza_ssa_params& p) {
+  const bool unb = p.n_local == LOZA_UNBOUNDED;
+  return SsaWindow{p.block_size, unb ? 0 : p.n_sink * p.block_size, unb ? -1 : p.n_local};
+}
+
+// Most units of `unit` keys (RowWalk) that a query at any position below
+// max_seqlen reads. Once the window is full the count repeats with period
+// max(b, unit) (both powers of two), so the positions of the first window and
+// the last few periods before max_seqlen cover every value it takes.
+int max_row_units(const loza_ssa_params& p, int32_t max_seqlen, int unit) {
+  const SsaWindow w = host_window(p);
+  if (w.n_local < 0) return (max_seqlen - 1) / unit + 1;
+  const int64_t period = std::max(p.block_size, unit);
+  const int64_t span = std::min<int64_t>(max_seqlen, (int64_t)(p.n_sink + p.n_local + 2) * p.block_size + 4 * period);
+  int best = 0;
+  for (int64_t i = 0; i < span; ++i) best = std::max(best, RowWalk(w, (int)i, unit).count);
+  for (int64_t i = std::max<int64_t>(span, max_seqlen - 4 * period - unit); i < max_seqlen; ++i)
+    best = std::max(best, RowWalk(w, (int)i, unit).count);
+  return best;
+}
+
+// Most key tiles (BlockWalk) a query tile of a sequence of max_seqlen reads.
+int max_tiles(const loza_ssa_params& p, int32_t max_seqlen) {
+  const int nq = (max_seqlen + kTile - 1) / kTile;
+  const SsaWindow w = host_window(p);
+  if (w.n_local < 0) return nq;
+  const int n_sink = p.n_sink, b = p.block_size;
+  const int64_t period = std::max(1, b / kTile);
+  const int64_t span = std::min<int64_t>(nq, ((int64_t)(n_sink + p.n_local + 2) * b) / kTile + 4 * period + 2);
+  int best = 0;
+  for (int64_t q = 0; q < span; ++q) best = std::max(best, BlockWalk((int)q, n_sink, w.n_local, b).count);
+  for (int64_t q = std::max<int64_t>(span, nq - 4 * period - 2); q < nq; ++q)
+    best = std::max(best, BlockWalk((int)q, n_sink, w.n_local, b).count);
+  return best;
 }
 
 int sm_count() {
@@ -102,10 +147,7 @@ struct DecodePlan {
   bool half_block;  // 64-row units resident for both MMAs (decode_mla_hb.cuh)
 };
 DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t batch) {
-  const int max_blocks = (max_seqlen + kTile - 1) / kTile;
-  const int count = p.n_local == LOZA_UNBOUNDED
-                        ? max_blocks
-                        : (p.n_sink + p.n_local < max_blocks ? p.n_sink + p.n_local : max_blocks);
+  const int count = max_row_units(p, max_seqlen, kTile);  // selected 128-row blocks
   const int sms = sm_count();
   if (count > 8 && (int64_t)batch * 16 <= sms) {
     int ns = (sms + batch - 1) / batch;
@@ -116,7 +158,7 @@ DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t bat
   if (count <= 16 && (int64_t)batch * 2 <= sms) {
     // half blocks: up to 4 CTAs per sequence in one cluster, each pulling
     // its share of the rows once
-    const int nh = 2 * count;
+    const int nh = max_row_units(p, max_seqlen, kHbRows);
     int ns = 1;
     while (ns < kHbMaxSplit && ns * 2 <= nh && (int64_t)batch * ns * 2 <= sms) ns *= 2;
     const int hps = (nh + ns - 1) / ns;
@@ -139,6 +181,24 @@ DecodeWorkspace decode_workspace(int32_t batch, const DecodePlan& plan) {
   w.ticket_off = w.ml_off + parts * sizeof(float4);
   w.total = w.ticket_off + ((size_t)batch * sizeof(int) + 255) / 256 * 256;
   return w;
+}
+
+// 4-D bf16 map {64 columns, rows, ntiles, 1}: column tile i of row r at
+// base + r * row_stride + i * tile_stride_bytes (128-byte swizzle); a box
+// {64, box_rows, box_tiles, 1} lands as box_tiles consecutive [box_rows x 64]
+// tiles.
+bool make_map_tiles4(CUtensorMap* m, const void* base, int64_t rows, int ntiles, int64_t row_stride,
+                     int64_t tile_stride_bytes, uint32_t box_rows, uint32_t box_tiles) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)ntiles, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)row_stride * 2, (cuuint64_t)tile_stride_bytes,
+                           (cuuint64_t)row_stride * 2 * (cuuint64_t)rows};
+  cuuint32_t box[4] = {64, box_rows, box_tiles, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 4-D bf16 map {64 columns, rows, 9 column tiles, batch} over a latent tensor
@@ -211,6 +271,7 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
   prm->bps = plan->bps;
   prm->n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
   prm->n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
+  prm->block = p.block_size;
   prm->scale_log2 = p.scale * 1.4426950408889634f;
   return LOZA_OK;
 }
@@ -382,8 +443,10 @@ size_t mla_scratch_per_cta(int max_blocks) {
   return (size_t)max_blocks * (kTile * kTile * 2 + 256 * 4);
 }
 size_t mla_workspace_bytes(int max_blocks) { return (size_t)sm_count() * mla_scratch_per_cta(max_blocks); }
-// The two-pass kernel keeps one bit per key block of a query tile.
-bool mla_window_ok(int n_sink, int n_local) { return n_local >= 0 && n_sink + n_local <= 32; }
+// The two-pass kernel keeps one bit per key tile of a query tile.
+bool mla_window_ok(const loza_ssa_params& p, int32_t max_seqlen) {
+  return p.n_local != LOZA_UNBOUNDED && max_tiles(p, max_seqlen) <= kMlaMaxBlocks;
+}
 
 loza_status launch_prefill_mla(PrefillMlaParams& prm, void* workspace, cudaStream_t stream) {
   using LY = PrefillMlaLayout;
@@ -579,11 +642,12 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
     return 0;
   }
   if (op == LOZA_OP_PREFILL) {
-    if (n_kv_heads == 1 && d_qk == 576 && d_v == 512 && n_heads % 2 == 0 && mla_window_ok(p.n_sink, p.n_local))
-      return mla_workspace_bytes(p.n_sink + p.n_local);
+    if (n_kv_heads == 1 && d_qk == 576 && d_v == 512 && n_heads % 2 == 0 && mla_window_ok(p, max_seqlen))
+      return mla_workspace_bytes(max_tiles(p, max_seqlen));
     return 0;
   }
   if (op == LOZA_OP_PREFILL_HOST) {
+    if (!window_block128(p)) return 0;
     if (total_tokens < max_seqlen || total_tokens > INT32_MAX || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v))
       return 0;
     const HostChunkPlan h = host_chunk_plan(max_seqlen, p);
@@ -592,6 +656,7 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
     return host_layout(h, host_chunk_cap(batch, total_tokens), pf, n_heads, n_kv_heads, d_qk, d_v).total;
   }
   if (op == LOZA_OP_BACKWARD) {
+    if (!window_block128(p)) return 0;
     if (n_kv_heads != n_heads || p.n_local == LOZA_UNBOUNDED || total_tokens < 1) return 0;
     if (!((d_qk == 64 && d_v == 64) || (d_qk == 192 && d_v == 128))) return 0;
     return bwd_workspace(batch, total_tokens, max_seqlen, n_heads, d_qk, d_v, p).total;
@@ -630,6 +695,7 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
   prm.d_v = d_v;
   prm.n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
   prm.n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
+  prm.block = p.block_size;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
 
   int dvt;
@@ -642,26 +708,32 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
 
   const int64_t v_head_stride = latent_v ? d_qk : d_v;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0 && mla_window_ok(prm.n_sink, prm.n_local) && workspace != nullptr &&
-      aligned16(workspace) && workspace_bytes >= mla_workspace_bytes(prm.n_sink + prm.n_local)) {
+  if (dvt == 256 && n_kv_heads == 1 && n_heads % 2 == 0 && mla_window_ok(p, max_seqlen) && workspace != nullptr &&
+      aligned16(workspace) && workspace_bytes >= mla_workspace_bytes(max_tiles(p, max_seqlen))) {
     // absorbed MLA, bounded window: S once, the value dimension in two passes
     PrefillMlaParams mp;
     std::memset(&mp, 0, sizeof(mp));
     mp.cu_seqlens = cu_seqlens;
     mp.out = prm.out;
     mp.lse = lse;
-    mp.max_blocks = prm.n_sink + prm.n_local;
+    mp.max_blocks = max_tiles(p, max_seqlen);
     mp.n_heads = n_heads;
     mp.n_qtiles = (max_seqlen + kTile - 1) / kTile;
     if ((int64_t)batch * mp.n_qtiles * (n_heads / 2) > INT32_MAX) return LOZA_ERR_UNSUPPORTED;
     mp.total_tiles = batch * mp.n_qtiles * (n_heads / 2);
     mp.n_sink = prm.n_sink;
     mp.n_local = prm.n_local;
+    mp.block = prm.block;
     mp.scale_log2 = prm.scale_log2;
     if (!make_map_3d(&mp.tm_q, q, d_qk, n_heads, total_tokens, d_qk, q_row_stride) ||
         !make_map_3d(&mp.tm_k, k, d_qk, 1, total_tokens, d_qk, k_row_stride, 64) ||
         !make_map_3d(&mp.tm_v, v, d_v, 1, total_tokens, v_head_stride, v_row_stride) ||
-        !make_map_3d(&mp.tm_v64, v, d_v, 1, total_tokens, v_head_stride, v_row_stride, 64))
+        !make_map_3d(&mp.tm_v64, v, d_v, 1, total_tokens, v_head_stride, v_row_stride, 64) ||
+        !make_map_tiles4(&mp.tm_k2, k, total_tokens, 9, k_row_stride, 128, 64, 2) ||
+        !make_map_tiles4(&mp.tm_v2[0], static_cast<const uint16_t*>(v) + 256, total_tokens, 2, v_row_stride, 256, 64,
+                         2) ||
+        !make_map_tiles4(&mp.tm_v2[1], static_cast<const uint16_t*>(v) + 320, total_tokens, 2, v_row_stride, 256, 64,
+                         2))
       return LOZA_ERR_CUDA;
     return launch_prefill_mla(mp, workspace, st);
   }
@@ -678,6 +750,7 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
     pp.total_tiles = batch * pp.n_qtiles * n_heads;
     pp.n_sink = prm.n_sink;
     pp.n_local = prm.n_local;
+    pp.block = prm.block;
     pp.scale_log2 = prm.scale_log2;
     if (!make_map_3d(&pp.tm_q, q, d_qk, n_heads, total_tokens, d_qk, q_row_stride) ||
         !make_map_3d(&pp.tm_k, k, d_qk, 1, total_tokens, d_qk, k_row_stride, 64) ||
@@ -692,7 +765,10 @@ loza_status loza_ssa_prefill(const void* q, const void* k, const void* v, const 
 
   switch (dvt) {
     case 64: return launch_prefill<64, 64, 8>(prm, max_seqlen, batch, st);
-    case 128: return launch_prefill_mha2(prm, max_seqlen, batch, st);
+    case 128:
+      // the two-tile kernel's union walk assumes blocks of 128 tokens
+      return p.block_size == kTile ? launch_prefill_mha2(prm, max_seqlen, batch, st)
+                                   : launch_prefill<192, 128, 8>(prm, max_seqlen, batch, st);
     default: return launch_prefill<576, 256, 5>(prm, max_seqlen, batch, st);
   }
 }
@@ -710,7 +786,7 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, c
     if (cu_seqlens[n + 1] < cu_seqlens[n] || cu_seqlens[n + 1] - cu_seqlens[n] > max_seqlen)
       return LOZA_ERR_INVALID_ARG;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
-  if (!window_ok(p) || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v)) return LOZA_ERR_UNSUPPORTED;
+  if (!window_block128(p) || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v)) return LOZA_ERR_UNSUPPORTED;
   const bool latent_v = (v == k);
   if (latent_v && d_v > d_qk) return LOZA_ERR_INVALID_ARG;
   const size_t need = loza_ssa_workspace_size(LOZA_OP_PREFILL_HOST, batch, total_tokens, max_seqlen, n_heads,
@@ -884,6 +960,7 @@ loza_status loza_ssa_decode(const void* q, const void* k_cache, const void* v_ca
   prm.n_kv_heads = n_kv_heads;
   prm.n_sink = n_sink;
   prm.n_local = n_local;
+  prm.block = p.block_size;
   prm.scale_log2 = scale_log2;
   if (cache_batch_stride % d_qk != 0 || cache_row_stride % d_qk != 0) return LOZA_ERR_INVALID_ARG;
   const dim3 grid(n_heads, batch);
@@ -907,7 +984,7 @@ loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const
       max_seqlen > total_tokens)
     return LOZA_ERR_INVALID_ARG;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
-  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (!window_block128(p)) return LOZA_ERR_UNSUPPORTED;
   if (p.n_local == LOZA_UNBOUNDED) return LOZA_ERR_UNSUPPORTED;
   if (n_kv_heads != n_heads || n_heads > 65535 / (p.n_sink > 0 ? p.n_sink : 1)) return LOZA_ERR_UNSUPPORTED;
   const bool d64 = (d_qk == 64 && d_v == 64), d192 = (d_qk == 192 && d_v == 128);

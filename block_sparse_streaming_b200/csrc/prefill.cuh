@@ -51,6 +51,7 @@ struct PrefillParams {
   int dv_slices;       // d_v / DVT
   int n_sink;          // already 0 for the unbounded window
   int n_local;         // < 0: unbounded (full causal)
+  int block;           // b, tokens per block of the window
   float scale_log2;    // scale * log2(e)
 };
 
@@ -85,15 +86,71 @@ struct PrefillLayout {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// Key block visited at step `it` of query block qb (sinks first, diagonal last).
+// The keys query position i sees (LoZA page 1 section 01 (1): the sink
+// blocks and the l most recent blocks of b tokens, token-causal):
+//   A(i) = {t <= i : t < sink_end or t >= lo(i)},  sink_end = s * b,
+//   lo(i) = max(0, (floor(i / b) - l + 1) * b)   (l < 0: unbounded, lo = 0).
+// b = 128, s = 1, l = 7 is the pages' configuration; b = 1 makes every token
+// a block, which is page 4's fixed part of the streaming-aware index (s = 16
+// sink tokens and an l = 1,024-token sliding window).
+struct SsaWindow {
+  int b, sink_end, n_local;
+  __host__ __device__ __forceinline__ int lo(int i) const {
+    return n_local < 0 ? 0 : max(0, (i / b - n_local + 1) * b);
+  }
+};
+
+// Key tiles (kTile = 128 keys) that query tile qb reads, sinks first, then
+// the local tiles in order (the diagonal last), each tile once. A tile needs
+// the per-row mask (visible(i, t) of SsaWindow) if it is the diagonal or if
+// some of its keys are neither sinks for every row nor inside every row's
+// local range; with b = 128 only the diagonal does.
 struct BlockWalk {
   int sinks, local_lo, count;
-  __device__ __forceinline__ BlockWalk(int qb, int n_sink, int n_local) {
-    sinks = min(n_sink, qb + 1);
-    local_lo = n_local < 0 ? sinks : max(n_sink, qb - n_local + 1);
+  int sink_end, lo_last;  // lo() of the tile's last row
+  __host__ __device__ __forceinline__ BlockWalk(int qb, int n_sink, int n_local, int b = kTile) {
+    const SsaWindow w{b, n_sink * b, n_local};
+    sink_end = w.sink_end;
+    sinks = min((sink_end + kTile - 1) / kTile, qb + 1);
+    local_lo = max(sinks, w.lo(qb * kTile) / kTile);
+    lo_last = w.lo(qb * kTile + kTile - 1);
     count = sinks + max(0, qb - local_lo + 1);
   }
-  __device__ __forceinline__ int block(int it) const { return it < sinks ? it : local_lo + (it - sinks); }
+  __host__ __device__ __forceinline__ int block(int it) const { return it < sinks ? it : local_lo + (it - sinks); }
+  __host__ __device__ __forceinline__ bool masked(int kb, int qb) const {
+    return kb == qb || !(kb * kTile + kTile <= sink_end || kb * kTile >= lo_last);
+  }
+};
+
+// Whether key t (relative to the tile start `base`, as j = t - base) is
+// visible from query position i: j <= i - base and (j < sink_end - base or
+// j >= lo(i) - base). The three bounds are per row; the test is per key.
+struct RowMask {
+  int a, e, f;
+  __device__ __forceinline__ RowMask(const SsaWindow& w, int i, int base)
+      : a(i - base), e(w.sink_end - base), f(w.lo(i) - base) {}
+  __device__ __forceinline__ bool visible(int j) const { return j <= a && (j < e || j >= f); }
+  // bit j of the result: visible(j0 + j), for j = 0 .. 63
+  __device__ __forceinline__ uint64_t bits64(int j0) const {
+    auto below = [](int x) -> uint64_t {  // bits j with j < x
+      return x <= 0 ? 0ull : (x >= 64 ? ~0ull : ((1ull << x) - 1ull));
+    };
+    return below(a - j0 + 1) & (below(e - j0) | ~below(f - j0));
+  }
+};
+
+// The units (of `unit` keys) that a single query position i reads, sinks
+// first, then the local range in order, each unit once; each holds at least
+// one visible key. Used by the decode kernels.
+struct RowWalk {
+  int sinks, local_lo, count;
+  __host__ __device__ __forceinline__ RowWalk(const SsaWindow& w, int i, int unit) {
+    const int last = i / unit;
+    sinks = min((w.sink_end + unit - 1) / unit, last + 1);
+    local_lo = max(sinks, w.lo(i) / unit);
+    count = sinks + max(0, last - local_lo + 1);
+  }
+  __host__ __device__ __forceinline__ int unit_at(int it) const { return it < sinks ? it : local_lo + (it - sinks); }
 };
 
 template <int DQK, int DVT, int NSTAGE>
@@ -114,7 +171,8 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
   const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
   if (qb * kTile >= seq_len) return;  // whole CTA leaves before any setup
   const int hk = head / (p.n_heads / p.n_kv_heads);
-  const BlockWalk walk(qb, p.n_sink, p.n_local);
+  const BlockWalk walk(qb, p.n_sink, p.n_local, p.block);
+  const SsaWindow win{p.block, walk.sink_end, p.n_local};
   const int nb = walk.count;
 
   const int warp = threadIdx.x >> 5;
@@ -275,12 +333,15 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
       if (lane == 0) mbar_arrive(bar(LY::BAR_ROW + quarter));
       ok = warp_wait(bar(LY::BAR_ROW + quarter), b & 1, abort_flag);
       if (!ok) break;
-      // the diagonal block is token-causal: keys after this row's query do not exist
-      if (walk.block(b) == qb) {
+      // keys this row does not see: after its query (the diagonal tile), or
+      // between the sinks and its local range (tiles at the window's edges)
+      if (walk.masked(walk.block(b), qb)) {
+        const RowMask rm(win, qpos, walk.block(b) * kTile);
+        const uint64_t vo = rm.bits64(64 * (half ^ 1)), vs = rm.bits64(64 * half);
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          if (64 * (half ^ 1) + j > row) so[j] = -INFINITY;
-          if (64 * half + j > row) s[j] = -INFINITY;
+          if (!((vo >> j) & 1ull)) so[j] = -INFINITY;
+          if (!((vs >> j) & 1ull)) s[j] = -INFINITY;
         }
       }
       float mx;
@@ -301,7 +362,9 @@ ssa_prefill_kernel(const __grid_constant__ PrefillParams p) {
         m_run = mx;
       }
       const float2 c2 = make_float2(c, c);
-      const float2 nm2 = make_float2(-m_run, -m_run);
+      // a row that has seen no key yet (all masked so far) takes P = 0
+      const float nm = m_run == -INFINITY ? 0.f : -m_run;
+      const float2 nm2 = make_float2(nm, nm);
       float2 l2[4], r2[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) l2[i] = r2[i] = make_float2(0.f, 0.f);

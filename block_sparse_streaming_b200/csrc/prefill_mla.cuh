@@ -38,6 +38,9 @@ struct PrefillMlaParams {
   CUtensorMap tm_v;    // value [T, 1, 512]          box {64, 1, 128}
   CUtensorMap tm_v64;  // value [T, 1, 512]          box {64, 1, 64}
   CUtensorMap tm_p;    // P scratch as lines of 64 bf16  box {64, 128}, unswizzled
+  // 4-D views {64 columns, rows, column tile, 1}: two [64 x 64] tiles per request
+  CUtensorMap tm_k2;   // latent, tiles of 64 columns (stride 128 B), box {64, 64, 2, 1}
+  CUtensorMap tm_v2[2];  // value columns 256 + 64r + 128m (m = 0, 1; r = CTA rank), box {64, 64, 2, 1}
   const int32_t* cu_seqlens;
   __nv_bfloat16* out;  // [T, H, 512]
   float* lse;          // [T, H]
@@ -49,6 +52,7 @@ struct PrefillMlaParams {
   int total_tiles;     // batch * n_qtiles * n_heads / 2
   int n_sink;
   int n_local;
+  int block;           // b, tokens per block of the window
   float scale_log2;
 };
 
@@ -159,6 +163,8 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       tma_prefetch_desc(&p.tm_v);
       tma_prefetch_desc(&p.tm_v64);
       tma_prefetch_desc(&p.tm_p);
+      tma_prefetch_desc(&p.tm_k2);
+      tma_prefetch_desc(&p.tm_v2[rank]);
     }
     __syncwarp();
     int slot = 0;
@@ -193,7 +199,7 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
     int t = next_tile(pair, tl);
     if (t < p.total_tiles) load_q(tl);
     while (t < p.total_tiles && ok) {
-      const BlockWalk walk(tl.qb, p.n_sink, p.n_local);
+      const BlockWalk walk(tl.qb, p.n_sink, p.n_local, p.block);
       const int nb = walk.count;
       // pass 1: K halves of every block, value columns [0, 256)
       for (int it = 0; it <= nb && ok; ++it) {
@@ -202,10 +208,13 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
           for (int k = 0; k < 5 && ok; ++k) {
             if (!acquire(mla_k_slot_bytes(k))) break;
             if (elect_one()) {
+              // column tiles 2k and 2k+1 in one request (a TMA request has a
+              // fixed cost); the rope tile 8 alone
               const uint32_t dst = sbase + LY::RING_OFF + slot * kChunkBytes;
-              tma_load_3d_pair(dst, &p.tm_k, lead_bar(LY::BAR_FULL + slot), 128 * k, 0, krow);
               if (2 * k + 1 < 9)
-                tma_load_3d_pair(dst + kMlaHalfK, &p.tm_k, lead_bar(LY::BAR_FULL + slot), 128 * k + 64, 0, krow);
+                tma_load_4d_pair(dst, &p.tm_k2, lead_bar(LY::BAR_FULL + slot), 0, krow, 2 * k, 0);
+              else
+                tma_load_3d_pair(dst, &p.tm_k, lead_bar(LY::BAR_FULL + slot), 128 * k, 0, krow);
             }
             __syncwarp();
             advance();
@@ -248,12 +257,9 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
           __syncwarp();
           advance();
           if (!acquire(kChunkBytes)) break;
-          if (elect_one()) {
-            const uint32_t dst = sbase + LY::RING_OFF + slot * kChunkBytes;
-            for (int m = 0; m < 2; ++m)
-              tma_load_3d_pair(dst + m * kMlaHalfK, &p.tm_v64, lead_bar(LY::BAR_FULL + slot),
-                               256 + 128 * m + 64 * (int)rank, 0, vrow + 64 * kh);
-          }
+          if (elect_one())  // this CTA's columns of both 128-column groups, one request
+            tma_load_4d_pair(sbase + LY::RING_OFF + slot * kChunkBytes, &p.tm_v2[rank], lead_bar(LY::BAR_FULL + slot),
+                             0, vrow + 64 * kh, 0, 0);
           __syncwarp();
           advance();
         }
@@ -293,7 +299,7 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
       };
       for (int t = pair; t < p.total_tiles && ok; t += npairs) {
         if (!tl.load(p, t)) continue;
-        const int nb = BlockWalk(tl.qb, p.n_sink, p.n_local).count;
+        const int nb = BlockWalk(tl.qb, p.n_sink, p.n_local, p.block).count;
         const uint32_t ra = (uint32_t)(ntile & 1) * 256;
         const uint32_t tmem_o1 = tmem + (256 - ra);
         const uint32_t tmem_o2 = tmem + ra;
@@ -481,7 +487,7 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
     };
     for (int t = pair; t < p.total_tiles && ok; t += npairs) {
       if (!tl.load(p, t)) continue;
-      const BlockWalk walk(tl.qb, p.n_sink, p.n_local);
+      const BlockWalk walk(tl.qb, p.n_sink, p.n_local, p.block);
       const int nb = walk.count;
       const int head = 2 * tl.hp + (int)rank;
       // m_run: running row maximum of scale*log2(e)*s (the reference of P);
@@ -511,11 +517,16 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
         ok = warp_wait(bar(LY::BAR_ROW + quarter), n_row & 1, abort_flag);
         ++n_row;
         if (!ok) break;
-        if (walk.block(b) == tl.qb) {  // token-causal inside the diagonal block
+        if (walk.masked(walk.block(b), tl.qb)) {
+          // keys this row does not see: after its query (the diagonal tile), or
+          // between the sinks and its local range (tiles at the window's edges)
+          const SsaWindow win{p.block, walk.sink_end, p.n_local};
+          const RowMask rm(win, tl.qb * kTile + row, walk.block(b) * kTile);
+          const uint64_t vo = rm.bits64(64 * (half ^ 1)), vs = rm.bits64(64 * half);
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            if (64 * (half ^ 1) + j > row) so[j] = -INFINITY;
-            if (64 * half + j > row) s[j] = -INFINITY;
+            if (!((vo >> j) & 1ull)) so[j] = -INFINITY;
+            if (!((vs >> j) & 1ull)) s[j] = -INFINITY;
           }
         }
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -533,7 +544,9 @@ ssa_prefill_mla_kernel(const __grid_constant__ PrefillMlaParams p) {
           m_run = mx;
         }
         const float2 c2 = make_float2(c, c);
-        const float2 nm2 = make_float2(-m_run, -m_run);
+        // a row that has seen no key yet (all masked so far) takes P = 0
+        const float nm = m_run == -INFINITY ? 0.f : -m_run;
+        const float2 nm2 = make_float2(nm, nm);
         float2 l2[4], r2[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) l2[i] = r2[i] = make_float2(0.f, 0.f);

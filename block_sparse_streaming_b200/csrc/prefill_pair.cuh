@@ -59,6 +59,7 @@ struct PrefillPairParams {
   int total_tiles;     // batch * n_qtiles * n_heads (head pairs x 2 value slices)
   int n_sink;
   int n_local;         // < 0: unbounded
+  int block;           // b, tokens per block of the window
   float scale_log2;
 };
 
@@ -191,7 +192,7 @@ ssa_prefill_pair_kernel(const __grid_constant__ PrefillPairParams p) {
     PairTile tl;
     for (int t = pair; t < p.total_tiles && ok; t += npairs) {
       if (!tl.load(p, t)) continue;
-      const BlockWalk walk(tl.qb, p.n_sink, p.n_local);
+      const BlockWalk walk(tl.qb, p.n_sink, p.n_local, p.block);
       const int nb = walk.count;
       const int head = 2 * tl.hp + (int)rank;
       // Q of this tile once the previous tile's last S MMA has read Q
@@ -250,7 +251,7 @@ ssa_prefill_pair_kernel(const __grid_constant__ PrefillPairParams p) {
       PairTile tl;
       for (int t = pair; t < p.total_tiles && ok; t += npairs) {
         if (!tl.load(p, t)) continue;
-        const int nb = BlockWalk(tl.qb, p.n_sink, p.n_local).count;
+        const int nb = BlockWalk(tl.qb, p.n_sink, p.n_local, p.block).count;
         ok = warp_wait(bar(LY::BAR_Q), ntile & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
@@ -334,7 +335,7 @@ ssa_prefill_pair_kernel(const __grid_constant__ PrefillPairParams p) {
     PairTile tl;
     for (int t = pair; t < p.total_tiles && ok; t += npairs) {
       if (!tl.load(p, t)) continue;
-      const BlockWalk walk(tl.qb, p.n_sink, p.n_local);
+      const BlockWalk walk(tl.qb, p.n_sink, p.n_local, p.block);
       const int nb = walk.count;
       // m_run: running row maximum of scale*log2(e)*s (the reference of P);
       // l_run: this warp's share of the running sum of 2^(x - m_run) (exact,
@@ -353,11 +354,16 @@ ssa_prefill_pair_kernel(const __grid_constant__ PrefillPairParams p) {
         // keys of both warps of the row: neither warp may store P before its
         // partner has loaded all of S.
         named_barrier_sync(2 + quarter, 64);
-        if (walk.block(b) == tl.qb) {  // token-causal: keys after this row's query do not exist
+        if (walk.masked(walk.block(b), tl.qb)) {
+          // keys this row does not see: after its query (the diagonal tile), or
+          // between the sinks and its local range (tiles at the window's edges)
+          const SsaWindow win{p.block, walk.sink_end, p.n_local};
+          const RowMask rm(win, tl.qb * kTile + row, walk.block(b) * kTile);
+          const uint64_t vo = rm.bits64(64 * (half ^ 1)), vs = rm.bits64(64 * half);
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            if (64 * (half ^ 1) + j > row) so[j] = -INFINITY;
-            if (64 * half + j > row) s[j] = -INFINITY;
+            if (!((vo >> j) & 1ull)) so[j] = -INFINITY;
+            if (!((vs >> j) & 1ull)) s[j] = -INFINITY;
           }
         }
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -375,7 +381,9 @@ ssa_prefill_pair_kernel(const __grid_constant__ PrefillPairParams p) {
           m_run = mx;
         }
         const float2 c2 = make_float2(c, c);
-        const float2 nm2 = make_float2(-m_run, -m_run);
+        // a row that has seen no key yet (all masked so far) takes P = 0
+        const float nm = m_run == -INFINITY ? 0.f : -m_run;
+        const float2 nm2 = make_float2(nm, nm);
         float2 l2[4], r2[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) l2[i] = r2[i] = make_float2(0.f, 0.f);

@@ -316,6 +316,17 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* desc,
       : "memory");
 }
 
+// 4-D box load (see tma_load_4d) whose bytes are counted on an mbarrier of
+// either CTA of the pair.
+__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const void* desc, uint32_t bar, int32_t c0, int32_t c1,
+                                                 int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* desc, uint32_t bar, int32_t c0,
                                                  int32_t c1) {
   asm volatile(

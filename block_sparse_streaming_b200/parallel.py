@@ -122,6 +122,12 @@ def local_queries(q_own, plan: ShardPlan):
     return torch.cat([pre, q_own], dim=0)
 
 
+def _require_block128(params):
+    """The shard plan moves whole blocks of 128 tokens (the pages' b)."""
+    if params.block_size != BLOCK:
+        raise ValueError(f"sharding needs block_size {BLOCK}, got {params.block_size}")
+
+
 def own_outputs(out_local, lse_local, plan: ShardPlan):
     """The rows of the own blocks in the local outputs."""
     off = plan.n_pre * BLOCK
@@ -135,6 +141,7 @@ def prefill_sharded(q_own, k_own, v_own, params, plan: ShardPlan, group=None, la
     Returns (out, lse) of the own rows."""
     import torch
     from . import loza_ssa_prefill
+    _require_block128(params)
     k_loc = exchange_kv(k_own, plan, params.n_sink, params.n_local, group)
     if latent_v:
         v_loc = k_loc[..., : v_own.shape[-1]]
@@ -224,6 +231,7 @@ def backward_sharded(q_own, k_own, v_own, out_own, dout_own, lse_own, params, pl
     Returns (dq, dk, dv) of the own rows."""
     import torch
     from . import loza_ssa_backward
+    _require_block128(params)
     k_loc = exchange_kv(k_own, plan, params.n_sink, params.n_local, group).contiguous()
     v_loc = exchange_kv(v_own, plan, params.n_sink, params.n_local, group).contiguous()
     q_loc = local_rows(q_own, plan).contiguous()

@@ -38,8 +38,21 @@
  *     heads are contiguous with head stride = head dim.
  *   - Every row stride times 2 bytes and every base pointer must be 16-byte
  *     aligned (TMA requirement); otherwise LOZA_ERR_INVALID_ARG.
- *   - Only block_size == 128 is compiled; n_sink >= 0, n_local >= 1, or
- *     n_local == LOZA_UNBOUNDED for full causal attention (n_sink ignored).
+ *   - Window: block_size b a power of two from 1 to 65,536; n_sink >= 0,
+ *     n_local >= 1 (n_sink * b and n_local * b at most 2^30), or n_local ==
+ *     LOZA_UNBOUNDED for full causal attention (n_sink ignored). The keys of
+ *     query position i are then {t <= i : t < n_sink * b or t >= lo(i)}, lo(i)
+ *     = max(0, (floor(i / b) - n_local + 1) * b). b = 1 makes every token a
+ *     block: {1, 16, 1024} is the fixed part of the streaming-aware index of
+ *     page 4 ("LongCat Sparse Attention ...", agihunt.info), 16 sink tokens
+ *     and a 1,024-token sliding window that includes the query. The prefill
+ *     and decode entry points take any such window; loza_ssa_backward,
+ *     loza_ssa_prefill_host and the sharded prefill need b = 128
+ *     (LOZA_ERR_UNSUPPORTED otherwise). Keys are read in tiles of 128 (64 in
+ *     the half-block decode): the cache rows of positions below seqlens[n]
+ *     that share a tile with a visible key are read and must hold finite
+ *     values (they are the sequence's own context); rows at or past
+ *     seqlens[n] never reach the result, whatever they hold.
  */
 #ifndef LOZA_SSA_H
 #define LOZA_SSA_H
@@ -55,7 +68,8 @@ extern "C" {
 typedef struct CUstream_st *loza_stream_t;
 
 /* Window parameters {b, s, l, scale}; the pages' configuration is
- * {128, 1, 7, scale}. scale multiplies q.k before the softmax. */
+ * {128, 1, 7, scale}; {1, 16, 1024, scale} is page 4's token-granular sink
+ * and sliding window. scale multiplies q.k before the softmax. */
 typedef struct {
     int32_t block_size;
     int32_t n_sink;
@@ -267,7 +281,7 @@ loza_status loza_ssa_backward(const void *q, const void *k, const void *v, const
 
 /*
  * Absorbed decode (n_kv_heads 1, d_qk 576, d_v 512, n_heads 64) from a paged
- * latent cache: the pool holds num_pages pages of 128 rows (one SSA block
+ * latent cache: the pool holds num_pages pages of 128 rows (one 128-row tile
  * each), row r of page g at kv_pool + (g * 128 + r) * pool_row_stride
  * elements; logical block kb of sequence n (rows 128kb .. 128kb+127 of its
  * context) is page block_table[n * bt_stride + kb]. Every block the window

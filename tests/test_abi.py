@@ -63,7 +63,10 @@ def _call_prefill(L, a):
     (dict(batch=0), -1),
     (dict(max_seqlen=300), -1),            # longer than the packed batch
     (dict(dqk=96, dv=96, qs=384, ks=384, vs=384), -2),    # head dims not compiled
-    (dict(params=bss.Params(0.1, block_size=64)), -2),    # only b = 128
+    (dict(params=bss.Params(0.1, block_size=96)), -2),    # b must be a power of two
+    (dict(params=bss.Params(0.1, block_size=0)), -2),
+    (dict(params=bss.Params(0.1, block_size=1 << 17)), -2),  # at most 65,536
+    (dict(params=bss.Params(0.1, block_size=1 << 16, n_local=1 << 15)), -2),  # window beyond 2^30 keys
     (dict(params=bss.Params(0.1, n_local=0)), -2),
     (dict(H=4, Hkv=2, ks=128, vs=128), -2),              # grouped heads not compiled
 ])
@@ -141,6 +144,7 @@ def _call_prefill_host(L, q=1 << 20, k=1 << 21, v=1 << 22, cu=(0, 4096), batch=N
     (dict(dqk=96, dv=96), -2),                        # head dims not compiled
     (dict(dqk=576, dv=512, H=3, Hkv=1), -2),          # absorbed needs an even head count
     (dict(params=bss.Params(0.1, n_local=0)), -2),    # empty local window
+    (dict(params=bss.Params(0.1, 64, 2, 14)), -2),    # chunks move whole blocks of 128 tokens
     (dict(ws=0), -1),                                 # no workspace
     (dict(ws=(1 << 28) + 16), -1),                    # workspace not 256-byte aligned
     (dict(ws_bytes=1024), -3),                        # workspace too small
@@ -191,4 +195,19 @@ def test_prefill_host_binding_rejects_before_any_device_work(L):
     with pytest.raises(bss.LozaError) as e:  # the whole 576-wide latent as V: no such head dims
         bss.loza_ssa_prefill_host(q, lat, lat, p)
     assert e.value.status == -2
+    assert L.loza_launch_count() == count
+
+
+def test_backward_needs_blocks_of_128(L):
+    """The backward works in blocks of 128 tokens: another block size is
+    refused (LOZA_ERR_UNSUPPORTED) before anything runs, and the workspace
+    query reports 0 for it."""
+    vp = ctypes.c_void_p
+    count = L.loza_launch_count()
+    for params in (bss.Params(0.125, 64, 2, 14), bss.Params(0.125, 1, 16, 1024)):
+        rc = L.loza_ssa_backward(vp(1 << 20), vp(1 << 21), vp(1 << 22), vp(1 << 23), vp(1 << 24), vp(1 << 25),
+                                 vp(1 << 26), 1, 256, 256, 4, 4, 64, 64, params, vp(1 << 27), vp(1 << 28),
+                                 vp(1 << 29), vp(1 << 30), 1 << 30, vp(0))
+        assert rc == -2
+        assert bss.workspace_size(bss.LOZA_OP_BACKWARD, 1, 256, 256, 4, 4, 64, 64, params) == 0
     assert L.loza_launch_count() == count

@@ -108,3 +108,20 @@ def test_rejects_bad_windows(oracle_mod):
         oracle_mod.forward_tokens(q, k, v, cu, 1, 1, 0, 0, 1.0)
     with pytest.raises(ValueError):
         oracle_mod.forward_tokens(q, k, v, cu, 1, 1, -1, 4, 1.0)
+
+
+@pytest.mark.parametrize("sink,window", [(16, 1024), (0, 300), (5, 1)])
+def test_token_window_is_the_block_window_with_single_token_blocks(oracle_mod, sink, window):
+    """With blocks of one token, s sink blocks and l local blocks select the
+    tokens t < s and i - l < t <= i: the token window of S = s sink tokens and a
+    W = l token sliding window. The block oracle (b = 1) and the token oracle
+    list their keys by different routines; they must agree on every row of a
+    packed batch."""
+    lens = [2500, 1, 700]
+    T, H = sum(lens), 2
+    q, k, v = draw(510 + window, T, H, H, 16, 16)
+    cu = synth.cu_seqlens(lens)
+    o_t, l_t = oracle_mod.forward_tokens(q, k, v, cu, H, H, sink, window, 0.25)
+    o_b, l_b = oracle_mod.forward(q, k, v, cu, H, H, 1, sink, window, 0.25)
+    np.testing.assert_allclose(o_t, o_b, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l_t, l_b, rtol=0, atol=1e-12)
