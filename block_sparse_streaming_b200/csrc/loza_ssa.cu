@@ -158,11 +158,12 @@ DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t bat
   if (count <= 16 && (int64_t)batch * 2 <= sms) {
     // half blocks: up to 4 CTAs per sequence in one cluster, each pulling
     // its share of the rows once
+    // (the on-chip merge splits the 512 value columns evenly: nsplit is 1, 2
+    // or 4, and a split may get no half block)
     const int nh = max_row_units(p, max_seqlen, kHbRows);
     int ns = 1;
     while (ns < kHbMaxSplit && ns * 2 <= nh && (int64_t)batch * ns * 2 <= sms) ns *= 2;
-    const int hps = (nh + ns - 1) / ns;
-    return {hps, (nh + hps - 1) / hps, true, true};
+    return {(nh + ns - 1) / ns, ns, true, true};
   }
   int ns = 1;
   while (ns < 4 && ns * 2 <= count && (int64_t)batch * ns * 2 <= sms) ns *= 2;
@@ -280,8 +281,8 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
 loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t batch, uint8_t* ws,
                               cudaStream_t st) {
   if (plan.half_block) {
-    // the kernel's merge buffers hold at most kHbMaxSplit splits
-    if (plan.nsplit < 1 || plan.nsplit > kHbMaxSplit) return LOZA_ERR_UNSUPPORTED;
+    // the kernel's merge gives each split 512 / nsplit whole value columns
+    if (plan.nsplit != 1 && plan.nsplit != 2 && plan.nsplit != 4) return LOZA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(ssa_decode_mla_hb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DecodeHbLayout::SMEM_BYTES) != cudaSuccess)
       return LOZA_ERR_CUDA;
@@ -310,8 +311,8 @@ loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t
       return LOZA_ERR_CUDA;
     ssa_decode_mla_kernel<false><<<dim3(plan.nsplit, batch), kDecThreads, DecodeLayout::SMEM_BYTES, st>>>(prm);
   } else {
-    // the cluster merge handles at most 4 splits
-    if (plan.nsplit < 1 || plan.nsplit > 4) return LOZA_ERR_UNSUPPORTED;
+    // the cluster merge gives each split 512 / nsplit whole value columns
+    if (plan.nsplit != 1 && plan.nsplit != 2 && plan.nsplit != 4) return LOZA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(ssa_decode_mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DecodeLayout::SMEM_BYTES) != cudaSuccess)
       return LOZA_ERR_CUDA;
