@@ -25,6 +25,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ssa_ref.c")
+_SRC_HI = os.path.join(_HERE, "hi_ref.c")
 _LIB_PATH = os.path.join(_HERE, "libssa_oracle.so")
 _lib = None
 
@@ -37,11 +38,11 @@ _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 def build(force: bool = False) -> str:
     """Compile ssa_ref.c into libssa_oracle.so next to it (gcc -O2 -fopenmp)."""
     if (not force and os.path.exists(_LIB_PATH)
-            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+            and os.path.getmtime(_LIB_PATH) >= max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_HI))):
         return _LIB_PATH
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
-                    "-o", tmp, _SRC, "-lm"], check=True)
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99", "-ffp-contract=off",
+                    "-o", tmp, _SRC, _SRC_HI, "-lm"], check=True)
     os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -79,6 +80,18 @@ def _load():
         lib.ssa_oracle_merge.argtypes = [_u16p, _f64p, _u16p, _f64p, ctypes.c_int64, ctypes.c_int, _f64p, _f64p]
         lib.ssa_oracle_mix.restype = ctypes.c_int
         lib.ssa_oracle_mix.argtypes = [_u16p, _u16p, ctypes.c_int64, ctypes.c_double, _f64p]
+        _f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+        lib.hi_oracle_page_keys.restype = ctypes.c_int
+        lib.hi_oracle_page_keys.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, _i32p, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int64, _f32p]
+        lib.hi_oracle_select.restype = ctypes.c_int
+        lib.hi_oracle_select.argtypes = [_u16p, _u16p, ctypes.c_int64, ctypes.c_int64, _f32p, ctypes.c_int64, _i32p,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, _i32p]
+        lib.hi_oracle_decode.restype = ctypes.c_int
+        lib.hi_oracle_decode.argtypes = [_u16p, _u16p, ctypes.c_int64, ctypes.c_int64, _i32p, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_double, _i32p, ctypes.c_int, _f64p, _f64p]
         lib.ssa_oracle_visible_count.restype = ctypes.c_int64
         lib.ssa_oracle_visible_count.argtypes = [
             ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
@@ -213,3 +226,56 @@ def mix(o_full, o_ssa, alpha):
     if _load().ssa_oracle_mix(a.reshape(-1), b.reshape(-1), a.size, float(alpha), o.reshape(-1)) != 0:
         raise ValueError("oracle mix rejected its arguments")
     return o
+
+
+# ---------------------------------------------------------------------------
+# Hierarchical index (page 4: pages of 128 tokens, top pages, then top tokens)
+# ---------------------------------------------------------------------------
+HI_PAGE = 128
+
+
+def hi_page_keys(k_index, seqlens):
+    """Mean index key of every whole 128-token page: k_index [B, Lcap, d] bf16
+    bits -> float32 [B, Lcap // 128, d] (pages past a sequence's end are 0)."""
+    k = _u16(k_index)
+    B, Lcap, d = k.shape
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    pages = Lcap // HI_PAGE
+    out = np.zeros((B, pages, d), np.float32)
+    if _load().hi_oracle_page_keys(k, Lcap * d, d, sl, B, d, pages, out) != 0:
+        raise ValueError("oracle page keys rejected its arguments")
+    return out
+
+
+def hi_select(q_index, k_index, page_keys, seqlens, block_size, n_sink, n_local, top_pages, top_k):
+    """Tokens chosen by the hierarchical index for each sequence's decode query:
+    int32 [B, top_k], ascending, unused entries -1. q_index [B, d]; k_index
+    [B, Lcap, d] bf16 bits; page_keys from hi_page_keys."""
+    q, k = _u16(q_index), _u16(k_index)
+    B, Lcap, d = k.shape
+    pk = np.ascontiguousarray(page_keys, dtype=np.float32)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    out = np.full((B, max(top_k, 1)), -1, np.int32)
+    if _load().hi_oracle_select(q, k, Lcap * d, d, pk, pk.shape[1], sl, B, d, block_size, n_sink, n_local,
+                                top_pages, top_k, out) != 0:
+        raise ValueError("oracle select rejected its arguments")
+    return out[:, :top_k]
+
+
+def hi_decode(q, kv_cache, seqlens, n_heads, block_size, n_sink, n_local, scale, selected, d_v=512):
+    """O [B, H, d_v], LSE [B, H] (float64) of each decode query over its fixed
+    window and its selected tokens; kv_cache [B, Lcap, 1, d_qk] latent bits."""
+    q, kv = _u16(q), _u16(kv_cache)
+    B = q.shape[0]
+    d_qk = q.shape[-1]
+    Lcap = kv.shape[1]
+    sel = np.ascontiguousarray(selected, dtype=np.int32).reshape(B, -1)
+    top_k = sel.shape[1]
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    o = np.zeros((B, n_heads, d_v), np.float64)
+    lse = np.zeros((B, n_heads), np.float64)
+    if _load().hi_oracle_decode(q, kv, Lcap * kv.shape[-1], kv.shape[-1], sl, B, n_heads, d_qk, d_v, block_size,
+                                n_sink, n_local, float(scale), sel if top_k else np.zeros((B, 1), np.int32),
+                                top_k, o, lse) != 0:
+        raise ValueError("oracle HI decode rejected its arguments")
+    return o, lse
