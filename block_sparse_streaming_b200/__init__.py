@@ -43,6 +43,11 @@ EXPORTED = [
     "loza_status_string",
     "loza_device_status",
     "loza_launch_count",
+    "loza_hi_page_keys",
+    "loza_hi_workspace_size",
+    "loza_hi_select",
+    "loza_ssa_decode_selected",
+    "loza_hi_decode",
 ]
 
 
@@ -103,6 +108,19 @@ def lib() -> ctypes.CDLL:
         L.loza_device_status.argtypes = [_vp]
         L.loza_launch_count.restype = ctypes.c_uint64
         L.loza_launch_count.argtypes = []
+        L.loza_hi_page_keys.restype = ctypes.c_int
+        L.loza_hi_page_keys.argtypes = [_vp, _i64, _i64, _vp, _i32, _i32, _i32, _vp, _vp]
+        L.loza_hi_workspace_size.restype = _sz
+        L.loza_hi_workspace_size.argtypes = [_i32, _i32, _i32, _i32, Params]
+        L.loza_hi_select.restype = ctypes.c_int
+        L.loza_hi_select.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _i32, _i32, _i32, Params, _i32, _i32, _vp, _vp,
+                                     _sz, _vp]
+        L.loza_ssa_decode_selected.restype = ctypes.c_int
+        L.loza_ssa_decode_selected.argtypes = [_vp, _vp, _i64, _i64, _vp, _i32, _i32, _i32, ctypes.c_float, _vp,
+                                               _vp, _vp]
+        L.loza_hi_decode.restype = ctypes.c_int
+        L.loza_hi_decode.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _i32, _i32, Params,
+                                     _i32, _i32, _vp, _vp, _vp, _sz, _vp]
         _lib = L
     return _lib
 
@@ -376,4 +394,117 @@ def loza_ssa_decode_paged(q, kv_pool, block_table, seqlens, max_seqlen: int, par
                                      block_table.shape[1], _ptr(seqlens), B, int(max_seqlen), H, params, _ptr(out),
                                      _ptr(lse), _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check(rc, "loza_ssa_decode_paged")
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Hierarchical index decode (page 4's streaming-aware and hierarchical index)
+# ---------------------------------------------------------------------------
+def _contiguous(t, name):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _latent_cache(kv_cache):
+    import torch
+    _require(kv_cache, "kv_cache", torch.bfloat16, 4)
+    if kv_cache.shape[2] != 1 or kv_cache.shape[3] < 576 or kv_cache.stride(3) != 1:
+        raise ValueError("kv_cache must be [batch, rows, 1, 576] with contiguous latent rows")
+
+
+def _index_keys(k_index):
+    import torch
+    _require(k_index, "k_index", torch.bfloat16, 3)
+    if k_index.stride(2) != 1:
+        raise ValueError("k_index: the index dimension must be contiguous")
+    return k_index.shape[2], k_index.stride(0), k_index.stride(1)
+
+
+def loza_hi_page_keys(k_index, seqlens, max_seqlen: int, page_keys=None, stream=None):
+    """Mean index key of every whole 128-token page: k_index [B, Lcap, d] bf16 ->
+    page_keys [B, max_seqlen // 128, d] float32."""
+    import torch
+    d, bs, rs = _index_keys(k_index)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B = k_index.shape[0]
+    if page_keys is None:
+        page_keys = torch.zeros((B, int(max_seqlen) // 128, d), dtype=torch.float32, device=k_index.device)
+    rc = lib().loza_hi_page_keys(_ptr(k_index), bs, rs, _ptr(seqlens), B, int(max_seqlen), d, _ptr(page_keys),
+                                 _stream_ptr(stream))
+    _check(rc, "loza_hi_page_keys")
+    return page_keys
+
+
+def hi_workspace_size(batch, max_seqlen, top_pages, top_k, params: Params) -> int:
+    return int(lib().loza_hi_workspace_size(batch, max_seqlen, top_pages, top_k, params))
+
+
+def loza_hi_select(q_index, k_index, page_keys, seqlens, max_seqlen: int, params: Params, top_pages: int, top_k: int,
+                   selected=None, workspace=None, stream=None):
+    """Tokens the hierarchical index selects: int32 [B, top_k], ascending, -1 padded."""
+    import torch
+    d, bs, rs = _index_keys(k_index)
+    _require(q_index, "q_index", torch.bfloat16, 2)
+    _require(page_keys, "page_keys", torch.float32, 3)
+    _contiguous(q_index, "q_index")
+    _contiguous(page_keys, "page_keys")
+    B = k_index.shape[0]
+    if selected is None:
+        selected = torch.empty((B, top_k), dtype=torch.int32, device=k_index.device)
+    if workspace is None:
+        workspace = torch.empty(max(16, hi_workspace_size(B, int(max_seqlen), top_pages, top_k, params)),
+                                dtype=torch.uint8, device=k_index.device)
+    rc = lib().loza_hi_select(_ptr(q_index), _ptr(k_index), bs, rs, _ptr(page_keys), _ptr(seqlens), B,
+                              int(max_seqlen), d, params, top_pages, top_k, _ptr(selected), _ptr(workspace),
+                              workspace.numel(), _stream_ptr(stream))
+    _check(rc, "loza_hi_select")
+    return selected
+
+
+def loza_ssa_decode_selected(q, kv_cache, selected, scale: float, out=None, lse=None, stream=None):
+    """Attention of each decode query over its selected tokens (absorbed latent
+    cache [B, Lcap, 1, 576]); returns (out [B, 64, 512], lse [B, 64])."""
+    import torch
+    _require(q, "q", torch.bfloat16, 3)
+    _latent_cache(kv_cache)
+    _require(selected, "selected", torch.int32, 2)
+    _contiguous(q, "q")
+    _contiguous(selected, "selected")
+    B, H, _ = q.shape
+    if out is None:
+        out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    rc = lib().loza_ssa_decode_selected(_ptr(q), _ptr(kv_cache), kv_cache.stride(0), kv_cache.stride(1),
+                                        _ptr(selected), selected.shape[1], B, H, float(scale), _ptr(out), _ptr(lse),
+                                        _stream_ptr(stream))
+    _check(rc, "loza_ssa_decode_selected")
+    return out, lse
+
+
+def loza_hi_decode(q, kv_cache, q_index, k_index, page_keys, seqlens, max_seqlen: int, params: Params,
+                   top_pages: int, top_k: int, out=None, lse=None, workspace=None, stream=None):
+    """Decode over the window `params` and the tokens the hierarchical index
+    selects, merged; returns (out [B, 64, 512], lse [B, 64])."""
+    import torch
+    _require(q, "q", torch.bfloat16, 3)
+    _latent_cache(kv_cache)
+    d, bs, rs = _index_keys(k_index)
+    _require(q_index, "q_index", torch.bfloat16, 2)
+    _require(page_keys, "page_keys", torch.float32, 3)
+    for t, name in ((q, "q"), (q_index, "q_index"), (page_keys, "page_keys")):
+        _contiguous(t, name)
+    B, H, _ = q.shape
+    if out is None:
+        out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(16, hi_workspace_size(B, int(max_seqlen), top_pages, top_k, params)),
+                                dtype=torch.uint8, device=q.device)
+    rc = lib().loza_hi_decode(_ptr(q), _ptr(kv_cache), kv_cache.stride(0), kv_cache.stride(1), _ptr(q_index),
+                              _ptr(k_index), bs, rs, _ptr(page_keys), _ptr(seqlens), B, int(max_seqlen), d, params,
+                              top_pages, top_k, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                              _stream_ptr(stream))
+    _check(rc, "loza_hi_decode")
     return out, lse

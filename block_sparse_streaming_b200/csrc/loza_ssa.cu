@@ -21,6 +21,7 @@
 #include "decode_mla_hb.cuh"
 #include "merge.cuh"
 #include "backward.cuh"
+#include "hi_index.cuh"
 
 namespace loza {
 namespace {
@@ -526,6 +527,43 @@ unsigned stream_grid(int64_t n) {
   return (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + per - 1) / per, cap));
 }
 
+// Hierarchical index (page 4): workspace of loza_hi_select / loza_hi_decode.
+struct HiWorkspace {
+  size_t sel_pages, n_pages, tok_keys, selected, o_sel, l_sel, o_win, l_win, dec, total;
+};
+size_t hi_align(size_t x) { return (x + 255) / 256 * 256; }
+HiWorkspace hi_workspace(int32_t batch, int32_t top_pages, int32_t top_k, size_t decode_ws) {
+  HiWorkspace w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = hi_align(off + bytes);
+    return at;
+  };
+  w.sel_pages = take((size_t)batch * top_pages * 4);
+  w.n_pages = take((size_t)batch * 4);
+  w.tok_keys = take((size_t)batch * top_pages * kHiPage * 8);
+  w.selected = take((size_t)batch * std::max(top_k, 1) * 4);
+  w.o_sel = take((size_t)batch * kDecHeads * 512 * 2);
+  w.l_sel = take((size_t)batch * kDecHeads * 4);
+  w.o_win = take((size_t)batch * kDecHeads * 512 * 2);
+  w.l_win = take((size_t)batch * kDecHeads * 4);
+  w.dec = take(decode_ws);
+  w.total = off;
+  return w;
+}
+
+bool hi_args_ok(const void* k_index, int64_t index_batch_stride, int64_t index_row_stride, int32_t batch,
+                int32_t max_seqlen, int32_t d_index) {
+  if (!k_index || !aligned16(k_index)) return false;
+  if (batch < 1 || batch > 65535 || max_seqlen < 1) return false;
+  if (d_index < 8 || d_index > kHiMaxDim || d_index % 8 != 0) return false;
+  if (!stride_ok(index_row_stride) || !stride_ok(index_batch_stride) || index_row_stride < d_index ||
+      index_batch_stride < (int64_t)max_seqlen * index_row_stride)
+    return false;
+  return true;
+}
+
 }  // namespace
 }  // namespace loza
 
@@ -1020,6 +1058,160 @@ loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d64) return launch_backward<64, 64>(prm, out, dout, T * n_heads, nq_max, batch, st);
   return launch_backward<192, 128>(prm, out, dout, T * n_heads, nq_max, batch, st);
+}
+
+loza_status loza_hi_page_keys(const void* k_index, int64_t index_batch_stride, int64_t index_row_stride,
+                              const int32_t* seqlens, int32_t batch, int32_t max_seqlen, int32_t d_index,
+                              float* page_keys, loza_stream_t stream) {
+  if (!seqlens || !page_keys) return LOZA_ERR_INVALID_ARG;
+  if (!hi_args_ok(k_index, index_batch_stride, index_row_stride, batch, max_seqlen, d_index))
+    return LOZA_ERR_INVALID_ARG;
+  const int64_t pages = max_seqlen / kHiPage;
+  if (pages < 1) return LOZA_OK;
+  const int64_t per_seq = pages * d_index;
+  const unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((per_seq + 255) / 256, 4 * sm_count()));
+  hi_page_keys_kernel<<<dim3(gx, batch), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(k_index), index_batch_stride, index_row_stride, seqlens, d_index, pages,
+      page_keys);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
+size_t loza_hi_workspace_size(int32_t batch, int32_t max_seqlen, int32_t top_pages, int32_t top_k,
+                              loza_ssa_params p) {
+  if (batch < 1 || max_seqlen < 1 || top_pages < 1 || top_k < 0 || top_k > kHiMaxTopK || !window_ok(p)) return 0;
+  const size_t dec = decode_workspace(batch, decode_plan(p, max_seqlen, batch)).total;
+  return hi_workspace(batch, top_pages, top_k, dec).total;
+}
+
+}  // extern "C"
+
+namespace loza {
+namespace {
+// Validate and enqueue the selection; `w` is the workspace layout.
+loza_status hi_select_launch(const void* q_index, const void* k_index, int64_t index_batch_stride,
+                             int64_t index_row_stride, const float* page_keys, const int32_t* seqlens,
+                             int32_t batch, int32_t max_seqlen, int32_t d_index, const loza_ssa_params& p,
+                             int32_t top_pages, int32_t top_k, int32_t* selected, uint8_t* ws, const HiWorkspace& w,
+                             cudaStream_t st) {
+  HiParams hp;
+  std::memset(&hp, 0, sizeof(hp));
+  hp.q_index = static_cast<const __nv_bfloat16*>(q_index);
+  hp.k_index = static_cast<const __nv_bfloat16*>(k_index);
+  hp.batch_stride = index_batch_stride;
+  hp.row_stride = index_row_stride;
+  hp.page_keys = page_keys;
+  hp.pages_per_seq = max_seqlen / kHiPage;
+  hp.seqlens = seqlens;
+  hp.d = d_index;
+  hp.block = p.block_size;
+  hp.n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
+  hp.n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
+  hp.top_pages = top_pages;
+  hp.top_k = top_k;
+  hp.sel_pages = reinterpret_cast<int32_t*>(ws + w.sel_pages);
+  hp.n_pages = reinterpret_cast<int32_t*>(ws + w.n_pages);
+  hp.tok_keys = reinterpret_cast<unsigned long long*>(ws + w.tok_keys);
+  hp.selected = selected;
+  int npow2 = 1;
+  while (npow2 < hp.pages_per_seq) npow2 <<= 1;
+  const int smem = npow2 * 8;
+  if (cudaFuncSetAttribute(hi_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return LOZA_ERR_CUDA;
+  hi_pages_kernel<<<batch, 1024, smem, st>>>(hp);
+  hi_tokens_kernel<<<dim3((top_pages + kHiTokPagesPerCta - 1) / kHiTokPagesPerCta, batch), kHiPage, 0, st>>>(hp);
+  hi_topk_kernel<<<batch, 1024, 0, st>>>(hp);
+  g_launches.fetch_add(3, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+
+loza_status hi_attend_launch(const void* q, const void* kv_cache, int64_t cache_batch_stride,
+                             int64_t cache_row_stride, const int32_t* selected, int32_t top_k, int32_t batch,
+                             float scale, void* out, float* lse, cudaStream_t st) {
+  using LY = HiAttnLayout;
+  if (cudaFuncSetAttribute(hi_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM_BYTES) !=
+      cudaSuccess)
+    return LOZA_ERR_CUDA;
+  hi_attend_kernel<<<dim3(batch, kDecHeads / 8), 256, LY::SMEM_BYTES, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kv_cache), cache_batch_stride,
+      cache_row_stride, selected, top_k, scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(out), lse);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
+}  // namespace
+}  // namespace loza
+
+extern "C" {
+
+loza_status loza_hi_select(const void* q_index, const void* k_index, int64_t index_batch_stride,
+                           int64_t index_row_stride, const float* page_keys, const int32_t* seqlens, int32_t batch,
+                           int32_t max_seqlen, int32_t d_index, loza_ssa_params p, int32_t top_pages, int32_t top_k,
+                           int32_t* selected, void* workspace, size_t workspace_bytes, loza_stream_t stream) {
+  if (!q_index || !page_keys || !seqlens || !selected || !aligned16(q_index)) return LOZA_ERR_INVALID_ARG;
+  if (!hi_args_ok(k_index, index_batch_stride, index_row_stride, batch, max_seqlen, d_index))
+    return LOZA_ERR_INVALID_ARG;
+  if (top_pages < 1 || top_k < 1 || top_k > kHiMaxTopK) return LOZA_ERR_INVALID_ARG;
+  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (max_seqlen / kHiPage > kHiMaxPages) return LOZA_ERR_UNSUPPORTED;
+  const size_t need = loza_hi_workspace_size(batch, max_seqlen, top_pages, top_k, p);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LOZA_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return LOZA_ERR_WORKSPACE;
+  const HiWorkspace w = hi_workspace(batch, top_pages, top_k, 0);
+  return hi_select_launch(q_index, k_index, index_batch_stride, index_row_stride, page_keys, seqlens, batch,
+                          max_seqlen, d_index, p, top_pages, top_k, selected, static_cast<uint8_t*>(workspace), w,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+loza_status loza_ssa_decode_selected(const void* q, const void* kv_cache, int64_t cache_batch_stride,
+                                     int64_t cache_row_stride, const int32_t* selected, int32_t top_k,
+                                     int32_t batch, int32_t n_heads, float scale, void* out, float* lse,
+                                     loza_stream_t stream) {
+  if (!q || !kv_cache || !selected || !out || !lse) return LOZA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || top_k < 0) return LOZA_ERR_INVALID_ARG;
+  if (!stride_ok(cache_row_stride) || !stride_ok(cache_batch_stride) || cache_row_stride < 576)
+    return LOZA_ERR_INVALID_ARG;
+  if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
+  return hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, selected, top_k, batch, scale, out,
+                          lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+loza_status loza_hi_decode(const void* q, const void* kv_cache, int64_t cache_batch_stride, int64_t cache_row_stride,
+                           const void* q_index, const void* k_index, int64_t index_batch_stride,
+                           int64_t index_row_stride, const float* page_keys, const int32_t* seqlens, int32_t batch,
+                           int32_t max_seqlen, int32_t d_index, loza_ssa_params p, int32_t top_pages, int32_t top_k,
+                           void* out, float* lse, void* workspace, size_t workspace_bytes, loza_stream_t stream) {
+  if (!q_index || !page_keys || !seqlens || !aligned16(q_index)) return LOZA_ERR_INVALID_ARG;
+  if (!hi_args_ok(k_index, index_batch_stride, index_row_stride, batch, max_seqlen, d_index))
+    return LOZA_ERR_INVALID_ARG;
+  if (top_pages < 1 || top_k < 1 || top_k > kHiMaxTopK) return LOZA_ERR_INVALID_ARG;
+  if (max_seqlen / kHiPage > kHiMaxPages || !window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LOZA_ERR_INVALID_ARG;
+  if (workspace_bytes < loza_hi_workspace_size(batch, max_seqlen, top_pages, top_k, p)) return LOZA_ERR_WORKSPACE;
+  // the window part: validation and the decode plan as for loza_ssa_decode
+  DecodeParams prm;
+  DecodePlan plan;
+  const loza_status rc = setup_decode_mla(q, kv_cache, nullptr, seqlens, batch, max_seqlen, cache_batch_stride,
+                                          cache_row_stride, kDecHeads, p, out, lse, &prm, &plan);
+  if (rc != LOZA_OK) return rc;
+  const HiWorkspace w = hi_workspace(batch, top_pages, top_k, decode_workspace(batch, plan).total);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* sel = reinterpret_cast<int32_t*>(ws + w.selected);
+  loza_status r = hi_select_launch(q_index, k_index, index_batch_stride, index_row_stride, page_keys, seqlens,
+                                   batch, max_seqlen, d_index, p, top_pages, top_k, sel, ws, w, st);
+  if (r != LOZA_OK) return r;
+  // the selected part and the window part, then their log-sum-exp merge
+  r = hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, sel, top_k, batch, p.scale, ws + w.o_sel,
+                       reinterpret_cast<float*>(ws + w.l_sel), st);
+  if (r != LOZA_OK) return r;
+  prm.out = reinterpret_cast<__nv_bfloat16*>(ws + w.o_win);
+  prm.lse = reinterpret_cast<float*>(ws + w.l_win);
+  r = launch_decode_mla(prm, plan, batch, ws + w.dec, st);
+  if (r != LOZA_OK) return r;
+  return loza_ssa_merge(ws + w.o_win, reinterpret_cast<const float*>(ws + w.l_win), ws + w.o_sel,
+                        reinterpret_cast<const float*>(ws + w.l_sel), (int64_t)batch * kDecHeads, 512, out, lse,
+                        stream);
 }
 
 loza_status loza_ssa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -215,6 +215,86 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
                             void *workspace, size_t workspace_bytes, loza_stream_t stream);
 
 /*
+ * Hierarchical index decode (page 4, "LongCat Sparse Attention: Taming the
+ * Lightning via Streaming-aware Hierarchical Cross-Layer Indexing",
+ * agihunt.info: its streaming-aware index gives every query fixed sink and
+ * window tokens plus dynamically selected tokens, and its hierarchical index
+ * selects those in two stages, top pages of 128 tokens first, then top tokens
+ * within them). The fixed part is the SSA window `p` of this library; the
+ * dynamic part is chosen among the tokens outside it, so the parts are
+ * disjoint, and the two are merged by their log-sum-exp (loza_ssa_merge).
+ * Scoring (the pages give none): the dot product of the sequence's index
+ * query with a token's index key, both supplied by the caller (as an indexer
+ * produces them); a page is scored by the mean of its 128 index keys. Scores
+ * are fp32 fused multiply-adds over the index dimension in order, so the
+ * selection is one exact set; ties go to the lower page / token index.
+ * Common arguments:
+ *   k_index   index keys: token t of sequence n at k_index + n *
+ *             index_batch_stride + t * index_row_stride elements, d_index bf16
+ *             each (d_index a multiple of 8, at most 512; strides * 2 multiples
+ *             of 16; index_batch_stride >= max_seqlen * index_row_stride)
+ *   q_index   [batch, d_index] bf16, one index query per sequence
+ *   page_keys [batch, max_seqlen / 128, d_index] fp32 (from loza_hi_page_keys)
+ *   seqlens   device int32 [batch], 1 <= seqlens[n] <= max_seqlen; the decode
+ *             query is position seqlens[n] - 1, as in loza_ssa_decode
+ * Limits: max_seqlen / 128 <= 8192 pages; 1 <= top_k <= 2048; top_pages >= 1.
+ *
+ * loza_hi_page_keys: the mean index key of every whole page (tokens 128p ..
+ * 128p+127 all below seqlens[n]): fp32 sums in token order times 1/128. Pages
+ * past a sequence's end are not written. Maintained by the caller as its cache
+ * fills (a page's mean never changes once the page is whole).
+ */
+loza_status loza_hi_page_keys(const void *k_index, int64_t index_batch_stride, int64_t index_row_stride,
+                              const int32_t *seqlens, int32_t batch, int32_t max_seqlen, int32_t d_index,
+                              float *page_keys, loza_stream_t stream);
+
+/* Bytes of device workspace loza_hi_select and loza_hi_decode need (0 for an
+ * unsupported request). */
+size_t loza_hi_workspace_size(int32_t batch, int32_t max_seqlen, int32_t top_pages, int32_t top_k,
+                              loza_ssa_params p);
+
+/*
+ * The tokens the hierarchical index selects for each sequence's decode query:
+ * the top_pages whole pages holding a token outside the window, by page score,
+ * then the top_k tokens outside the window in those pages, by token score.
+ *   selected  device int32 [batch, top_k]: the tokens in ascending order, then
+ *             -1 where fewer than top_k were available
+ *   workspace loza_hi_workspace_size(...) bytes, 256-byte aligned
+ */
+loza_status loza_hi_select(const void *q_index, const void *k_index, int64_t index_batch_stride,
+                           int64_t index_row_stride, const float *page_keys, const int32_t *seqlens, int32_t batch,
+                           int32_t max_seqlen, int32_t d_index, loza_ssa_params p, int32_t top_pages, int32_t top_k,
+                           int32_t *selected, void *workspace, size_t workspace_bytes, loza_stream_t stream);
+
+/*
+ * Softmax attention of each sequence's decode query over an explicit list of
+ * its tokens (absorbed MLA: 64 heads, the 576-wide latent row as K, its first
+ * 512 columns as V): out [batch, 64, 512] bf16, lse [batch, 64] fp32 (natural
+ * log; -inf and O = 0 when a sequence has no token). selected: device int32
+ * [batch, top_k], entries < 0 ignored; every other entry must name a row the
+ * cache holds for its sequence (not checked: the call has no sequence
+ * lengths). q is [batch, 64, 576] contiguous and the cache layout is
+ * loza_ssa_decode's.
+ */
+loza_status loza_ssa_decode_selected(const void *q, const void *kv_cache, int64_t cache_batch_stride,
+                                     int64_t cache_row_stride, const int32_t *selected, int32_t top_k,
+                                     int32_t batch, int32_t n_heads, float scale, void *out, float *lse,
+                                     loza_stream_t stream);
+
+/*
+ * The whole decode: loza_hi_select, loza_ssa_decode_selected over the
+ * selection, loza_ssa_decode over the window p, and the log-sum-exp merge of
+ * the two into out [batch, 64, 512] bf16 and lse [batch, 64]. Same cache
+ * arguments as loza_ssa_decode (absorbed MLA, 64 heads, 576 / 512).
+ *   workspace loza_hi_workspace_size(...) bytes, 256-byte aligned
+ */
+loza_status loza_hi_decode(const void *q, const void *kv_cache, int64_t cache_batch_stride, int64_t cache_row_stride,
+                           const void *q_index, const void *k_index, int64_t index_batch_stride,
+                           int64_t index_row_stride, const float *page_keys, const int32_t *seqlens, int32_t batch,
+                           int32_t max_seqlen, int32_t d_index, loza_ssa_params p, int32_t top_pages, int32_t top_k,
+                           void *out, float *lse, void *workspace, size_t workspace_bytes, loza_stream_t stream);
+
+/*
  * Decode without any caller-provided device memory. (The LoZA pages have no
  * counterpart to this entry point; it exists for callers of this library.)
  *
