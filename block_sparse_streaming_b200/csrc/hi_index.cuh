@@ -256,7 +256,10 @@ __global__ void __launch_bounds__(1024) hi_topk_kernel(const HiParams p) {
     thr = prefix;
     for (int64_t t = threadIdx.x; t < N; t += blockDim.x) {
       const unsigned long long k = keys[t];
-      if (k != 0ull && k >= thr) sel[atomicAdd(&n_out, 1)] = k;
+      if (k != 0ull && k >= thr) {
+        const int slot = atomicAdd(&n_out, 1);  // < k_eff: the keys are distinct
+        if (slot < kHiMaxTopK) sel[slot] = k;
+      }
     }
   }
   __syncthreads();
