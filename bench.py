@@ -532,6 +532,102 @@ def long_secondary(bss, device, stream, peaks, peak_kind):
     return res, dec
 
 
+HI_WINDOW = (1, 16, 1024)   # page 4: 16 sink tokens and a 1,024-token window (b = 1)
+HI_TOP_PAGES, HI_TOP_K, HI_DIM = 1024, 1024, 128
+
+
+def token_window_rows(L, win=HI_WINDOW):
+    b, s, l = win
+    i = L - 1
+    lo = max(0, (i // b - l + 1) * b)
+    return min(s * b, L) + (L - max(lo, min(s * b, L)))
+
+
+def hi_secondary(bss, device, stream, peaks, peak_kind, batch=32, ctx=1 << 20, steps=10):
+    """Hierarchical index decode (page 4): 32 sequences of 1,048,576 tokens,
+    16 sink tokens + a 1,024-token window + 1,024 tokens selected from the top
+    1,024 pages of 128, index keys of 128 bf16. Times the whole call and, apart,
+    its three parts (the selection, the window decode, the attention over the
+    selection with the merge); the page keys are maintained as the cache fills
+    and are computed once, outside the step."""
+    import torch
+    seed = synth.workload_seed(4) * 1000 + 70
+    q = synth.torch_normal_bf16((batch, H, DQK), seed, device)
+    cache = synth.torch_normal_bf16((batch, ctx, 1, DQK), seed + 1, device)
+    k_idx = synth.torch_normal_bf16((batch, ctx, HI_DIM), seed + 2, device)
+    q_idx = synth.torch_normal_bf16((batch, HI_DIM), seed + 3, device)
+    lens = [ctx] * batch
+    seqlens = torch.tensor(lens, dtype=torch.int32, device=device)
+    params = bss.Params(SCALE, *HI_WINDOW)
+    pk = bss.loza_hi_page_keys(k_idx, seqlens, ctx, stream=stream)
+    out = torch.empty((batch, H, DV), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((batch, H), dtype=torch.float32, device=device)
+    o_w = torch.empty_like(out)
+    l_w = torch.empty_like(lse)
+    ws = torch.empty(max(16, bss.hi_workspace_size(batch, ctx, HI_TOP_PAGES, HI_TOP_K, params)), dtype=torch.uint8,
+                     device=device)
+    ws_dec = torch.empty(max(16, bss.workspace_size(bss.LOZA_OP_DECODE, batch, 0, ctx, H, 1, DQK, DV, params)),
+                         dtype=torch.uint8, device=device)
+    sel = torch.empty((batch, HI_TOP_K), dtype=torch.int32, device=device)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=device)
+
+    def flush():
+        flush_w.zero_()
+        flush_r.sum()
+        torch.cuda._sleep(400000)
+
+    calls = {
+        "hi_decode": lambda: bss.loza_hi_decode(q, cache, q_idx, k_idx, pk, seqlens, ctx, params, HI_TOP_PAGES,
+                                                HI_TOP_K, out=out, lse=lse, workspace=ws, stream=stream),
+        "select": lambda: bss.loza_hi_select(q_idx, k_idx, pk, seqlens, ctx, params, HI_TOP_PAGES, HI_TOP_K,
+                                             selected=sel, workspace=ws, stream=stream),
+        "window_decode": lambda: bss.loza_ssa_decode(q, cache, None, seqlens, ctx, params, out=o_w, lse=l_w,
+                                                     workspace=ws_dec, stream=stream),
+        "attend_selected": lambda: bss.loza_ssa_decode_selected(q, cache, sel, SCALE, out=o_w, lse=l_w,
+                                                                stream=stream),
+        "page_keys": lambda: bss.loza_hi_page_keys(k_idx, seqlens, ctx, page_keys=pk, stream=stream),
+    }
+    ms = {}
+    launches = {}
+    for name, fn in calls.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        c0 = bss.launch_count()
+        ms[name], _ = time_launches(fn, stream, steps if name != "page_keys" else 3, flush=flush)
+        launches[name] = (bss.launch_count() - c0) // (steps if name != "page_keys" else 3)
+    if bss.device_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait in the HI decode")
+    # algorithmic bytes of one step
+    n_pages = ctx // 128
+    b_select = batch * (n_pages * HI_DIM * 4 + HI_TOP_PAGES * 128 * HI_DIM * 2 + HI_DIM * 2)
+    b_window = batch * (token_window_rows(ctx) * DQK * 2 + H * DQK * 2)
+    b_attend = batch * (HI_TOP_K * DQK * 2 + H * DQK * 2)
+    b_out = batch * H * (DV * 2 + 4)
+    total = b_select + b_window + b_attend + b_out
+    dense_bytes = batch * (ctx * DQK * 2 + H * (DQK * 2 + DV * 2 + 4))
+    parts = {"select": b_select, "window_decode": b_window + b_out, "attend_selected": b_attend + b_out}
+    del q, cache, k_idx, q_idx, pk, ws, ws_dec
+    torch.cuda.empty_cache()
+    hbm = float(peaks["hbm_gbs"])
+    gbs = total / (ms["hi_decode"] / 1000.0) / 1e9
+    return {"workload": f"hierarchical index decode (MLA-absorbed), {batch} seqs x {ctx} tokens, "
+                        f"window 16 sink + 1,024 tokens, top {HI_TOP_PAGES} pages of 128, top {HI_TOP_K} tokens, "
+                        f"index keys {HI_DIM} bf16",
+            "metric": "HI decode GB/s (bytes touched)", "value": gbs, "unit": "GB/s",
+            "ms_per_call": ms["hi_decode"], "bytes_per_call": total, "launches_per_call": launches["hi_decode"],
+            "roofline": hbm_roofline(total, ms["hi_decode"], peaks, peak_kind, "hi_decode (all its kernels)"),
+            "parts": {k: {"ms_per_call": ms[k], "bytes_per_call": parts[k],
+                          "GB/s": parts[k] / (ms[k] / 1000.0) / 1e9,
+                          "frac_of_hbm": parts[k] / (ms[k] / 1000.0) / 1e9 / hbm, "launches": launches[k]}
+                      for k in parts},
+            "page_keys_once": {"ms": ms["page_keys"], "bytes": batch * (ctx * HI_DIM * 2 + n_pages * HI_DIM * 4)},
+            "dense_decode_bytes_per_call": dense_bytes,
+            "timing": "mean of per-call CUDA events; L2 flushed (256 MB write, then 256 MB read) and a ~0.2 ms "
+                      "device sleep before each call"}
+
+
 def train_secondary(bss, device, stream, peaks, peak_kind, train_len=None):
     """Workload 5: varlen forward + backward, per-head 192/128 dims, 64 heads
     (train_len: one sequence of that many tokens instead, for profiling)."""
@@ -675,6 +771,8 @@ def run_ours(args, rank, world, local_rank):
         secondary["merge"] = merge_secondary(bss, device, stream, peaks, peak_kind)
     if args.workload in ("default", "long"):
         secondary["long"], secondary["decode_1m"] = long_secondary(bss, device, stream, peaks, peak_kind)
+    if args.workload in ("default", "hi"):
+        secondary["hi_decode"] = hi_secondary(bss, device, stream, peaks, peak_kind)
     if args.workload in ("default", "train"):
         secondary["train"] = train_secondary(bss, device, stream, peaks, peak_kind, args.train_len)
 
@@ -803,10 +901,10 @@ def main():
                          "sequence, a smaller cache)")
     ap.add_argument("--train-len", type=int, default=None,
                     help="training workload as one sequence of this length (profiling)")
-    ap.add_argument("--workload", choices=["default", "prefill", "decode", "long", "train"], default="default",
+    ap.add_argument("--workload", choices=["default", "prefill", "decode", "long", "hi", "train"], default="default",
                     help="default: the prefill line with every other workload as secondary lines (the "
                          "64-sequence decode, the branch merge, workload 4's long prefill and 1M decode, "
-                         "workload 5's training); the others: the prefill line plus only that one")
+                         "the hierarchical index decode at 1M, workload 5's training); the others: the prefill line plus only that one")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

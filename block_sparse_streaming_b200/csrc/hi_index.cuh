@@ -29,8 +29,8 @@
 //                         largest (score, token) key, the tokens at or above
 //                         it, sorted by position
 //   hi_attend_kernel      softmax attention of the 64 heads over the selected
-//                         latent rows (CUDA cores, fp32), giving O and LSE to
-//                         merge with the window's
+//                         latent rows (CUDA cores, fp32); optionally merged
+//                         with the window part's fp32 O and LSE in its epilogue
 #pragma once
 
 #include <cuda_bf16.h>
@@ -292,6 +292,8 @@ __global__ void __launch_bounds__(256) hi_attend_kernel(const __nv_bfloat16* __r
                                                         const __nv_bfloat16* __restrict__ kv, int64_t batch_stride,
                                                         int64_t row_stride, const int32_t* __restrict__ selected,
                                                         int top_k, float scale_log2,
+                                                        const float* __restrict__ o_win,
+                                                        const float* __restrict__ lse_win,
                                                         __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   using LY = HiAttnLayout;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -373,15 +375,45 @@ __global__ void __launch_bounds__(256) hi_attend_kernel(const __nv_bfloat16* __r
       }
     }
   }
-  // no selected token: O = 0, LSE = -inf (the merge then keeps the other part)
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  __nv_bfloat16* o = out + ((int64_t)n * 64 + head) * 512 + 16 * lane;
-#pragma unroll
-  for (int e = 0; e < 16; e += 2) {
-    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
-    *reinterpret_cast<__nv_bfloat162*>(o + e) = b2;
+  // This part alone (no selected token: O = 0, LSE = -inf), or, given the
+  // window part's unrounded O and its LSE, the log-sum-exp merge of the two
+  // (weights exp(LSE_part - LSE), LSE = log(exp(LSE_win) + exp(LSE_sel))).
+  const int64_t row = (int64_t)n * 64 + head;
+  float w_sel = l > 0.f ? 1.f / l : 0.f;  // multiplies acc
+  float w_win = 0.f;
+  float lse2 = l > 0.f ? m + log2f(l) : -INFINITY;  // log2 units
+  if (o_win) {
+    const float a = lse_win[row] * 1.4426950408889634f;
+    const float mx = fmaxf(a, lse2);
+    if (mx == -INFINITY) {
+      w_sel = 0.f;
+    } else {
+      const float ea = exp2f(a - mx), eb = exp2f(lse2 - mx);
+      const float inv = 1.f / (ea + eb);
+      w_win = ea * inv;
+      w_sel = l > 0.f ? exp2f(m - mx) * inv : 0.f;  // eb / l
+      lse2 = mx + log2f(ea + eb);
+    }
   }
-  if (lane == 0) lse[(int64_t)n * 64 + head] = l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  __nv_bfloat16* o = out + row * 512 + 16 * lane;
+  if (o_win) {
+    const float4* ow = reinterpret_cast<const float4*>(o_win + row * 512 + 16 * lane);
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+      const float4 v = ow[e4];
+      acc[4 * e4] = fmaf(w_win, v.x, acc[4 * e4] * w_sel);
+      acc[4 * e4 + 1] = fmaf(w_win, v.y, acc[4 * e4 + 1] * w_sel);
+      acc[4 * e4 + 2] = fmaf(w_win, v.z, acc[4 * e4 + 2] * w_sel);
+      acc[4 * e4 + 3] = fmaf(w_win, v.w, acc[4 * e4 + 3] * w_sel);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] *= w_sel;
+  }
+#pragma unroll
+  for (int e = 0; e < 16; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(o + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
+  if (lane == 0) lse[row] = lse2 == -INFINITY ? -INFINITY : lse2 * 0.69314718055994530942f;
 }
 
 }  // namespace loza

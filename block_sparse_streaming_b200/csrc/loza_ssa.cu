@@ -529,7 +529,7 @@ unsigned stream_grid(int64_t n) {
 
 // Hierarchical index (page 4): workspace of loza_hi_select / loza_hi_decode.
 struct HiWorkspace {
-  size_t sel_pages, n_pages, tok_keys, selected, o_sel, l_sel, o_win, l_win, dec, total;
+  size_t sel_pages, n_pages, tok_keys, selected, o_win, l_win, dec, total;
 };
 size_t hi_align(size_t x) { return (x + 255) / 256 * 256; }
 HiWorkspace hi_workspace(int32_t batch, int32_t top_pages, int32_t top_k, size_t decode_ws) {
@@ -544,9 +544,7 @@ HiWorkspace hi_workspace(int32_t batch, int32_t top_pages, int32_t top_k, size_t
   w.n_pages = take((size_t)batch * 4);
   w.tok_keys = take((size_t)batch * top_pages * kHiPage * 8);
   w.selected = take((size_t)batch * std::max(top_k, 1) * 4);
-  w.o_sel = take((size_t)batch * kDecHeads * 512 * 2);
-  w.l_sel = take((size_t)batch * kDecHeads * 4);
-  w.o_win = take((size_t)batch * kDecHeads * 512 * 2);
+  w.o_win = take((size_t)batch * kDecHeads * 512 * 4);  // fp32: rounded once, after the merge
   w.l_win = take((size_t)batch * kDecHeads * 4);
   w.dec = take(decode_ws);
   w.total = off;
@@ -1127,14 +1125,16 @@ loza_status hi_select_launch(const void* q_index, const void* k_index, int64_t i
 
 loza_status hi_attend_launch(const void* q, const void* kv_cache, int64_t cache_batch_stride,
                              int64_t cache_row_stride, const int32_t* selected, int32_t top_k, int32_t batch,
-                             float scale, void* out, float* lse, cudaStream_t st) {
+                             float scale, const float* o_win, const float* lse_win, void* out, float* lse,
+                             cudaStream_t st) {
   using LY = HiAttnLayout;
   if (cudaFuncSetAttribute(hi_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM_BYTES) !=
       cudaSuccess)
     return LOZA_ERR_CUDA;
   hi_attend_kernel<<<dim3(batch, kDecHeads / 8), 256, LY::SMEM_BYTES, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kv_cache), cache_batch_stride,
-      cache_row_stride, selected, top_k, scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(out), lse);
+      cache_row_stride, selected, top_k, scale * 1.4426950408889634f, o_win, lse_win,
+      static_cast<__nv_bfloat16*>(out), lse);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
@@ -1172,8 +1172,8 @@ loza_status loza_ssa_decode_selected(const void* q, const void* kv_cache, int64_
   if (!stride_ok(cache_row_stride) || !stride_ok(cache_batch_stride) || cache_row_stride < 576)
     return LOZA_ERR_INVALID_ARG;
   if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
-  return hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, selected, top_k, batch, scale, out,
-                          lse, reinterpret_cast<cudaStream_t>(stream));
+  return hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, selected, top_k, batch, scale, nullptr,
+                          nullptr, out, lse, reinterpret_cast<cudaStream_t>(stream));
 }
 
 loza_status loza_hi_decode(const void* q, const void* kv_cache, int64_t cache_batch_stride, int64_t cache_row_stride,
@@ -1201,17 +1201,16 @@ loza_status loza_hi_decode(const void* q, const void* kv_cache, int64_t cache_ba
   loza_status r = hi_select_launch(q_index, k_index, index_batch_stride, index_row_stride, page_keys, seqlens,
                                    batch, max_seqlen, d_index, p, top_pages, top_k, sel, ws, w, st);
   if (r != LOZA_OK) return r;
-  // the selected part and the window part, then their log-sum-exp merge
-  r = hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, sel, top_k, batch, p.scale, ws + w.o_sel,
-                       reinterpret_cast<float*>(ws + w.l_sel), st);
-  if (r != LOZA_OK) return r;
-  prm.out = reinterpret_cast<__nv_bfloat16*>(ws + w.o_win);
-  prm.lse = reinterpret_cast<float*>(ws + w.l_win);
+  // the window part in fp32, then the selected part, merged by log-sum-exp in
+  // the attention kernel's epilogue (one bf16 rounding of the result)
+  float* o_win = reinterpret_cast<float*>(ws + w.o_win);
+  float* l_win = reinterpret_cast<float*>(ws + w.l_win);
+  prm.out_f32 = o_win;
+  prm.lse = l_win;
   r = launch_decode_mla(prm, plan, batch, ws + w.dec, st);
   if (r != LOZA_OK) return r;
-  return loza_ssa_merge(ws + w.o_win, reinterpret_cast<const float*>(ws + w.l_win), ws + w.o_sel,
-                        reinterpret_cast<const float*>(ws + w.l_sel), (int64_t)batch * kDecHeads, 512, out, lse,
-                        stream);
+  return hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, sel, top_k, batch, p.scale, o_win, l_win,
+                          out, lse, st);
 }
 
 loza_status loza_ssa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -222,7 +222,7 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  * selects those in two stages, top pages of 128 tokens first, then top tokens
  * within them). The fixed part is the SSA window `p` of this library; the
  * dynamic part is chosen among the tokens outside it, so the parts are
- * disjoint, and the two are merged by their log-sum-exp (loza_ssa_merge).
+ * disjoint, and the two are merged by their log-sum-exp.
  * Scoring (the pages give none): the dot product of the sequence's index
  * query with a token's index key, both supplied by the caller (as an indexer
  * produces them); a page is scored by the mean of its 128 index keys. Scores
@@ -282,10 +282,11 @@ loza_status loza_ssa_decode_selected(const void *q, const void *kv_cache, int64_
                                      loza_stream_t stream);
 
 /*
- * The whole decode: loza_hi_select, loza_ssa_decode_selected over the
- * selection, loza_ssa_decode over the window p, and the log-sum-exp merge of
- * the two into out [batch, 64, 512] bf16 and lse [batch, 64]. Same cache
- * arguments as loza_ssa_decode (absorbed MLA, 64 heads, 576 / 512).
+ * The whole decode: loza_hi_select, then loza_ssa_decode over the window p
+ * (its O kept in fp32 in the workspace), then the attention over the
+ * selection, whose epilogue merges the two parts by their log-sum-exp into
+ * out [batch, 64, 512] bf16 and lse [batch, 64] (one rounding to bf16). Same
+ * cache arguments as loza_ssa_decode (absorbed MLA, 64 heads, 576 / 512).
  *   workspace loza_hi_workspace_size(...) bytes, 256-byte aligned
  */
 loza_status loza_hi_decode(const void *q, const void *kv_cache, int64_t cache_batch_stride, int64_t cache_row_stride,
