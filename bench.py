@@ -547,9 +547,9 @@ def hi_secondary(bss, device, stream, peaks, peak_kind, batch=32, ctx=1 << 20, s
     """Hierarchical index decode (page 4): 32 sequences of 1,048,576 tokens,
     16 sink tokens + a 1,024-token window + 1,024 tokens selected from the top
     1,024 pages of 128, index keys of 128 bf16. Times the whole call and, apart,
-    its three parts (the selection, the window decode, the attention over the
-    selection with the merge); the page keys are maintained as the cache fills
-    and are computed once, outside the step."""
+    its two parts (the selection; the attention over the window and the
+    selection), and the window alone for comparison; the page keys are
+    maintained as the cache fills and are computed once, outside the step."""
     import torch
     seed = synth.workload_seed(4) * 1000 + 70
     q = synth.torch_normal_bf16((batch, H, DQK), seed, device)
@@ -566,6 +566,8 @@ def hi_secondary(bss, device, stream, peaks, peak_kind, batch=32, ctx=1 << 20, s
     l_w = torch.empty_like(lse)
     ws = torch.empty(max(16, bss.hi_workspace_size(batch, ctx, HI_TOP_PAGES, HI_TOP_K, params)), dtype=torch.uint8,
                      device=device)
+    ws_sel = torch.empty(max(16, bss.hi_workspace_size(batch, ctx, 1, HI_TOP_K, params)), dtype=torch.uint8,
+                         device=device)
     ws_dec = torch.empty(max(16, bss.workspace_size(bss.LOZA_OP_DECODE, batch, 0, ctx, H, 1, DQK, DV, params)),
                          dtype=torch.uint8, device=device)
     sel = torch.empty((batch, HI_TOP_K), dtype=torch.int32, device=device)
@@ -582,10 +584,10 @@ def hi_secondary(bss, device, stream, peaks, peak_kind, batch=32, ctx=1 << 20, s
                                                 HI_TOP_K, out=out, lse=lse, workspace=ws, stream=stream),
         "select": lambda: bss.loza_hi_select(q_idx, k_idx, pk, seqlens, ctx, params, HI_TOP_PAGES, HI_TOP_K,
                                              selected=sel, workspace=ws, stream=stream),
-        "window_decode": lambda: bss.loza_ssa_decode(q, cache, None, seqlens, ctx, params, out=o_w, lse=l_w,
-                                                     workspace=ws_dec, stream=stream),
-        "attend_selected": lambda: bss.loza_ssa_decode_selected(q, cache, sel, SCALE, out=o_w, lse=l_w,
-                                                                stream=stream),
+        "decode_selected": lambda: bss.loza_ssa_decode_selected(q, cache, seqlens, ctx, params, sel, out=o_w,
+                                                                lse=l_w, workspace=ws_sel, stream=stream),
+        "window_only_decode": lambda: bss.loza_ssa_decode(q, cache, None, seqlens, ctx, params, out=o_w, lse=l_w,
+                                                          workspace=ws_dec, stream=stream),
         "page_keys": lambda: bss.loza_hi_page_keys(k_idx, seqlens, ctx, page_keys=pk, stream=stream),
     }
     ms = {}
@@ -602,13 +604,12 @@ def hi_secondary(bss, device, stream, peaks, peak_kind, batch=32, ctx=1 << 20, s
     # algorithmic bytes of one step
     n_pages = ctx // 128
     b_select = batch * (n_pages * HI_DIM * 4 + HI_TOP_PAGES * 128 * HI_DIM * 2 + HI_DIM * 2)
-    b_window = batch * (token_window_rows(ctx) * DQK * 2 + H * DQK * 2)
-    b_attend = batch * (HI_TOP_K * DQK * 2 + H * DQK * 2)
-    b_out = batch * H * (DV * 2 + 4)
-    total = b_select + b_window + b_attend + b_out
+    b_attend = batch * ((token_window_rows(ctx) + HI_TOP_K) * DQK * 2 + H * (DQK * 2 + DV * 2 + 4))
+    total = b_select + b_attend
     dense_bytes = batch * (ctx * DQK * 2 + H * (DQK * 2 + DV * 2 + 4))
-    parts = {"select": b_select, "window_decode": b_window + b_out, "attend_selected": b_attend + b_out}
-    del q, cache, k_idx, q_idx, pk, ws, ws_dec
+    parts = {"select": b_select, "decode_selected": b_attend,
+             "window_only_decode": batch * (token_window_rows(ctx) * DQK * 2 + H * (DQK * 2 + DV * 2 + 4))}
+    del q, cache, k_idx, q_idx, pk, ws, ws_sel, ws_dec
     torch.cuda.empty_cache()
     hbm = float(peaks["hbm_gbs"])
     gbs = total / (ms["hi_decode"] / 1000.0) / 1e9
@@ -772,7 +773,7 @@ def run_ours(args, rank, world, local_rank):
     if args.workload in ("default", "long"):
         secondary["long"], secondary["decode_1m"] = long_secondary(bss, device, stream, peaks, peak_kind)
     if args.workload in ("default", "hi"):
-        secondary["hi_decode"] = hi_secondary(bss, device, stream, peaks, peak_kind)
+        secondary["hi_decode"] = hi_secondary(bss, device, stream, peaks, peak_kind, args.hi_batch, args.hi_ctx)
     if args.workload in ("default", "train"):
         secondary["train"] = train_secondary(bss, device, stream, peaks, peak_kind, args.train_len)
 
@@ -901,6 +902,8 @@ def main():
                          "sequence, a smaller cache)")
     ap.add_argument("--train-len", type=int, default=None,
                     help="training workload as one sequence of this length (profiling)")
+    ap.add_argument("--hi-batch", type=int, default=32, help="sequences of the hierarchical index decode line")
+    ap.add_argument("--hi-ctx", type=int, default=1 << 20, help="tokens per sequence of that line (a multiple of 128)")
     ap.add_argument("--workload", choices=["default", "prefill", "decode", "long", "hi", "train"], default="default",
                     help="default: the prefill line with every other workload as secondary lines (the "
                          "64-sequence decode, the branch merge, workload 4's long prefill and 1M decode, "

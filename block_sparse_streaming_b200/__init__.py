@@ -116,8 +116,8 @@ def lib() -> ctypes.CDLL:
         L.loza_hi_select.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _i32, _i32, _i32, Params, _i32, _i32, _vp, _vp,
                                      _sz, _vp]
         L.loza_ssa_decode_selected.restype = ctypes.c_int
-        L.loza_ssa_decode_selected.argtypes = [_vp, _vp, _i64, _i64, _vp, _i32, _i32, _i32, ctypes.c_float, _vp,
-                                               _vp, _vp]
+        L.loza_ssa_decode_selected.argtypes = [_vp, _vp, _i64, _i64, _vp, _i32, _i32, Params, _vp, _i32, _vp, _vp,
+                                               _vp, _sz, _vp]
         L.loza_hi_decode.restype = ctypes.c_int
         L.loza_hi_decode.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _i32, _i32, Params,
                                      _i32, _i32, _vp, _vp, _vp, _sz, _vp]
@@ -422,13 +422,14 @@ def _index_keys(k_index):
 
 def loza_hi_page_keys(k_index, seqlens, max_seqlen: int, page_keys=None, stream=None):
     """Mean index key of every whole 128-token page: k_index [B, Lcap, d] bf16 ->
-    page_keys [B, max_seqlen // 128, d] float32."""
+    page_keys [B, d, max_seqlen // 128] float32 (pages innermost)."""
     import torch
     d, bs, rs = _index_keys(k_index)
     _require(seqlens, "seqlens", torch.int32, 1)
     B = k_index.shape[0]
     if page_keys is None:
-        page_keys = torch.zeros((B, int(max_seqlen) // 128, d), dtype=torch.float32, device=k_index.device)
+        page_keys = torch.zeros((B, d, int(max_seqlen) // 128), dtype=torch.float32, device=k_index.device)
+    _contiguous(page_keys, "page_keys")
     rc = lib().loza_hi_page_keys(_ptr(k_index), bs, rs, _ptr(seqlens), B, int(max_seqlen), d, _ptr(page_keys),
                                  _stream_ptr(stream))
     _check(rc, "loza_hi_page_keys")
@@ -461,23 +462,31 @@ def loza_hi_select(q_index, k_index, page_keys, seqlens, max_seqlen: int, params
     return selected
 
 
-def loza_ssa_decode_selected(q, kv_cache, selected, scale: float, out=None, lse=None, stream=None):
-    """Attention of each decode query over its selected tokens (absorbed latent
-    cache [B, Lcap, 1, 576]); returns (out [B, 64, 512], lse [B, 64])."""
+def loza_ssa_decode_selected(q, kv_cache, seqlens, max_seqlen: int, params: Params, selected, out=None, lse=None,
+                             workspace=None, stream=None):
+    """Attention of each decode query over its window `params` and the tokens of
+    `selected` (int32 [B, top_k]; entries that are negative, past the query or
+    inside the window are ignored). Absorbed latent cache [B, Lcap, 1, 576];
+    returns (out [B, 64, 512], lse [B, 64])."""
     import torch
     _require(q, "q", torch.bfloat16, 3)
     _latent_cache(kv_cache)
     _require(selected, "selected", torch.int32, 2)
+    _require(seqlens, "seqlens", torch.int32, 1)
     _contiguous(q, "q")
     _contiguous(selected, "selected")
     B, H, _ = q.shape
+    top_k = selected.shape[1]
     if out is None:
         out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(16, hi_workspace_size(B, int(max_seqlen), 1, top_k, params)),
+                                dtype=torch.uint8, device=q.device)
     rc = lib().loza_ssa_decode_selected(_ptr(q), _ptr(kv_cache), kv_cache.stride(0), kv_cache.stride(1),
-                                        _ptr(selected), selected.shape[1], B, H, float(scale), _ptr(out), _ptr(lse),
-                                        _stream_ptr(stream))
+                                        _ptr(seqlens), B, int(max_seqlen), params, _ptr(selected), top_k, _ptr(out),
+                                        _ptr(lse), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check(rc, "loza_ssa_decode_selected")
     return out, lse
 

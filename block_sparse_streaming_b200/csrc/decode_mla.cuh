@@ -68,7 +68,6 @@ struct DecodeParams {
   float4* ws_ml;       // workspace mode: [B, nsplit, H] partial (m in log2 units, l exact, l of bf16 P, -)
   int* ws_ticket;      // workspace mode: [B] arrival counters (zero on entry)
   __nv_bfloat16* out;  // [B, H, 512]
-  float* out_f32;      // when set, O goes here in fp32 [B, H, 512] instead (a part merged later)
   float* lse;          // [B, H]
   int nsplit;
   int bps;             // selected blocks per split
@@ -594,14 +593,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
             if (wgt[s2 * 64 + h] != 0.f) acc[i] += src[(size_t)h * W];  // a split without blocks sent no data
           }
         }
-        const int64_t o0 = (int64_t)seq * kDecHeads * 512 + d;
-        if (p.out_f32) {
+        __nv_bfloat16* dst = p.out + (int64_t)seq * kDecHeads * 512 + d;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) p.out_f32[o0 + (int64_t)(32 * grp + i) * 512] = acc[i];
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) p.out[o0 + (int64_t)(32 * grp + i) * 512] = __float2bfloat16_rn(acc[i]);
-        }
+        for (int i = 0; i < 32; ++i) dst[(int64_t)(32 * grp + i) * 512] = __float2bfloat16_rn(acc[i]);
       }
     }
     tc_fence_before();
@@ -653,11 +647,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
             acc.w += o.w * w;
           }
         }
-        const int64_t o0 = ((int64_t)seq * kDecHeads + h) * 512 + d4;
-        if (p.out_f32)
-          *reinterpret_cast<float4*>(p.out_f32 + o0) = acc;
-        else
-          *reinterpret_cast<uint2*>(p.out + o0) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+        __nv_bfloat16* dst = p.out + ((int64_t)seq * kDecHeads + h) * 512 + d4;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
       }
       if (threadIdx.x == 0) p.ws_ticket[seq] = 0;  // ready for the next call
     }

@@ -571,14 +571,9 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
           acc[4 * q4 + 3] = fmaf(v.w, w.w, acc[4 * q4 + 3]);
         }
       }
-      const int64_t o0 = (int64_t)seq * kDecHeads * 512 + d;
-      if (p.out_f32) {
+      __nv_bfloat16* dst = p.out + (int64_t)seq * kDecHeads * 512 + d;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) p.out_f32[o0 + (int64_t)(32 * grp + i) * 512] = acc[i];
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) p.out[o0 + (int64_t)(32 * grp + i) * 512] = __float2bfloat16_rn(acc[i]);
-      }
+      for (int i = 0; i < 32; ++i) dst[(int64_t)(32 * grp + i) * 512] = __float2bfloat16_rn(acc[i]);
     }
   }
   // no split leaves while a bulk copy out of its shared memory may still run

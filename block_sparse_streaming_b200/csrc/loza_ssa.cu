@@ -527,12 +527,33 @@ unsigned stream_grid(int64_t n) {
   return (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + per - 1) / per, cap));
 }
 
-// Hierarchical index (page 4): workspace of loza_hi_select / loza_hi_decode.
+// Hierarchical index (page 4): the window part and the selected tokens are
+// packed per sequence (hi_gather_kernel) and attended by the absorbed decode
+// with the unbounded window: every packed row is visible.
+constexpr int64_t kHiMaxWindowRows = 65536;  // rows of a bounded window the packed block holds at most
+
+loza_ssa_params hi_packed_params(float scale) {
+  loza_ssa_params q;
+  q.block_size = kTile;
+  q.n_sink = 0;
+  q.n_local = LOZA_UNBOUNDED;
+  q.scale = scale;
+  return q;
+}
+
+bool hi_window_ok(const loza_ssa_params& p) {
+  if (!window_ok(p)) return false;
+  return p.n_local == LOZA_UNBOUNDED ||
+         ((int64_t)p.n_sink + p.n_local) * p.block_size <= kHiMaxWindowRows;
+}
+
 struct HiWorkspace {
-  size_t sel_pages, n_pages, tok_keys, selected, o_win, l_win, dec, total;
+  size_t page_scored, sel_pages, n_pages, hist1, tok_keys, selected, n_sel, counts, packed, dec, total;
+  int cap_rows;  // packed rows per sequence (0: the unbounded window, decoded in place)
 };
 size_t hi_align(size_t x) { return (x + 255) / 256 * 256; }
-HiWorkspace hi_workspace(int32_t batch, int32_t top_pages, int32_t top_k, size_t decode_ws) {
+HiWorkspace hi_workspace(int32_t batch, int32_t max_seqlen, int32_t top_pages, int32_t top_k,
+                         const loza_ssa_params& p) {
   HiWorkspace w;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -540,13 +561,25 @@ HiWorkspace hi_workspace(int32_t batch, int32_t top_pages, int32_t top_k, size_t
     off = hi_align(off + bytes);
     return at;
   };
+  const int64_t pages = std::max<int64_t>(max_seqlen / kHiPage, 1);
+  w.page_scored = take((size_t)batch * pages * 8);
   w.sel_pages = take((size_t)batch * top_pages * 4);
   w.n_pages = take((size_t)batch * 4);
+  w.hist1 = take((size_t)batch * kHiBins * 4);
   w.tok_keys = take((size_t)batch * top_pages * kHiPage * 8);
   w.selected = take((size_t)batch * std::max(top_k, 1) * 4);
-  w.o_win = take((size_t)batch * kDecHeads * 512 * 4);  // fp32: rounded once, after the merge
-  w.l_win = take((size_t)batch * kDecHeads * 4);
-  w.dec = take(decode_ws);
+  w.n_sel = take((size_t)batch * 4);
+  w.counts = take((size_t)batch * 4);
+  if (p.n_local == LOZA_UNBOUNDED) {
+    w.cap_rows = 0;
+    w.packed = take(0);
+    w.dec = take(decode_workspace(batch, decode_plan(p, max_seqlen, batch)).total);
+  } else {
+    const int64_t rows = std::min<int64_t>(max_seqlen, ((int64_t)p.n_sink + p.n_local) * p.block_size + top_k);
+    w.cap_rows = (int)((rows + kTile - 1) / kTile * kTile);
+    w.packed = take((size_t)batch * w.cap_rows * 576 * 2);
+    w.dec = take(decode_workspace(batch, decode_plan(hi_packed_params(p.scale), w.cap_rows, batch)).total);
+  }
   w.total = off;
   return w;
 }
@@ -555,11 +588,26 @@ bool hi_args_ok(const void* k_index, int64_t index_batch_stride, int64_t index_r
                 int32_t max_seqlen, int32_t d_index) {
   if (!k_index || !aligned16(k_index)) return false;
   if (batch < 1 || batch > 65535 || max_seqlen < 1) return false;
-  if (d_index < 8 || d_index > kHiMaxDim || d_index % 8 != 0) return false;
+  if (d_index < kHiDimStep || d_index > kHiMaxDim || d_index % kHiDimStep != 0) return false;
   if (!stride_ok(index_row_stride) || !stride_ok(index_batch_stride) || index_row_stride < d_index ||
       index_batch_stride < (int64_t)max_seqlen * index_row_stride)
     return false;
   return true;
+}
+
+// Index keys as a 3-D tensor {d, rows, batch}: 128-row x 64-column tiles with
+// the 128-byte swizzle.
+bool make_map_index(CUtensorMap* m, const void* k_index, int32_t d, int32_t rows, int32_t batch,
+                    int64_t row_stride, int64_t batch_stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)batch_stride * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kHiDimStep, (cuuint32_t)kHiPage, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_index), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -1066,27 +1114,27 @@ loza_status loza_hi_page_keys(const void* k_index, int64_t index_batch_stride, i
     return LOZA_ERR_INVALID_ARG;
   const int64_t pages = max_seqlen / kHiPage;
   if (pages < 1) return LOZA_OK;
-  const int64_t per_seq = pages * d_index;
-  const unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((per_seq + 255) / 256, 4 * sm_count()));
-  hi_page_keys_kernel<<<dim3(gx, batch), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(k_index), index_batch_stride, index_row_stride, seqlens, d_index, pages,
-      page_keys);
+  hi_page_keys_kernel<<<dim3((unsigned)((pages + 31) / 32), d_index / 64, batch), 256, 0,
+                        reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(k_index),
+                                                                  index_batch_stride, index_row_stride, seqlens,
+                                                                  d_index, pages, page_keys);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
 size_t loza_hi_workspace_size(int32_t batch, int32_t max_seqlen, int32_t top_pages, int32_t top_k,
                               loza_ssa_params p) {
-  if (batch < 1 || max_seqlen < 1 || top_pages < 1 || top_k < 0 || top_k > kHiMaxTopK || !window_ok(p)) return 0;
-  const size_t dec = decode_workspace(batch, decode_plan(p, max_seqlen, batch)).total;
-  return hi_workspace(batch, top_pages, top_k, dec).total;
+  if (batch < 1 || batch > 65535 || max_seqlen < 1 || top_pages < 1 || top_k < 0 || top_k > kHiMaxTopK ||
+      !hi_window_ok(p))
+    return 0;
+  return hi_workspace(batch, max_seqlen, top_pages, top_k, p).total;
 }
 
 }  // extern "C"
 
 namespace loza {
 namespace {
-// Validate and enqueue the selection; `w` is the workspace layout.
+// Enqueue the selection (validated by the caller) into `selected`.
 loza_status hi_select_launch(const void* q_index, const void* k_index, int64_t index_batch_stride,
                              int64_t index_row_stride, const float* page_keys, const int32_t* seqlens,
                              int32_t batch, int32_t max_seqlen, int32_t d_index, const loza_ssa_params& p,
@@ -1094,49 +1142,77 @@ loza_status hi_select_launch(const void* q_index, const void* k_index, int64_t i
                              cudaStream_t st) {
   HiParams hp;
   std::memset(&hp, 0, sizeof(hp));
+  if (!make_map_index(&hp.tm_index, k_index, d_index, max_seqlen, batch, index_row_stride, index_batch_stride))
+    return LOZA_ERR_CUDA;
   hp.q_index = static_cast<const __nv_bfloat16*>(q_index);
-  hp.k_index = static_cast<const __nv_bfloat16*>(k_index);
-  hp.batch_stride = index_batch_stride;
-  hp.row_stride = index_row_stride;
   hp.page_keys = page_keys;
   hp.pages_per_seq = max_seqlen / kHiPage;
   hp.seqlens = seqlens;
+  hp.batch = batch;
   hp.d = d_index;
   hp.block = p.block_size;
   hp.n_sink = p.n_local == LOZA_UNBOUNDED ? 0 : p.n_sink;
   hp.n_local = p.n_local == LOZA_UNBOUNDED ? -1 : p.n_local;
   hp.top_pages = top_pages;
   hp.top_k = top_k;
+  hp.page_scored = reinterpret_cast<unsigned long long*>(ws + w.page_scored);
   hp.sel_pages = reinterpret_cast<int32_t*>(ws + w.sel_pages);
   hp.n_pages = reinterpret_cast<int32_t*>(ws + w.n_pages);
+  hp.hist1 = reinterpret_cast<int32_t*>(ws + w.hist1);
   hp.tok_keys = reinterpret_cast<unsigned long long*>(ws + w.tok_keys);
   hp.selected = selected;
-  int npow2 = 1;
-  while (npow2 < hp.pages_per_seq) npow2 <<= 1;
-  const int smem = npow2 * 8;
-  if (cudaFuncSetAttribute(hi_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  hp.n_sel = reinterpret_cast<int32_t*>(ws + w.n_sel);
+  if (cudaFuncSetAttribute(hi_tokens_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           HiTokLayout::SMEM_ALLOC) != cudaSuccess ||
+      cudaFuncSetAttribute(hi_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           HiTopkLayout::SMEM_BYTES) != cudaSuccess)
     return LOZA_ERR_CUDA;
-  hi_pages_kernel<<<batch, 1024, smem, st>>>(hp);
-  hi_tokens_kernel<<<dim3((top_pages + kHiTokPagesPerCta - 1) / kHiTokPagesPerCta, batch), kHiPage, 0, st>>>(hp);
-  hi_topk_kernel<<<batch, 1024, 0, st>>>(hp);
-  g_launches.fetch_add(3, std::memory_order_relaxed);
+  int launches = 3;
+  if (hp.pages_per_seq >= 1) {
+    hi_page_scores_kernel<<<dim3((unsigned)((hp.pages_per_seq + 255) / 256), batch), 256, 0, st>>>(hp);
+    ++launches;
+  }
+  hi_page_select_kernel<<<batch, 1024, 0, st>>>(hp);
+  const int64_t items = (int64_t)batch * ((top_pages + kHiTokPages - 1) / kHiTokPages);
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(items, 3 * (int64_t)sm_count()));
+  hi_tokens_kernel<<<grid, kHiTokThreads, HiTokLayout::SMEM_ALLOC, st>>>(hp);
+  hi_topk_kernel<<<batch, 1024, HiTopkLayout::SMEM_BYTES, st>>>(hp);
+  g_launches.fetch_add(launches, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
 
-loza_status hi_attend_launch(const void* q, const void* kv_cache, int64_t cache_batch_stride,
-                             int64_t cache_row_stride, const int32_t* selected, int32_t top_k, int32_t batch,
-                             float scale, const float* o_win, const float* lse_win, void* out, float* lse,
-                             cudaStream_t st) {
-  using LY = HiAttnLayout;
-  if (cudaFuncSetAttribute(hi_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM_BYTES) !=
-      cudaSuccess)
-    return LOZA_ERR_CUDA;
-  hi_attend_kernel<<<dim3(batch, kDecHeads / 8), 256, LY::SMEM_BYTES, st>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kv_cache), cache_batch_stride,
-      cache_row_stride, selected, top_k, scale * 1.4426950408889634f, o_win, lse_win,
-      static_cast<__nv_bfloat16*>(out), lse);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+// Validate the attention part of loza_ssa_decode_selected / loza_hi_decode and
+// prepare its decode: over the packed rows (bounded window) or over the cache
+// itself (unbounded window: the selection adds no token).
+loza_status hi_attend_setup(const void* q, const void* kv_cache, int64_t cache_batch_stride,
+                            int64_t cache_row_stride, const int32_t* seqlens, int32_t batch, int32_t max_seqlen,
+                            const loza_ssa_params& p, void* out, float* lse, uint8_t* ws, const HiWorkspace& w,
+                            DecodeParams* prm, DecodePlan* plan) {
+  // the cache and the outputs, as loza_ssa_decode checks them
+  loza_status rc = setup_decode_mla(q, kv_cache, nullptr, seqlens, batch, max_seqlen, cache_batch_stride,
+                                    cache_row_stride, kDecHeads, p, out, lse, prm, plan);
+  if (rc != LOZA_OK || w.cap_rows == 0) return rc;
+  return setup_decode_mla(q, ws + w.packed, nullptr, reinterpret_cast<const int32_t*>(ws + w.counts), batch,
+                          w.cap_rows, (int64_t)w.cap_rows * 576, 576, kDecHeads, hi_packed_params(p.scale), out,
+                          lse, prm, plan);
+}
+
+// Pack the window and the selection (list: compact, n_sel entries per
+// sequence) and run the decode prepared by hi_attend_setup.
+loza_status hi_attend_launch(const void* kv_cache, int64_t cache_batch_stride, int64_t cache_row_stride,
+                             const int32_t* seqlens, int32_t batch, const loza_ssa_params& p, const int32_t* list,
+                             int32_t top_k, uint8_t* ws, const HiWorkspace& w, DecodeParams& prm,
+                             const DecodePlan& plan, cudaStream_t st) {
+  if (w.cap_rows > 0) {
+    const SsaWindow win{p.block_size, p.n_sink * p.block_size, p.n_local};
+    hi_gather_kernel<<<dim3(w.cap_rows / 32, batch), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(kv_cache), cache_batch_stride, cache_row_stride, seqlens, win, list,
+        std::max(top_k, 1), reinterpret_cast<const int32_t*>(ws + w.n_sel), w.cap_rows,
+        reinterpret_cast<__nv_bfloat16*>(ws + w.packed), reinterpret_cast<int32_t*>(ws + w.counts));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (cudaGetLastError() != cudaSuccess) return LOZA_ERR_CUDA;
+  }
+  return launch_decode_mla(prm, plan, batch, ws + w.dec, st);
 }
 }  // namespace
 }  // namespace loza
@@ -1151,29 +1227,43 @@ loza_status loza_hi_select(const void* q_index, const void* k_index, int64_t ind
   if (!hi_args_ok(k_index, index_batch_stride, index_row_stride, batch, max_seqlen, d_index))
     return LOZA_ERR_INVALID_ARG;
   if (top_pages < 1 || top_k < 1 || top_k > kHiMaxTopK) return LOZA_ERR_INVALID_ARG;
-  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
-  if (max_seqlen / kHiPage > kHiMaxPages) return LOZA_ERR_UNSUPPORTED;
-  const size_t need = loza_hi_workspace_size(batch, max_seqlen, top_pages, top_k, p);
+  if (!hi_window_ok(p) || max_seqlen / kHiPage > kHiMaxPages) return LOZA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LOZA_ERR_INVALID_ARG;
-  if (workspace_bytes < need) return LOZA_ERR_WORKSPACE;
-  const HiWorkspace w = hi_workspace(batch, top_pages, top_k, 0);
+  const HiWorkspace w = hi_workspace(batch, max_seqlen, top_pages, top_k, p);
+  if (workspace_bytes < w.total) return LOZA_ERR_WORKSPACE;
   return hi_select_launch(q_index, k_index, index_batch_stride, index_row_stride, page_keys, seqlens, batch,
                           max_seqlen, d_index, p, top_pages, top_k, selected, static_cast<uint8_t*>(workspace), w,
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 loza_status loza_ssa_decode_selected(const void* q, const void* kv_cache, int64_t cache_batch_stride,
-                                     int64_t cache_row_stride, const int32_t* selected, int32_t top_k,
-                                     int32_t batch, int32_t n_heads, float scale, void* out, float* lse,
+                                     int64_t cache_row_stride, const int32_t* seqlens, int32_t batch,
+                                     int32_t max_seqlen, loza_ssa_params p, const int32_t* selected, int32_t top_k,
+                                     void* out, float* lse, void* workspace, size_t workspace_bytes,
                                      loza_stream_t stream) {
-  if (!q || !kv_cache || !selected || !out || !lse) return LOZA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out)) return LOZA_ERR_INVALID_ARG;
-  if (batch < 1 || batch > 65535 || top_k < 0) return LOZA_ERR_INVALID_ARG;
-  if (!stride_ok(cache_row_stride) || !stride_ok(cache_batch_stride) || cache_row_stride < 576)
-    return LOZA_ERR_INVALID_ARG;
-  if (n_heads != kDecHeads) return LOZA_ERR_UNSUPPORTED;
-  return hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, selected, top_k, batch, scale, nullptr,
-                          nullptr, out, lse, reinterpret_cast<cudaStream_t>(stream));
+  if (top_k < 0 || top_k > kHiMaxTopK || (top_k > 0 && !selected)) return LOZA_ERR_INVALID_ARG;
+  if (!hi_window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (batch < 1 || batch > 65535 || max_seqlen < 1) return LOZA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LOZA_ERR_INVALID_ARG;
+  const HiWorkspace w = hi_workspace(batch, max_seqlen, 1, top_k, p);
+  if (workspace_bytes < w.total) return LOZA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeParams prm;
+  DecodePlan plan;
+  loza_status rc = hi_attend_setup(q, kv_cache, cache_batch_stride, cache_row_stride, seqlens, batch, max_seqlen,
+                                   p, out, lse, ws, w, &prm, &plan);
+  if (rc != LOZA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* list = reinterpret_cast<int32_t*>(ws + w.selected);
+  if (w.cap_rows > 0) {
+    const SsaWindow win{p.block_size, p.n_sink * p.block_size, p.n_local};
+    hi_compact_kernel<<<batch, 1024, 0, st>>>(selected, top_k, seqlens, win, list,
+                                               reinterpret_cast<int32_t*>(ws + w.n_sel));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (cudaGetLastError() != cudaSuccess) return LOZA_ERR_CUDA;
+  }
+  return hi_attend_launch(kv_cache, cache_batch_stride, cache_row_stride, seqlens, batch, p, list, top_k, ws, w,
+                          prm, plan, st);
 }
 
 loza_status loza_hi_decode(const void* q, const void* kv_cache, int64_t cache_batch_stride, int64_t cache_row_stride,
@@ -1185,32 +1275,25 @@ loza_status loza_hi_decode(const void* q, const void* kv_cache, int64_t cache_ba
   if (!hi_args_ok(k_index, index_batch_stride, index_row_stride, batch, max_seqlen, d_index))
     return LOZA_ERR_INVALID_ARG;
   if (top_pages < 1 || top_k < 1 || top_k > kHiMaxTopK) return LOZA_ERR_INVALID_ARG;
-  if (max_seqlen / kHiPage > kHiMaxPages || !window_ok(p)) return LOZA_ERR_UNSUPPORTED;
+  if (max_seqlen / kHiPage > kHiMaxPages || !hi_window_ok(p)) return LOZA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LOZA_ERR_INVALID_ARG;
-  if (workspace_bytes < loza_hi_workspace_size(batch, max_seqlen, top_pages, top_k, p)) return LOZA_ERR_WORKSPACE;
-  // the window part: validation and the decode plan as for loza_ssa_decode
+  const HiWorkspace w = hi_workspace(batch, max_seqlen, top_pages, top_k, p);
+  if (workspace_bytes < w.total) return LOZA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeParams prm;
   DecodePlan plan;
-  const loza_status rc = setup_decode_mla(q, kv_cache, nullptr, seqlens, batch, max_seqlen, cache_batch_stride,
-                                          cache_row_stride, kDecHeads, p, out, lse, &prm, &plan);
+  loza_status rc = hi_attend_setup(q, kv_cache, cache_batch_stride, cache_row_stride, seqlens, batch, max_seqlen,
+                                   p, out, lse, ws, w, &prm, &plan);
   if (rc != LOZA_OK) return rc;
-  const HiWorkspace w = hi_workspace(batch, top_pages, top_k, decode_workspace(batch, plan).total);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int32_t* sel = reinterpret_cast<int32_t*>(ws + w.selected);
-  loza_status r = hi_select_launch(q_index, k_index, index_batch_stride, index_row_stride, page_keys, seqlens,
-                                   batch, max_seqlen, d_index, p, top_pages, top_k, sel, ws, w, st);
-  if (r != LOZA_OK) return r;
-  // the window part in fp32, then the selected part, merged by log-sum-exp in
-  // the attention kernel's epilogue (one bf16 rounding of the result)
-  float* o_win = reinterpret_cast<float*>(ws + w.o_win);
-  float* l_win = reinterpret_cast<float*>(ws + w.l_win);
-  prm.out_f32 = o_win;
-  prm.lse = l_win;
-  r = launch_decode_mla(prm, plan, batch, ws + w.dec, st);
-  if (r != LOZA_OK) return r;
-  return hi_attend_launch(q, kv_cache, cache_batch_stride, cache_row_stride, sel, top_k, batch, p.scale, o_win, l_win,
-                          out, lse, st);
+  if (w.cap_rows > 0) {  // an unbounded window leaves no token to select
+    rc = hi_select_launch(q_index, k_index, index_batch_stride, index_row_stride, page_keys, seqlens, batch,
+                          max_seqlen, d_index, p, top_pages, top_k, sel, ws, w, st);
+    if (rc != LOZA_OK) return rc;
+  }
+  return hi_attend_launch(kv_cache, cache_batch_stride, cache_row_stride, seqlens, batch, p, sel, top_k, ws, w, prm,
+                          plan, st);
 }
 
 loza_status loza_ssa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -222,7 +222,8 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  * selects those in two stages, top pages of 128 tokens first, then top tokens
  * within them). The fixed part is the SSA window `p` of this library; the
  * dynamic part is chosen among the tokens outside it, so the parts are
- * disjoint, and the two are merged by their log-sum-exp.
+ * disjoint, and the query attends to both at once (one softmax over their
+ * union, the same as merging the two parts by their log-sum-exp).
  * Scoring (the pages give none): the dot product of the sequence's index
  * query with a token's index key, both supplied by the caller (as an indexer
  * produces them); a page is scored by the mean of its 128 index keys. Scores
@@ -231,12 +232,17 @@ loza_status loza_ssa_decode(const void *q, const void *k_cache, const void *v_ca
  * Common arguments:
  *   k_index   index keys: token t of sequence n at k_index + n *
  *             index_batch_stride + t * index_row_stride elements, d_index bf16
- *             each (d_index a multiple of 8, at most 512; strides * 2 multiples
- *             of 16; index_batch_stride >= max_seqlen * index_row_stride)
- *   q_index   [batch, d_index] bf16, one index query per sequence
- *   page_keys [batch, max_seqlen / 128, d_index] fp32 (from loza_hi_page_keys)
+ *             each (d_index a multiple of 64, at most 512; 16-byte aligned;
+ *             strides * 2 multiples of 16; index_batch_stride >= max_seqlen *
+ *             index_row_stride)
+ *   q_index   [batch, d_index] bf16 contiguous, one index query per sequence
+ *   page_keys [batch, d_index, max_seqlen / 128] fp32, the page dimension
+ *             innermost (from loza_hi_page_keys)
  *   seqlens   device int32 [batch], 1 <= seqlens[n] <= max_seqlen; the decode
  *             query is position seqlens[n] - 1, as in loza_ssa_decode
+ *   p         the window: as loza_ssa_decode's, with at most 65,536 rows
+ *             ((n_sink + n_local) * block_size); LOZA_UNBOUNDED leaves no
+ *             token outside the window, so nothing is selected
  * Limits: max_seqlen / 128 <= 8192 pages; 1 <= top_k <= 2048; top_pages >= 1.
  *
  * loza_hi_page_keys: the mean index key of every whole page (tokens 128p ..
@@ -249,7 +255,8 @@ loza_status loza_hi_page_keys(const void *k_index, int64_t index_batch_stride, i
                               float *page_keys, loza_stream_t stream);
 
 /* Bytes of device workspace loza_hi_select and loza_hi_decode need (0 for an
- * unsupported request). */
+ * unsupported request); loza_ssa_decode_selected needs the size for
+ * top_pages = 1. */
 size_t loza_hi_workspace_size(int32_t batch, int32_t max_seqlen, int32_t top_pages, int32_t top_k,
                               loza_ssa_params p);
 
@@ -267,26 +274,31 @@ loza_status loza_hi_select(const void *q_index, const void *k_index, int64_t ind
                            int32_t *selected, void *workspace, size_t workspace_bytes, loza_stream_t stream);
 
 /*
- * Softmax attention of each sequence's decode query over an explicit list of
- * its tokens (absorbed MLA: 64 heads, the 576-wide latent row as K, its first
- * 512 columns as V): out [batch, 64, 512] bf16, lse [batch, 64] fp32 (natural
- * log; -inf and O = 0 when a sequence has no token). selected: device int32
- * [batch, top_k], entries < 0 ignored; every other entry must name a row the
- * cache holds for its sequence (not checked: the call has no sequence
- * lengths). q is [batch, 64, 576] contiguous and the cache layout is
- * loza_ssa_decode's.
+ * Softmax attention of each sequence's decode query (position seqlens[n] - 1)
+ * over its window p and the tokens of a given selection (absorbed MLA: 64
+ * heads, the 576-wide latent row as K, its first 512 columns as V): out
+ * [batch, 64, 512] bf16, lse [batch, 64] fp32 (natural log). q [batch, 64,
+ * 576] bf16 contiguous; the cache layout is loza_ssa_decode's.
+ *   selected  device int32 [batch, top_k] (0 <= top_k <= 2048): entries that
+ *             name a token before the query and outside the window are
+ *             attended, every other entry (negative, past the query, inside
+ *             the window) is ignored; the entries must be distinct
+ *   workspace loza_hi_workspace_size(batch, max_seqlen, 1, top_k, p) bytes,
+ *             256-byte aligned
+ * The window rows and the selected rows are packed per sequence in the
+ * workspace and attended by the tensor-core decode.
  */
 loza_status loza_ssa_decode_selected(const void *q, const void *kv_cache, int64_t cache_batch_stride,
-                                     int64_t cache_row_stride, const int32_t *selected, int32_t top_k,
-                                     int32_t batch, int32_t n_heads, float scale, void *out, float *lse,
+                                     int64_t cache_row_stride, const int32_t *seqlens, int32_t batch,
+                                     int32_t max_seqlen, loza_ssa_params p, const int32_t *selected, int32_t top_k,
+                                     void *out, float *lse, void *workspace, size_t workspace_bytes,
                                      loza_stream_t stream);
 
 /*
- * The whole decode: loza_hi_select, then loza_ssa_decode over the window p
- * (its O kept in fp32 in the workspace), then the attention over the
- * selection, whose epilogue merges the two parts by their log-sum-exp into
- * out [batch, 64, 512] bf16 and lse [batch, 64] (one rounding to bf16). Same
- * cache arguments as loza_ssa_decode (absorbed MLA, 64 heads, 576 / 512).
+ * The whole decode: loza_hi_select, then loza_ssa_decode_selected over the
+ * window p and that selection, into out [batch, 64, 512] bf16 and lse
+ * [batch, 64]. Same cache arguments as loza_ssa_decode (absorbed MLA, 64
+ * heads, 576 / 512).
  *   workspace loza_hi_workspace_size(...) bytes, 256-byte aligned
  */
 loza_status loza_hi_decode(const void *q, const void *kv_cache, int64_t cache_batch_stride, int64_t cache_row_stride,

@@ -27,7 +27,8 @@ def _index(**over):
 @pytest.mark.parametrize("over", [
     dict(k=0), dict(k=(1 << 21) + 8),          # null / misaligned index keys
     dict(seqlens=0),
-    dict(d=12, rs=12, bs=4096 * 12),            # d_index not a multiple of 8
+    dict(d=12, rs=12, bs=4096 * 12),            # d_index not a multiple of 64
+    dict(d=32, rs=32, bs=4096 * 32),
     dict(d=520, rs=520, bs=4096 * 520),         # d_index above 512
     dict(d=0),
     dict(rs=32),                                # row stride below d_index
@@ -56,6 +57,8 @@ def test_workspace_size():
     assert size(4, 1 << 20, 0, 1024, p) == 0         # no page recalled
     assert size(0, 1 << 20, 1024, 1024, p) == 0
     assert size(4, 1 << 20, 1024, 1024, bss.Params(0.07, block_size=3)) == 0
+    assert size(4, 1 << 20, 1024, 1024, bss.Params(0.07, block_size=128, n_sink=1, n_local=512)) == 0  # window > 64K rows
+    assert size(4, 1 << 20, 1024, 1024, bss.Params(0.07, block_size=128, n_sink=1, n_local=-1)) > 0   # unbounded
 
 
 def _select(L, ws_bytes=1 << 30, ws=1 << 24, top_pages=16, top_k=256, params=None, q_index=1 << 20, **over):
@@ -84,18 +87,22 @@ def test_select_rejects_before_launch(L, kw, code):
     assert L.loza_launch_count() == count
 
 
-@pytest.mark.parametrize("q,kv,rs,top_k,heads,code", [
-    (0, 1 << 21, 576, 64, 64, INVALID),
-    (1 << 20, (1 << 21) + 2, 576, 64, 64, INVALID),
-    (1 << 20, 1 << 21, 512, 64, 64, INVALID),     # latent row narrower than 576
-    (1 << 20, 1 << 21, 580, 64, 64, INVALID),     # row stride not 16-byte
-    (1 << 20, 1 << 21, 576, -1, 64, INVALID),
-    (1 << 20, 1 << 21, 576, 64, 32, UNSUPPORTED),  # absorbed decode has 64 heads
+@pytest.mark.parametrize("q,kv,rs,top_k,sel,params,ws_bytes,code", [
+    (0, 1 << 21, 576, 64, 1 << 22, None, 1 << 30, INVALID),
+    (1 << 20, (1 << 21) + 2, 576, 64, 1 << 22, None, 1 << 30, INVALID),
+    (1 << 20, 1 << 21, 512, 64, 1 << 22, None, 1 << 30, INVALID),     # latent row narrower than 576
+    (1 << 20, 1 << 21, 580, 64, 1 << 22, None, 1 << 30, INVALID),     # row stride not 16-byte
+    (1 << 20, 1 << 21, 576, -1, 1 << 22, None, 1 << 30, INVALID),
+    (1 << 20, 1 << 21, 576, 2049, 1 << 22, None, 1 << 30, INVALID),
+    (1 << 20, 1 << 21, 576, 64, 0, None, 1 << 30, INVALID),           # no list
+    (1 << 20, 1 << 21, 576, 64, 1 << 22, bss.Params(0.07, block_size=6), 1 << 30, UNSUPPORTED),
+    (1 << 20, 1 << 21, 576, 64, 1 << 22, None, 4096, WORKSPACE),
 ])
-def test_decode_selected_rejects_before_launch(L, q, kv, rs, top_k, heads, code):
+def test_decode_selected_rejects_before_launch(L, q, kv, rs, top_k, sel, params, ws_bytes, code):
+    p = params or bss.Params(0.07, block_size=1, n_sink=16, n_local=1024)
     count = L.loza_launch_count()
-    rc = L.loza_ssa_decode_selected(vp(q), vp(kv), 4096 * 576, rs, vp(1 << 22), top_k, 2, heads, 0.07, vp(1 << 23),
-                                    vp(1 << 24), vp(0))
+    rc = L.loza_ssa_decode_selected(vp(q), vp(kv), 4096 * rs, rs, vp(1 << 23), 2, 4096, p, vp(sel), top_k,
+                                    vp(1 << 24), vp(1 << 25), vp(1 << 26), ws_bytes, vp(0))
     assert rc == code
     assert L.loza_launch_count() == count
 

@@ -51,7 +51,13 @@ def window_tile_rows(L, win, tile=128):
 
 
 def index_inputs(g, B, Lcap, d, ints=False):
-    if ints:  # small integers: exact scores with many ties
+    """Index queries and keys: N(0, 1) in bf16; small integers (ints=True:
+    exact scores, many ties); or 0/1 keys against an all-ones query
+    (ints="binary": scores crowd into a few values)."""
+    if ints == "binary":
+        ones = np.full((B, d), 0x3F80, np.uint16)
+        return ones, synth.bf16_bits(g.integers(0, 2, size=(B, Lcap, d)).astype(np.float32))
+    if ints:
         draw = lambda shape: synth.bf16_bits(g.integers(-3, 4, size=shape).astype(np.float32))
     else:
         draw = lambda shape: synth.normal_bits(g, shape)
@@ -74,25 +80,26 @@ def test_page_keys_bit_exact(bss, oracle_mod):
     lens = [5000, 129, 100, 128, 4096]
     q_idx, k_idx = index_inputs(g, len(lens), 5120, 64)
     pk, _ = gpu_select(bss, q_idx, k_idx, lens, 5120, TOKEN_WINDOW, 4, 16)
-    ref = oracle_mod.hi_page_keys(k_idx, lens)
+    ref = oracle_mod.hi_page_keys(k_idx, lens)          # [B, pages, d]; the library's is [B, d, pages]
     for n, L in enumerate(lens):
-        np.testing.assert_array_equal(pk[n, :L // 128], ref[n, :L // 128])
+        np.testing.assert_array_equal(pk[n, :, :L // 128].T, ref[n, :L // 128])
 
 
 SELECT_CASES = [
     # (window, top_pages, top_k, d, integer keys)
     (TOKEN_WINDOW, 8, 500, 64, False),
     (TOKEN_WINDOW, 1024, 1024, 128, False),   # page 4's budget: 1,024 pages and 1,024 tokens
-    ((128, 1, 7), 64, 2048, 32, False),       # the SSA block window; the largest top_k
-    ((64, 2, 3), 3, 100, 8, False),           # fewer tokens kept than the pages hold
-    ((1, 0, 50), 10 ** 4, 7, 16, False),      # more pages asked than exist
-    (TOKEN_WINDOW, 6, 300, 16, True),         # many equal scores: ties go to the lower index
+    ((128, 1, 7), 64, 2048, 64, False),       # the SSA block window; the largest top_k
+    ((64, 2, 3), 3, 100, 192, False),         # fewer tokens kept than the pages hold
+    ((1, 0, 50), 10 ** 4, 7, 64, False),      # more pages asked than exist
+    (TOKEN_WINDOW, 6, 300, 64, True),         # many equal scores: ties go to the lower index
+    (TOKEN_WINDOW, 150, 2000, 64, "binary"),  # more than 4,096 keys share the threshold's top digit
     ((128, 1, 7), 40, 1500, 512, False),      # the widest index key
 ]
 
 
 @pytest.mark.parametrize("win,top_pages,top_k,d,ints", SELECT_CASES,
-                         ids=[f"w{c[0][0]}-{c[0][1]}-{c[0][2]}-p{c[1]}-k{c[2]}-d{c[3]}{'-int' if c[4] else ''}"
+                         ids=[f"w{c[0][0]}-{c[0][1]}-{c[0][2]}-p{c[1]}-k{c[2]}-d{c[3]}{'-' + str(c[4]) if c[4] else ''}"
                               for c in SELECT_CASES])
 def test_selection_is_the_oracles(bss, oracle_mod, win, top_pages, top_k, d, ints):
     g = synth.rng(910 + top_k + d)
@@ -122,14 +129,30 @@ def test_unbounded_window_selects_nothing(bss):
     """With full causal attention as the window no token lies outside it."""
     g = synth.rng(921)
     lens = [5000, 300]
-    q_idx, k_idx = index_inputs(g, 2, 5000, 32)
+    q_idx, k_idx = index_inputs(g, 2, 5000, 64)
     _, sel = gpu_select(bss, q_idx, k_idx, lens, 5000, (128, 1, -1), 4, 64)
     assert (sel == -1).all()
 
 
+def filled_cache(g, lens, Lcap, win, extra_rows, poison=True):
+    """Latent cache [B, Lcap, 1, 576]: the rows of the tiles the window reads
+    and the rows in extra_rows[n] carry seeded values, every other row is NaN
+    (or zero); returns the device cache and its host copy."""
+    import torch
+    B = len(lens)
+    cache = torch.full((B, Lcap, 1, D), float("nan") if poison else 0.0, dtype=torch.bfloat16, device="cuda")
+    host = np.empty((B, Lcap, 1, D), np.uint16)
+    for n, L in enumerate(lens):
+        rows = np.union1d(window_tile_rows(L, win), extra_rows[n])
+        vals = synth.normal_bits(g, (len(rows), 1, D))
+        host[n, rows] = vals
+        cache[n, torch.from_numpy(rows).cuda()] = to_dev(vals)
+    return cache, host
+
+
 def attention_case(bss, oracle_mod, seed, lens, Lcap, win, top_pages, top_k, d_index=64, poison=True):
-    """The whole decode on the GPU against the oracle; also the two parts apart
-    (the selected part through loza_ssa_decode_selected)."""
+    """The whole decode on the GPU against the oracle, and the same selection
+    through loza_ssa_decode_selected."""
     import torch
     B = len(lens)
     g = synth.rng(seed)
@@ -137,13 +160,7 @@ def attention_case(bss, oracle_mod, seed, lens, Lcap, win, top_pages, top_k, d_i
     ref_sel = oracle_mod.hi_select(q_idx, k_idx, oracle_mod.hi_page_keys(k_idx, lens), lens, *win, top_pages,
                                    top_k)
     q = synth.normal_bits(g, (B, H, D))
-    cache = torch.full((B, Lcap, 1, D), float("nan") if poison else 0.0, dtype=torch.bfloat16, device="cuda")
-    host = np.empty((B, Lcap, 1, D), np.uint16)
-    for n, L in enumerate(lens):
-        rows = np.union1d(window_tile_rows(L, win), ref_sel[n][ref_sel[n] >= 0])
-        vals = synth.normal_bits(g, (len(rows), 1, D))
-        host[n, rows] = vals
-        cache[n, torch.from_numpy(rows).cuda()] = to_dev(vals)
+    cache, host = filled_cache(g, lens, Lcap, win, [r[r >= 0] for r in ref_sel], poison)
     scale = 1.0 / math.sqrt(192.0)
     p = bss.Params(scale, *win)
     seq = dev_i32(lens)
@@ -151,20 +168,15 @@ def attention_case(bss, oracle_mod, seed, lens, Lcap, win, top_pages, top_k, d_i
     pk = bss.loza_hi_page_keys(k_dev, seq, Lcap)
     q_dev = to_dev(q)
     out, lse = bss.loza_hi_decode(q_dev, cache, to_dev(q_idx), k_dev, pk, seq, Lcap, p, top_pages, top_k)
-    # the selected part alone, from the oracle's selection
-    o_s, l_s = bss.loza_ssa_decode_selected(q_dev, cache, dev_i32(ref_sel), scale)
+    o_s, l_s = bss.loza_ssa_decode_selected(q_dev, cache, seq, Lcap, p, dev_i32(ref_sel))
     torch.cuda.synchronize()
     assert bss.device_status() == 0
     o_ref, lse_ref = oracle_mod.hi_decode(q, host, lens, H, *win, scale, ref_sel)
-    assert_close_o(from_dev(out), o_ref, f"HI decode O {win} p{top_pages} k{top_k}")
-    assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, f"HI decode LSE {win} p{top_pages} k{top_k}")
-    # an empty window (no sinks, no local keys) leaves the selection alone
-    has = (ref_sel >= 0).any(axis=1)
-    o_sr, l_sr = oracle_mod.hi_decode(q[has], host[has], np.asarray(lens)[has], H, 1, 0, 0, scale, ref_sel[has])
-    assert_close_o(from_dev(o_s)[has], o_sr, f"selected part O {win}")
-    assert_close_lse(l_s.cpu().numpy().astype(np.float64)[has], l_sr, f"selected part LSE {win}")
-    empty_l = l_s.cpu().numpy()[~has]
-    assert np.all(empty_l == -np.inf) and not from_dev(o_s)[~has].any()
+    tag = f"{win} p{top_pages} k{top_k}"
+    assert_close_o(from_dev(out), o_ref, f"HI decode O {tag}")
+    assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, f"HI decode LSE {tag}")
+    # the same computation from the oracle's selection: bit for bit the same
+    assert torch.equal(out, o_s) and torch.equal(lse, l_s)
     res = (out.clone(), lse.clone())
     del cache
     return res
@@ -184,6 +196,59 @@ def test_hi_decode_batches_and_budgets(bss, oracle_mod):
     lens = g.integers(1, 9000, size=40).tolist()
     attention_case(bss, oracle_mod, 932, lens, 9216, TOKEN_WINDOW, 4, 64)
     attention_case(bss, oracle_mod, 933, [40000], 40960, TOKEN_WINDOW, 1024, 1024)
+
+
+def test_decode_selected_with_a_caller_list(bss, oracle_mod):
+    """A caller's own list: unsorted, with -1 holes and entries that the call
+    must ignore (inside the window, past the query); the rest is attended with
+    the window."""
+    import torch
+    g = synth.rng(935)
+    lens, Lcap, win = [6000, 3000, 1200, 40], 6144, TOKEN_WINDOW
+    B, top_k = len(lens), 700
+    lists = np.full((B, top_k), -1, np.int32)
+    kept = []
+    for n, L in enumerate(lens):
+        outside = np.array([t for t in range(L) if t >= 16 and t < max(0, L - 1024)], np.int64)
+        take = g.choice(outside, size=min(len(outside), 500), replace=False) if len(outside) else outside
+        ignored = np.concatenate([np.arange(0, min(16, L)), np.arange(max(0, L - 5), L), L + np.arange(3)])
+        entries = np.concatenate([take, ignored])
+        slots = g.choice(top_k, size=len(entries), replace=False)
+        lists[n, slots] = entries
+        kept.append(np.sort(take).astype(np.int32))
+    q = synth.normal_bits(g, (B, H, D))
+    cache, host = filled_cache(g, lens, Lcap, win, kept)
+    scale = 1.0 / math.sqrt(192.0)
+    out, lse = bss.loza_ssa_decode_selected(to_dev(q), cache, dev_i32(lens), Lcap, bss.Params(scale, *win),
+                                            dev_i32(lists))
+    torch.cuda.synchronize()
+    assert bss.device_status() == 0
+    ref_list = np.full((B, top_k), -1, np.int32)
+    for n, k in enumerate(kept):
+        ref_list[n, :len(k)] = k
+    o_ref, lse_ref = oracle_mod.hi_decode(q, host, lens, H, *win, scale, ref_list)
+    assert_close_o(from_dev(out), o_ref, "decode over a caller list O")
+    assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, "decode over a caller list LSE")
+
+
+def test_hi_decode_unbounded_window_is_full_attention(bss, oracle_mod):
+    import torch
+    g = synth.rng(936)
+    lens, Lcap = [3000, 129, 1], 3072
+    B = len(lens)
+    q_idx, k_idx = index_inputs(g, B, Lcap, 64)
+    q = synth.normal_bits(g, (B, H, D))
+    kv = synth.normal_bits(g, (B, Lcap, 1, D))
+    scale = 1.0 / math.sqrt(192.0)
+    seq = dev_i32(lens)
+    k_dev = to_dev(k_idx)
+    pk = bss.loza_hi_page_keys(k_dev, seq, Lcap)
+    out, lse = bss.loza_hi_decode(to_dev(q), to_dev(kv), to_dev(q_idx), k_dev, pk, seq, Lcap,
+                                  bss.Params(scale, 128, 1, -1), 8, 256)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle_mod.decode(q, kv, None, np.array(lens, np.int32), H, 1, 128, 0, -1, scale, d_v=512)
+    assert_close_o(from_dev(out), o_ref, "HI decode, unbounded window O")
+    assert_close_lse(lse.cpu().numpy().astype(np.float64), lse_ref, "HI decode, unbounded window LSE")
 
 
 def test_hi_decode_nan_bounds_bitwise(bss, oracle_mod):
@@ -216,19 +281,14 @@ def test_hi_decode_one_million_tokens(bss, oracle_mod):
     sel = bss.loza_hi_select(to_dev(q_idx), k_dev, pk, seq, Lcap, bss.Params(0.1, *TOKEN_WINDOW), top_pages, top_k)
     torch.cuda.synchronize()
     pk_ref = oracle_mod.hi_page_keys(k_idx, lens)
-    np.testing.assert_array_equal(pk.cpu().numpy()[0], pk_ref[0])
-    np.testing.assert_array_equal(pk.cpu().numpy()[1, :lens[1] // 128], pk_ref[1, :lens[1] // 128])
+    pk_h = pk.cpu().numpy()
+    np.testing.assert_array_equal(pk_h[0].T, pk_ref[0])
+    np.testing.assert_array_equal(pk_h[1, :, :lens[1] // 128].T, pk_ref[1, :lens[1] // 128])
     ref_sel = oracle_mod.hi_select(q_idx, k_idx, pk_ref, lens, *TOKEN_WINDOW, top_pages, top_k)
     np.testing.assert_array_equal(sel.cpu().numpy(), ref_sel)
     # the decode over window and selection, with every other cache row NaN
     q = synth.normal_bits(g, (B, H, D))
-    cache = torch.full((B, Lcap, 1, D), float("nan"), dtype=torch.bfloat16, device="cuda")
-    host = np.empty((B, Lcap, 1, D), np.uint16)
-    for n, L in enumerate(lens):
-        rows = np.union1d(window_tile_rows(L, TOKEN_WINDOW), ref_sel[n][ref_sel[n] >= 0])
-        vals = synth.normal_bits(g, (len(rows), 1, D))
-        host[n, rows] = vals
-        cache[n, torch.from_numpy(rows).cuda()] = to_dev(vals)
+    cache, host = filled_cache(g, lens, Lcap, TOKEN_WINDOW, [r[r >= 0] for r in ref_sel])
     scale = 1.0 / math.sqrt(192.0)
     out, lse = bss.loza_hi_decode(to_dev(q), cache, to_dev(q_idx), k_dev, pk, seq, Lcap,
                                   bss.Params(scale, *TOKEN_WINDOW), top_pages, top_k)
