@@ -24,13 +24,19 @@
 //   hi_page_keys_kernel     mean index key of every whole page (maintained as
 //                           the cache fills; not part of a decode step)
 //   hi_page_scores_kernel   a thread per page: its key (0 for a non-candidate)
-//   hi_page_select_kernel   a CTA per sequence: the top pages (radix select)
+//                           and a histogram of the keys' top digit
+//   hi_page_select_kernel   a CTA per sequence: the top pages (one pass over
+//                           the keys from that histogram, radix select among
+//                           the keys sharing the threshold's top digit)
 //   hi_tokens_kernel        persistent; the index keys of the recalled pages
 //                           arrive by TMA in 128-row x 64-column tiles and a
 //                           thread per token forms its score; writes the keys
 //                           and a histogram of their top digit per sequence
-//   hi_topk_kernel          a CTA per sequence: the top_k tokens, starting
-//                           from that histogram; sorted by position
+//   hi_topk_collect_kernel  many CTAs per sequence: from that histogram, the
+//                           keys at or above the threshold's top digit
+//   hi_topk_kernel          a CTA per sequence: the top_k tokens (radix
+//                           select among the threshold's digit), in order of
+//                           position through a bitmap
 //   hi_compact_kernel       (caller-given lists only) the valid entries
 //   hi_gather_kernel        the latent rows of the window and the selection,
 //                           packed per sequence for the tensor-core decode
@@ -52,7 +58,8 @@ constexpr int kHiDimStep = 64;      // the index dimension is a multiple of this
 constexpr int kHiBits = 11;         // radix digit
 constexpr int kHiBins = 1 << kHiBits;
 constexpr int kHiTopShift = 64 - kHiBits;  // the first digit: bits 53..63
-constexpr int kHiCand = 4096;       // keys sharing the threshold's first digit that the top-k sorts on chip
+constexpr int kHiCand = 4096;       // keys sharing the threshold's first digit that are sorted out on chip
+constexpr int kHiTiny = 64;         // a digit shared by at most this many keys is resolved by direct ranking
 
 struct HiParams {
   CUtensorMap tm_index;           // index keys {d, rows, batch}, box {64, 128, 1}, 128-byte swizzle
@@ -66,8 +73,13 @@ struct HiParams {
   unsigned long long* page_scored;  // [B, pages_per_seq] page keys, 0 = not a candidate
   int32_t* sel_pages;             // [B, top_pages] recalled pages (any order)
   int32_t* n_pages;               // [B] recalled page count
-  int32_t* hist1;                 // [B, kHiBins] top-digit histogram of the token keys
+  // zero on entry (one memset per call): histograms of top digits and list counters
+  int32_t* page_hist;             // [B, kHiBins] of the page keys
+  int32_t* hist1;                 // [B, kHiBins] of the token keys
+  int32_t* counters;              // [B, 4]: [3] the length of the sequence's tok_cand list
+  unsigned long long* page_cand;  // [B, pages_per_seq] page keys at or above the threshold's top digit
   unsigned long long* tok_keys;   // [B, top_pages * 128] token keys, 0 = none
+  unsigned long long* tok_cand;   // [B, top_pages * 128] token keys at or above the threshold's top digit
   int32_t* selected;              // [B, top_k] selected tokens, ascending, then -1
   int32_t* n_sel;                 // [B] selected count
 };
@@ -98,6 +110,7 @@ __device__ __forceinline__ SsaWindow hi_window(const HiParams& p) {
 // Add 1 to hist[bin] for every lane with bin >= 0, one shared-memory atomic
 // per distinct bin of the warp (scores crowd into few top digits). Whole warp.
 __device__ __forceinline__ void hi_hist_add(int* hist, int bin) {
+  if (!__any_sync(0xffffffffu, bin >= 0)) return;
   const unsigned peers = __match_any_sync(0xffffffffu, bin);
   if (bin >= 0 && (threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
 }
@@ -106,81 +119,140 @@ __device__ __forceinline__ void hi_hist_add(int* hist, int bin) {
 // Whole warp; returns the lane's slot (meaningless where !take).
 __device__ __forceinline__ int hi_warp_slot(int* counter, bool take) {
   const unsigned m = __ballot_sync(0xffffffffu, take);
+  if (!m) return 0;
   const int lane = threadIdx.x & 31;
-  const int leader = m ? __ffs(m) - 1 : 0;
+  const int leader = __ffs(m) - 1;
   int base = 0;
-  if (m && lane == leader) base = atomicAdd(counter, __popc(m));
+  if (lane == leader) base = atomicAdd(counter, __popc(m));
   base = __shfl_sync(0xffffffffu, base, leader);
   return base + __popc(m & ((1u << lane) - 1u));
 }
 
+// Warp 0 of a block (all 32 lanes): the bin of hist[0, kHiBins) holding the
+// rank-th largest element, counting from the top bin, the element's rank
+// within that bin and the bin's count, into sh[0] (rank), sh[1] (bin) and
+// sh[2] (count); sh is left as it was
+// if the counts hold fewer than rank elements. Lane j first sums bins
+// [64j, 64j + 64) (hist 16-byte aligned), a suffix scan over the lanes finds
+// the lane whose bins hold the rank, and its 64 bins, two per lane, are
+// resolved the same way.
+__device__ __forceinline__ void hi_find_bin(const int* hist, int rank, int* sh) {
+  const int lane = threadIdx.x & 31;
+  const int4* h4 = reinterpret_cast<const int4*>(hist + 64 * lane);
+  int own = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int4 v = h4[j];
+    own += v.x + v.y + v.z + v.w;
+  }
+  int above = 0;  // elements in the bins of the lanes above this one
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_down_sync(0xffffffffu, above + own, o);
+    if (lane + o < 32) above += x;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, above < rank && above + own >= rank);
+  if (!hit) return;
+  const int L = __ffs(hit) - 1;
+  const int r = rank - __shfl_sync(0xffffffffu, above, L);  // rank among lane L's bins
+  const int b0 = hist[64 * L + 2 * lane], b1 = hist[64 * L + 2 * lane + 1];
+  const int own2 = b0 + b1;
+  int above2 = 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_down_sync(0xffffffffu, above2 + own2, o);
+    if (lane + o < 32) above2 += x;
+  }
+  if (above2 < r && above2 + own2 >= r) {
+    const int rr = r - above2;  // the higher bin of the pair first
+    if (b1 >= rr) {
+      sh[0] = rr;
+      sh[1] = 64 * L + 2 * lane + 1;
+      sh[2] = b1;
+    } else {
+      sh[0] = rr - b1;
+      sh[1] = 64 * L + 2 * lane;
+      sh[2] = b0;
+    }
+  }
+}
+
+// Block-wide pass over keys[0, N): f(key) on every thread, the same number
+// of times on every lane (0 past the end), with kHiScanDepth loads in flight
+// per thread so that a pass over global memory is not one round trip per key.
+constexpr int kHiScanDepth = 8;
+template <typename F>
+__device__ __forceinline__ void hi_for_keys(const unsigned long long* keys, int64_t N, F&& f) {
+  const int64_t step = (int64_t)blockDim.x * kHiScanDepth;
+  for (int64_t base = 0; base < N; base += step) {
+    unsigned long long kk[kHiScanDepth];
+#pragma unroll
+    for (int j = 0; j < kHiScanDepth; ++j) {
+      const int64_t t = base + (int64_t)j * blockDim.x + threadIdx.x;
+      kk[j] = t < N ? keys[t] : 0ull;
+    }
+#pragma unroll
+    for (int j = 0; j < kHiScanDepth; ++j)
+      if (base + (int64_t)j * blockDim.x < N) f(kk[j]);  // block-uniform: rows past the end are skipped
+  }
+}
+
 // Block-wide: the rank-th largest non-zero key of keys[0, N) among those
 // equal to `prefix` on the bits `mask` already fixed, deciding the digits
-// from bit `shift` down (1 <= rank <= that count). `hist` holds kHiBins
-// ints, `sh` two ints.
+// from bit `shift` down (1 <= rank <= that count). Once the digits so far
+// leave at most kHiTiny keys, those are gathered and ranked directly. `hist`
+// holds kHiBins ints (16-byte aligned), `sh` four ints, `tiny` kHiTiny + 1
+// keys, all in shared memory.
 __device__ unsigned long long hi_radix_kth(const unsigned long long* keys, int64_t N, int rank,
                                            unsigned long long prefix, unsigned long long mask, int shift, int* hist,
-                                           int* sh) {
-  const int64_t n_iter = (N + blockDim.x - 1) / blockDim.x * blockDim.x;  // warp-uniform trip count
+                                           int* sh, unsigned long long* tiny) {
   for (; shift > -kHiBits; shift -= kHiBits) {
     const int s0 = max(shift, 0);
     const int width = shift >= 0 ? kHiBits : kHiBits + shift;  // the last digit holds the remaining bits
     const unsigned long long dmask = ((1ull << width) - 1ull) << s0;
     for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) hist[b] = 0;
+    if (threadIdx.x == 0) sh[2] = kHiTiny + 1;
     __syncthreads();
-    for (int64_t t = threadIdx.x; t < n_iter; t += blockDim.x) {
-      const unsigned long long k = t < N ? keys[t] : 0ull;
+    hi_for_keys(keys, N, [&](unsigned long long k) {
       const bool in = k != 0ull && (k & mask) == prefix;
       hi_hist_add(hist, in ? (int)((k & dmask) >> s0) : -1);
-    }
+    });
     __syncthreads();
-    if (threadIdx.x < 32) {
-      // the digit holding the rank-th largest key, counted from the top: lane
-      // j sums bins [64j, 64j + 64), a suffix scan over the lanes gives the
-      // count above each lane's bins, and the lane where the rank falls scans
-      const int lane = threadIdx.x;
-      int own = 0;
-      for (int b = 64 * lane; b < 64 * lane + 64; ++b) own += hist[b];
-      int above = 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_down_sync(0xffffffffu, above + own, o);
-        if (lane + o < 32) above += x;
-      }
-      if (above < rank && above + own >= rank) {
-        int r = rank - above, dg = 64 * lane + 63;
-        for (; dg > 64 * lane && hist[dg] < r; --dg) r -= hist[dg];
-        sh[0] = r;
-        sh[1] = dg;
-      }
-    }
+    if (threadIdx.x < 32) hi_find_bin(hist, rank, sh);
     __syncthreads();
     rank = sh[0];
     prefix |= (unsigned long long)sh[1] << s0;
     mask |= dmask;
+    const int cnt = sh[2];
     __syncthreads();
-  }
-  return prefix;
-}
-
-// Bitonic sort of n (a power of two) keys in shared memory, largest first.
-__device__ void hi_sort_desc(unsigned long long* keys, int n) {
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int t = threadIdx.x; t < n; t += blockDim.x) {
-        const int u = t ^ j;
-        if (u > t) {
-          const unsigned long long a = keys[t], b = keys[u];
-          const bool desc = (t & k) == 0;
-          if (desc ? a < b : a > b) {
-            keys[t] = b;
-            keys[u] = a;
-          }
-        }
+    if (s0 == 0) break;  // every bit decided
+    if (cnt <= kHiTiny) {
+      // the few keys with this prefix: the one with rank - 1 larger keys among them
+      if (threadIdx.x == 0) {
+        sh[3] = 0;
+        tiny[kHiTiny] = prefix;
       }
       __syncthreads();
+      hi_for_keys(keys, N, [&](unsigned long long k) {
+        const bool in = k != 0ull && (k & mask) == prefix;
+        const int slot = hi_warp_slot(&sh[3], in);
+        if (in && slot < kHiTiny) tiny[slot] = k;
+      });
+      __syncthreads();
+      const int c = min(sh[3], kHiTiny);
+      if ((int)threadIdx.x < c) {
+        const unsigned long long k = tiny[threadIdx.x];
+        int larger = 0;
+        for (int j = 0; j < c; ++j) larger += tiny[j] > k;
+        if (larger == rank - 1) tiny[kHiTiny] = k;
+      }
+      __syncthreads();
+      const unsigned long long r = tiny[kHiTiny];
+      __syncthreads();
+      return r;
     }
   }
+  return prefix;
 }
 
 // Block-wide sum of one int per thread; `scratch` holds 33 ints.
@@ -235,58 +307,94 @@ __global__ void __launch_bounds__(256) hi_page_keys_kernel(const __nv_bfloat16* 
 
 // ---------------------------------------------------------------------------
 // Page scores: grid (ceil(pages / 256), B), 256 threads, a thread per page.
-// A page is a candidate if it is whole and meets [sink_end, lo(i)).
+// A page is a candidate if it is whole and meets [sink_end, lo(i)). Also the
+// histogram of the keys' top digits per sequence (page_hist, zero on entry).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) hi_page_scores_kernel(const __grid_constant__ HiParams p) {
   __shared__ float q[kHiMaxDim];
+  __shared__ int hist[kHiBins];
   const int n = blockIdx.y;
   const int L = p.seqlens[n];
   const int i = L - 1;
   const SsaWindow w = hi_window(p);
   const int64_t full = min((int64_t)max(L, 0) / kHiPage, p.pages_per_seq);
   for (int c = threadIdx.x; c < p.d; c += blockDim.x) q[c] = __bfloat162float(p.q_index[(int64_t)n * p.d + c]);
+  for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) hist[b] = 0;
   __syncthreads();
   const int64_t pg = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (pg >= p.pages_per_seq) return;
   unsigned long long key = 0;
   if (pg < full && w.n_local >= 0 && pg * kHiPage + kHiPage - 1 >= w.sink_end && pg * kHiPage < w.lo(i)) {
     const float* pk = p.page_keys + (int64_t)n * p.d * p.pages_per_seq + pg;
     float s = 0.f;
+#pragma unroll 16
     for (int c = 0; c < p.d; ++c) s = __fmaf_rn(q[c], pk[(int64_t)c * p.pages_per_seq], s);
     key = hi_key(s, pg);
   }
-  p.page_scored[(int64_t)n * p.pages_per_seq + pg] = key;
+  if (pg < p.pages_per_seq) p.page_scored[(int64_t)n * p.pages_per_seq + pg] = key;
+  hi_hist_add(hist, key ? (int)(key >> kHiTopShift) : -1);
+  __syncthreads();
+  for (int b = threadIdx.x; b < kHiBins; b += blockDim.x)
+    if (hist[b]) atomicAdd(&p.page_hist[(int64_t)n * kHiBins + b], hist[b]);
+}
+
+// Top-k by the histogram of top digits: the digit d1 of the k-th largest key
+// and its rank r1 among the keys of that digit (warp 0 writes sh[0..2]:
+// r1, d1, count of d1; defaults r1 = 1, d1 = 0). Block-wide; hist in shared
+// memory (16-byte aligned) holds the histogram.
+__device__ __forceinline__ void hi_first_digit(const int* hist, int k, int* sh) {
+  if (threadIdx.x < 32) hi_find_bin(hist, k, sh);
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
-// Page selection: a CTA (1024 threads) per sequence. The top_pages largest
-// page keys (all candidates if fewer); also clears the sequence's token-key
-// histogram for the token stage.
+// Page selection: a CTA (1024 threads) per sequence. From the histogram of
+// the page keys' top digits, the digit d1 of the top_pages-th key: the keys
+// with top digit >= d1 are listed (on chip, or in the workspace if many), the
+// r1-th largest of digit d1 found among them by the remaining digits, and
+// every listed key at or above it is recalled.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) hi_page_select_kernel(const __grid_constant__ HiParams p) {
-  __shared__ int hist[kHiBins];
-  __shared__ int sh[34];
-  __shared__ int n_out;
+  __shared__ __align__(16) int hist[kHiBins];
+  __shared__ __align__(16) unsigned long long list_s[kHiCand];
+  __shared__ unsigned long long tiny[kHiTiny + 1];
+  __shared__ int sh[40];
   const int n = blockIdx.x;
-  for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) p.hist1[(int64_t)n * kHiBins + b] = 0;
   const unsigned long long* keys = p.page_scored + (int64_t)n * p.pages_per_seq;
   const int64_t N = p.pages_per_seq;
   int v = 0;
-  for (int64_t t = threadIdx.x; t < N; t += blockDim.x) v += keys[t] != 0ull;
+  for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) {
+    hist[b] = p.page_hist[(int64_t)n * kHiBins + b];
+    v += hist[b];
+  }
+  if (threadIdx.x == 0) {
+    sh[34] = 1;
+    sh[35] = 0;
+    sh[38] = 0;  // listed
+    sh[39] = 0;  // recalled
+  }
   const int n_valid = hi_block_sum(v, sh);
   const int m = min(n_valid, p.top_pages);
-  unsigned long long thr = 1ull;  // every real key is >= 1
-  if (m > 0 && m < n_valid) thr = hi_radix_kth(keys, N, m, 0ull, 0ull, kHiTopShift, hist, sh);
-  if (threadIdx.x == 0) n_out = 0;
-  __syncthreads();
   if (m > 0) {
-    const int64_t n_iter = (N + blockDim.x - 1) / blockDim.x * blockDim.x;
-    for (int64_t t = threadIdx.x; t < n_iter; t += blockDim.x) {
-      const unsigned long long k = t < N ? keys[t] : 0ull;
+    hi_first_digit(hist, m, sh + 34);
+    const int r1 = sh[34], d1 = sh[35] & (kHiBins - 1);
+    const int n_list = m - r1 + hist[d1];
+    const bool on_chip = n_list <= kHiCand;
+    unsigned long long* list = on_chip ? list_s : p.page_cand + (int64_t)n * p.pages_per_seq;
+    hi_for_keys(keys, N, [&](unsigned long long k) {
+      const bool in = k != 0ull && (int)(k >> kHiTopShift) >= d1;
+      const int s = hi_warp_slot(&sh[38], in);
+      if (in && s < n_list) list[s] = k;
+    });
+    __syncthreads();
+    const unsigned long long pre = (unsigned long long)d1 << kHiTopShift;
+    const unsigned long long msk = (unsigned long long)(kHiBins - 1) << kHiTopShift;
+    const unsigned long long thr = hi_radix_kth(list, n_list, r1, pre, msk, kHiTopShift - kHiBits, hist, sh, tiny);
+    int32_t* out = p.sel_pages + (int64_t)n * p.top_pages;
+    hi_for_keys(list, n_list, [&](unsigned long long k) {
       const bool take = k != 0ull && k >= thr;
-      const int slot = hi_warp_slot(&n_out, take);
-      if (take && slot < p.top_pages) p.sel_pages[(int64_t)n * p.top_pages + slot] = (int32_t)hi_key_index(k);
-    }
+      const int s = hi_warp_slot(&sh[39], take);
+      if (take && s < p.top_pages) out[s] = (int32_t)hi_key_index(k);
+    });
   }
   if (threadIdx.x == 0) p.n_pages[n] = m;
 }
@@ -435,31 +543,22 @@ __global__ void __launch_bounds__(kHiTokThreads) hi_tokens_kernel(const __grid_c
 }
 
 // ---------------------------------------------------------------------------
-// Token selection: a CTA (1024 threads) per sequence. The histogram of the
-// keys' top digits gives the digit d1 of the top_k-th largest key: keys with
-// a larger top digit are selected outright, those with digit d1 are the
-// candidates, sorted out on chip by the remaining digits (or, if more than
-// kHiCand share d1, by passes over the keys). The selection is then sorted by
-// position. Dynamic shared memory: HiTopkLayout::SMEM_BYTES.
+// Token selection, first pass: grid (ceil(top_pages * 128 / kHiCollectKeys),
+// B), 256 threads. From the histogram of the token keys' top digits every
+// CTA derives the digit d1 of the top_k-th largest key, lists the keys of its
+// slice with top digit >= d1 on chip and appends them to the sequence's list
+// tok_cand (its length in counters[n * 4 + 3], zero on entry).
 // ---------------------------------------------------------------------------
-struct HiTopkLayout {
-  static constexpr int SEL_OFF = 0;                          // [kHiMaxTopK] u64
-  static constexpr int CAND_OFF = SEL_OFF + kHiMaxTopK * 8;  // [kHiCand] u64
-  static constexpr int HIST_OFF = CAND_OFF + kHiCand * 8;    // [kHiBins] int
-  static constexpr int SH_OFF = HIST_OFF + kHiBins * 4;      // [40] int
-  static constexpr int SMEM_BYTES = SH_OFF + 40 * 4;
-};
-
-__global__ void __launch_bounds__(1024) hi_topk_kernel(const __grid_constant__ HiParams p) {
-  using LY = HiTopkLayout;
-  extern __shared__ __align__(16) uint8_t smem[];
-  unsigned long long* sel = reinterpret_cast<unsigned long long*>(smem + LY::SEL_OFF);
-  unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + LY::CAND_OFF);
-  int* hist = reinterpret_cast<int*>(smem + LY::HIST_OFF);
-  int* sh = reinterpret_cast<int*>(smem + LY::SH_OFF);  // [0..32] sums, [34..35] digit search, [36..37] counters
-  const int n = blockIdx.x;
+constexpr int kHiCollectKeys = 8192;
+constexpr int kHiCollectList = 2048;
+__global__ void __launch_bounds__(256) hi_topk_collect_kernel(const __grid_constant__ HiParams p) {
+  __shared__ __align__(16) int hist[kHiBins];
+  __shared__ unsigned long long list_s[kHiCollectList];
+  __shared__ int sh[40];
+  const int n = blockIdx.y;
   const int64_t N = (int64_t)p.n_pages[n] * kHiPage;
-  const unsigned long long* keys = p.tok_keys + (int64_t)n * p.top_pages * kHiPage;
+  const int64_t t0 = (int64_t)blockIdx.x * kHiCollectKeys;
+  if (t0 >= N) return;
   int v = 0;
   for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) {
     hist[b] = p.hist1[(int64_t)n * kHiBins + b];
@@ -468,70 +567,137 @@ __global__ void __launch_bounds__(1024) hi_topk_kernel(const __grid_constant__ H
   if (threadIdx.x == 0) {
     sh[34] = 1;
     sh[35] = 0;
-    sh[36] = 0;
-    sh[37] = 0;
+    sh[38] = 0;
   }
-  const int n_valid = hi_block_sum(v, sh);
-  const int k_eff = min(n_valid, p.top_k);
+  const int k_eff = min(hi_block_sum(v, sh), p.top_k);
+  if (k_eff <= 0) return;
+  hi_first_digit(hist, k_eff, sh + 34);
+  const int d1 = sh[35] & (kHiBins - 1);
+  int32_t* cnt = p.counters + (int64_t)n * 4;
+  unsigned long long* list = p.tok_cand + (int64_t)n * p.top_pages * kHiPage;
+  const int64_t cap = (int64_t)p.top_pages * kHiPage;
+  hi_for_keys(p.tok_keys + (int64_t)n * p.top_pages * kHiPage + t0, min((int64_t)kHiCollectKeys, N - t0),
+              [&](unsigned long long k) {
+                const bool in = k != 0ull && (int)(k >> kHiTopShift) >= d1;
+                const int s = hi_warp_slot(&sh[38], in);
+                if (in && s < kHiCollectList) list_s[s] = k;
+                const bool spill = in && s >= kHiCollectList;  // a crowded slice: straight to the list
+                const int g = hi_warp_slot(&cnt[3], spill);
+                if (spill && g < cap) list[g] = k;
+              });
+  __syncthreads();
+  const int nl = min(sh[38], kHiCollectList);
+  if (threadIdx.x == 0) sh[0] = nl ? atomicAdd(&cnt[3], nl) : 0;
+  __syncthreads();
+  const int base = sh[0];
+  for (int t = threadIdx.x; t < nl; t += blockDim.x)
+    if (base + t < cap) list[base + t] = list_s[t];
+}
+
+// ---------------------------------------------------------------------------
+// Token selection, second pass: a CTA (1024 threads) per sequence. Among the
+// listed keys (top digit >= d1; on chip when at most kHiCand), the r1-th
+// largest of digit d1 by the remaining digits is the threshold; the listed
+// keys at or above it are the selection. Their positions go into a bitmap of
+// the sequence's whole pages, read back in order. Dynamic shared memory:
+// HiTopkLayout::bytes(pages_per_seq).
+// ---------------------------------------------------------------------------
+struct HiTopkLayout {
+  static constexpr int LIST_OFF = 0;                            // [kHiCand] u64
+  static constexpr int TINY_OFF = LIST_OFF + kHiCand * 8;       // [kHiTiny + 1] u64
+  static constexpr int HIST_OFF = TINY_OFF + (kHiTiny + 2) * 8;  // [kHiBins] int
+  static constexpr int SH_OFF = HIST_OFF + kHiBins * 4;         // [64] int
+  static constexpr int BITS_OFF = SH_OFF + 64 * 4;              // [pages * 4] u32 bitmap
+  static constexpr int bytes(int64_t pages) { return BITS_OFF + (int)(pages * 4 * 4); }
+};
+
+__global__ void __launch_bounds__(1024) hi_topk_kernel(const __grid_constant__ HiParams p) {
+  using LY = HiTopkLayout;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  unsigned long long* list_s = reinterpret_cast<unsigned long long*>(smem + LY::LIST_OFF);
+  unsigned long long* tiny = reinterpret_cast<unsigned long long*>(smem + LY::TINY_OFF);
+  int* hist = reinterpret_cast<int*>(smem + LY::HIST_OFF);
+  int* sh = reinterpret_cast<int*>(smem + LY::SH_OFF);  // [0..32] sums, [34..36] first digit, [40..43] radix
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + LY::BITS_OFF);
+  const int n = blockIdx.x;
+  const int nwords = (int)(p.pages_per_seq * 4);
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) bits[w] = 0u;
+  int v = 0;
+  for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) {
+    hist[b] = p.hist1[(int64_t)n * kHiBins + b];
+    v += hist[b];
+  }
+  if (threadIdx.x == 0) {
+    sh[34] = 1;
+    sh[35] = 0;
+  }
+  const int k_eff = min(hi_block_sum(v, sh), p.top_k);
   if (k_eff > 0) {
-    if (threadIdx.x < 32) {
-      // the top digit d1 of the k_eff-th largest key and its rank r1 among the keys of that digit
-      const int lane = threadIdx.x;
-      int own = 0;
-      for (int b = 64 * lane; b < 64 * lane + 64; ++b) own += hist[b];
-      int above = 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_down_sync(0xffffffffu, above + own, o);
-        if (lane + o < 32) above += x;
-      }
-      if (above < k_eff && above + own >= k_eff) {
-        int r = k_eff - above, dg = 64 * lane + 63;
-        for (; dg > 64 * lane && hist[dg] < r; --dg) r -= hist[dg];
-        sh[34] = r;
-        sh[35] = dg;
-      }
-    }
-    __syncthreads();
+    hi_first_digit(hist, k_eff, sh + 34);
     const int r1 = sh[34], d1 = sh[35] & (kHiBins - 1);
-    const int c1 = hist[d1];
-    const bool on_chip = c1 <= kHiCand;
-    const int64_t n_iter = (N + blockDim.x - 1) / blockDim.x * blockDim.x;
-    for (int64_t t = threadIdx.x; t < n_iter; t += blockDim.x) {
-      const unsigned long long k = t < N ? keys[t] : 0ull;
-      const int dg = k ? (int)(k >> kHiTopShift) : -1;
-      const bool take = dg > d1;
-      const int s = hi_warp_slot(&sh[36], take);
-      if (take && s < kHiMaxTopK) sel[s] = k;
-      const bool keep = on_chip && dg == d1;
-      const int c = hi_warp_slot(&sh[37], keep);
-      if (keep && c < kHiCand) cand[c] = k;
-    }
+    const int n_list = min((int64_t)p.counters[(int64_t)n * 4 + 3], (int64_t)p.top_pages * kHiPage);
+    const unsigned long long* list_g = p.tok_cand + (int64_t)n * p.top_pages * kHiPage;
+    const bool on_chip = n_list <= kHiCand;
+    if (on_chip)
+      for (int t = threadIdx.x; t < n_list; t += blockDim.x) list_s[t] = list_g[t];
     __syncthreads();
+    const unsigned long long* list = on_chip ? list_s : list_g;
     const unsigned long long pre = (unsigned long long)d1 << kHiTopShift;
     const unsigned long long msk = (unsigned long long)(kHiBins - 1) << kHiTopShift;
-    const unsigned long long* src = on_chip ? cand : keys;
-    const int64_t n_src = on_chip ? c1 : N;
-    // the r1-th largest key of digit d1, by the digits below it
-    const unsigned long long thr = hi_radix_kth(src, n_src, r1, pre, msk, kHiTopShift - kHiBits, hist, sh + 34);
-    const int64_t n_iter2 = (n_src + blockDim.x - 1) / blockDim.x * blockDim.x;
-    for (int64_t t = threadIdx.x; t < n_iter2; t += blockDim.x) {
-      const unsigned long long k = t < n_src ? src[t] : 0ull;
-      const bool take = k != 0ull && (k & msk) == pre && k >= thr;
-      const int s = hi_warp_slot(&sh[36], take);
-      if (take && s < kHiMaxTopK) sel[s] = k;
-    }
+    const unsigned long long thr =
+        hi_radix_kth(list, n_list, r1, pre, msk, kHiTopShift - kHiBits, hist, sh + 40, tiny);
+    hi_for_keys(list, n_list, [&](unsigned long long k) {
+      if (k != 0ull && k >= thr) {
+        const uint32_t pos = hi_key_index(k);
+        if (pos < (uint32_t)nwords * 32u) atomicOr(&bits[pos >> 5], 1u << (pos & 31));
+      }
+    });
   }
   __syncthreads();
-  // by position: keys whose value is 2^32 - 1 - position, sorted largest first
-  int npow2 = 1;
-  while (npow2 < k_eff) npow2 <<= 1;
-  for (int t = threadIdx.x; t < npow2; t += blockDim.x)
-    sel[t] = t < k_eff ? (unsigned long long)(0xFFFFFFFFu - hi_key_index(sel[t])) : 0ull;
+  // positions in order: warp w reads the words [w * per, (w + 1) * per), 32
+  // consecutive words at a time (lane = word)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+  const int per = (nwords + n_warps - 1) / n_warps;
+  const int wb = warp * per, we = min(wb + per, nwords);
+  int cnt = 0;
+  for (int w = wb + lane; w < we; w += 32) cnt += __popc(bits[w]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) sh[warp] = cnt;
   __syncthreads();
-  if (k_eff > 1) hi_sort_desc(sel, npow2);
-  for (int t = threadIdx.x; t < p.top_k; t += blockDim.x)
-    p.selected[(int64_t)n * p.top_k + t] = t < k_eff ? (int32_t)(0xFFFFFFFFu - (uint32_t)sel[t]) : -1;
+  if (warp == 0) {
+    const int wv = lane < n_warps ? sh[lane] : 0;
+    int wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += x;
+    }
+    sh[lane] = wi - wv;  // positions before this warp's words
+  }
+  __syncthreads();
+  int at = sh[warp];
+  int32_t* out = p.selected + (int64_t)n * p.top_k;
+  for (int w0 = wb; w0 < we; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t b = w < we ? bits[w] : 0u;
+    const int c = __popc(b);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    int q = at + incl - c;
+    while (b) {
+      const int j = __ffs(b) - 1;
+      b &= b - 1;
+      if (q < p.top_k) out[q] = w * 32 + j;
+      ++q;
+    }
+    at += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  for (int t = k_eff + threadIdx.x; t < p.top_k; t += blockDim.x) out[t] = -1;
   if (threadIdx.x == 0) p.n_sel[n] = k_eff;
 }
 
@@ -593,17 +759,36 @@ __global__ void __launch_bounds__(256) hi_gather_kernel(const __nv_bfloat16* __r
   const int ns = min(n_sel[n], top_k);
   const int count = min(sink_rows + ns + local_rows, cap_rows);
   if (blockIdx.x == 0 && threadIdx.x == 0) counts[n] = count;
+  // the 32 rows' tokens first (-1: past the packed rows, not written; -2: an
+  // entry that names no row of the sequence, written as zeros), then all 9
+  // copies of each thread in flight at once
+  __shared__ int64_t src[32];
   const int j0 = blockIdx.x * 32;
-  for (int e = threadIdx.x; e < 32 * 72; e += blockDim.x) {
-    const int j = j0 + e / 72, c = e % 72;
-    if (j >= count) continue;
-    int64_t tok;
-    if (j < sink_rows) tok = j;
-    else if (j < sink_rows + ns) tok = sel[(int64_t)n * top_k + (j - sink_rows)];
-    else tok = lo + (j - sink_rows - ns);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (tok >= 0 && tok < L) v = reinterpret_cast<const uint4*>(kv + n * batch_stride + tok * row_stride)[c];
-    reinterpret_cast<uint4*>(packed + ((int64_t)n * cap_rows + j) * 576)[c] = v;
+  if (threadIdx.x < 32) {
+    const int j = j0 + threadIdx.x;
+    int64_t tok = -1;
+    if (j < count) {
+      if (j < sink_rows) tok = j;
+      else if (j < sink_rows + ns) tok = sel[(int64_t)n * top_k + (j - sink_rows)];
+      else tok = lo + (j - sink_rows - ns);
+      if (tok >= L) tok = -1;
+    }
+    src[threadIdx.x] = j < count ? (tok < 0 ? -2 : tok) : -1;
+  }
+  __syncthreads();
+  static_assert(32 * 72 % 256 == 0, "whole copies per thread");
+  uint4 v[32 * 72 / 256];
+#pragma unroll
+  for (int it = 0; it < 32 * 72 / 256; ++it) {
+    const int e = threadIdx.x + it * 256, r = e / 72, c = e % 72;
+    const int64_t tok = src[r];
+    v[it] = tok >= 0 ? reinterpret_cast<const uint4*>(kv + n * batch_stride + tok * row_stride)[c]
+                     : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int it = 0; it < 32 * 72 / 256; ++it) {
+    const int e = threadIdx.x + it * 256, r = e / 72, c = e % 72;
+    if (src[r] != -1) reinterpret_cast<uint4*>(packed + ((int64_t)n * cap_rows + j0 + r) * 576)[c] = v[it];
   }
 }
 

@@ -130,7 +130,7 @@ int sm_count() {
 // the GPU in one wave.
 //   - a few sequences with long windows (more than 8 blocks, batch * 16 <= SMs):
 //     the block kernel, many splits, merged through the workspace;
-//   - windows of at most 16 blocks while two CTAs per sequence fit (batch * 2
+//   - windows of at most 24 blocks while two CTAs per sequence fit (batch * 2
 //     <= SMs): the half-block kernel, up to 4 splits per sequence in a
 //     cluster, merged on chip;
 //   - otherwise the block kernel with up to 4 splits per sequence in a
@@ -156,7 +156,7 @@ DecodePlan decode_plan(const loza_ssa_params& p, int32_t max_seqlen, int32_t bat
     const int bps = (count + ns - 1) / ns;
     return {bps, (count + bps - 1) / bps, false, false};
   }
-  if (count <= 16 && (int64_t)batch * 2 <= sms) {
+  if (count <= 24 && (int64_t)batch * 2 <= sms) {
     // half blocks: up to 4 CTAs per sequence in one cluster, each pulling
     // its share of the rows once
     // (the on-chip merge splits the 512 value columns evenly: nsplit is 1, 2
@@ -548,7 +548,8 @@ bool hi_window_ok(const loza_ssa_params& p) {
 }
 
 struct HiWorkspace {
-  size_t page_scored, sel_pages, n_pages, hist1, tok_keys, selected, n_sel, counts, packed, dec, total;
+  size_t page_scored, sel_pages, n_pages, zeroed, zeroed_bytes, page_hist, hist1, counters, page_cand, tok_keys,
+      tok_cand, selected, n_sel, counts, packed, dec, total;
   int cap_rows;  // packed rows per sequence (0: the unbounded window, decoded in place)
 };
 size_t hi_align(size_t x) { return (x + 255) / 256 * 256; }
@@ -565,8 +566,15 @@ HiWorkspace hi_workspace(int32_t batch, int32_t max_seqlen, int32_t top_pages, i
   w.page_scored = take((size_t)batch * pages * 8);
   w.sel_pages = take((size_t)batch * top_pages * 4);
   w.n_pages = take((size_t)batch * 4);
-  w.hist1 = take((size_t)batch * kHiBins * 4);
+  // histograms and list counters, cleared by one memset per call
+  w.zeroed_bytes = (size_t)batch * (2 * kHiBins + 4) * 4;
+  w.zeroed = take(w.zeroed_bytes);
+  w.page_hist = w.zeroed;
+  w.hist1 = w.page_hist + (size_t)batch * kHiBins * 4;
+  w.counters = w.hist1 + (size_t)batch * kHiBins * 4;
+  w.page_cand = take((size_t)batch * pages * 8);
   w.tok_keys = take((size_t)batch * top_pages * kHiPage * 8);
+  w.tok_cand = take((size_t)batch * top_pages * kHiPage * 8);
   w.selected = take((size_t)batch * std::max(top_k, 1) * 4);
   w.n_sel = take((size_t)batch * 4);
   w.counts = take((size_t)batch * 4);
@@ -1158,16 +1166,21 @@ loza_status hi_select_launch(const void* q_index, const void* k_index, int64_t i
   hp.page_scored = reinterpret_cast<unsigned long long*>(ws + w.page_scored);
   hp.sel_pages = reinterpret_cast<int32_t*>(ws + w.sel_pages);
   hp.n_pages = reinterpret_cast<int32_t*>(ws + w.n_pages);
+  hp.page_hist = reinterpret_cast<int32_t*>(ws + w.page_hist);
   hp.hist1 = reinterpret_cast<int32_t*>(ws + w.hist1);
+  hp.counters = reinterpret_cast<int32_t*>(ws + w.counters);
+  hp.page_cand = reinterpret_cast<unsigned long long*>(ws + w.page_cand);
   hp.tok_keys = reinterpret_cast<unsigned long long*>(ws + w.tok_keys);
+  hp.tok_cand = reinterpret_cast<unsigned long long*>(ws + w.tok_cand);
   hp.selected = selected;
   hp.n_sel = reinterpret_cast<int32_t*>(ws + w.n_sel);
   if (cudaFuncSetAttribute(hi_tokens_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            HiTokLayout::SMEM_ALLOC) != cudaSuccess ||
       cudaFuncSetAttribute(hi_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           HiTopkLayout::SMEM_BYTES) != cudaSuccess)
+                           HiTopkLayout::bytes(hp.pages_per_seq)) != cudaSuccess)
     return LOZA_ERR_CUDA;
-  int launches = 3;
+  if (cudaMemsetAsync(ws + w.zeroed, 0, w.zeroed_bytes, st) != cudaSuccess) return LOZA_ERR_CUDA;
+  int launches = 4;
   if (hp.pages_per_seq >= 1) {
     hi_page_scores_kernel<<<dim3((unsigned)((hp.pages_per_seq + 255) / 256), batch), 256, 0, st>>>(hp);
     ++launches;
@@ -1176,7 +1189,9 @@ loza_status hi_select_launch(const void* q_index, const void* k_index, int64_t i
   const int64_t items = (int64_t)batch * ((top_pages + kHiTokPages - 1) / kHiTokPages);
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(items, 3 * (int64_t)sm_count()));
   hi_tokens_kernel<<<grid, kHiTokThreads, HiTokLayout::SMEM_ALLOC, st>>>(hp);
-  hi_topk_kernel<<<batch, 1024, HiTopkLayout::SMEM_BYTES, st>>>(hp);
+  const int64_t slices = ((int64_t)top_pages * kHiPage + kHiCollectKeys - 1) / kHiCollectKeys;
+  hi_topk_collect_kernel<<<dim3((unsigned)slices, batch), 256, 0, st>>>(hp);
+  hi_topk_kernel<<<batch, 1024, HiTopkLayout::bytes(hp.pages_per_seq), st>>>(hp);
   g_launches.fetch_add(launches, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
