@@ -183,3 +183,28 @@ def test_decode_is_the_lse_merge_of_its_two_parts(oracle_mod):
         wa, wb = np.exp(lw[n] - m), np.exp(ls - m)
         np.testing.assert_allclose(o[n], (wa[:, None] * ow[n] + wb[:, None] * os_) / (wa + wb)[:, None], atol=1e-12)
         np.testing.assert_allclose(l[n], m + np.log(wa + wb), atol=1e-12)
+
+
+@pytest.mark.parametrize("win,sel", [((1, 0, 50), [0, 5, 77]), ((4, 1, 3), [31, 4, 200]), ((1, 16, 1024), [])])
+def test_decode_brute_force_small(oracle_mod, win, sel):
+    """Tiny case by brute force: the keys are the window's (token-distance
+    form, written out) plus an explicit selection that includes token 0 when
+    the window has no sinks; one numpy softmax over them."""
+    b, s, l = win
+    g = synth.rng(807)
+    H, D, L = 3, 32, 300
+    q = synth.normal_bits(g, (1, H, D))
+    kv = synth.normal_bits(g, (1, L, 1, D))
+    i = L - 1
+    keys = sorted(set(t for t in range(L) if in_window(t, i, b, s, l)) | set(sel))
+    assert len(keys) == len(set(t for t in range(L) if in_window(t, i, b, s, l))) + len(sel)  # disjoint
+    qf = synth.bits_to_f32(q).astype(np.float64)[0]
+    kf = synth.bits_to_f32(kv).astype(np.float64)[0, :, 0]
+    z = 0.2 * qf @ kf[keys].T
+    w = np.exp(z)
+    o_ref = (w @ kf[keys, :D]) / w.sum(1, keepdims=True)
+    lse_ref = np.log(w.sum(1))
+    selected = np.array([sel], np.int32) if sel else np.full((1, 0), -1, np.int32)
+    o, lse = oracle_mod.hi_decode(q, kv, [L], H, b, s, l, 0.2, selected, d_v=D)
+    np.testing.assert_allclose(o[0], o_ref, atol=1e-12)
+    np.testing.assert_allclose(lse[0], lse_ref, atol=1e-12)
