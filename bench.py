@@ -768,7 +768,7 @@ def run_ours(args, rank, world, local_rank):
     if args.workload in ("default", "decode"):
         secondary["decode"] = decode_secondary(bss, device, stream, peaks, peak_kind, args.decode_batch,
                                                args.decode_ctx)
-    if args.workload == "default":
+    if args.workload in ("default", "merge"):
         secondary["merge"] = merge_secondary(bss, device, stream, peaks, peak_kind)
     if args.workload in ("default", "long"):
         secondary["long"], secondary["decode_1m"] = long_secondary(bss, device, stream, peaks, peak_kind)
@@ -904,7 +904,7 @@ def main():
                     help="training workload as one sequence of this length (profiling)")
     ap.add_argument("--hi-batch", type=int, default=32, help="sequences of the hierarchical index decode line")
     ap.add_argument("--hi-ctx", type=int, default=1 << 20, help="tokens per sequence of that line (a multiple of 128)")
-    ap.add_argument("--workload", choices=["default", "prefill", "decode", "long", "hi", "train"], default="default",
+    ap.add_argument("--workload", choices=["default", "prefill", "decode", "merge", "long", "hi", "train"], default="default",
                     help="default: the prefill line with every other workload as secondary lines (the "
                          "64-sequence decode, the branch merge, workload 4's long prefill and 1M decode, "
                          "the hierarchical index decode at 1M, workload 5's training); the others: the prefill line plus only that one")
