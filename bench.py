@@ -78,9 +78,11 @@ def kernel_source_hash(files=None):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key):
+def profiled_traffic(kernel_key, scale=1.0):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    the current kernel sources; else None. `scale`: this launch's units over
+    those of the recorded launch, for a kernel whose traffic grows in
+    proportion to them (the record says which units)."""
     p = os.path.join(ROOT, "profiles", "ncu_counters.json")
     if not os.path.exists(p):
         return None
@@ -88,7 +90,7 @@ def profiled_traffic(kernel_key):
     e = d.get(kernel_key)
     if not e or e.get("source_hash") != kernel_source_hash(e.get("source_files")):
         return None
-    return e.get("dram_bytes_per_launch")
+    return int(round(e.get("dram_bytes_per_launch") * scale))
 
 
 class ClockSampler:
@@ -400,7 +402,8 @@ def decode_secondary(bss, device, stream, peaks, peak_kind, batch=None, ctx=None
            "metric": "SSA decode GB/s (bytes touched)", "value": ssa["GB/s"], "unit": "GB/s",
            "ms_per_call": ssa["ms"], "bytes_per_call": ssa["bytes"],
            "roofline": {"bound": "hbm", "achieved": ssa["GB/s"], "peak": hbm, "unit": "GB/s",
-                        "frac": ssa["GB/s"] / hbm, "traffic": profiled_traffic(DECODE_KERNEL),
+                        "frac": ssa["GB/s"] / hbm,
+                        "traffic": profiled_traffic(DECODE_KERNEL, len(lens) / w["batch"]),
                         "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)",
                         "kernel": DECODE_KERNEL},
            "timing": "mean of per-call CUDA events; before each call (outside the events) the L2 is flushed "
@@ -462,19 +465,19 @@ def merge_secondary(bss, device, stream, peaks, peak_kind, steps=20):
             "timing": "mean of per-call CUDA events; inputs larger than L2"}
 
 
-def tensor_roofline(flop, ms, peaks, peak_kind, kernel):
+def tensor_roofline(flop, ms, peaks, peak_kind, kernel, traffic_scale=1.0):
     pk = float(peaks["bf16_tflops"])
     a = flop / (ms / 1000.0) / 1e12
     return {"bound": "tensor", "achieved": a, "peak": pk, "unit": "TFLOP/s", "frac": a / pk,
-            "traffic": profiled_traffic(kernel),
+            "traffic": profiled_traffic(kernel, traffic_scale),
             "peak_kind": f"{peak_kind} bf16 dense burst (MEASURED_PEAKS.json bf16_tflops)", "kernel": kernel}
 
 
-def hbm_roofline(nbytes, ms, peaks, peak_kind, kernel):
+def hbm_roofline(nbytes, ms, peaks, peak_kind, kernel, traffic_scale=1.0):
     hbm = float(peaks["hbm_gbs"])
     a = nbytes / (ms / 1000.0) / 1e9
     return {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
-            "traffic": profiled_traffic(kernel),
+            "traffic": profiled_traffic(kernel, traffic_scale),
             "peak_kind": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)", "kernel": kernel}
 
 
@@ -508,7 +511,7 @@ def long_secondary(bss, device, stream, peaks, peak_kind):
         kern = "ssa_prefill_mla_kernel" if (nl > 0 and ws is not None) else "ssa_prefill_pair_kernel"
         lines[name] = {"ms_per_call": ms, "launches_timed": n, "algorithmic_tflop": fl / 1e12,
                        "TFLOP/s": fl / (ms / 1000) / 1e12,
-                       "roofline": tensor_roofline(fl, ms, peaks, peak_kind, kern)}
+                       "roofline": tensor_roofline(fl, ms, peaks, peak_kind, kern, traffic_scale=L / SEQLEN)}
         del ws
     del q, lat, out, lse
     torch.cuda.empty_cache()
@@ -524,7 +527,8 @@ def long_secondary(bss, device, stream, peaks, peak_kind):
     dec = {"workload": f"MLA-absorbed SSA decode, {w['decode_batch']} seqs x {w['decode_ctx']} tokens",
            "metric": "SSA decode GB/s (bytes touched)", "value": ssa["GB/s"], "unit": "GB/s",
            "ms_per_call": ssa["ms"], "bytes_per_call": ssa["bytes"],
-           "roofline": hbm_roofline(ssa["bytes"], ssa["ms"], peaks, peak_kind, DECODE_KERNEL),
+           "roofline": hbm_roofline(ssa["bytes"], ssa["ms"], peaks, peak_kind, DECODE_KERNEL,
+                                    traffic_scale=w["decode_batch"] / synth.WORKLOADS[3]["batch"]),
            "dense": {"ms_per_call": dense["ms"], "bytes_per_call": dense["bytes"], "GB/s": dense["GB/s"],
                      "frac_of_hbm": dense["GB/s"] / float(peaks["hbm_gbs"]),
                      "dense_over_ssa_time": dense["ms"] / ssa["ms"]},
