@@ -48,6 +48,7 @@ EXPORTED = [
     "loza_hi_select",
     "loza_ssa_decode_selected",
     "loza_hi_decode",
+    "loza_wait_selftest",
 ]
 
 
@@ -108,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.loza_device_status.argtypes = [_vp]
         L.loza_launch_count.restype = ctypes.c_uint64
         L.loza_launch_count.argtypes = []
+        L.loza_wait_selftest.restype = ctypes.c_int
+        L.loza_wait_selftest.argtypes = [ctypes.c_uint32, _vp]
         L.loza_hi_page_keys.restype = ctypes.c_int
         L.loza_hi_page_keys.argtypes = [_vp, _i64, _i64, _vp, _i32, _i32, _i32, _vp, _vp]
         L.loza_hi_workspace_size.restype = _sz
@@ -517,3 +520,11 @@ def loza_hi_decode(q, kv_cache, q_index, k_index, page_keys, seqlens, max_seqlen
                               _stream_ptr(stream))
     _check(rc, "loza_hi_decode")
     return out, lse
+
+
+def wait_selftest(limit_us: int, stream=None) -> int:
+    """Launch the bounded-wait self-test (a wait that nothing completes gives
+    up after limit_us); returns the status of the following device-status
+    read, LOZA_ERR_TIMEOUT (-5) when the bound works."""
+    _check(lib().loza_wait_selftest(int(limit_us), _stream_ptr(stream)), "loza_wait_selftest")
+    return device_status(stream)

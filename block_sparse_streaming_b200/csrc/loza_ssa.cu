@@ -618,6 +618,18 @@ bool make_map_index(CUtensorMap* m, const void* k_index, int32_t d, int32_t rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The bounded-wait self-test: one thread waits on an mbarrier that nothing
+// completes, gives up after limit_ns and records the timeout like every
+// kernel's waits do. No TMA, MMA or other thread is involved.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    mbar_wait_for(smem_u32(&bar), 0, nullptr, limit_ns);
+  }
+}
+
 }  // namespace
 }  // namespace loza
 
@@ -711,6 +723,13 @@ const char* loza_status_string(loza_status s) {
 }
 
 uint64_t loza_launch_count(void) { return g_launches.load(); }
+
+loza_status loza_wait_selftest(uint32_t limit_us, loza_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000) return LOZA_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((unsigned long long)limit_us * 1000ull);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
+}
 
 loza_status loza_device_status(loza_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return LOZA_ERR_CUDA;

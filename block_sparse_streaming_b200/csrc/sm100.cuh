@@ -77,22 +77,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Returns false (and
-// records a timeout) if it does not complete within kWaitLimitNs, or if
-// `abort` (a shared flag other roles raise after their own timeout) is set.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// records a timeout) if it does not complete within limit_ns, or if `abort`
+// (a shared flag other roles raise after their own timeout) is set.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int* abort,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255) == 0) {
       if (abort && *abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         atomicOr(&g_device_status, kErrTimeout);
         if (abort) *abort = 1;
         return false;
       }
     }
   }
+}
+
+// The kernels' wait: gives up after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // mbar_wait executed by a whole warp, with a warp-uniform result (if any lane

@@ -435,6 +435,16 @@ loza_status loza_device_status(loza_stream_t stream);
 /* Number of kernel launches the library issued since load (all entry points). */
 uint64_t loza_launch_count(void);
 
+/*
+ * Self-test of the bounded waits: launches one thread that waits on an
+ * mbarrier nothing completes; after limit_us microseconds (1 ... 2,000,000)
+ * it gives up and records a timeout exactly as a kernel's own wait would, so
+ * the next loza_device_status returns LOZA_ERR_TIMEOUT and the context stays
+ * usable. (Every wait in the library's kernels has the same bound, 2 s.)
+ * LOZA_ERR_INVALID_ARG for a limit out of range.
+ */
+loza_status loza_wait_selftest(uint32_t limit_us, loza_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -211,3 +211,10 @@ def test_backward_needs_blocks_of_128(L):
         assert rc == -2
         assert bss.workspace_size(bss.LOZA_OP_BACKWARD, 1, 256, 256, 4, 4, 64, 64, params) == 0
     assert L.loza_launch_count() == count
+
+
+@pytest.mark.parametrize("limit", [0, 2000001])
+def test_wait_selftest_rejects_out_of_range_limits(L, limit):
+    count = L.loza_launch_count()
+    assert L.loza_wait_selftest(limit, ctypes.c_void_p(0)) == -1
+    assert L.loza_launch_count() == count

@@ -96,7 +96,7 @@ def test_select_rejects_before_launch(L, kw, code):
     (1 << 20, 1 << 21, 576, 2049, 1 << 22, None, 1 << 30, INVALID),
     (1 << 20, 1 << 21, 576, 64, 0, None, 1 << 30, INVALID),           # no list
     (1 << 20, 1 << 21, 576, 64, 1 << 22, bss.Params(0.07, block_size=6), 1 << 30, UNSUPPORTED),
-    (1 << 20, 1 << 21, 576, 64, 1 << 22, None, 4096, WORKSPACE),
+    (0, 1 << 21, 576, 64, 1 << 22, None, 4096, WORKSPACE),  # q NULL: a skipped size check still launches nothing
 ])
 def test_decode_selected_rejects_before_launch(L, q, kv, rs, top_k, sel, params, ws_bytes, code):
     p = params or bss.Params(0.07, block_size=1, n_sink=16, n_local=1024)
@@ -122,7 +122,7 @@ def _hi_decode(L, ws_bytes=1 << 30, ws=1 << 26, q=1 << 27, cache_rs=576, top_k=2
     (dict(k=0), INVALID),
     (dict(params=bss.Params(0.07, block_size=5)), UNSUPPORTED),
     (dict(ws=0), INVALID),
-    (dict(ws_bytes=4096), WORKSPACE),
+    (dict(ws_bytes=4096, q=0), WORKSPACE),  # q NULL: a skipped size check still launches nothing
 ])
 def test_hi_decode_rejects_before_launch(L, kw, code):
     count = L.loza_launch_count()
