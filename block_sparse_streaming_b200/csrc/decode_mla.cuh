@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ssa_decode_mla_kernel(const __
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int split = blockIdx.x;
   const int seq = blockIdx.y;
+  griddep_wait();  // in a chain of launches, the sequence lengths and cache rows may come from the kernel before
   const int L = p.seqlens[seq];
   const int i_q = L - 1;                 // decode query position
   const int jq = i_q / kTile;            // its block

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kHbThreads, 1) ssa_decode_mla_hb_kernel(const 
   const int split = blockIdx.x;  // == rank in the cluster
   const int seq = blockIdx.y;
   const int ns = p.nsplit;
+  griddep_wait();  // in a chain of launches, the sequence lengths and cache rows may come from the kernel before
   const int L = p.seqlens[seq];
   const int i_q = L - 1;                                 // decode query position
   // the half blocks (64-row units) of the window of position i_q, sinks

@@ -335,6 +335,7 @@ __global__ void __launch_bounds__(256) hi_page_scores_kernel(const __grid_consta
   __syncthreads();
   for (int b = threadIdx.x; b < kHiBins; b += blockDim.x)
     if (hist[b]) atomicAdd(&p.page_hist[(int64_t)n * kHiBins + b], hist[b]);
+  griddep_launch_dependents();
 }
 
 // Top-k by the histogram of top digits: the digit d1 of the k-th largest key
@@ -361,6 +362,7 @@ __global__ void __launch_bounds__(1024) hi_page_select_kernel(const __grid_const
   const int n = blockIdx.x;
   const unsigned long long* keys = p.page_scored + (int64_t)n * p.pages_per_seq;
   const int64_t N = p.pages_per_seq;
+  griddep_wait();  // the page keys and their histogram
   int v = 0;
   for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) {
     hist[b] = p.page_hist[(int64_t)n * kHiBins + b];
@@ -397,6 +399,7 @@ __global__ void __launch_bounds__(1024) hi_page_select_kernel(const __grid_const
     });
   }
   if (threadIdx.x == 0) p.n_pages[n] = m;
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -442,6 +445,7 @@ __global__ void __launch_bounds__(kHiTokThreads) hi_tokens_kernel(const __grid_c
   }
   for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) hist[b] = 0;
   __syncthreads();
+  griddep_wait();  // the recalled pages
   const int n_ch = p.d / kHiDimStep;
   const int groups = (p.top_pages + kHiTokPages - 1) / kHiTokPages;
   const int64_t items = (int64_t)p.batch * groups;
@@ -479,6 +483,7 @@ __global__ void __launch_bounds__(kHiTokThreads) hi_tokens_kernel(const __grid_c
       for (uint32_t j = it > (uint32_t)kHiTokStages ? it - kHiTokStages : 0; j < it; ++j)
         mbar_wait(full(j % kHiTokStages), (j / kHiTokStages) & 1, nullptr);
     }
+    griddep_launch_dependents();
     return;
   }
   // consumers: thread t scores token t of each page
@@ -540,6 +545,7 @@ __global__ void __launch_bounds__(kHiTokThreads) hi_tokens_kernel(const __grid_c
     }
     named_barrier_sync(1, 128);
   }
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -556,9 +562,13 @@ __global__ void __launch_bounds__(256) hi_topk_collect_kernel(const __grid_const
   __shared__ unsigned long long list_s[kHiCollectList];
   __shared__ int sh[40];
   const int n = blockIdx.y;
+  griddep_wait();  // the token keys and their histogram
   const int64_t N = (int64_t)p.n_pages[n] * kHiPage;
   const int64_t t0 = (int64_t)blockIdx.x * kHiCollectKeys;
-  if (t0 >= N) return;
+  if (t0 >= N) {
+    griddep_launch_dependents();
+    return;
+  }
   int v = 0;
   for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) {
     hist[b] = p.hist1[(int64_t)n * kHiBins + b];
@@ -570,7 +580,10 @@ __global__ void __launch_bounds__(256) hi_topk_collect_kernel(const __grid_const
     sh[38] = 0;
   }
   const int k_eff = min(hi_block_sum(v, sh), p.top_k);
-  if (k_eff <= 0) return;
+  if (k_eff <= 0) {
+    griddep_launch_dependents();
+    return;
+  }
   hi_first_digit(hist, k_eff, sh + 34);
   const int d1 = sh[35] & (kHiBins - 1);
   int32_t* cnt = p.counters + (int64_t)n * 4;
@@ -592,6 +605,7 @@ __global__ void __launch_bounds__(256) hi_topk_collect_kernel(const __grid_const
   const int base = sh[0];
   for (int t = threadIdx.x; t < nl; t += blockDim.x)
     if (base + t < cap) list[base + t] = list_s[t];
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -622,6 +636,7 @@ __global__ void __launch_bounds__(1024) hi_topk_kernel(const __grid_constant__ H
   const int n = blockIdx.x;
   const int nwords = (int)(p.pages_per_seq * 4);
   for (int w = threadIdx.x; w < nwords; w += blockDim.x) bits[w] = 0u;
+  griddep_wait();  // the lists of the first pass
   int v = 0;
   for (int b = threadIdx.x; b < kHiBins; b += blockDim.x) {
     hist[b] = p.hist1[(int64_t)n * kHiBins + b];
@@ -699,6 +714,7 @@ __global__ void __launch_bounds__(1024) hi_topk_kernel(const __grid_constant__ H
   }
   for (int t = k_eff + threadIdx.x; t < p.top_k; t += blockDim.x) out[t] = -1;
   if (threadIdx.x == 0) p.n_sel[n] = k_eff;
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -751,6 +767,7 @@ __global__ void __launch_bounds__(256) hi_gather_kernel(const __nv_bfloat16* __r
                                                         __nv_bfloat16* __restrict__ packed,
                                                         int32_t* __restrict__ counts) {
   const int n = blockIdx.y;
+  griddep_wait();  // the selection
   const int L = seqlens[n];
   const int i = L - 1;
   const int sink_rows = (int)min((int64_t)w.sink_end, (int64_t)L);
@@ -790,6 +807,7 @@ __global__ void __launch_bounds__(256) hi_gather_kernel(const __nv_bfloat16* __r
     const int e = threadIdx.x + it * 256, r = e / 72, c = e % 72;
     if (src[r] != -1) reinterpret_cast<uint4*>(packed + ((int64_t)n * cap_rows + j0 + r) * 576)[c] = v[it];
   }
+  griddep_launch_dependents();
 }
 
 }  // namespace loza

@@ -280,7 +280,9 @@ loza_status setup_decode_mla(const void* q, const void* k_cache, const void* v_c
 
 // Point the kernel at its workspace (unless the plan merges on chip) and launch.
 loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t batch, uint8_t* ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool after = false) {
+  // after: launched with programmatic stream serialization behind the kernel
+  // that produced its rows and lengths (the kernels wait for it first)
   if (plan.half_block) {
     // the kernel's merge gives each split 512 / nsplit whole value columns
     if (plan.nsplit != 1 && plan.nsplit != 2 && plan.nsplit != 4) return LOZA_ERR_UNSUPPORTED;
@@ -292,13 +294,15 @@ loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t
     cfg.blockDim = dim3(kHbThreads, 1, 1);
     cfg.dynamicSmemBytes = DecodeHbLayout::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = plan.nsplit;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = after ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, ssa_decode_mla_hb_kernel, prm) != cudaSuccess) return LOZA_ERR_CUDA;
   } else if (!plan.cluster) {
     const DecodeWorkspace wl = decode_workspace(batch, plan);
@@ -322,13 +326,15 @@ loza_status launch_decode_mla(DecodeParams& prm, const DecodePlan& plan, int32_t
     cfg.blockDim = dim3(kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = DecodeLayout::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = plan.nsplit;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = after ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, ssa_decode_mla_kernel<true>, prm) != cudaSuccess) return LOZA_ERR_CUDA;
   }
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -601,6 +607,25 @@ bool hi_args_ok(const void* k_index, int64_t index_batch_stride, int64_t index_r
       index_batch_stride < (int64_t)max_seqlen * index_row_stride)
     return false;
   return true;
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the kernel before it in the stream finishes (it calls griddep_wait before
+// reading that kernel's results), hiding the launch gap of a chain.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Index keys as a 3-D tensor {d, rows, batch}: 128-row x 64-column tiles with
@@ -1204,13 +1229,21 @@ loza_status hi_select_launch(const void* q_index, const void* k_index, int64_t i
     hi_page_scores_kernel<<<dim3((unsigned)((hp.pages_per_seq + 255) / 256), batch), 256, 0, st>>>(hp);
     ++launches;
   }
-  hi_page_select_kernel<<<batch, 1024, 0, st>>>(hp);
+  // each kernel after the first waits (griddep_wait) for the one before it
   const int64_t items = (int64_t)batch * ((top_pages + kHiTokPages - 1) / kHiTokPages);
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(items, 3 * (int64_t)sm_count()));
-  hi_tokens_kernel<<<grid, kHiTokThreads, HiTokLayout::SMEM_ALLOC, st>>>(hp);
   const int64_t slices = ((int64_t)top_pages * kHiPage + kHiCollectKeys - 1) / kHiCollectKeys;
-  hi_topk_collect_kernel<<<dim3((unsigned)slices, batch), 256, 0, st>>>(hp);
-  hi_topk_kernel<<<batch, 1024, HiTopkLayout::bytes(hp.pages_per_seq), st>>>(hp);
+  const bool chained = hp.pages_per_seq >= 1;  // page selection follows the page scores
+  auto launch = [&](auto kernel, dim3 g, dim3 b, size_t sm, bool after) {
+    if (after) return launch_after(kernel, g, b, sm, st, hp);
+    kernel<<<g, b, sm, st>>>(hp);
+    return cudaGetLastError();
+  };
+  if (launch(hi_page_select_kernel, dim3(batch), dim3(1024), 0, chained) != cudaSuccess ||
+      launch(hi_tokens_kernel, dim3(grid), dim3(kHiTokThreads), HiTokLayout::SMEM_ALLOC, true) != cudaSuccess ||
+      launch(hi_topk_collect_kernel, dim3((unsigned)slices, batch), dim3(256), 0, true) != cudaSuccess ||
+      launch(hi_topk_kernel, dim3(batch), dim3(1024), HiTopkLayout::bytes(hp.pages_per_seq), true) != cudaSuccess)
+    return LOZA_ERR_CUDA;
   g_launches.fetch_add(launches, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
 }
@@ -1239,12 +1272,15 @@ loza_status hi_attend_launch(const void* kv_cache, int64_t cache_batch_stride, i
                              const DecodePlan& plan, cudaStream_t st) {
   if (w.cap_rows > 0) {
     const SsaWindow win{p.block_size, p.n_sink * p.block_size, p.n_local};
-    hi_gather_kernel<<<dim3(w.cap_rows / 32, batch), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(kv_cache), cache_batch_stride, cache_row_stride, seqlens, win, list,
-        std::max(top_k, 1), reinterpret_cast<const int32_t*>(ws + w.n_sel), w.cap_rows,
-        reinterpret_cast<__nv_bfloat16*>(ws + w.packed), reinterpret_cast<int32_t*>(ws + w.counts));
+    // after the selection or the compaction of a caller's list
+    if (launch_after(hi_gather_kernel, dim3(w.cap_rows / 32, batch), dim3(256), 0, st,
+                     static_cast<const __nv_bfloat16*>(kv_cache), cache_batch_stride, cache_row_stride, seqlens, win,
+                     list, std::max(top_k, 1), reinterpret_cast<const int32_t*>(ws + w.n_sel), w.cap_rows,
+                     reinterpret_cast<__nv_bfloat16*>(ws + w.packed),
+                     reinterpret_cast<int32_t*>(ws + w.counts)) != cudaSuccess)
+      return LOZA_ERR_CUDA;
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (cudaGetLastError() != cudaSuccess) return LOZA_ERR_CUDA;
+    return launch_decode_mla(prm, plan, batch, ws + w.dec, st, /*after=*/true);
   }
   return launch_decode_mla(prm, plan, batch, ws + w.dec, st);
 }

@@ -108,6 +108,14 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
+// Programmatic dependent launch. griddep_wait: wait until the kernel before
+// this one in the stream has completed and its writes are visible (a no-op
+// when this kernel was not launched with programmatic stream serialization).
+// griddep_launch_dependents: let the next kernel start launching; its own
+// griddep_wait still waits for this grid's completion.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA,
 // tensor cores) before they read that memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
