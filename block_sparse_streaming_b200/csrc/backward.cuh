@@ -5,22 +5,26 @@
 // selected keys (recomputed from the forward LSE), D_i = dO_i . O_i,
 // dP = dO V^T, dS = P o (dP - D):
 //     dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO.
-// Gradients are written by exactly one owner CTA per output tile (no atomics):
-//   ssa_bwd_dq_kernel     owner of a 128-query tile; walks the <= s+l key
-//                         blocks its window selects (S, dP, dQ += dS K).
-//   ssa_bwd_dkdv_kernel   owner of a 128-key block; walks the query blocks
-//                         that select it: j = k .. k+l-1 ("local" part). A sink
-//                         block (k < s) is also selected by every later query
-//                         block; those "far" query blocks are handled by extra
-//                         CTAs in fixed chunks, and every contribution to a
-//                         sink block goes to an fp32 partial in the workspace.
-//   ssa_bwd_sink_reduce   adds a sink block's partials in a fixed order
+// Gradients are written by exactly one owner CTA per output tile (no atomics).
+// Tiles are 128 tokens; the window (any power-of-two block size b) is applied
+// per element where a tile is only partly visible:
+//   ssa_bwd_dq_kernel     owner of a 128-query tile; walks the key tiles its
+//                         window reads (S, dP, dQ += dS K).
+//   ssa_bwd_dkdv_kernel   owner of a 128-key tile; walks the query tiles that
+//                         see it through the local window: k .. (with b = 128,
+//                         l tiles; bwd_local_end in general). A tile holding a
+//                         sink key is also seen by every later query tile;
+//                         those "far" query tiles are handled by extra CTAs in
+//                         fixed chunks, and every contribution to such a tile
+//                         goes to an fp32 partial in the workspace.
+//   ssa_bwd_sink_reduce   adds a sink tile's partials in a fixed order
 //                         (deterministic) and writes its dK, dV.
 //   ssa_bwd_preprocess    D = rowsum(dO o O), bandwidth bound.
 #pragma once
 
 #include <cuda.h>
 
+#include "prefill.cuh"
 #include "sm100.cuh"
 
 namespace loza {
@@ -39,11 +43,31 @@ struct BwdParams {
   float* partial;      // sink partials [B][s][H][nslots][128][DQK + DV]
   int n_heads;
   int n_sink, n_local;
-  int nslots;          // partial slots per (sequence, sink block, head)
+  int block;           // b, tokens per block of the window (a power of two)
+  int sink_end;        // s * b: keys below it are sinks
+  int n_sink_tiles;    // 128-key tiles holding a sink key: ceil(s * b / 128)
+  int nslots;          // partial slots per (sequence, sink tile, head)
   int far_mode;        // dK/dV kernel: 0 = owners, 1 = far sink chunks
   float scale;         // softmax scale
   float scale_log2;    // scale * log2(e)
 };
+
+// Query tiles [k, bwd_local_end(k)) see key tile k through the local part of
+// the window: the last query that does is the last i with lo(i) <= 128k + 127,
+// i.e. i < (floor((128k + 127) / b) + l) * b. Beyond it only sink keys are seen.
+__host__ __device__ __forceinline__ int bwd_local_end(int k, int b, int n_local) {
+  const int64_t i_end = ((int64_t)(k * kTile + kTile - 1) / b + n_local) * b;  // first query past the range
+  return (int)((i_end - 1) / kTile + 1);
+}
+
+// Bits q = 0 .. 63 of the queries i0 + q that see key t: t <= i and (t is a
+// sink or i < (floor(t / b) + l) * b).
+__device__ __forceinline__ uint64_t bwd_key_mask(int64_t t, int64_t i0, int b, int sink_end, int n_local) {
+  const int64_t lo = t - i0;
+  const int64_t hi = t < sink_end ? 64 : ((t / b + n_local) * b - i0);
+  auto below = [](int64_t x) -> uint64_t { return x <= 0 ? 0ull : (x >= 64 ? ~0ull : ((1ull << x) - 1ull)); };
+  return below(hi) & ~below(lo);
+}
 
 // ---------------------------------------------------------------------------
 // D = rowsum(dO o O) over DV columns; one half-warp per (token, head) row.
@@ -114,7 +138,8 @@ __global__ void __launch_bounds__(kBwdDqThreads, 1) ssa_bwd_dq_kernel(const __gr
   const int seq_start = p.cu_seqlens[seq];
   const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
   if (qb * kTile >= seq_len) return;
-  const BlockWalk walk(qb, p.n_sink, p.n_local);
+  const BlockWalk walk(qb, p.n_sink, p.n_local, p.block);
+  const SsaWindow win{p.block, walk.sink_end, p.n_local};
   const int nb = walk.count;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = smem_u32(smem);
@@ -276,16 +301,18 @@ __global__ void __launch_bounds__(kBwdDqThreads, 1) ssa_bwd_dq_kernel(const __gr
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(LY::BAR_FREE));
-      const bool diag = walk.block(b) == qb;
+      // keys of this tile the row does not see (the diagonal, and tiles at
+      // the window's edges when b < 128): bit j for key 64 * half + j
+      const int kb = walk.block(b);
+      const uint64_t vis = walk.masked(kb, qb) ? RowMask(win, qpos, kb * kTile).bits64(64 * half) : ~0ull;
       uint32_t pk[2][16];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         float ds2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int key = 64 * half + 2 * i + e;
           float pr = ex2_approx(fmaf(s[2 * i + e], c2, -lse2));
-          if (diag && key > row) pr = 0.f;
+          if (!((vis >> (2 * i + e)) & 1ull)) pr = 0.f;
           ds2[e] = pr * (dp[2 * i + e] - dd);
         }
         pk[i >> 4][i & 15] = pack_bf16(ds2[0], ds2[1]);
@@ -344,8 +371,8 @@ __global__ void __launch_bounds__(kBwdDqThreads, 1) ssa_bwd_dq_kernel(const __gr
 }
 
 // ---------------------------------------------------------------------------
-// dK / dV: one CTA per (key block, head, sequence) in owner mode, or per
-// (far chunk, sink block x head, sequence) in far mode.
+// dK / dV: one CTA per (key tile, head, sequence) in owner mode, or per
+// (far chunk, sink tile x head, sequence) in far mode.
 // TMEM: S^T [0,128) (P^T and later dS^T packed into [0,64)), dP^T [64,192),
 //       dV [192, 192+DV), dK [192+DV, 192+DV+DQK).
 // ---------------------------------------------------------------------------
@@ -384,13 +411,13 @@ __global__ void __launch_bounds__(kBwdDkvThreads, 1) ssa_bwd_dkdv_kernel(const _
     head = blockIdx.y;
     if (kblk >= nq) return;
     j_lo = kblk;
-    j_hi = min(nq, kblk + p.n_local);
-    if (kblk < p.n_sink) slot = 0;
+    j_hi = min(nq, bwd_local_end(kblk, p.block, p.n_local));
+    if (kblk < p.n_sink_tiles) slot = 0;
   } else {
-    kblk = blockIdx.y % p.n_sink;
-    head = blockIdx.y / p.n_sink;
-    if (kblk >= nq) return;  // no such sink block: its partial slots are never read
-    j_lo = kblk + p.n_local + blockIdx.x * kSinkChunk;
+    kblk = blockIdx.y % p.n_sink_tiles;
+    head = blockIdx.y / p.n_sink_tiles;
+    if (kblk >= nq) return;  // no such sink tile: its partial slots are never read
+    j_lo = bwd_local_end(kblk, p.block, p.n_local) + blockIdx.x * kSinkChunk;
     j_hi = min(nq, j_lo + kSinkChunk);
     slot = 1 + blockIdx.x;
   }
@@ -400,7 +427,7 @@ __global__ void __launch_bounds__(kBwdDkvThreads, 1) ssa_bwd_dkdv_kernel(const _
   // sink partial destination: [seq][kblk][head][slot][128][DQK+DV]
   float* part = nullptr;
   if (slot >= 0)
-    part = p.partial + ((((int64_t)seq * p.n_sink + kblk) * p.n_heads + head) * p.nslots + slot) *
+    part = p.partial + ((((int64_t)seq * p.n_sink_tiles + kblk) * p.n_heads + head) * p.nslots + slot) *
                            (int64_t)(kTile * (DQK + DV));
   if (nj == 0) {
     // empty far chunk: its partial contributes zero
@@ -554,7 +581,10 @@ __global__ void __launch_bounds__(kBwdDkvThreads, 1) ssa_bwd_dkdv_kernel(const _
       ok = warp_wait(bar(LY::BAR_S), jj & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
-      const bool diag = (j == kblk);
+      // queries of block j that see this row's key (causality, and the
+      // window's end for a key that is not a sink): bit q for query 64 * half + q
+      const uint64_t vis = bwd_key_mask((int64_t)kblk * kTile + key, (int64_t)j * kTile + 64 * half, p.block,
+                                        p.sink_end, p.n_local);
       float pr[64];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -568,9 +598,8 @@ __global__ void __launch_bounds__(kBwdDkvThreads, 1) ssa_bwd_dkdv_kernel(const _
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = 32 * c + 4 * i4 + e;
-            const int col = 64 * half + i;  // query row of block j
             float v = ex2_approx(fmaf(sx[4 * i4 + e], p.scale_log2, -lv[e]));
-            if (diag && col < key) v = 0.f;
+            if (!((vis >> i) & 1ull)) v = 0.f;
             pr[i] = v;
           }
         }
@@ -684,13 +713,14 @@ __global__ void __launch_bounds__(kBwdDkvThreads, 1) ssa_bwd_dkdv_kernel(const _
 }
 
 // ---------------------------------------------------------------------------
-// Sink blocks: dK, dV = sum of the partial slots, in slot order.
-// grid (128 key rows, s * H, B); thread = column of [DQK | DV].
+// Sink tiles (the 128-key tiles holding a sink key): dK, dV = sum of the
+// partial slots, in slot order. grid (128 key rows, sink tiles * H, B);
+// thread = column of [DQK | DV].
 // ---------------------------------------------------------------------------
 template <int DQK, int DV>
 __global__ void __launch_bounds__(DQK + DV) ssa_bwd_sink_reduce(const BwdParams p) {
   const int key = blockIdx.x;
-  const int kblk = blockIdx.y % p.n_sink, head = blockIdx.y / p.n_sink, seq = blockIdx.z;
+  const int kblk = blockIdx.y % p.n_sink_tiles, head = blockIdx.y / p.n_sink_tiles, seq = blockIdx.z;
   const int seq_start = p.cu_seqlens[seq];
   const int seq_len = p.cu_seqlens[seq + 1] - seq_start;
   const int nq = (seq_len + kTile - 1) / kTile;
@@ -698,9 +728,9 @@ __global__ void __launch_bounds__(DQK + DV) ssa_bwd_sink_reduce(const BwdParams 
   if (kblk >= nq || kpos >= seq_len) return;
   const int col = threadIdx.x;
   // slots that received work: 0 (local) and the far chunks that start inside the sequence
-  const int far = max(0, nq - (kblk + p.n_local));
+  const int far = max(0, nq - bwd_local_end(kblk, p.block, p.n_local));
   const int used = min(p.nslots, 1 + (far + kSinkChunk - 1) / kSinkChunk);
-  const float* base = p.partial + (((int64_t)seq * p.n_sink + kblk) * p.n_heads + head) * p.nslots *
+  const float* base = p.partial + (((int64_t)seq * p.n_sink_tiles + kblk) * p.n_heads + head) * p.nslots *
                                       (int64_t)(kTile * (DQK + DV));
   float acc = 0.f;
   for (int s = 0; s < used; ++s) acc += base[(int64_t)s * kTile * (DQK + DV) + (int64_t)key * (DQK + DV) + col];

@@ -347,16 +347,21 @@ struct BwdWorkspace {
   size_t d_off, part_off, total;
   int nslots;
 };
+// 128-key tiles that hold a sink key.
+int bwd_sink_tiles(const loza_ssa_params& p) {
+  return (int)(((int64_t)p.n_sink * p.block_size + kTile - 1) / kTile);
+}
 BwdWorkspace bwd_workspace(int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t n_heads, int d_qk,
                            int d_v, const loza_ssa_params& p) {
   BwdWorkspace w;
   const int nq_max = (max_seqlen + kTile - 1) / kTile;
-  // sink block 0 has the most "far" query blocks: those at or after block l
-  const int far = nq_max > p.n_local ? nq_max - p.n_local : 0;
+  // sink tile 0 has the most "far" query tiles: those past its local range
+  const int far = std::max(0, nq_max - bwd_local_end(0, p.block_size, p.n_local));
   w.nslots = 1 + (far + kSinkChunk - 1) / kSinkChunk;
   w.d_off = 0;
   w.part_off = ((size_t)total_tokens * n_heads * sizeof(float) + 255) / 256 * 256;
-  w.total = w.part_off + (size_t)batch * p.n_sink * n_heads * w.nslots * kTile * (d_qk + d_v) * sizeof(float);
+  w.total = w.part_off +
+            (size_t)batch * bwd_sink_tiles(p) * n_heads * w.nslots * kTile * (d_qk + d_v) * sizeof(float);
   return w;
 }
 
@@ -381,14 +386,14 @@ loza_status launch_backward(BwdParams& prm, const void* out, const void* dout, i
   ssa_bwd_dq_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdDqThreads, LQ::SMEM_BYTES, st>>>(prm);
   ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(nq_max, prm.n_heads, batch), kBwdDkvThreads, LK::SMEM_BYTES, st>>>(prm);
   g_launches.fetch_add(2, std::memory_order_relaxed);
-  if (prm.n_sink > 0) {
+  if (prm.n_sink_tiles > 0) {
     if (prm.nslots > 1) {
       prm.far_mode = 1;
-      ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(prm.nslots - 1, prm.n_heads * prm.n_sink, batch), kBwdDkvThreads,
+      ssa_bwd_dkdv_kernel<DQK, DV><<<dim3(prm.nslots - 1, prm.n_heads * prm.n_sink_tiles, batch), kBwdDkvThreads,
                                      LK::SMEM_BYTES, st>>>(prm);
       g_launches.fetch_add(1, std::memory_order_relaxed);
     }
-    ssa_bwd_sink_reduce<DQK, DV><<<dim3(kTile, prm.n_heads * prm.n_sink, batch), DQK + DV, 0, st>>>(prm);
+    ssa_bwd_sink_reduce<DQK, DV><<<dim3(kTile, prm.n_heads * prm.n_sink_tiles, batch), DQK + DV, 0, st>>>(prm);
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
   return cudaGetLastError() == cudaSuccess ? LOZA_OK : LOZA_ERR_CUDA;
@@ -793,7 +798,7 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
     return host_layout(h, host_chunk_cap(batch, total_tokens), pf, n_heads, n_kv_heads, d_qk, d_v).total;
   }
   if (op == LOZA_OP_BACKWARD) {
-    if (!window_block128(p)) return 0;
+    if (!window_ok(p)) return 0;
     if (n_kv_heads != n_heads || p.n_local == LOZA_UNBOUNDED || total_tokens < 1) return 0;
     if (!((d_qk == 64 && d_v == 64) || (d_qk == 192 && d_v == 128))) return 0;
     return bwd_workspace(batch, total_tokens, max_seqlen, n_heads, d_qk, d_v, p).total;
@@ -1121,9 +1126,10 @@ loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const
       max_seqlen > total_tokens)
     return LOZA_ERR_INVALID_ARG;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
-  if (!window_block128(p)) return LOZA_ERR_UNSUPPORTED;
+  if (!window_ok(p)) return LOZA_ERR_UNSUPPORTED;
   if (p.n_local == LOZA_UNBOUNDED) return LOZA_ERR_UNSUPPORTED;
-  if (n_kv_heads != n_heads || n_heads > 65535 / (p.n_sink > 0 ? p.n_sink : 1)) return LOZA_ERR_UNSUPPORTED;
+  const int sink_tiles = bwd_sink_tiles(p);
+  if (n_kv_heads != n_heads || n_heads > 65535 / std::max(sink_tiles, 1)) return LOZA_ERR_UNSUPPORTED;
   const bool d64 = (d_qk == 64 && d_v == 64), d192 = (d_qk == 192 && d_v == 128);
   if (!d64 && !d192) return LOZA_ERR_UNSUPPORTED;
   const BwdWorkspace wl = bwd_workspace(batch, total_tokens, max_seqlen, n_heads, d_qk, d_v, p);
@@ -1149,6 +1155,9 @@ loza_status loza_ssa_backward(const void* q, const void* k, const void* v, const
   prm.n_heads = n_heads;
   prm.n_sink = p.n_sink;
   prm.n_local = p.n_local;
+  prm.block = p.block_size;
+  prm.sink_end = p.n_sink * p.block_size;
+  prm.n_sink_tiles = sink_tiles;
   prm.nslots = wl.nslots;
   prm.scale = p.scale;
   prm.scale_log2 = p.scale * 1.4426950408889634f;

@@ -46,9 +46,10 @@
  *     block: {1, 16, 1024} is the fixed part of the streaming-aware index of
  *     page 4 ("LongCat Sparse Attention ...", agihunt.info), 16 sink tokens
  *     and a 1,024-token sliding window that includes the query. The prefill
- *     and decode entry points take any such window; loza_ssa_backward,
- *     loza_ssa_prefill_host and the sharded prefill need b = 128
- *     (LOZA_ERR_UNSUPPORTED otherwise). Keys are read in tiles of 128 (64 in
+ *     and decode entry points take any such window, and so does
+ *     loza_ssa_backward (bounded windows only); loza_ssa_prefill_host and
+ *     the sharded prefill and backward need b = 128 (LOZA_ERR_UNSUPPORTED
+ *     otherwise). Keys are read in tiles of 128 (64 in
  *     the half-block decode): the cache rows of positions below seqlens[n]
  *     that share a tile with a visible key are read and must hold finite
  *     values (they are the sequence's own context); rows at or past

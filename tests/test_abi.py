@@ -198,13 +198,16 @@ def test_prefill_host_binding_rejects_before_any_device_work(L):
     assert L.loza_launch_count() == count
 
 
-def test_backward_needs_blocks_of_128(L):
-    """The backward works in blocks of 128 tokens: another block size is
-    refused (LOZA_ERR_UNSUPPORTED) before anything runs, and the workspace
-    query reports 0 for it."""
+def test_backward_window_checks(L):
+    """The backward takes any bounded window whose block size is a power of
+    two (it sizes a workspace for b = 64 and for the token window b = 1); a
+    block size that is not a power of two and the unbounded window are
+    refused (LOZA_ERR_UNSUPPORTED) before anything runs."""
     vp = ctypes.c_void_p
+    for params in (bss.Params(0.125, 64, 2, 14), bss.Params(0.125, 1, 16, 1024), bss.Params(0.125, 256, 1, 3)):
+        assert bss.workspace_size(bss.LOZA_OP_BACKWARD, 1, 256, 256, 4, 4, 64, 64, params) > 0
     count = L.loza_launch_count()
-    for params in (bss.Params(0.125, 64, 2, 14), bss.Params(0.125, 1, 16, 1024)):
+    for params in (bss.Params(0.125, 96, 1, 7), bss.Params(0.125, 128, 1, bss.LOZA_UNBOUNDED)):
         rc = L.loza_ssa_backward(vp(1 << 20), vp(1 << 21), vp(1 << 22), vp(1 << 23), vp(1 << 24), vp(1 << 25),
                                  vp(1 << 26), 1, 256, 256, 4, 4, 64, 64, params, vp(1 << 27), vp(1 << 28),
                                  vp(1 << 29), vp(1 << 30), 1 << 30, vp(0))
