@@ -74,8 +74,7 @@ bool window_ok(const loza_ssa_params& p) {
   if ((int64_t)p.n_sink * b > (int64_t(1) << 30) || (int64_t)p.n_local * b > (int64_t(1) << 30)) return false;
   return true;
 }
-// The backward, the host-buffer prefill and the sharded prefill work in
-// whole blocks of 128 tokens.
+// The host-buffer prefill works in whole blocks of 128 tokens.
 bool window_block128(const loza_ssa_params& p) { return window_ok(p) && p.block_size == kTile; }
 
 SsaWindow host_window(const loza_ssa_params& p) {

@@ -1,137 +1,164 @@
 """Sharding one long sequence's SSA prefill over ranks (one process per GPU).
 
-Rank r owns the query blocks [j0, j1) of the sequence (contiguous, equal
-shares of whole 128-token blocks) and the K/V rows of those blocks. A query in
-block j reads the sink blocks 0 .. s-1 and the local blocks j-l+1 .. j (page 1
-section 01 of the LoZA pages), so the rank also needs
+The window of query i (page 1 section 01 of the LoZA pages, blocks of b
+tokens) is the sink rows [0, s*b) and the local rows [lo(i), i] with
+lo(i) = max(0, (floor(i/b) - l + 1) * b). Rank r owns the rows [row0, row1)
+of the sequence (equal shares of whole units of U = max(b, 128) rows, so a
+share starts on a block and on a kernel tile) and the K/V rows of those rows.
+Its own queries then read
 
-    the sink blocks 0 .. s-1          (broadcast from rank 0) and
-    the halo blocks j0-l+1 .. j0-1    (sent by the left neighbour),
+    the sink rows [0, s*b)                     (broadcast from rank 0) and
+    the halo rows [row0 - (l-1)*b, row0)       (sent by the left neighbour),
 
-one exchange before any compute. It then runs the one-GPU prefill on a local
-sequence [sinks | halo | own blocks]: local block t = j - j0 + s + l - 1 of an
-own block j has the window {0 .. s-1} U {t-l+1 .. t}, which is exactly the
-sinks, the halo and the own blocks up to j, so the outputs of the own rows are
-those of the whole-sequence prefill. The query rows of the prepended blocks are
-zeros; their outputs are dropped (s + l - 1 blocks per rank).
+one exchange before any compute. It runs the one-GPU prefill on a local
+sequence
+
+    [sinks (s*b) | gap (zeros) | halo ((l-1)*b) | own rows],
+
+with the prefix (sinks, gap, halo) of P rows, P the smallest multiple of U that
+holds the sinks rounded up to whole 128-row tiles plus the halo. An own row i
+sits at local row i' = i - row0 + P. Because row0 and P are both multiples of U,
+floor(i'/b) - floor(i/b) = (P - row0)/b, so the local window of i' is the sinks
+plus [lo(i) - row0 + P, i']: the halo and the own rows up to i, the same keys
+as in the whole sequence. The gap rows lie past the sinks and before every own
+row's window, so no own query sees them. Because row0 and P are multiples of
+128, each own row and key keeps its place inside its 128-row tile, and the
+halo never shares a tile with the sinks (on either side). The kernels
+therefore walk the same key tiles in the same order, and the own rows'
+outputs are bit-identical to the whole-sequence prefill. The query rows of
+the prefix are zeros; their outputs are dropped.
 
 The exchange uses torch.distributed point-to-point send/recv and broadcast
 (NCCL over NVLink on GPUs, gloo on CPU) into each rank's own memory; kernels
-only ever read local memory. Every rank's share must hold at least s + l - 1
-blocks, so a halo never reaches past the left neighbour and a rank's halo
-never overlaps the sinks.
+only ever read local memory. Every rank's share must hold at least P rows, so a
+halo never reaches past the left neighbour and never overlaps the sink tiles.
 """
 from __future__ import annotations
 
 from dataclasses import dataclass
 
-BLOCK = 128
+TILE = 128  # rows of a query / key tile of the kernels
 
 
 @dataclass(frozen=True)
 class ShardPlan:
     rank: int
     world: int
-    j0: int          # first own query block
-    j1: int          # one past the last own query block (clipped to the sequence)
-    n_pre: int       # blocks prepended to the local sequence (0 on rank 0)
+    row0: int        # first own row
+    row1: int        # one past the last own row
+    pre_rows: int    # rows of the local prefix [sinks | gap | halo] (0 on rank 0)
     seq_len: int
+    sink_rows: int   # s * b
+    halo_rows: int   # (l - 1) * b
 
     @property
     def own_rows(self):
-        return self.j0 * BLOCK, min(self.j1 * BLOCK, self.seq_len)
+        return self.row0, self.row1
 
     @property
     def local_len(self):
-        lo, hi = self.own_rows
-        return self.n_pre * BLOCK + (hi - lo)
+        return self.pre_rows + (self.row1 - self.row0)
 
 
-def shard_plan(seq_len: int, world: int, rank: int, n_sink: int = 1, n_local: int = 7) -> ShardPlan:
-    """Equal shares of whole blocks (the last rank takes the ragged tail)."""
+def _round_up(x, m):
+    return (x + m - 1) // m * m
+
+
+def shard_plan(seq_len: int, world: int, rank: int, n_sink: int = 1, n_local: int = 7,
+               block: int = 128) -> ShardPlan:
+    """Equal shares of whole units of max(b, 128) rows (the last rank takes the ragged tail)."""
     if world < 1 or not 0 <= rank < world:
         raise ValueError("bad rank / world")
     if n_local < 1 or n_sink < 0:
         raise ValueError("sharding needs a bounded window (n_local >= 1)")
-    nb = (seq_len + BLOCK - 1) // BLOCK
-    per = (nb + world - 1) // world
-    need = n_sink + n_local - 1
-    if world > 1 and per < need:
-        raise ValueError(f"each rank needs at least {need} blocks ({need * BLOCK} tokens)")
-    if world > 1 and (world - 1) * per >= nb:
+    if block < 1 or block & (block - 1):
+        raise ValueError("block size must be a power of two")
+    unit = max(block, TILE)
+    sink_rows, halo_rows = n_sink * block, (n_local - 1) * block
+    pre = _round_up(_round_up(sink_rows, TILE) + halo_rows, unit)
+    n_units = (seq_len + unit - 1) // unit
+    per = (n_units + world - 1) // world
+    if world > 1 and per * unit < pre:
+        raise ValueError(f"each rank needs at least {pre} rows")
+    if world > 1 and (world - 1) * per >= n_units:
         raise ValueError("more ranks than shares of this sequence")
-    j0 = min(rank * per, nb)
-    j1 = min(j0 + per, nb)
-    return ShardPlan(rank, world, j0, j1, 0 if j0 == 0 else need, seq_len)
+    row0 = min(rank * per * unit, seq_len)
+    row1 = min(row0 + per * unit, seq_len)
+    return ShardPlan(rank, world, row0, row1, 0 if row0 == 0 else pre, seq_len, sink_rows, halo_rows)
 
 
-def exchange_kv(kv_own, plan: ShardPlan, n_sink: int = 1, n_local: int = 7, group=None):
-    """Assemble this rank's local K (or V, or latent) rows [sinks | halo | own]
-    from its own rows (a [rows, ...] tensor of the own blocks, on this rank's
-    device). Every rank must call it (collective: one broadcast, one
-    send/recv pair per neighbour)."""
+def _prefix(sinks, halo, plan: ShardPlan):
+    """[sinks | gap of zero rows | halo], the local prefix."""
+    import torch
+    gap = plan.pre_rows - plan.sink_rows - plan.halo_rows
+    zeros = torch.zeros((gap,) + tuple(sinks.shape[1:]), dtype=sinks.dtype, device=sinks.device)
+    return torch.cat([sinks, zeros, halo], dim=0)
+
+
+def exchange_kv(kv_own, plan: ShardPlan, group=None):
+    """Assemble this rank's local K (or V, or latent) rows [sinks | gap | halo |
+    own] from its own rows (a [rows, ...] tensor, on this rank's device).
+    Every rank must call it (collective: one broadcast, one send/recv pair per
+    neighbour)."""
     import torch
     import torch.distributed as dist
-    halo_rows = (n_local - 1) * BLOCK
-    sink_rows = n_sink * BLOCK
     # rows travel as raw bytes, which every backend moves
     dtype = kv_own.dtype
     kv_own = kv_own.contiguous().view(torch.uint8)
     tail = kv_own.shape[1:]
-    # sink blocks from rank 0 (its own first rows)
-    sinks = torch.empty((sink_rows,) + tail, dtype=kv_own.dtype, device=kv_own.device)
+    # the sink rows from rank 0 (its own first rows)
+    sinks = torch.empty((plan.sink_rows,) + tail, dtype=kv_own.dtype, device=kv_own.device)
     if plan.rank == 0:
-        sinks.copy_(kv_own[:sink_rows])
+        sinks.copy_(kv_own[:plan.sink_rows])
     if plan.world > 1:
         dist.broadcast(sinks, src=0, group=group)
-    # halo: the left neighbour's last l-1 blocks (its share is whole blocks, at least that many)
-    halo = torch.empty((halo_rows,) + tail, dtype=kv_own.dtype, device=kv_own.device)
+    # the halo: the left neighbour's last (l-1)*b rows (its share holds at least that many)
+    halo = torch.empty((plan.halo_rows,) + tail, dtype=kv_own.dtype, device=kv_own.device)
     ops = []
     if plan.world > 1:
         if plan.rank + 1 < plan.world:
-            ops.append(dist.P2POp(dist.isend, kv_own[kv_own.shape[0] - halo_rows:].contiguous(), plan.rank + 1,
+            ops.append(dist.P2POp(dist.isend, kv_own[kv_own.shape[0] - plan.halo_rows:].contiguous(), plan.rank + 1,
                                   group=group))
         if plan.rank > 0:
             ops.append(dist.P2POp(dist.irecv, halo, plan.rank - 1, group=group))
         if ops:
             for req in dist.batch_isend_irecv(ops):
                 req.wait()
-    if plan.n_pre == 0:
+    if plan.pre_rows == 0:
         return kv_own.view(dtype)
-    return torch.cat([sinks, halo, kv_own], dim=0).view(dtype)
+    return torch.cat([_prefix(sinks, halo, plan), kv_own], dim=0).view(dtype)
 
 
-def local_kv_from_full(kv_full, plan: ShardPlan, n_sink: int = 1, n_local: int = 7):
-    """The local rows [sinks | halo | own] that exchange_kv assembles, taken
-    directly from the whole sequence's rows (for one process standing in for
-    every rank)."""
+def local_kv_from_full(kv_full, plan: ShardPlan):
+    """The local rows that exchange_kv assembles, taken directly from the
+    whole sequence's rows (for one process standing in for every rank)."""
     import torch
     lo, hi = plan.own_rows
-    if plan.n_pre == 0:
+    if plan.pre_rows == 0:
         return kv_full[lo:hi]
-    halo_lo = lo - (n_local - 1) * BLOCK
-    return torch.cat([kv_full[: n_sink * BLOCK], kv_full[halo_lo:lo], kv_full[lo:hi]], dim=0)
+    prefix = _prefix(kv_full[:plan.sink_rows], kv_full[lo - plan.halo_rows:lo], plan)
+    return torch.cat([prefix, kv_full[lo:hi]], dim=0)
 
 
 def local_queries(q_own, plan: ShardPlan):
-    """Local query rows: zeros for the prepended blocks, then the own rows."""
+    """Local query rows: zeros for the prefix, then the own rows."""
     import torch
-    if plan.n_pre == 0:
+    if plan.pre_rows == 0:
         return q_own
-    pre = torch.zeros((plan.n_pre * BLOCK,) + tuple(q_own.shape[1:]), dtype=q_own.dtype, device=q_own.device)
+    pre = torch.zeros((plan.pre_rows,) + tuple(q_own.shape[1:]), dtype=q_own.dtype, device=q_own.device)
     return torch.cat([pre, q_own], dim=0)
 
 
-def _require_block128(params):
-    """The shard plan moves whole blocks of 128 tokens (the pages' b)."""
-    if params.block_size != BLOCK:
-        raise ValueError(f"sharding needs block_size {BLOCK}, got {params.block_size}")
+def _check_params(params, plan: ShardPlan):
+    """The plan must have been made for this window."""
+    if (params.n_local < 1 or plan.sink_rows != params.n_sink * params.block_size or
+            plan.halo_rows != (params.n_local - 1) * params.block_size):
+        raise ValueError("shard plan made for another window")
 
 
 def own_outputs(out_local, lse_local, plan: ShardPlan):
-    """The rows of the own blocks in the local outputs."""
-    off = plan.n_pre * BLOCK
-    return out_local[off:], lse_local[off:]
+    """The own rows of the local outputs."""
+    return out_local[plan.pre_rows:], lse_local[plan.pre_rows:]
 
 
 def prefill_sharded(q_own, k_own, v_own, params, plan: ShardPlan, group=None, latent_v: bool = False):
@@ -141,12 +168,12 @@ def prefill_sharded(q_own, k_own, v_own, params, plan: ShardPlan, group=None, la
     Returns (out, lse) of the own rows."""
     import torch
     from . import loza_ssa_prefill
-    _require_block128(params)
-    k_loc = exchange_kv(k_own, plan, params.n_sink, params.n_local, group)
+    _check_params(params, plan)
+    k_loc = exchange_kv(k_own, plan, group)
     if latent_v:
         v_loc = k_loc[..., : v_own.shape[-1]]
     else:
-        v_loc = exchange_kv(v_own, plan, params.n_sink, params.n_local, group)
+        v_loc = exchange_kv(v_own, plan, group)
     q_loc = local_queries(q_own, plan)
     cu = torch.tensor([0, q_loc.shape[0]], dtype=torch.int32, device=q_own.device)
     out, lse = loza_ssa_prefill(q_loc, k_loc, v_loc, cu, q_loc.shape[0], params)
@@ -156,47 +183,47 @@ def prefill_sharded(q_own, k_own, v_own, params, plan: ShardPlan, group=None, la
 # ---------------------------------------------------------------------------
 # Backward of the sharded prefill.
 #
-# Each rank runs the one-GPU backward on its local sequence [sinks | halo |
-# own]: the prepended rows get zero dO (and zero O), so their queries add
+# Each rank runs the one-GPU backward on its local sequence [sinks | gap |
+# halo | own]: the prefix rows get zero dO (and zero O), so their queries add
 # nothing to any gradient, and the own rows' dQ is exact. The key gradients of
-# the prepended rows are partial sums that belong to other ranks:
-#   halo rows (local blocks s .. s+l-2): the left neighbour's last l-1 blocks,
-#       sent back to it and added to its own dK, dV;
-#   sink rows (local blocks 0 .. s-1): every rank's share of the sink blocks'
-#       gradients, summed onto rank 0 (which owns the sinks) by a reduce.
+# the prefix rows are partial sums that belong to other ranks:
+#   halo rows: the left neighbour's last (l-1)*b rows, sent back to it and
+#       added to its own dK, dV;
+#   sink rows: every rank's share of the sink rows' gradients, summed onto
+#       rank 0 (which owns the sinks) by a reduce;
+#   gap rows: seen by no query with a nonzero dO, so zero, and dropped.
 # The additions are done in fp32.
 # ---------------------------------------------------------------------------
 def local_rows(x_own, plan: ShardPlan):
-    """Zero rows for the prepended blocks, then the own rows (q, out, dout, lse)."""
+    """Zero rows for the prefix, then the own rows (q, out, dout, lse)."""
     return local_queries(x_own, plan)
 
 
-def split_key_grads(dk_loc, dv_loc, plan: ShardPlan, n_sink: int = 1, n_local: int = 7):
-    """The local backward's dK, dV (rows [sinks | halo | own]) as fp32 parts:
-    (own dK, own dV, halo dK, halo dV, sink dK, sink dV); the halo and sink
-    parts are None on rank 0, which has no prepended rows."""
-    off = plan.n_pre * BLOCK
+def split_key_grads(dk_loc, dv_loc, plan: ShardPlan):
+    """The local backward's dK, dV (rows [sinks | gap | halo | own]) as fp32
+    parts: (own dK, own dV, halo dK, halo dV, sink dK, sink dV); the halo and
+    sink parts are None on rank 0, which has no prefix."""
+    off = plan.pre_rows
     own = (dk_loc[off:].float(), dv_loc[off:].float())
-    if plan.n_pre == 0:
+    if off == 0:
         return own + (None, None, None, None)
-    s_rows, h_rows = n_sink * BLOCK, (n_local - 1) * BLOCK
-    halo = (dk_loc[s_rows:s_rows + h_rows].float(), dv_loc[s_rows:s_rows + h_rows].float())
-    sink = (dk_loc[:s_rows].float(), dv_loc[:s_rows].float())
+    h0 = off - plan.halo_rows
+    halo = (dk_loc[h0:off].float(), dv_loc[h0:off].float())
+    sink = (dk_loc[:plan.sink_rows].float(), dv_loc[:plan.sink_rows].float())
     return own + halo + sink
 
 
-def settle_key_grads(dk_loc, dv_loc, plan: ShardPlan, n_sink: int = 1, n_local: int = 7, group=None):
-    """From the local backward's dK, dV (rows [sinks | halo | own]) return this
-    rank's own dK, dV with the other ranks' contributions added (fp32 sums,
-    then the input dtype): its right neighbour's halo part is added to its
-    last l-1 blocks, and on rank 0 every rank's sink part to its first s
-    blocks. Every rank must call it (collective)."""
+def settle_key_grads(dk_loc, dv_loc, plan: ShardPlan, group=None):
+    """From the local backward's dK, dV (rows [sinks | gap | halo | own])
+    return this rank's own dK, dV with the other ranks' contributions added
+    (fp32 sums, then the input dtype): its right neighbour's halo part is added
+    to its last (l-1)*b rows, and on rank 0 every rank's sink part to its
+    first s*b rows. Every rank must call it (collective)."""
     import torch
     import torch.distributed as dist
     out_dtype = dk_loc.dtype
-    dk, dv, hk, hv, sk_part, sv_part = split_key_grads(dk_loc, dv_loc, plan, n_sink, n_local)
-    halo_rows = (n_local - 1) * BLOCK
-    sink_rows = n_sink * BLOCK
+    dk, dv, hk, hv, sk_part, sv_part = split_key_grads(dk_loc, dv_loc, plan)
+    halo_rows, sink_rows = plan.halo_rows, plan.sink_rows
     if plan.world > 1:
         ops = []
         recv_k = recv_v = None
@@ -231,14 +258,14 @@ def backward_sharded(q_own, k_own, v_own, out_own, dout_own, lse_own, params, pl
     Returns (dq, dk, dv) of the own rows."""
     import torch
     from . import loza_ssa_backward
-    _require_block128(params)
-    k_loc = exchange_kv(k_own, plan, params.n_sink, params.n_local, group).contiguous()
-    v_loc = exchange_kv(v_own, plan, params.n_sink, params.n_local, group).contiguous()
+    _check_params(params, plan)
+    k_loc = exchange_kv(k_own, plan, group).contiguous()
+    v_loc = exchange_kv(v_own, plan, group).contiguous()
     q_loc = local_rows(q_own, plan).contiguous()
     o_loc = local_rows(out_own, plan).contiguous()
     do_loc = local_rows(dout_own, plan).contiguous()
     lse_loc = local_rows(lse_own, plan).contiguous()
     cu = torch.tensor([0, q_loc.shape[0]], dtype=torch.int32, device=q_own.device)
     dq, dk, dv = loza_ssa_backward(q_loc, k_loc, v_loc, o_loc, do_loc, lse_loc, cu, q_loc.shape[0], params)
-    dk_own, dv_own = settle_key_grads(dk, dv, plan, params.n_sink, params.n_local, group)
-    return dq[plan.n_pre * BLOCK:], dk_own, dv_own
+    dk_own, dv_own = settle_key_grads(dk, dv, plan, group)
+    return dq[plan.pre_rows:], dk_own, dv_own

@@ -47,9 +47,9 @@
  *     page 4 ("LongCat Sparse Attention ...", agihunt.info), 16 sink tokens
  *     and a 1,024-token sliding window that includes the query. The prefill
  *     and decode entry points take any such window, and so does
- *     loza_ssa_backward (bounded windows only); loza_ssa_prefill_host and
- *     the sharded prefill and backward need b = 128 (LOZA_ERR_UNSUPPORTED
- *     otherwise). Keys are read in tiles of 128 (64 in
+ *     loza_ssa_backward (bounded windows only); loza_ssa_prefill_host
+ *     needs b = 128 (LOZA_ERR_UNSUPPORTED otherwise). Keys are read in
+ *     tiles of 128 (64 in
  *     the half-block decode): the cache rows of positions below seqlens[n]
  *     that share a tile with a visible key are read and must hold finite
  *     values (they are the sequence's own context); rows at or past
