@@ -74,8 +74,6 @@ bool window_ok(const loza_ssa_params& p) {
   if ((int64_t)p.n_sink * b > (int64_t(1) << 30) || (int64_t)p.n_local * b > (int64_t(1) << 30)) return false;
   return true;
 }
-// The host-buffer prefill works in whole blocks of 128 tokens.
-bool window_block128(const loza_ssa_params& p) { return window_ok(p) && p.block_size == kTile; }
 
 SsaWindow host_window(const loza_ssa_params& p) {
   const bool unb = p.n_local == LOZA_UNBOUNDED;
@@ -788,7 +786,7 @@ size_t loza_ssa_workspace_size(int op, int32_t batch, int64_t total_tokens, int3
     return 0;
   }
   if (op == LOZA_OP_PREFILL_HOST) {
-    if (!window_block128(p)) return 0;
+    if (!window_ok(p)) return 0;
     if (total_tokens < max_seqlen || total_tokens > INT32_MAX || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v))
       return 0;
     const HostChunkPlan h = host_chunk_plan(max_seqlen, p);
@@ -927,7 +925,7 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, c
     if (cu_seqlens[n + 1] < cu_seqlens[n] || cu_seqlens[n + 1] - cu_seqlens[n] > max_seqlen)
       return LOZA_ERR_INVALID_ARG;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return LOZA_ERR_INVALID_ARG;
-  if (!window_block128(p) || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v)) return LOZA_ERR_UNSUPPORTED;
+  if (!window_ok(p) || !host_shape_ok(n_heads, n_kv_heads, d_qk, d_v)) return LOZA_ERR_UNSUPPORTED;
   const bool latent_v = (v == k);
   if (latent_v && d_v > d_qk) return LOZA_ERR_INVALID_ARG;
   const size_t need = loza_ssa_workspace_size(LOZA_OP_PREFILL_HOST, batch, total_tokens, max_seqlen, n_heads,
@@ -1001,23 +999,28 @@ loza_status loza_ssa_prefill_host(const void* q, const void* k, const void* v, c
     uint8_t* vd = latent_v ? kd : slot + w.v_off;
     uint8_t* od = slot + w.o_off;
     float* ld = reinterpret_cast<float*>(slot + w.l_off);
-    const int64_t pre_rows = ck.pre * kTile, own = ck.q1 - ck.q0;
+    const int64_t pre_rows = ck.pre, own = ck.q1 - ck.q0;
 
     // copy in: the slot's inputs are free once the chunk that used them ran
     if (g >= (size_t)slots) LOZA_CU(cudaStreamWaitEvent(hp.h2d, hp.run_done[sl], 0));
     if (pre_rows > 0) LOZA_CU(cudaMemsetAsync(qd, 0, (size_t)pre_rows * q_row, hp.h2d));
     LOZA_CU(cudaMemcpyAsync(qd + (size_t)pre_rows * q_row, qh + (size_t)(r0 + ck.q0) * q_row, (size_t)own * q_row,
                             cudaMemcpyDefault, hp.h2d));
+    // K (and V) rows: run 0, the gap as zero rows (read with the tiles around it
+    // and masked, so they must be finite), run 1
+    const int64_t at1 = ck.n0 + ck.gap;
     LOZA_CU(cudaMemcpyAsync(kd, kh + (size_t)(r0 + ck.src0) * k_row, (size_t)ck.n0 * k_row, cudaMemcpyDefault,
                             hp.h2d));
+    if (ck.gap > 0) LOZA_CU(cudaMemsetAsync(kd + (size_t)ck.n0 * k_row, 0, (size_t)ck.gap * k_row, hp.h2d));
     if (ck.n1 > 0)
-      LOZA_CU(cudaMemcpyAsync(kd + (size_t)ck.n0 * k_row, kh + (size_t)(r0 + ck.src1) * k_row, (size_t)ck.n1 * k_row,
+      LOZA_CU(cudaMemcpyAsync(kd + (size_t)at1 * k_row, kh + (size_t)(r0 + ck.src1) * k_row, (size_t)ck.n1 * k_row,
                               cudaMemcpyDefault, hp.h2d));
     if (!latent_v) {
       LOZA_CU(cudaMemcpyAsync(vd, vh + (size_t)(r0 + ck.src0) * v_row, (size_t)ck.n0 * v_row, cudaMemcpyDefault,
                               hp.h2d));
+      if (ck.gap > 0) LOZA_CU(cudaMemsetAsync(vd + (size_t)ck.n0 * v_row, 0, (size_t)ck.gap * v_row, hp.h2d));
       if (ck.n1 > 0)
-        LOZA_CU(cudaMemcpyAsync(vd + (size_t)ck.n0 * v_row, vh + (size_t)(r0 + ck.src1) * v_row,
+        LOZA_CU(cudaMemcpyAsync(vd + (size_t)at1 * v_row, vh + (size_t)(r0 + ck.src1) * v_row,
                                 (size_t)ck.n1 * v_row, cudaMemcpyDefault, hp.h2d));
     }
     LOZA_CU(cudaEventRecord(hp.in_done[sl], hp.h2d));

@@ -4,18 +4,24 @@
 // so that the PCIe copies in both directions overlap each other and the
 // kernels.
 //
-// A query in block j reads the sink blocks 0 .. s-1 and the local blocks
-// j-l+1 .. j (LongCat ZigZag Attention, page 1 section 01 (1)-(2)). A chunk of
-// own query blocks [j0, j1) therefore needs the K/V rows of the sinks, of the
-// halo blocks j0-l+1 .. j0-1 and of its own blocks. It runs the one-GPU prefill
-// on the local sequence [sinks | halo | own]: local block t = j - j0 + s + l - 1
-// of own block j has the window {0 .. s-1} U {t-l+1 .. t}, which is exactly
-// the sinks, the halo and the own blocks up to j, so the own rows come out as
-// in the whole-sequence prefill (the same kernel, the same keys in the same
-// order). The prepended query rows are zeros; their outputs are not copied
-// back. A chunk with j0 <= s + l - 1 has no gap between sinks and halo: its
-// local sequence is simply rows [0, end of chunk), with j0 prepended blocks.
-// The unbounded (full causal) window runs as one chunk.
+// The window of query i (LongCat ZigZag Attention, page 1 section 01 (1)-(2),
+// blocks of b tokens) is the sink rows [0, s*b) and the local rows [lo(i), i],
+// lo(i) = max(0, (floor(i/b) - l + 1) * b). A chunk of own query rows [q0, q1)
+// (q0 a multiple of U = max(b, 128)) therefore needs the K/V rows of the sinks,
+// of the halo [q0 - (l-1)*b, q0) and its own rows. It runs the one-GPU prefill
+// on the local sequence [sinks | gap | halo | own], whose prefix (sinks, gap of
+// zero rows, halo) holds P rows: the smallest multiple of U that fits the sinks
+// rounded up to whole 128-row tiles, plus the halo (P = (s + l - 1) * 128 and
+// no gap for b = 128). An own row i sits at local row i - q0 + P; q0 and P are
+// multiples of U, so floor(i/b) moves by whole blocks and the local window is
+// the sinks plus the halo and own rows up to i, the keys of the whole sequence;
+// the gap lies past the sinks and before every own row's window. Every row and
+// key keeps its place in its 128-row tile and the halo never shares a tile with
+// the sinks, so the kernels walk the same tiles in the same order and the own
+// rows come out bit for bit as in the whole-sequence prefill. The prepended
+// query rows are zeros; their outputs are not copied back. A chunk with q0 <= P
+// runs on rows [0, q1) of the sequence itself (q0 rows prepended). The
+// unbounded (full causal) window runs as one chunk.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -30,73 +36,83 @@ namespace {
 
 constexpr int kHostSlots = 3;          // chunks in flight: copy in, compute, copy out
 constexpr int64_t kHostChunks = 16;    // aim: about this many chunks per sequence
-constexpr int64_t kHostMinBlocks = 8;  // chunk size bounds, in blocks of 128 rows
-constexpr int64_t kHostMaxBlocks = 64;
+constexpr int64_t kHostMinRows = 1024; // chunk size bounds, in rows (rounded to whole units)
+constexpr int64_t kHostMaxRows = 8192;
 
 struct HostChunkPlan {
-  int64_t nb;        // blocks in the sequence
-  int64_t cb;        // own blocks per chunk
+  int64_t unit;      // rows per unit: max(b, 128)
+  int64_t nu;        // units in the sequence
+  int64_t cu;        // own units per chunk
   int64_t n_chunks;
-  int64_t pre_max;   // prepended blocks at most
+  int64_t pre;       // rows of the prefix [sinks | gap | halo] of a chunk past it (0: unbounded)
   int64_t rows_max;  // local rows of the largest chunk
 };
 
 HostChunkPlan host_chunk_plan(int64_t seq_len, const loza_ssa_params& p) {
   HostChunkPlan h;
-  h.nb = (seq_len + kTile - 1) / kTile;
+  const int64_t b = p.block_size;
+  h.unit = std::max<int64_t>(b, kTile);
+  h.nu = (seq_len + h.unit - 1) / h.unit;
   if (p.n_local == LOZA_UNBOUNDED) {
-    h.pre_max = 0;
-    h.cb = h.nb;
+    h.pre = 0;
+    h.cu = h.nu;
   } else {
-    h.pre_max = (int64_t)p.n_sink + p.n_local - 1;
-    int64_t cb = (h.nb + kHostChunks - 1) / kHostChunks;
-    // at least as many own blocks as prepended ones, so that the zero query
+    const int64_t sink_tiles_rows = ((int64_t)p.n_sink * b + kTile - 1) / kTile * kTile;
+    const int64_t halo = ((int64_t)p.n_local - 1) * b;
+    h.pre = (sink_tiles_rows + halo + h.unit - 1) / h.unit * h.unit;
+    const int64_t pre_units = h.pre / h.unit;
+    const int64_t min_units = (kHostMinRows + h.unit - 1) / h.unit;
+    const int64_t max_units = std::max<int64_t>(1, kHostMaxRows / h.unit);
+    int64_t cu = (h.nu + kHostChunks - 1) / kHostChunks;
+    // at least as many own rows as prepended ones, so that the zero query
     // rows cost at most as much as the own rows
-    cb = std::max(cb, std::max(h.pre_max, kHostMinBlocks));
-    cb = std::min(cb, std::max(kHostMaxBlocks, h.pre_max));
-    h.cb = std::min(cb, h.nb);
+    cu = std::max(cu, std::max(pre_units, min_units));
+    cu = std::min(cu, std::max(max_units, pre_units));
+    h.cu = std::min(cu, h.nu);
   }
-  h.n_chunks = (h.nb + h.cb - 1) / h.cb;
+  h.n_chunks = (h.nu + h.cu - 1) / h.cu;
   // a local sequence never holds more rows than the prefix up to its chunk's end
-  h.rows_max = std::min((h.pre_max + h.cb) * kTile, seq_len);
+  h.rows_max = std::min(h.pre + h.cu * h.unit, seq_len);
   return h;
 }
 
-// One chunk: own query rows [q0, q1), `pre` prepended blocks, and the K/V rows
-// copied into the local sequence as up to two runs of host rows.
+// One chunk: own query rows [q0, q1), `pre` prepended rows, and the K/V rows
+// of the local sequence: run 0 of host rows -> local row 0, then `gap` zero
+// rows, then run 1 -> local row n0 + gap.
 struct HostChunk {
   int64_t q0, q1, pre;
-  int64_t src0, n0, src1, n1;  // run 0 -> local row 0, run 1 -> local row n0
-  int64_t local_len() const { return pre * kTile + (q1 - q0); }
+  int64_t src0, n0, gap, src1, n1;
+  int64_t local_len() const { return pre + (q1 - q0); }
 };
 
 HostChunk host_chunk(const HostChunkPlan& h, int64_t c, int64_t seq_len, const loza_ssa_params& p) {
   HostChunk k;
-  const int64_t j0 = c * h.cb;
-  const int64_t j1 = std::min(j0 + h.cb, h.nb);
-  k.q0 = j0 * kTile;
-  k.q1 = std::min(j1 * kTile, seq_len);
-  if (p.n_local == LOZA_UNBOUNDED || j0 <= h.pre_max) {
-    k.pre = j0;
+  k.q0 = c * h.cu * h.unit;
+  k.q1 = std::min(k.q0 + h.cu * h.unit, seq_len);
+  if (p.n_local == LOZA_UNBOUNDED || k.q0 <= h.pre) {
+    k.pre = k.q0;
     k.src0 = 0;
     k.n0 = k.q1;
+    k.gap = 0;
     k.src1 = 0;
     k.n1 = 0;
   } else {
-    k.pre = h.pre_max;
+    const int64_t b = p.block_size;
+    k.pre = h.pre;
     k.src0 = 0;
-    k.n0 = (int64_t)p.n_sink * kTile;
-    k.src1 = (j0 - p.n_local + 1) * kTile;
+    k.n0 = (int64_t)p.n_sink * b;
+    k.src1 = k.q0 - ((int64_t)p.n_local - 1) * b;
+    k.gap = h.pre - k.n0 - (k.q0 - k.src1);
     k.n1 = k.q1 - k.src1;
   }
   return k;
 }
 
-// Upper bound of the chunks of a packed batch: a sequence of nb blocks is one
-// chunk if nb < kHostMinBlocks, otherwise chunks of at least kHostMinBlocks
-// blocks, at most nb / kHostMinBlocks + 1 of them.
+// Upper bound of the chunks of a packed batch: every chunk of a sequence but
+// its last holds at least kHostMinRows own rows, so a sequence of L rows has at
+// most L / kHostMinRows + 1 chunks.
 int64_t host_chunk_cap(int32_t batch, int64_t total_tokens) {
-  return 2 * (int64_t)batch + total_tokens / (kTile * kHostMinBlocks) + 1;
+  return 2 * (int64_t)batch + total_tokens / kHostMinRows + 1;
 }
 
 struct HostLayout {

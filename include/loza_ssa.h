@@ -47,9 +47,8 @@
  *     page 4 ("LongCat Sparse Attention ...", agihunt.info), 16 sink tokens
  *     and a 1,024-token sliding window that includes the query. The prefill
  *     and decode entry points take any such window, and so does
- *     loza_ssa_backward (bounded windows only); loza_ssa_prefill_host
- *     needs b = 128 (LOZA_ERR_UNSUPPORTED otherwise). Keys are read in
- *     tiles of 128 (64 in
+ *     loza_ssa_backward (bounded windows only) and loza_ssa_prefill_host.
+ *     Keys are read in tiles of 128 (64 in
  *     the half-block decode): the cache rows of positions below seqlens[n]
  *     that share a tile with a visible key are read and must hold finite
  *     values (they are the sequence's own context); rows at or past
@@ -157,13 +156,17 @@ loza_status loza_ssa_prefill(const void *q, const void *k, const void *v,
  * run asynchronously and overlap; pageable memory gives the same results but
  * the copies serialise) or device memory; they are addressed through the
  * unified address space.
- * How it runs: each sequence's query blocks are cut into chunks (about 16 per
- * sequence, 8 to 64 blocks of 128 rows each, at least s + l - 1 blocks; the
- * unbounded window is one chunk per sequence). A chunk's own blocks
- * [j0, j1) run as the local sequence [sink blocks | blocks j0-l+1 .. j0-1 |
- * own blocks] with zero query rows for the prepended blocks: by the window
- * rule (page 1 section 01 (1) of the LoZA pages) every own query sees exactly
- * its keys of the whole sequence. Up to three chunks are in flight: the
+ * How it runs: each sequence's query rows are cut into chunks of whole units
+ * of U = max(b, 128) rows (about 16 chunks per sequence, of 1,024 to 8,192
+ * rows, at least as many as the prefix below; the unbounded window is one
+ * chunk per sequence). A chunk's own rows [q0, q1) run as the local sequence
+ * [sink rows | zero rows | rows q0-(l-1)b .. q0-1 | own rows] with zero query
+ * rows before the own ones; the prefix is the smallest multiple of U that
+ * holds the sink rows rounded up to whole 128-row tiles plus the (l-1)b halo
+ * rows (exactly s + l - 1 blocks for b = 128). By the window rule (page 1
+ * section 01 (1) of the LoZA pages) every own query then sees exactly its
+ * keys of the whole sequence, each in the same place of its 128-row tile, so
+ * the kernels read them in the same order. Up to three chunks are in flight: the
  * copy-in of one, the kernels of the next and the copy-out of a third
  * overlap, on two copy streams that the library creates on the first call per
  * device and keeps until exit. The call is asynchronous on `stream`: when

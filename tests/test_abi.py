@@ -144,7 +144,7 @@ def _call_prefill_host(L, q=1 << 20, k=1 << 21, v=1 << 22, cu=(0, 4096), batch=N
     (dict(dqk=96, dv=96), -2),                        # head dims not compiled
     (dict(dqk=576, dv=512, H=3, Hkv=1), -2),          # absorbed needs an even head count
     (dict(params=bss.Params(0.1, n_local=0)), -2),    # empty local window
-    (dict(params=bss.Params(0.1, 64, 2, 14)), -2),    # chunks move whole blocks of 128 tokens
+    (dict(params=bss.Params(0.1, 96, 1, 7)), -2),     # block size not a power of two
     (dict(ws=0), -1),                                 # no workspace
     (dict(ws=(1 << 28) + 16), -1),                    # workspace not 256-byte aligned
     (dict(ws_bytes=1024), -3),                        # workspace too small
@@ -174,6 +174,13 @@ def test_prefill_host_workspace_size():
     # the unbounded window runs as one chunk per sequence: a slot of the longest sequence
     dense = size(1, 8192, 8192, 4, 4, 64, 64, bss.Params(0.125, n_local=bss.LOZA_UNBOUNDED))
     assert dense >= 8192 * 4 * (64 * 2 * 4 + 4)
+    # other block sizes: slots of whole max(b, 128)-row units plus the chunk's prefix
+    row = 64 * 576 * 2 + 64 * 512 * 2 + 2 * 576 * 2 + 64 * 4
+    tok = size(1, 1 << 20, 1 << 20, 64, 1, 576, 512, bss.Params(0.1, 1, 16, 1024))  # prefix 1,152 rows
+    assert huge < tok < 3 * (1152 + 8192) * row + (256 << 20)
+    wide = size(1, 1 << 20, 1 << 20, 64, 1, 576, 512, bss.Params(0.1, 1024, 1, 4))
+    assert wide > 3 * (4 * 1024) * 64 * 576 * 2   # prefix 4,096 rows + at least one 1,024-row unit
+    assert size(1, 4096, 4096, 64, 1, 576, 512, bss.Params(0.1, 96, 1, 7)) == 0
 
 
 def test_prefill_host_binding_rejects_before_any_device_work(L):

@@ -31,15 +31,24 @@ def host_bf16(bits, pinned):
 
 
 def check_host_call(bss, oracle_mod, params, qh, kh, vh, qd, kd, vd, q_bits, k_bits, v_bits, Hkv, rows=None,
-                    lens=None):
+                    lens=None, poison=False):
     """Run the host entry point, then compare it bit for bit with the device call
     and element by element with the oracle (on ``rows``, all rows if None).
-    lens: the packed sequence lengths (one sequence of all rows if None)."""
+    lens: the packed sequence lengths (one sequence of all rows if None).
+    poison: hand the call a workspace of 0xFF bytes (bf16 NaN), so that any
+    slot row the chunks read without writing it first shows in the outputs."""
     import torch
     L, H = qh.shape[0], qh.shape[1]
     lens = [L] if lens is None else lens
     cu_np = synth.cu_seqlens(lens)
-    out_h, lse_h = bss.loza_ssa_prefill_host(qh, kh, vh, params, cu_seqlens=None if len(lens) == 1 else cu_np)
+    ws = None
+    if poison:
+        size = bss.workspace_size(bss.LOZA_OP_PREFILL_HOST, len(lens), L, max(lens), H, Hkv, qh.shape[2],
+                                  vh.shape[2], params)
+        assert size > 0
+        ws = torch.full((size,), 255, dtype=torch.uint8, device="cuda")
+    out_h, lse_h = bss.loza_ssa_prefill_host(qh, kh, vh, params, cu_seqlens=None if len(lens) == 1 else cu_np,
+                                             workspace=ws)
     torch.cuda.synchronize()
     assert bss.device_status() == 0
     assert out_h.device.type == "cpu" and lse_h.device.type == "cpu"
@@ -48,7 +57,7 @@ def check_host_call(bss, oracle_mod, params, qh, kh, vh, qd, kd, vd, q_bits, k_b
     torch.cuda.synchronize()
     assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16)), "O differs from the device call"
     assert torch.equal(lse_h.view(torch.int32), lse_d.cpu().view(torch.int32)), "LSE differs from the device call"
-    o_ref, lse_ref = oracle_mod.forward(q_bits, k_bits, v_bits, cu_np, H, Hkv, 128, params.n_sink,
+    o_ref, lse_ref = oracle_mod.forward(q_bits, k_bits, v_bits, cu_np, H, Hkv, params.block_size, params.n_sink,
                                         params.n_local, params.scale, rows=rows)
     o_got = out_h.to(torch.float32).numpy().astype(np.float64)
     lse_got = lse_h.numpy().astype(np.float64)
@@ -60,7 +69,7 @@ def check_host_call(bss, oracle_mod, params, qh, kh, vh, qd, kd, vd, q_bits, k_b
 
 
 def host_case(bss, oracle_mod, seed, L, H, Hkv, dqk, dv, scale, n_sink=1, n_local=7, latent=False,
-              pinned=True, lens=None):
+              pinned=True, lens=None, block=128, poison=False):
     """L tokens, one sequence or packed as `lens` (summing to L)."""
     g = synth.rng(seed)
     q = synth.normal_bits(g, (L, H, dqk))
@@ -76,9 +85,9 @@ def host_case(bss, oracle_mod, seed, L, H, Hkv, dqk, dv, scale, n_sink=1, n_loca
         v_bits = synth.normal_bits(g, (L, Hkv, dv))
         kh, vh = host_bf16(k_bits, pinned), host_bf16(v_bits, pinned)
         kd, vd = to_dev(k_bits), to_dev(v_bits)
-    params = bss.Params(scale, 128, n_sink, n_local)
+    params = bss.Params(scale, block, n_sink, n_local)
     check_host_call(bss, oracle_mod, params, host_bf16(q, pinned), kh, vh, to_dev(q), kd, vd, q, k_bits, v_bits,
-                    Hkv, lens=lens)
+                    Hkv, lens=lens, poison=poison)
 
 
 @pytest.mark.parametrize("L", [1, 200, 3000, 5000])
@@ -111,6 +120,30 @@ def test_host_absorbed_packed(bss, oracle_mod, lens):
 def test_host_packed_d64_and_192(bss, oracle_mod, n_sink, n_local):
     host_case(bss, oracle_mod, 460, 4300, 2, 2, 64, 64, 0.125, n_sink, n_local, lens=[2500, 300, 1500])
     host_case(bss, oracle_mod, 461, 3100, 2, 2, 192, 128, 1 / math.sqrt(192), n_sink, n_local, lens=[1100, 2000])
+
+
+# (b, s, l): page 4's token window, and block sizes below and above 128; most
+# leave a gap of zero rows between the sinks and the halo of a chunk's prefix
+GENERAL = [(1, 16, 1024), (64, 2, 14), (256, 1, 3), (32, 3, 20), (1, 0, 300), (512, 1, 2)]
+
+
+@pytest.mark.parametrize("block,n_sink,n_local", GENERAL)
+def test_host_general_windows(bss, oracle_mod, block, n_sink, n_local):
+    """Other block sizes: chunks of whole max(b, 128)-row units, the later ones
+    on [sinks | zero gap | halo | own]; the workspace starts as NaN bytes.
+    Bit for bit the device call, and the oracle."""
+    host_case(bss, oracle_mod, 470 + block + n_sink, 9000, 2, 2, 64, 64, 0.125, n_sink, n_local, block=block,
+              poison=True)
+
+
+@pytest.mark.parametrize("block,n_sink,n_local", [(1, 16, 1024), (64, 2, 14)])
+def test_host_general_windows_absorbed_and_192(bss, oracle_mod, block, n_sink, n_local):
+    """The absorbed two-pass kernel and the per-head 192/128 kernel under other
+    block sizes, packed batches, poisoned workspace."""
+    host_case(bss, oracle_mod, 480 + block, 5600, 4, 1, 576, 512, 1 / math.sqrt(192), n_sink, n_local,
+              latent=True, lens=[4000, 1, 1599], block=block, poison=True)
+    host_case(bss, oracle_mod, 490 + block, 4300, 2, 2, 192, 128, 1 / math.sqrt(192), n_sink, n_local,
+              lens=[2500, 300, 1500], block=block, poison=True)
 
 
 def test_host_pageable(bss, oracle_mod):
